@@ -1,0 +1,140 @@
+"""ctypes wrapper around the plain-C oracle (``moe_oracle.c``) -- test infrastructure only.
+
+Arrays are NumPy; bf16 tensors are passed as their raw 16-bit patterns (``np.uint16``).
+The wrapper only marshals arguments: every arithmetic step is in ``moe_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_moe.so")
+
+F32 = 0
+BF16 = 1
+
+_lib = None
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle_moe.so (gcc, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", _SRC, "-o", _LIB, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build_oracle()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_router_logits.argtypes = [P, P, I, I, I, I, P]
+        lib.oracle_route.argtypes = [P, P, I, I, I, P, P]
+        lib.oracle_permute.argtypes = [P, I, I, I, P, P, P, P]
+        lib.oracle_expert_ffn.argtypes = [P, P, P, P, I, I, I, P]
+        lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
+                                           ctypes.c_double, P, I, P, P, P, P, P]
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _as_input(a):
+    """Contiguous fp32 or bf16-bits array and its dtype code."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return a, BF16
+    if a.dtype == np.float32:
+        return a, F32
+    raise TypeError(f"oracle inputs are float32 or bf16 bits (uint16), got {a.dtype}")
+
+
+def oracle_num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def oracle_router_logits(x, w_r):
+    x, dt = _as_input(x)
+    w_r, dt2 = _as_input(w_r)
+    assert dt == dt2
+    T, d = x.shape
+    E = w_r.shape[0]
+    out = np.empty((T, E), np.float32)
+    _load().oracle_router_logits(_ptr(x), _ptr(w_r), dt, T, d, E, _ptr(out))
+    return out
+
+
+def oracle_route(logits, bias, k):
+    logits = np.ascontiguousarray(logits, np.float32)
+    T, E = logits.shape
+    bias = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    idx = np.empty((T, k), np.int32)
+    gates = np.empty((T, k), np.float32)
+    _load().oracle_route(_ptr(logits), _ptr(bias), T, E, k, _ptr(idx), _ptr(gates))
+    return idx, gates
+
+
+def oracle_permute(idx, E):
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.empty(T * k, np.int32)
+    slot_row = np.empty(T * k, np.int32)
+    _load().oracle_permute(_ptr(idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm),
+                           _ptr(slot_row))
+    return counts, offsets, perm, slot_row.reshape(T, k)
+
+
+def oracle_expert_ffn(x_row, wg, wu, wd):
+    x_row, dt = _as_input(x_row)
+    wg, _ = _as_input(wg)
+    wu, _ = _as_input(wu)
+    wd, _ = _as_input(wd)
+    f, d = wg.shape
+    y = np.empty(d, np.float64)
+    _load().oracle_expert_ffn(_ptr(x_row), _ptr(wg), _ptr(wu), _ptr(wd), dt, d, f, _ptr(y))
+    return y
+
+
+def oracle_moe_forward(x, w_r, bias, w_gate, w_up, w_down, k, n_shared=1, routed_scale=1.0,
+                       tokens=None, logits_in=None):
+    """Layer output (float64) for `tokens` (default: all), plus idx, gates, logits."""
+    x, dt = _as_input(x)
+    w_r, _ = _as_input(w_r)
+    w_gate, _ = _as_input(w_gate)
+    w_up, _ = _as_input(w_up)
+    w_down, _ = _as_input(w_down)
+    T, d = x.shape
+    E = w_r.shape[0]
+    f = w_gate.shape[1]
+    assert w_gate.shape[0] == E + n_shared
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tokens = np.ascontiguousarray(tokens, np.int32)
+    n = len(tokens)
+    out = np.empty((n, d), np.float64)
+    idx = np.empty((n, k), np.int32)
+    gates = np.empty((n, k), np.float32)
+    logits = np.empty((n, E), np.float32)
+    if logits_in is not None:
+        logits_in = np.ascontiguousarray(logits_in, np.float32)
+        assert logits_in.shape == (n, E)
+    bias = np.ascontiguousarray(bias, np.float32)
+    _load().oracle_moe_forward(_ptr(x), _ptr(w_r), _ptr(bias), _ptr(w_gate), _ptr(w_up),
+                               _ptr(w_down), dt, d, E, k, f, n_shared, float(routed_scale),
+                               _ptr(tokens), n, _ptr(logits_in), _ptr(out), _ptr(idx),
+                               _ptr(gates), _ptr(logits))
+    return out, idx, gates, logits

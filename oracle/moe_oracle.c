@@ -1,0 +1,254 @@
+/*
+ * moe_oracle.c -- plain, slow CPU oracle for one fine-grained sparse-MoE FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this
+ * file.  Only the test suite, the smoke check and the CPU-baseline leg of the benchmark
+ * use it.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (the plain definition, no blocking, no fusion, no reordering):
+ *
+ *   Sources (page title, then the passage):
+ *   [P2 2.2]   "Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active Parameters",
+ *              section 2.2 (sparse-MoE backbone): each MoE layer has 288 routed experts and
+ *              one shared expert; every token activates its top-k = 8 experts.
+ *   [P2 2.2.2] same page, section 2.2.2 (expert-parallel load balancing): loss-free load
+ *              balancing; S_t is the top-K expert set of token t, s_{t,e} = 1[e in S_t],
+ *              p_{t,e} the routing probability.
+ *   [P3 MoE]   "Step 3.5 Flash 技术论文深度解读：196B MoE 如何做到 11B 激活打 37B",
+ *              architecture item 1 (fine-grained MoE, 288 experts top-8): parameter table
+ *              (288 routed + 1 shared, top-8, routed-expert hidden size 1280) and the note
+ *              under it: balancing by bias adjustment, not an auxiliary loss.
+ *   [P3 stab]  same page, training stability, "local activation explosion", root cause 3:
+ *              the experts are SwiGLU with gate and up projection branches.
+ *   [P2 4.1.2] first page above, section 4.1.2 (expert collapse): aggregation of the
+ *              routed experts needs an explicit scale (value not given: routed_scale).
+ *   [P2 3.2.4] first page above, section 3.2.4 (GPU kernel optimisation): fused MoE
+ *              gather/scatter with grouped GEMM -- the expert-sorted permutation below.
+ *
+ *   Readings where the pages are silent (each is listed in the design notes):
+ *   - router score: logits l[t,e] = x_t . W_r[e]; the bias b_e is added for SELECTION only
+ *     (s = fl32(l + b)); the gates are a softmax over the k selected UNBIASED logits,
+ *     i.e. the full softmax renormalised over S_t.
+ *   - ties in top-k: larger fp32 score first; equal scores -> lower expert id first;
+ *     -0.0 == +0.0 (float compare); NaN ranks below every number (NaNs by id).
+ *   - the slots of a token are ordered by that same ranking (descending biased score).
+ *   - the shared expert is always on with weight 1; out = shared + routed_scale*sum g*y.
+ *   - expert-sorted order: group e holds its (t, j) pairs in ascending t.
+ *
+ * Arithmetic: inputs are decoded exactly to double (bf16 -> float is exact), every dot
+ * product is accumulated in double; logits are rounded ONCE to fp32 (they are an fp32
+ * output of the router); s = l + b is an fp32 add (the selection is decided in the same
+ * precision as the GPU's); gates are computed in double and rounded once to fp32; the
+ * expert FFNs and the combine stay in double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+/* exact bf16 (stored as its 16 high bits) -> double */
+static double orc_bf16_to_double(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* element i of a row-major matrix stored either as fp32 or as bf16 bits */
+static double orc_elem(const void *base, int dtype, size_t i) {
+  if (dtype == ORC_BF16) return orc_bf16_to_double(((const uint16_t *)base)[i]);
+  return (double)((const float *)base)[i];
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + exp(-z))   [P3 stab: SwiGLU experts] */
+static double orc_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* ranking used for top-k: returns 1 if (sa, ea) ranks strictly before (sb, eb) */
+static int orc_ranks_before(float sa, int ea, float sb, int eb) {
+  int na = isnan(sa), nb = isnan(sb);
+  if (na != nb) return nb;          /* a number ranks before a NaN */
+  if (!na && sa != sb) return sa > sb;
+  return ea < eb;                   /* equal scores (or both NaN): lower id first */
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Router logits: l[t,e] = sum_i x[t,i] * W_r[e,i], double accumulation, one fp32 round. */
+/* [P2 2.2.2]: p_{t,e} is a distribution over experts computed from these logits.        */
+void oracle_router_logits(const void *x, const void *w_r, int dtype, int T, int d, int E,
+                          float *logits) {
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i)
+        acc += orc_elem(x, dtype, (size_t)t * d + i) * orc_elem(w_r, dtype, (size_t)e * d + i);
+      logits[(size_t)t * E + e] = (float)acc;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Selection and gates for one token.                                                     */
+/* [P3 MoE] bias for selection only; [P2 2.2.2] S_t = top-K set; gates renormalised.       */
+static void orc_route_token(const float *l, const float *bias, int E, int k, int *idx,
+                            float *gates) {
+  /* s = fl32(l + b): the fp32 add decides the selection */
+  float *s = (float *)malloc(sizeof(float) * (size_t)E);
+  int *order = (int *)malloc(sizeof(int) * (size_t)E);
+  for (int e = 0; e < E; ++e) {
+    s[e] = l[e] + (bias ? bias[e] : 0.0f);
+    order[e] = e;
+  }
+  /* full insertion sort of all E experts by the ranking, then take the first k */
+  for (int a = 1; a < E; ++a) {
+    int cur = order[a];
+    int b = a - 1;
+    while (b >= 0 && orc_ranks_before(s[cur], cur, s[order[b]], order[b])) {
+      order[b + 1] = order[b];
+      --b;
+    }
+    order[b + 1] = cur;
+  }
+  /* gates: softmax over the k selected unbiased logits (max-shifted), double */
+  double m = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    double v = (double)l[order[j]];
+    if (v > m) m = v;
+  }
+  double z = 0.0;
+  for (int j = 0; j < k; ++j) z += exp((double)l[order[j]] - m);
+  for (int j = 0; j < k; ++j) {
+    idx[j] = order[j];
+    gates[j] = (float)(exp((double)l[order[j]] - m) / z);
+  }
+  free(s);
+  free(order);
+}
+
+void oracle_route(const float *logits, const float *bias, int T, int E, int k, int *idx,
+                  float *gates) {
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t)
+    orc_route_token(logits + (size_t)t * E, bias, E, k, idx + (size_t)t * k,
+                    gates + (size_t)t * k);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Expert-sorted permutation by counting sort.  [P2 3.2.4] gather/scatter grouping.        */
+/* counts[e] = |{t : e in S_t}|; offsets = exclusive prefix sum (offsets[E] = T*k);        */
+/* perm[offsets[e] + r] = t*k + j for the r-th token (ascending t) that chose e in slot j; */
+/* slot_row[t*k + j] = that position.                                                      */
+void oracle_permute(const int *idx, int T, int E, int k, int *counts, int *offsets,
+                    int *perm, int *slot_row) {
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int q = 0; q < T * k; ++q) counts[idx[q]] += 1;
+  offsets[0] = 0;
+  for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int *fill = (int *)calloc((size_t)E, sizeof(int));
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      int q = t * k + j;
+      int e = idx[q];
+      int p = offsets[e] + fill[e];
+      fill[e] += 1;
+      perm[p] = q;
+      slot_row[q] = p;
+    }
+  }
+  free(fill);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* One SwiGLU expert on one token, double:  [P3 stab]                                     */
+/*   g_r = x . W_g[r],  u_r = x . W_u[r],  h_r = silu(g_r) * u_r,  y_c = sum_r h_r W_d[c,r] */
+/* W_g, W_u are [f, d] row-major (d contiguous); W_d is [d, f] row-major (f contiguous).    */
+void oracle_expert_ffn(const void *x_row, const void *wg, const void *wu, const void *wd,
+                       int dtype, int d, int f, double *y) {
+  double *h = (double *)malloc(sizeof(double) * (size_t)f);
+  for (int r = 0; r < f; ++r) {
+    double g = 0.0, u = 0.0;
+    for (int i = 0; i < d; ++i) {
+      double xi = orc_elem(x_row, dtype, (size_t)i);
+      g += xi * orc_elem(wg, dtype, (size_t)r * d + i);
+      u += xi * orc_elem(wu, dtype, (size_t)r * d + i);
+    }
+    h[r] = orc_silu(g) * u;
+  }
+  for (int c = 0; c < d; ++c) {
+    double acc = 0.0;
+    for (int r = 0; r < f; ++r) acc += h[r] * orc_elem(wd, dtype, (size_t)c * f + r);
+    y[c] = acc;
+  }
+  free(h);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* The whole layer for a list of tokens (all of them, or a sample).                        */
+/*   out[i,:] = shared(x_t) + routed_scale * sum_j g[t,j] * expert_{idx[t,j]}(x_t)          */
+/* [P2 2.2] shared expert always on; [P2 4.1.2] explicit routed scale.                     */
+/* Expert e's weights start at element e*f*d of w_gate / w_up and e*d*f of w_down; the     */
+/* shared expert (if n_shared == 1) is expert index E in the same arrays.                  */
+/* If `logits_in` is non-null the router logits of the listed tokens are taken from it     */
+/* ([n_list, E]); otherwise they are computed by oracle_router_logits' definition.         */
+/* idx_out / gates_out / logits_out ([n_list, k] / [n_list, k] / [n_list, E]) may be null.  */
+void oracle_moe_forward(const void *x, const void *w_r, const float *bias, const void *w_gate,
+                        const void *w_up, const void *w_down, int dtype, int d, int E, int k,
+                        int f, int n_shared, double routed_scale, const int *tokens, int n_list,
+                        const float *logits_in, double *out, int *idx_out, float *gates_out,
+                        float *logits_out) {
+  const size_t esz = (dtype == ORC_BF16) ? 2 : 4;
+  const size_t wsz = (size_t)f * (size_t)d; /* elements per expert matrix */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < n_list; ++i) {
+    const int t = tokens[i];
+    const char *xr = (const char *)x + (size_t)t * d * esz;
+    float *l = (float *)malloc(sizeof(float) * (size_t)E);
+    if (logits_in) {
+      memcpy(l, logits_in + (size_t)i * E, sizeof(float) * (size_t)E);
+    } else {
+      for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c)
+          acc += orc_elem(xr, dtype, (size_t)c) * orc_elem(w_r, dtype, (size_t)e * d + c);
+        l[e] = (float)acc;
+      }
+    }
+    int *idx = (int *)malloc(sizeof(int) * (size_t)k);
+    float *g = (float *)malloc(sizeof(float) * (size_t)k);
+    orc_route_token(l, bias, E, k, idx, g);
+    double *o = out + (size_t)i * d;
+    double *y = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[j];
+      oracle_expert_ffn(xr, (const char *)w_gate + (size_t)e * wsz * esz,
+                        (const char *)w_up + (size_t)e * wsz * esz,
+                        (const char *)w_down + (size_t)e * wsz * esz, dtype, d, f, y);
+      for (int c = 0; c < d; ++c) o[c] += routed_scale * (double)g[j] * y[c];
+    }
+    if (n_shared) {
+      oracle_expert_ffn(xr, (const char *)w_gate + (size_t)E * wsz * esz,
+                        (const char *)w_up + (size_t)E * wsz * esz,
+                        (const char *)w_down + (size_t)E * wsz * esz, dtype, d, f, y);
+      for (int c = 0; c < d; ++c) o[c] += y[c];
+    }
+    if (idx_out) memcpy(idx_out + (size_t)i * k, idx, sizeof(int) * (size_t)k);
+    if (gates_out) memcpy(gates_out + (size_t)i * k, g, sizeof(float) * (size_t)k);
+    if (logits_out) memcpy(logits_out + (size_t)i * E, l, sizeof(float) * (size_t)E);
+    free(y);
+    free(g);
+    free(idx);
+    free(l);
+  }
+}
+
+/* number of OpenMP threads the oracle runs with (1 when built without OpenMP) */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+#else
+int oracle_num_threads(void) { return 1; }
+#endif

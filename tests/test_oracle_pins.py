@@ -1,0 +1,215 @@
+"""Pins for the CPU oracle (no GPU): closed forms, special cases that reduce to library
+routines, brute force on tiny inputs, invariants, and the independent NumPy restatement.
+
+Each pin is chosen so a plausible slip in the oracle fails it:
+  * dropped/transposed term in the expert FFN  -> textbook SwiGLU via torch (E = k = 1)
+  * wrong silu, wrong gate normalisation, sign -> silu antisymmetry closed form (golden)
+  * bias leaking into the gates                 -> topk_ties golden case 4 and 6
+  * wrong tie / NaN rule, wrong slot order      -> topk_ties golden + torch.topk
+  * permutation index slip                      -> numpy stable argsort + invariants
+  * routed/shared mix-up, missing routed scale  -> identical-experts invariance, zero W_down
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import (oracle_expert_ffn, oracle_moe_forward, oracle_permute, oracle_route,
+                    oracle_router_logits)
+from oracle import moe_numpy as onp
+from sparse_moe_layer_warp_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f(v):
+    return {"nan": math.nan, "-inf": -math.inf, "inf": math.inf}.get(v, v) if isinstance(v, str) else v
+
+
+def _small_inputs(name="tiny_fp32", **kw):
+    w = synth.WORKLOADS[name].replace(**kw)
+    inp = synth.make_inputs(w)
+    cv = synth.to_numpy_bits
+    return w, [cv(t) for t in (inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down)]
+
+
+# ----------------------------------------------------------------------------- golden
+def test_golden_silu_antisymmetry_closed_form():
+    g = json.load(open(os.path.join(GOLDEN, "silu_antisymmetry.json")))
+    arr = lambda k: np.array(g[k], np.float32)  # noqa: E731
+    for case in g["cases"]:
+        out, idx, gates, _ = oracle_moe_forward(arr("x"), arr("w_router"), arr("bias"),
+                                                arr("w_gate"), arr("w_up"), arr("w_down"),
+                                                k=g["k"], n_shared=1,
+                                                routed_scale=case["routed_scale"])
+        np.testing.assert_allclose(out, np.array(case["out"]), rtol=0, atol=1e-12)
+        assert (idx == np.array(case["idx"])[None, :]).all()
+        np.testing.assert_array_equal(gates, np.broadcast_to(np.float32(case["gates"]), gates.shape))
+
+
+def test_golden_topk_ties_nan_signed_zero():
+    g = json.load(open(os.path.join(GOLDEN, "topk_ties.json")))
+    for case in g["cases"]:
+        logits = np.array([[_f(v) for v in case["logits"]]], np.float32)
+        bias = np.array(case["bias"], np.float32)
+        idx, gates = oracle_route(logits, bias, case["k"])
+        assert idx[0].tolist() == case["idx"], case
+        np.testing.assert_allclose(gates[0], case["gates"], rtol=2e-7, atol=1e-30)
+        idx2, gates2, _ = onp.np_select(logits, bias, case["k"])
+        assert idx2[0].tolist() == case["idx"], case
+
+
+# ------------------------------------------------------------------- library reductions
+def test_topk_matches_torch_topk_without_ties():
+    logits = synth.make_logits(300, 288, seed=3).numpy()
+    bias = synth.make_bias(synth.WORKLOADS["decode_t16"], torch.Generator().manual_seed(1), "cpu").numpy()
+    s = torch.from_numpy(logits) + torch.from_numpy(bias)
+    ref = torch.topk(s, 8, dim=1, largest=True, sorted=True).indices.numpy()
+    idx, gates = oracle_route(logits, bias, 8)
+    assert (idx == ref).all()
+    # gates: softmax of the UNBIASED logits of the selection (torch.softmax as the library routine)
+    sel = np.take_along_axis(logits, idx.astype(np.int64), axis=1)
+    ref_g = torch.softmax(torch.from_numpy(sel).double(), dim=1).numpy()
+    np.testing.assert_allclose(gates, ref_g, rtol=1e-6, atol=0)
+
+
+def test_gates_k_equals_E_zero_bias_is_full_softmax():
+    logits = synth.make_logits(40, 16, seed=5).numpy()
+    idx, gates = oracle_route(logits, np.zeros(16, np.float32), 16)
+    full = torch.softmax(torch.from_numpy(logits).double(), dim=1).numpy()
+    got = np.zeros_like(full)
+    np.put_along_axis(got, idx.astype(np.int64), gates.astype(np.float64), axis=1)
+    np.testing.assert_allclose(got, full, rtol=1e-6, atol=1e-12)
+
+
+def test_gates_k1_is_one_and_sum_to_one():
+    logits = synth.make_logits(50, 24, seed=6).numpy()
+    _, g1 = oracle_route(logits, None, 1)
+    assert (g1 == 1.0).all()
+    idx, g = oracle_route(logits, None, 5)
+    assert np.abs(g.astype(np.float64).sum(1) - 1).max() < 1e-6
+    assert (g > 0).all()
+    for row in idx:
+        assert len(set(row.tolist())) == 5
+
+
+def test_router_logits_match_library_matmul():
+    w, (x, wr, *_rest) = _small_inputs()
+    got = oracle_router_logits(x, wr)
+    ref = (x.astype(np.float64) @ wr.astype(np.float64).T).astype(np.float32)
+    # double accumulation in either order rounds to the same fp32 except at most 1 ulp
+    assert np.max(np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32))) <= 1
+
+
+def test_expert_ffn_E1_k1_is_textbook_swiglu():
+    """E = k = 1: gate = 1 and the layer is FFN_0(x) + FFN_shared(x) (textbook SwiGLU)."""
+    w, (x, wr, b, wg, wu, wd) = _small_inputs(E=1, k=1)
+    wr = wr[:1]
+    b = b[:1]
+    out, idx, gates, _ = oracle_moe_forward(x, wr, b, wg[:2], wu[:2], wd[:2], k=1)
+    assert (idx == 0).all() and (gates == 1.0).all()
+    X = torch.from_numpy(x).double()
+    ref = torch.zeros_like(X)
+    for e in range(2):
+        Wg, Wu, Wd = (torch.from_numpy(a[e]).double() for a in (wg, wu, wd))
+        ref += (torch.nn.functional.silu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    y = oracle_expert_ffn(x[3], wg[0], wu[0], wd[0])
+    Wg, Wu, Wd = (torch.from_numpy(a[0]).double() for a in (wg, wu, wd))
+    y_ref = (torch.nn.functional.silu(X[3] @ Wg.T) * (X[3] @ Wu.T)) @ Wd.T
+    np.testing.assert_allclose(y, y_ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_identical_experts_make_routing_irrelevant():
+    """All routed experts equal => sum_j g_j y = y (gates sum to 1): closed form."""
+    w, (x, wr, b, wg, wu, wd) = _small_inputs()
+    E = w.E
+    for a in (wg, wu, wd):
+        a[:E] = a[0]
+    scale = 1.75
+    out, *_ = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k, routed_scale=scale)
+    X = torch.from_numpy(x).double()
+
+    def ffn(e):
+        Wg, Wu, Wd = (torch.from_numpy(a[e]).double() for a in (wg, wu, wd))
+        return (torch.nn.functional.silu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
+
+    ref = (scale * ffn(0) + ffn(E)).numpy()
+    # the gates are fp32 outputs, so they sum to 1 only within k * 2^-24
+    np.testing.assert_allclose(out, ref, rtol=0, atol=w.k * 2.0**-23 * scale * np.abs(ref).max())
+
+
+def test_zero_routed_down_gives_shared_only():
+    w, (x, wr, b, wg, wu, wd) = _small_inputs()
+    wd = wd.copy()
+    wd[: w.E] = 0
+    out, *_ = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k)
+    X = torch.from_numpy(x).double()
+    Wg, Wu, Wd = (torch.from_numpy(a[w.E]).double() for a in (wg, wu, wd))
+    ref = (torch.nn.functional.silu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------------- permutation
+@pytest.mark.parametrize("T,E,k,seed", [(64, 16, 2, 0), (37, 288, 8, 1), (1, 5, 5, 2), (300, 7, 3, 3)])
+def test_permute_is_stable_argsort_and_invariants(T, E, k, seed):
+    logits = synth.make_logits(T, E, seed=seed, ties=(seed % 2 == 1)).numpy()
+    idx, _ = oracle_route(logits, None, k)
+    counts, offsets, perm, slot_row = oracle_permute(idx, E)
+    flat = idx.reshape(-1)
+    assert (perm == np.argsort(flat, kind="stable")).all()
+    assert counts.sum() == T * k and offsets[0] == 0 and offsets[-1] == T * k
+    assert (np.diff(offsets) == counts).all()
+    assert sorted(perm.tolist()) == list(range(T * k))
+    assert (perm[slot_row.reshape(-1)] == np.arange(T * k)).all()
+    for e in range(E):
+        toks = perm[offsets[e]:offsets[e + 1]] // k
+        assert (np.diff(toks) > 0).all()
+        assert (flat[perm[offsets[e]:offsets[e + 1]]] == e).all()
+
+
+def test_route_k_distinct_and_brute_force_rank():
+    """Brute force: e is selected iff fewer than k experts rank before it."""
+    logits = synth.make_logits(30, 12, seed=9, ties=True).numpy()
+    bias = np.linspace(-0.2, 0.2, 12).astype(np.float32)
+    idx, _ = oracle_route(logits, bias, 4)
+    s = logits + bias
+    for t in range(30):
+        sel = set()
+        for e in range(12):
+            before = sum(1 for o in range(12) if s[t, o] > s[t, e] or (s[t, o] == s[t, e] and o < e))
+            if before < 4:
+                sel.add(e)
+        assert sel == set(idx[t].tolist())
+        assert len(set(idx[t].tolist())) == 4
+
+
+# ----------------------------------------------------------------- NumPy restatement
+@pytest.mark.parametrize("name,kw", [("tiny_fp32", {}),
+                                     ("tiny_fp32", {"dtype": "bf16", "E": 9, "k": 3, "T": 21}),
+                                     ("tiny_fp32", {"bias": "zipf", "seed": 4})])
+def test_c_oracle_matches_numpy_brute_force(name, kw):
+    w, (x, wr, b, wg, wu, wd) = _small_inputs(name, **kw)
+    out, idx, gates, logits = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k, routed_scale=1.0)
+    out2, idx2, gates2, logits2 = onp.np_moe_forward(x, wr, b, wg, wu, wd, k=w.k, logits=logits)
+    assert (idx == idx2).all()
+    np.testing.assert_allclose(gates, gates2, rtol=2e-7, atol=0)
+    np.testing.assert_allclose(out, out2, rtol=1e-9, atol=1e-9 * np.abs(out2).max())
+    # the oracle's own logits agree with the NumPy matmul to 1 ulp
+    assert np.max(np.abs(logits.view(np.int32).astype(np.int64) -
+                         onp.np_logits(x, wr).view(np.int32))) <= 1
+    c, o, p, s = oracle_permute(idx, w.E)
+    c2, o2, p2, s2 = onp.np_permute(idx, w.E)
+    assert (c == c2).all() and (o == o2).all() and (p == p2).all() and (s == s2).all()
+
+
+def test_sampled_tokens_equal_full_run():
+    w, (x, wr, b, wg, wu, wd) = _small_inputs()
+    full, idx, gates, _ = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k)
+    toks = np.array([5, 0, 63, 17], np.int32)
+    part, idx2, gates2, _ = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k, tokens=toks)
+    np.testing.assert_array_equal(part, full[toks])
+    np.testing.assert_array_equal(idx2, idx[toks])
