@@ -1,0 +1,405 @@
+"""Benchmark of the sparse-MoE FFN layer on B200: tokens/s of one layer forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole layer forward (router -> top-k -> permutation -> gather -> expert up +
+SwiGLU -> expert down -> combine) over one batch of T synthetic tokens already resident in
+HBM.  Each step uses a different seeded batch, and L2 is flushed (256 MiB write) between
+steps outside the timed intervals.  Times come from CUDA events the library records on its
+launch stream around each kernel stage (moe_forward_profiled), summed over the K timed
+steps, max over ranks.  N > 1 runs N independent replicas (one per GPU, no data-path
+collective): value = all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle (plain C, fp64) on the host cores instead, on a
+bounded sample of each step's batch; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s on 1 B200; achieved HBM GB/s / tensor-pipe % of peak"
+DEFAULT_WORKLOAD = "decode_t16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                 0x100: "display_clock_setting"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------ clocks sampler
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 5:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                bits = int(parts[4], 16)
+            except ValueError:
+                continue
+            for b, name in THROTTLE_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ roofline model
+def algorithmic(w, counts, T):
+    """Algorithmic bytes / flops of each stage for one forward (touched experts only)."""
+    import numpy as np
+
+    touched = int((np.asarray(counts) > 0).sum()) + w.n_shared
+    es = 2 if w.dtype == "bf16" else 4
+    Tk = T * w.k
+    P = Tk + w.n_shared * T
+    d, f, E = w.d, w.f, w.E
+    up_bytes = touched * 2 * f * d * es + (Tk + w.n_shared * T) * d * es + P * f * es
+    down_bytes = touched * d * f * es + P * f * es + P * d * es
+    up_flops = 2.0 * P * 2 * f * d
+    down_flops = 2.0 * P * d * f
+    layer_bytes = touched * 3 * f * d * es + E * d * es + 2 * T * d * es
+    layer_flops = up_flops + down_flops + 2.0 * T * d * E
+    return dict(touched=touched, up_bytes=up_bytes, down_bytes=down_bytes, up_flops=up_flops,
+                down_flops=down_flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
+
+
+def kernel_source_sha():
+    csrc = os.path.join(ROOT, "sparse_moe_layer_warp_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(f"{kernel}/{workload}")
+    if not ent or ent.get("source_sha") != kernel_source_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from sparse_moe_layer_warp_b200 import (MOE_PROFILE_STAGES, PROFILE_STAGE_NAMES, MoELayer,
+                                            moe_forward, moe_forward_profiled, synth)
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    T = w.T
+    inp = synth.make_inputs(w, device=dev)
+    layer = MoELayer(inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down, top_k=w.k,
+                     max_tokens=T, n_shared=w.n_shared, routed_scale=w.routed_scale)
+    nb = args.steps + args.warmup
+    batches = [synth.make_x(w, T, device=dev, seed=1000 * (rank + 1) + i) for i in range(nb)]
+    out = torch.empty_like(batches[0])
+    ws = layer.workspace(T)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # routing statistics of every timed batch (outside the timed region) for the roofline
+    algo = []
+    for i in range(args.warmup, nb):
+        r = layer.route(x=batches[i])
+        algo.append(algorithmic(w, r["counts"].cpu().numpy(), T))
+    st = torch.cuda.current_stream()
+
+    for i in range(args.warmup):
+        flush.zero_()
+        moe_forward(layer.handle, batches[i], T, out, ws)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(MOE_PROFILE_STAGES + 1)]
+           for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local_rank] if visible else local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        moe_forward_profiled(layer.handle, batches[args.warmup + i], T, out, ws, evs[i], st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(MOE_PROFILE_STAGES)]
+                         for i in range(args.steps)])
+    step_ms = np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)])
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = layer.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # end to end through the public API: pinned host x in, host out back, per step
+    hx = [b.cpu().pin_memory() for b in batches]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dx = torch.empty_like(batches[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        dx.copy_(hx[i], non_blocking=True)
+        moe_forward(layer.handle, dx, T, out, ws)
+        hout.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(st)
+    for i in range(args.steps):
+        dx.copy_(hx[args.warmup + i], non_blocking=True)
+        moe_forward(layer.handle, dx, T, out, ws)
+        hout.copy_(out, non_blocking=True)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    mean_stage = stage_ms.mean(axis=0)
+    names = list(PROFILE_STAGE_NAMES)
+    up_i, down_i = names.index("expert_up_swiglu"), names.index("expert_down")
+    dom = up_i if mean_stage[up_i] >= mean_stage[down_i] else down_i
+    dom_name = "grouped_gemm_up" if dom == up_i else "grouped_gemm_down"
+    key = "up" if dom == up_i else "down"
+    bytes_per = float(np.mean([a[f"{key}_bytes"] for a in algo]))
+    flops_per = float(np.mean([a[f"{key}_flops"] for a in algo]))
+    dur_s = mean_stage[dom] / 1e3
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops_per / bytes_per > ridge:
+        achieved = flops_per / dur_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        achieved = bytes_per / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = round(achieved / roof["peak"], 4)
+    roof["traffic"] = ncu_traffic(dom_name, args.workload)
+    roof["kernel"] = dom_name
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    roof["algorithmic_bytes_per_launch"] = int(bytes_per)
+    roof["algorithmic_flops_per_launch"] = int(flops_per)
+    layer_bytes = float(np.mean([a["layer_bytes"] for a in algo]))
+    layer_flops = float(np.mean([a["layer_flops"] for a in algo]))
+    step_s = total_ms / args.steps / 1e3
+    value = world * args.steps * T / (total_ms / 1e3)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; a different x batch every step; random-init weights)",
+        "config": {"workload": w.name, "tokens": T, "d_model": w.d, "n_experts": w.E,
+                   "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)"},
+        "roofline": roof,
+        "layer_roofline": {"algorithmic_bytes": int(layer_bytes), "algorithmic_flops": int(layer_flops),
+                           "hbm_frac": round(layer_bytes / step_s / 1e9 / peaks["hbm_gbs"], 4),
+                           "tensor_frac": round(layer_flops / step_s / 1e12 / peaks["bf16_tflops"], 4),
+                           "touched_experts_mean": float(np.mean([a["touched"] for a in algo]))},
+        "stages_ms": {n: round(float(v), 4) for n, v in zip(names, mean_stage)},
+        "e2e": {"value": round(world * args.steps * T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4)),
+                "d2h_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4))},
+        "gpu_launches": int(world * args.steps * (7 if w.dtype == "bf16" else 6)),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, batches[args.warmup], budget_s=args.cpu_budget)
+    return res
+
+
+# ------------------------------------------------------------------------ oracle timing
+def _host_weights(inp):
+    from sparse_moe_layer_warp_b200 import synth
+
+    cv = synth.to_numpy_bits
+    return [cv(t) for t in (inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down)]
+
+
+def cpu_baseline(w, inp, x_batch, budget_s=15.0, host=None):
+    """The oracle, as it stands, on a bounded sample of one batch (tokens/s)."""
+    import numpy as np
+
+    from oracle import oracle_moe_forward, oracle_num_threads
+    from sparse_moe_layer_warp_b200 import synth
+
+    wr, b, wg, wu, wd = host if host is not None else _host_weights(inp)
+    x = synth.to_numpy_bits(x_batch)
+    cores = oracle_num_threads()
+    n = min(x.shape[0], cores)
+    done, t0 = 0, time.perf_counter()
+    start = 0
+    while True:
+        toks = (np.arange(n) + start) % x.shape[0]
+        oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k, n_shared=w.n_shared,
+                           routed_scale=w.routed_scale, tokens=toks.astype(np.int32))
+        done += n
+        start += n
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 4 * x.shape[0]:
+            break
+    return {"value": round(done / el, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} tokens of one {w.name} batch ({el:.1f} s of plain-C fp64 oracle, "
+                      f"OpenMP over tokens)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+
+    from oracle import oracle_moe_forward, oracle_num_threads
+    from sparse_moe_layer_warp_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.make_inputs(w, device=dev)
+    host = _host_weights(inp)
+    wr, b, wg, wu, wd = host
+    cores = oracle_num_threads()
+    sample = min(w.T, max(1, cores))
+    xs = [synth.to_numpy_bits(synth.make_x(w, w.T, device=dev, seed=1000 + i))
+          for i in range(args.steps + args.warmup)]
+
+    def step(i):
+        toks = np.arange(sample, dtype=np.int32)
+        oracle_moe_forward(xs[i], wr, b, wg, wu, wd, k=w.k, n_shared=w.n_shared,
+                           routed_scale=w.routed_scale, tokens=toks)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    value = args.steps * sample / el
+    desc = (f"{sample} of the {w.T} tokens of each step's {w.name} batch, plain-C fp64 oracle, "
+            f"OpenMP over tokens")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "tokens": w.T, "d_model": w.d, "n_experts": w.E,
+                       "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        ap.error(f"WORLD_SIZE={world} but --gpus {args.gpus}")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch.distributed as dist
+    import datetime
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=None)
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,149 @@
+/*
+ * moe_layer.h -- C ABI of the B200 (sm_100a) sparse-MoE FFN layer library (libmoe_layer.so).
+ *
+ * One fine-grained sparse-MoE FFN layer as described in "Step 3.5 Flash: Open
+ * Frontier-Level Intelligence with 11B Active Parameters" (section 2.2: 288 routed experts
+ * plus one always-on shared expert, top-k = 8 per token; section 2.2.2: loss-free
+ * balancing, top-K set S_t and routing probabilities p_{t,e}; section 3.2.4: fused MoE
+ * gather/scatter with grouped GEMM; section 4.1.2: routed aggregation needs an explicit
+ * scale) and in the parameter table of "Step 3.5 Flash 技术论文深度解读" (architecture
+ * item 1: routed-expert hidden size 1280, balancing by a bias instead of an auxiliary
+ * loss; training-stability item: SwiGLU experts with gate and up branches).
+ *
+ * The layer, for token t with input row x_t (d = d_model, E routed experts, k = top_k,
+ * f = d_ff, G = E + n_shared expert weight sets):
+ *   l[t,e]  = x_t . W_r[e]                              router logits (fp32 accumulation)
+ *   s[t,e]  = l[t,e] + b[e]                             fp32 add; the bias only SELECTS
+ *   S_t     = the k experts with the largest s; equal scores -> lower expert id first,
+ *             -0.0 == +0.0, NaN below every number; slot j = rank j
+ *   g[t,j]  = exp(l[t,S_t[j]] - m) / sum_j' exp(l[t,S_t[j']] - m), m = max over S_t
+ *   FFN_e(x) = W_d[e] . (silu(W_g[e] . x) * (W_u[e] . x)),  silu(z) = z / (1 + exp(-z))
+ *   out_t   = FFN_E(x_t) [shared, if n_shared] + routed_scale * sum_j g[t,j] FFN_{S_t[j]}(x_t)
+ *
+ * Ownership and memory: every device buffer (weights, x, out, routing outputs, workspace)
+ * belongs to the caller.  The library never allocates device memory; it keeps the weight
+ * pointers (which must outlive the handle) and host-side TMA descriptors.  All calls that
+ * take a stream are asynchronous on that stream, never synchronise the host, and may be
+ * captured into a CUDA graph.  Argument, size and alignment errors are returned before
+ * anything is launched; a failed launch returns MOE_ERR_CUDA.  Device-side waits are
+ * bounded: a wait that gives up records a flag in the workspace, which
+ * moe_device_status() reports.
+ *
+ * Layouts (all row-major, innermost dimension contiguous):
+ *   x        [n_tokens, d]          dtype            out   [n_tokens, d]  dtype
+ *   w_router [E, d]                 dtype            bias  [E]            fp32
+ *   w_gate   [G, f, d]              dtype            w_up  [G, f, d]      dtype
+ *   w_down   [G, d, f]              dtype            (shared expert = index E)
+ *   logits   [n_tokens, E] fp32     topk_idx [n_tokens, k] int32   topk_gate [n_tokens, k] fp32
+ *   expert_counts [E] int32         expert_offsets [E + 1] int32 (exclusive prefix sum)
+ *   perm     [n_tokens * k] int32   perm[expert_offsets[e] + r] = t * k + j for the r-th
+ *                                   token (ascending t) that selected e, in slot j
+ *   slot_row [n_tokens, k] int32    inverse of perm: slot_row[t, j] = position of (t, j)
+ * For MOE_BF16 the tensor-core path needs d % 128 == 0, f % 128 == 0 and every device
+ * pointer 16-byte aligned.  MOE_F32 runs exact fp32 SIMT arithmetic (no TF32).
+ */
+#ifndef MOE_LAYER_H
+#define MOE_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, k > E, n_tokens > max_tokens ... */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape the kernels do not handle (see layout notes above) */
+  MOE_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
+  MOE_ERR_WORKSPACE = 4,     /* workspace null or smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 5,          /* a CUDA runtime / driver call or a launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 6 /* a bounded device-side wait gave up (moe_device_status) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer shape.  max_tokens bounds n_tokens of every call; n_shared is 0 or 1;
+ * routed_scale multiplies the gate-weighted routed sum (1.0 when the pages give no value). */
+typedef struct {
+  int max_tokens;
+  int d_model;
+  int n_experts;
+  int top_k;
+  int d_ff;
+  int n_shared;
+  moe_dtype dtype;
+  float routed_scale;
+} moe_config;
+
+/* Caller-owned device pointers to the layer's weights (layouts above). */
+typedef struct {
+  const void *w_router;
+  const float *router_bias; /* may be null: zero bias */
+  const void *w_gate;
+  const void *w_up;
+  const void *w_down;
+} moe_weights;
+
+typedef struct moe_layer *moe_handle;
+
+/* Validates the shape and the weight pointers, records them and encodes the weight TMA
+ * descriptors on the current CUDA device.  Host only: no device allocation, no launch, no
+ * synchronisation.  On success *out is a new handle (free it with moe_layer_destroy). */
+moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handle *out);
+
+/* Releases the host-side handle.  Does not touch any device buffer. */
+moe_status moe_layer_destroy(moe_handle h);
+
+/* Bytes of device workspace a call with n_tokens tokens needs (0 on bad arguments).
+ * The workspace holds the routing scratch, the expert-sorted activations, the SwiGLU
+ * outputs h and the per-row expert outputs y between the kernels of one call. */
+size_t moe_workspace_size(moe_handle h, int n_tokens);
+
+/* Clears the workspace's device status word (call once after allocating a workspace). */
+moe_status moe_workspace_init(moe_handle h, void *ws, size_t ws_bytes, void *stream);
+
+/* Router, selection and permutation ("fused MoE gather/scatter", section 3.2.4): computes
+ * logits (written to logits_out if non-null), topk_idx, topk_gate, expert_counts,
+ * expert_offsets, perm and slot_row.  `stream` is a cudaStream_t (null = default). */
+moe_status moe_route(moe_handle h, const void *x, int n_tokens, float *logits_out,
+                     int *topk_idx, float *topk_gate, int *expert_counts, int *expert_offsets,
+                     int *perm, int *slot_row, void *ws, size_t ws_bytes, void *stream);
+
+/* Same as moe_route but starting from caller-supplied fp32 logits [n_tokens, E]: selection
+ * and permutation are then fully determined by integer-exact rules, which makes the
+ * routing outputs comparable bit for bit. */
+moe_status moe_route_from_logits(moe_handle h, const float *logits, int n_tokens,
+                                 int *topk_idx, float *topk_gate, int *expert_counts,
+                                 int *expert_offsets, int *perm, int *slot_row, void *ws,
+                                 size_t ws_bytes, void *stream);
+
+/* The whole layer: out = shared + routed_scale * sum_j g_j FFN_{S_t[j]}(x_t).  bf16 runs
+ * the expert contractions on tcgen05 tensor cores with fp32 accumulation; h and the
+ * per-row expert outputs are rounded to bf16 and the combine sums in fp32. */
+moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* moe_forward that also records caller-created CUDA events (cudaEvent_t, passed as void*)
+ * on `stream` around its kernel stages, for per-kernel timing with no profiler attached:
+ *   events[0] before the router, then one event after each of the MOE_PROFILE_STAGES
+ *   stages: 1 router logits, 2 top-k + gates + chunk histograms, 3 permutation scatter,
+ *   4 row gather (bf16; empty for fp32), 5 expert up + SwiGLU, 6 expert down, 7 combine.
+ * n_events must be at least MOE_PROFILE_STAGES + 1; otherwise MOE_ERR_INVALID_ARG. */
+#define MOE_PROFILE_STAGES 7
+moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void *out,
+                                void *ws, size_t ws_bytes, void *stream, void *const *events,
+                                int n_events);
+
+/* Waits for `stream`, then reads and clears the workspace's device status word:
+ * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
+moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
+
+/* Static description of a status code. */
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_LAYER_H */

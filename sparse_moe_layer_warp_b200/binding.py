@@ -1,0 +1,230 @@
+"""Thin ctypes binding of ``libmoe_layer.so`` (C ABI declared in ``include/moe_layer.h``).
+
+Argument marshalling only: torch tensors supply device pointers and the current CUDA
+stream; every step of the layer runs in the library's kernels.  There is no fallback: if
+the shared library is missing or fails to load, importing the functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_layer.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_ALIGNMENT = 3
+MOE_ERR_WORKSPACE = 4
+MOE_ERR_CUDA = 5
+MOE_ERR_DEVICE_TIMEOUT = 6
+
+MOE_F32 = 0
+MOE_BF16 = 1
+
+# every entry point the header declares (checked by tests against the built library)
+EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_workspace_init",
+           "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
+           "moe_device_status", "moe_status_string")
+MOE_PROFILE_STAGES = 7
+PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
+                       "expert_up_swiglu", "expert_down", "combine")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("max_tokens", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int), ("d_ff", ctypes.c_int),
+                ("n_shared", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("routed_scale", ctypes.c_float)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: status {status} ({status_string(status)})")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe_layer.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} is missing: build it with `python -m "
+                          "sparse_moe_layer_warp_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.moe_layer_init.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights),
+                                       ctypes.POINTER(P)]
+        lib.moe_layer_destroy.argtypes = [P]
+        lib.moe_workspace_size.argtypes = [P, I]
+        lib.moe_workspace_size.restype = Z
+        lib.moe_workspace_init.argtypes = [P, P, Z, P]
+        lib.moe_route.argtypes = [P, P, I, P, P, P, P, P, P, P, P, Z, P]
+        lib.moe_route_from_logits.argtypes = [P, P, I, P, P, P, P, P, P, P, Z, P]
+        lib.moe_forward.argtypes = [P, P, I, P, P, Z, P]
+        lib.moe_forward_profiled.argtypes = [P, P, I, P, P, Z, P, ctypes.POINTER(P), I]
+        lib.moe_device_status.argtypes = [P, P, Z, P]
+        lib.moe_status_string.argtypes = [I]
+        lib.moe_status_string.restype = ctypes.c_char_p
+        for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
+                     "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
+                     "moe_device_status"):
+            getattr(lib, name).restype = I
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().moe_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoEError(fn, status)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------------ C-ABI mirrors
+def moe_layer_init(cfg: moe_config, w_router, router_bias, w_gate, w_up, w_down):
+    lib = load_library()
+    w = moe_weights(w_router.data_ptr(), None if router_bias is None else router_bias.data_ptr(),
+                    w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())
+    h = ctypes.c_void_p()
+    _check("moe_layer_init", lib.moe_layer_init(ctypes.byref(cfg), ctypes.byref(w),
+                                                ctypes.byref(h)))
+    return h
+
+
+def moe_layer_destroy(handle) -> None:
+    _check("moe_layer_destroy", load_library().moe_layer_destroy(handle))
+
+
+def moe_workspace_size(handle, n_tokens: int) -> int:
+    return int(load_library().moe_workspace_size(handle, int(n_tokens)))
+
+
+def moe_workspace_init(handle, ws, stream=None) -> None:
+    _check("moe_workspace_init", load_library().moe_workspace_init(
+        handle, _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route(handle, x, n_tokens, logits_out, topk_idx, topk_gate, expert_counts,
+              expert_offsets, perm, slot_row, ws, stream=None) -> None:
+    _check("moe_route", load_library().moe_route(
+        handle, _p(x), int(n_tokens), _p(logits_out), _p(topk_idx), _p(topk_gate),
+        _p(expert_counts), _p(expert_offsets), _p(perm), _p(slot_row), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route_from_logits(handle, logits, n_tokens, topk_idx, topk_gate, expert_counts,
+                          expert_offsets, perm, slot_row, ws, stream=None) -> None:
+    _check("moe_route_from_logits", load_library().moe_route_from_logits(
+        handle, _p(logits), int(n_tokens), _p(topk_idx), _p(topk_gate), _p(expert_counts),
+        _p(expert_offsets), _p(perm), _p(slot_row), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
+    _check("moe_forward", load_library().moe_forward(
+        handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_forward_profiled(handle, x, n_tokens, out, ws, events, stream=None) -> None:
+    """`events`: MOE_PROFILE_STAGES + 1 torch.cuda.Event(enable_timing=True) objects."""
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("moe_forward_profiled", load_library().moe_forward_profiled(
+        handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream), arr, len(events)))
+
+
+def moe_device_status(handle, ws, stream=None) -> int:
+    return int(load_library().moe_device_status(handle, _p(ws), ws.numel() * ws.element_size(),
+                                                 _stream(stream)))
+
+
+# ------------------------------------------------------------------ convenience wrapper
+class MoELayer:
+    """Owns a handle and a workspace; holds references to the weight tensors."""
+
+    def __init__(self, w_router, router_bias, w_gate, w_up, w_down, top_k: int,
+                 max_tokens: int, n_shared: int = 1, routed_scale: float = 1.0):
+        dt = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32}[w_router.dtype]
+        E, d = w_router.shape
+        f = w_gate.shape[1]
+        self.cfg = moe_config(int(max_tokens), int(d), int(E), int(top_k), int(f),
+                              int(n_shared), dt, float(routed_scale))
+        self.tensors = (w_router, router_bias, w_gate, w_up, w_down)
+        self.handle = moe_layer_init(self.cfg, *self.tensors)
+        self.device = w_router.device
+        self.ws = None
+        self.E, self.k, self.d = int(E), int(top_k), int(d)
+
+    def workspace(self, n_tokens: int):
+        need = moe_workspace_size(self.handle, n_tokens)
+        if self.ws is None or self.ws.numel() < need:
+            self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            moe_workspace_init(self.handle, self.ws)
+        return self.ws
+
+    def forward(self, x, out=None, stream=None):
+        T = x.shape[0]
+        out = torch.empty_like(x) if out is None else out
+        moe_forward(self.handle, x, T, out, self.workspace(T), stream)
+        return out
+
+    def route(self, x=None, logits=None, want_logits=False, stream=None):
+        T = (x if x is not None else logits).shape[0]
+        dev = self.device
+        r = dict(
+            idx=torch.empty((T, self.k), dtype=torch.int32, device=dev),
+            gates=torch.empty((T, self.k), dtype=torch.float32, device=dev),
+            counts=torch.empty((self.E,), dtype=torch.int32, device=dev),
+            offsets=torch.empty((self.E + 1,), dtype=torch.int32, device=dev),
+            perm=torch.empty((T * self.k,), dtype=torch.int32, device=dev),
+            slot_row=torch.empty((T, self.k), dtype=torch.int32, device=dev))
+        ws = self.workspace(T)
+        if logits is not None:
+            moe_route_from_logits(self.handle, logits, T, r["idx"], r["gates"], r["counts"],
+                                  r["offsets"], r["perm"], r["slot_row"], ws, stream)
+        else:
+            lg = torch.empty((T, self.E), dtype=torch.float32, device=dev) if want_logits else None
+            moe_route(self.handle, x, T, lg, r["idx"], r["gates"], r["counts"], r["offsets"],
+                      r["perm"], r["slot_row"], ws, stream)
+            if lg is not None:
+                r["logits"] = lg
+        return r
+
+    def device_status(self, stream=None) -> int:
+        return moe_device_status(self.handle, self.ws, stream)
+
+    def close(self):
+        if self.handle is not None:
+            moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,139 @@
+// expert_simt.cuh -- exact-fp32 expert FFNs (CUDA-core FFMA, no TF32) and the
+// gate-weighted combine shared by both precisions.
+//
+// Expert FFN: SwiGLU with gate and up branches ("Step 3.5 Flash 技术论文深度解读",
+// training stability, local activation explosion, root cause 3); the routed sum carries an
+// explicit scale ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active
+// Parameters", section 4.1.2) and the shared expert is always on (section 2.2).
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Row p of the expert-sorted space: p < Tk is pair perm[p] = t*k + j of expert
+// topk_idx[perm[p]]; p >= Tk is the shared expert on token p - Tk.
+__device__ __forceinline__ void sorted_row_owner(int p, int Tk, int k, int E,
+                                                 const int *__restrict__ perm,
+                                                 const int *__restrict__ topk_idx, int &t,
+                                                 int &g) {
+  if (p < Tk) {
+    const int pair = perm[p];
+    t = pair / k;
+    g = topk_idx[pair];
+  } else {
+    t = p - Tk;
+    g = E;
+  }
+}
+
+// h[p, r] = silu(x_t . W_g[g, r]) * (x_t . W_u[g, r]), one thread per (p, r), fp32.
+__global__ void __launch_bounds__(256) ffn_up_f32_kernel(
+    const float *__restrict__ x, const float *__restrict__ wg, const float *__restrict__ wu,
+    const int *__restrict__ perm, const int *__restrict__ topk_idx, int Tk, int k, int E,
+    int n_rows, int d, int f, float *__restrict__ h) {
+  const size_t total = (size_t)n_rows * f;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int p = (int)(i / f), r = (int)(i % f);
+    int t, g;
+    sorted_row_owner(p, Tk, k, E, perm, topk_idx, t, g);
+    const float *xr = x + (size_t)t * d;
+    const float *gr = wg + ((size_t)g * f + r) * d;
+    const float *ur = wu + ((size_t)g * f + r) * d;
+    float a = 0.f, b = 0.f;
+    for (int c = 0; c < d; ++c) {
+      a = fmaf(xr[c], gr[c], a);
+      b = fmaf(xr[c], ur[c], b);
+    }
+    h[i] = a / (1.f + expf(-a)) * b;
+  }
+}
+
+// y[p, c] = scale_p * sum_r h[p, r] W_d[g, c, r]; scale_p = routed_scale * gate of the pair
+// for routed rows, 1 for shared rows.  One thread per (p, c), fp32.
+__global__ void __launch_bounds__(256) ffn_down_f32_kernel(
+    const float *__restrict__ h, const float *__restrict__ wd, const int *__restrict__ perm,
+    const int *__restrict__ topk_idx, const float *__restrict__ topk_gate, float routed_scale,
+    int Tk, int k, int E, int n_rows, int d, int f, float *__restrict__ y) {
+  const size_t total = (size_t)n_rows * d;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int p = (int)(i / d), c = (int)(i % d);
+    int t, g;
+    sorted_row_owner(p, Tk, k, E, perm, topk_idx, t, g);
+    const float *hr = h + (size_t)p * f;
+    const float *wr = wd + ((size_t)g * d + c) * f;
+    float a = 0.f;
+    for (int r = 0; r < f; ++r) a = fmaf(hr[r], wr[r], a);
+    const float scale = (p < Tk) ? routed_scale * topk_gate[perm[p]] : 1.f;
+    y[i] = a * scale;
+  }
+}
+
+// out[t, :] = sum_{j < k} y[slot_row[t, j], :] (+ y[Tk + t, :] if shared), summed in fp32
+// in this fixed order and rounded once.  16-byte vectors, grid-stride.
+template <typename T>
+struct CombineIO;
+template <>
+struct CombineIO<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void add(const __nv_bfloat16 *p, float (&acc)[8]) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      acc[2 * i] += f.x;
+      acc[2 * i + 1] += f.y;
+    }
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&acc)[8]) {
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+  }
+};
+template <>
+struct CombineIO<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void add(const float *p, float (&acc)[4]) {
+    float4 u = *reinterpret_cast<const float4 *>(p);
+    acc[0] += u.x;
+    acc[1] += u.y;
+    acc[2] += u.z;
+    acc[3] += u.w;
+  }
+  __device__ __forceinline__ static void store(float *p, const float (&acc)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(const T *__restrict__ y,
+                                                      const int *__restrict__ slot_row,
+                                                      int n_tokens, int k, int Tk,
+                                                      int n_shared, int d,
+                                                      T *__restrict__ out) {
+  constexpr int V = CombineIO<T>::N;
+  const int vpr = d / V;
+  const size_t total = (size_t)n_tokens * vpr;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / vpr);
+    const int c = (int)(i % vpr) * V;
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int p = slot_row[(size_t)t * k + j];
+      CombineIO<T>::add(y + (size_t)p * d + c, acc);
+    }
+    if (n_shared) CombineIO<T>::add(y + (size_t)(Tk + t) * d + c, acc);
+    CombineIO<T>::store(out + (size_t)t * d + c, acc);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,356 @@
+// grouped_gemm.cuh -- persistent, warp-specialised grouped expert GEMM on tcgen05.
+//
+// "Fused MoE gather/scatter with grouped GEMM" ("Step 3.5 Flash: Open Frontier-Level
+// Intelligence with 11B Active Parameters", section 3.2.4) over SwiGLU experts with gate
+// and up branches ("Step 3.5 Flash 技术论文深度解读", training stability, root cause 3),
+// one always-on shared expert (first page, section 2.2) and an explicit routed scale
+// (first page, section 4.1.2).
+//
+// Orientation ("weights on M"): every unit computes D[128 weight rows, n tokens] =
+//   W[g][m0:m0+128, :] . B[rows of group g]^T
+// so the weight tile is the 128-row MMA A operand and the group's tokens are the N side
+// (N = 16 .. 256 in steps of 16, chosen per unit from the group's real token count).  In
+// decode a group holds one or two tokens, so this keeps the tensor-core work tiny while
+// every SM streams weight tiles from HBM through TMA.
+//
+//   MODE_UP   : A0 = W_gate, A1 = W_up (two accumulators), B = expert-sorted x rows
+//               (the shared group reads x directly); epilogue h = silu(G) * U -> bf16.
+//   MODE_DOWN : A0 = W_down, B = h rows; epilogue y = acc * scale -> bf16, scale =
+//               routed_scale * gate for routed rows and 1 for shared rows.
+//
+// Roles (192 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA issuer (warp 1
+// also owns the TMEM allocation), warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
+// Pipelines: STAGES shared-memory slots (full / empty mbarriers) and two TMEM accumulator
+// buffers (tmem_full / tmem_empty) so the epilogue of unit i overlaps the MMAs of i + 1.
+// Every wait is bounded (ptx_sm100.cuh); on a time-out the CTA drains its in-flight
+// copies and MMAs, frees TMEM and returns with the workspace status word set.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ptx_sm100.cuh"
+
+namespace moe {
+
+enum GemmMode { MODE_UP = 0, MODE_DOWN = 1 };
+
+struct GemmParams {
+  CUtensorMap tmA0;  // UP: W_gate [G*f, d]; DOWN: W_down [G*d, f]     box {64, 128}
+  CUtensorMap tmA1;  // UP: W_up [G*f, d]                               box {64, 128}
+  CUtensorMap tmB;   // UP: xs [Tk, d]; DOWN: h [Tk + n_shared*T, f]   box {64, BN}
+  CUtensorMap tmBs;  // UP: x [T, d] (shared group)                     box {64, BN}
+  const int *offsets;       // [E + 1] expert offsets in the sorted space
+  const int *perm;          // [Tk] (DOWN: gate lookup)
+  const float *topk_gate;   // [Tk] (DOWN)
+  __nv_bfloat16 *out;       // UP: h [P, f]; DOWN: y [P, d]
+  DevStatus *status;
+  float routed_scale;
+  int E, n_groups, T, Tk;
+  int M;      // weight rows per group: f (UP) or d (DOWN)
+  int K;      // reduction length: d (UP) or f (DOWN)
+  int ld_out; // f (UP) or d (DOWN)
+};
+
+constexpr int kBM = 128;         // weight rows per unit (MMA M)
+constexpr int kBK = 64;          // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kGemmThreads = 192;
+
+template <int MODE, int BN>
+struct GemmCfg {
+  static constexpr int NA = (MODE == MODE_UP) ? 2 : 1;
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = NA * BN;
+  static constexpr int TMEM_COLS_RAW = 2 * ACC_COLS;
+  static constexpr int TMEM_COLS = TMEM_COLS_RAW <= 32    ? 32
+                                   : TMEM_COLS_RAW <= 64  ? 64
+                                   : TMEM_COLS_RAW <= 128 ? 128
+                                   : TMEM_COLS_RAW <= 256 ? 256
+                                                          : 512;
+  static constexpr int SMEM_BUDGET = 208 * 1024;
+  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static_assert(STAGES >= 2, "pipeline too shallow");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of the MMA");
+  static_assert(TMEM_COLS_RAW <= 512, "TMEM has 512 columns");
+  // barriers: full[S], empty[S], tfull[2], tempty[2], drain[1]
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+  static constexpr size_t smem_bytes(int n_groups) {
+    return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
+           (size_t)(3 * n_groups + 1) * 4;
+  }
+};
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = GemmCfg<MODE, BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA0 = smem;
+  uint8_t *sA1 = sA0 + S * C::A_BYTES;  // only used by MODE_UP
+  uint8_t *sB = sA0 + C::NA * S * C::A_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + S * C::B_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *tfull = bars + 2 * S;
+  uint64_t *tempty = bars + 2 * S + 2;
+  uint64_t *drain = bars + 2 * S + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
+  int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
+  int *grp_row = grp_count + p.n_groups;                        // [G]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.n_groups;
+  const int mtiles = p.M / kBM;
+  const int kblocks = p.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmA0);
+    if (MODE == MODE_UP) {
+      tma_prefetch_desc(&p.tmA1);
+      tma_prefetch_desc(&p.tmBs);
+    }
+    tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  // group table: token count, first row in the sorted space, units per group
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int cnt, row;
+    if (g < p.E) {
+      row = p.offsets[g];
+      cnt = p.offsets[g + 1] - row;
+    } else {
+      row = p.Tk + (g - p.E) * p.T;
+      cnt = p.T;
+    }
+    grp_count[g] = cnt;
+    grp_row[g] = row;
+    unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of units per group (each lane a contiguous run)
+    const int per = (G + 31) / 32;
+    const int lo = min(G, lane * per), hi = min(G, lo + per);
+    int run = 0;
+    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int g = lo; g < hi; ++g) {
+      const int u = unit_prefix[g];
+      unit_prefix[g] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = unit_prefix[G];
+
+  // unit -> (group, m tile, n tile); n tile innermost so the units that share a weight
+  // tile run back to back on neighbouring CTAs (the tile is read from HBM once).
+  auto decode = [&](int u, int &g, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {  // last g with unit_prefix[g] <= u
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    g = lo;
+    const int nts = (grp_count[g] + BN - 1) / BN;
+    const int loc = u - unit_prefix[g];
+    mt = loc / nts;
+    nt = loc % nts;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();  // weights read once
+      const uint64_t pol_b = policy_evict_last();   // activations: re-read per m tile
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const int a_row = g * p.M + mt * kBM;
+        const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
+        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
+        const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
+        // a weight tile read by one unit only is streamed with evict-first priority; one
+        // shared by several token tiles keeps normal priority so its neighbours hit L2
+        const bool single_use = grp_count[g] <= BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (single_use) {
+            tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kb * kBK, a_row,
+                             pol_w);
+            if (MODE == MODE_UP)
+              tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kb * kBK,
+                               a_row, pol_w);
+          } else {
+            tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kb * kBK, a_row);
+            if (MODE == MODE_UP)
+              tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kb * kBK, a_row);
+          }
+          tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kb * kBK, b_row,
+                           pol_b);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 2)) break;
+        tc_fence_after();
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const int valid = min(BN, grp_count[g] - nt * BN);
+        const int n_mma = (valid + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA0 + stage * C::A_BYTES);
+          const uint32_t a1 = smem_u32(sA1 + stage * C::A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t accum = (kb | kk) ? 1u : 0u;
+            const uint64_t bd = sdesc_k_sw128(b + kk * 32);
+            tc_mma_bf16(d0, sdesc_k_sw128(a0 + kk * 32), bd, idesc, accum);
+            if (MODE == MODE_UP) tc_mma_bf16(d0 + BN, sdesc_k_sw128(a1 + kk * 32), bd, idesc, accum);
+          }
+          tc_commit(&empty[stage]);  // slot free once these MMAs have read it
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      // every MMA issued by this thread has completed once `drain` flips
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;              // TMEM lane quadrant of this warp
+    const int r = q * 32 + lane;         // weight row within the unit
+    int it = 0;
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, 4)) break;
+      tc_fence_after();
+      int g, mt, nt;
+      decode(u, g, mt, nt);
+      const int valid = min(BN, grp_count[g] - nt * BN);
+      const int row0 = grp_row[g] + nt * BN;
+      const int col = mt * kBM + r;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      for (int c0 = 0; c0 < valid; c0 += 16) {
+        uint32_t v0[16];
+        tmem_ld16(taddr + c0, v0);
+        if (MODE == MODE_UP) {
+          uint32_t v1[16];
+          tmem_ld16(taddr + BN + c0, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            if (c0 + n < valid) {
+              const float gv = __uint_as_float(v0[n]);
+              const float uv = __uint_as_float(v1[n]);
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              p.out[(size_t)(row0 + c0 + n) * p.ld_out + col] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            if (c0 + n < valid) {
+              const int pr = row0 + c0 + n;
+              const float scale = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[pr]] : 1.f;
+              p.out[(size_t)pr * p.ld_out + col] =
+                  __float2bfloat16_rn(__uint_as_float(v0[n]) * scale);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,473 @@
+// moe_layer.cu -- C ABI of the sparse-MoE FFN layer (declared in include/moe_layer.h) and
+// the host logic around the kernels: argument checks, workspace layout, TMA descriptors,
+// launch configuration.  The library never allocates device memory.
+//
+// One call of moe_forward launches, in stream order:
+//   router logits -> top-k + chunk histograms -> permutation scatter     (routing.cuh)
+//   bf16: row gather -> grouped GEMM up+SwiGLU -> grouped GEMM down     (grouped_gemm.cuh)
+//   fp32: SIMT up+SwiGLU -> SIMT down                                    (expert_simt.cuh)
+//   -> gate-weighted combine                                             (expert_simt.cuh)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "moe_layer.h"
+#include "expert_simt.cuh"
+#include "grouped_gemm.cuh"
+#include "ptx_sm100.cuh"
+#include "routing.cuh"
+
+using namespace moe;
+
+struct moe_layer {
+  moe_config cfg;
+  moe_weights w;
+  int device;
+  int num_sms;
+  int smem_optin;
+  CUtensorMap tm_wg, tm_wu, tm_wd;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] -> tiled map with box {64 columns, box_rows rows} and
+// 128-byte swizzle (the K-major operand layout of the tcgen05 descriptors).
+bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+
+// Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
+struct WsLayout {
+  size_t status, logits, idx, gate, counts, offsets, perm, slot_row, chunk_hist, xs, h, y,
+      total;
+};
+
+WsLayout ws_layout(const moe_config &c, int T) {
+  WsLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~static_cast<size_t>(255);
+    return o;
+  };
+  const size_t Tk = (size_t)T * c.top_k;
+  const size_t P = Tk + (size_t)c.n_shared * T;
+  const size_t nch = ((size_t)T + kChunk - 1) / kChunk;
+  L.status = take(sizeof(DevStatus));
+  L.logits = take((size_t)T * c.n_experts * 4);
+  L.idx = take(Tk * 4);
+  L.gate = take(Tk * 4);
+  L.counts = take((size_t)c.n_experts * 4);
+  L.offsets = take(((size_t)c.n_experts + 1) * 4);
+  L.perm = take(Tk * 4);
+  L.slot_row = take(Tk * 4);
+  L.chunk_hist = take(nch * c.n_experts * 4);
+  L.xs = (c.dtype == MOE_BF16) ? take(Tk * c.d_model * 2) : off;
+  L.h = take(P * c.d_ff * esize(c));
+  L.y = take(P * c.d_model * esize(c));
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+P *at(void *ws, size_t off) {
+  return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
+}
+
+moe_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int grid_for(size_t work, int per_block, int num_sms) {
+  size_t b = (work + per_block - 1) / per_block;
+  const size_t cap = (size_t)num_sms * 16;
+  if (b > cap) b = cap;
+  return b < 1 ? 1 : (int)b;
+}
+
+// Token tile of the grouped GEMM from the mean tokens per routed expert.
+int pick_bn(const moe_config &c, int T) {
+  const double mean = (double)T * c.top_k / c.n_experts;
+  if (mean <= 4.0) return 16;
+  if (mean <= 12.0) return 32;
+  if (mean <= 40.0) return 64;
+  return 128;
+}
+
+// ------------------------------------------------------------------ routing launches
+moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits,
+                         cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  constexpr int TB = 16;
+  if (T <= 32) {
+    dim3 grid(c.n_experts, (T + TB - 1) / TB);
+    if (c.dtype == MOE_BF16)
+      router_logits_rows_kernel<__nv_bfloat16, TB><<<grid, 128, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(x),
+          static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model, c.n_experts, logits);
+    else
+      router_logits_rows_kernel<float, TB><<<grid, 128, 0, st>>>(
+          static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
+          c.d_model, c.n_experts, logits);
+  } else {
+    dim3 grid((T + 63) / 64, (c.n_experts + 63) / 64);
+    if (c.dtype == MOE_BF16)
+      router_logits_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(x),
+          static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model, c.n_experts, logits);
+    else
+      router_logits_tiled_kernel<float><<<grid, 256, 0, st>>>(
+          static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
+          c.d_model, c.n_experts, logits);
+  }
+  return last_launch();
+}
+
+moe_status launch_select_permute(const moe_layer *L, const float *logits, int T, int *idx,
+                                 float *gate, int *counts, int *offsets, int *perm,
+                                 int *slot_row, int *chunk_hist, cudaStream_t st,
+                                 int mark_index = 0, void *const *events = nullptr) {
+  const moe_config &c = L->cfg;
+  const int nch = (T + kChunk - 1) / kChunk;
+  const int need = (c.n_experts + 31) / 32;
+  const float *bias = L->w.router_bias;
+  const int thr = kRouteWarps * 32;
+#define MOE_TOPK(V)                                                                       \
+  topk_hist_kernel<V><<<nch, thr, 0, st>>>(logits, bias, T, c.n_experts, c.top_k, idx, gate, \
+                                           chunk_hist)
+  if (need <= 1) MOE_TOPK(1);
+  else if (need <= 2) MOE_TOPK(2);
+  else if (need <= 4) MOE_TOPK(4);
+  else if (need <= 9) MOE_TOPK(9);
+  else if (need <= 16) MOE_TOPK(16);
+  else MOE_TOPK(32);
+#undef MOE_TOPK
+  if (last_launch() != MOE_OK) return MOE_ERR_CUDA;
+  if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  permute_scatter_kernel<<<nch, 256, 0, st>>>(idx, chunk_hist, T, c.n_experts, c.top_k, nch,
+                                              counts, offsets, perm, slot_row);
+  return last_launch();
+}
+
+// ------------------------------------------------------------------ grouped GEMM launch
+template <int MODE, int BN>
+moe_status launch_gemm_bn(const moe_layer *L, const GemmParams &p, cudaStream_t st) {
+  using C = GemmCfg<MODE, BN>;
+  const size_t smem = C::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  grouped_gemm_kernel<MODE, BN><<<L->num_sms, kGemmThreads, smem, st>>>(p);
+  return last_launch();
+}
+
+template <int MODE>
+moe_status launch_gemm(const moe_layer *L, int bn, const GemmParams &p, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_gemm_bn<MODE, 16>(L, p, st);
+    case 32: return launch_gemm_bn<MODE, 32>(L, p, st);
+    case 64: return launch_gemm_bn<MODE, 64>(L, p, st);
+    case 128: return launch_gemm_bn<MODE, 128>(L, p, st);
+  }
+  return MOE_ERR_UNSUPPORTED;
+}
+
+moe_status check_call(const moe_layer *L, int T, void *ws, size_t ws_bytes) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ws || ws_bytes < ws_layout(L->cfg, T).total) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+}  // namespace
+
+// =============================================================================== C ABI
+extern "C" {
+
+const char *moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+  }
+  return "unknown status";
+}
+
+moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handle *out) {
+  if (!cfg || !w || !out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const moe_config c = *cfg;
+  if (c.max_tokens < 1 || c.d_model < 1 || c.n_experts < 1 || c.top_k < 1 || c.d_ff < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (c.top_k > c.n_experts || (c.n_shared != 0 && c.n_shared != 1)) return MOE_ERR_INVALID_ARG;
+  if (c.dtype != MOE_F32 && c.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c.top_k > kMaxTopK || c.n_experts > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c.max_tokens * (c.top_k + c.n_shared) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c.d_model % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c.dtype == MOE_BF16 && (c.d_model % kBM != 0 || c.d_ff % kBM != 0))
+    return MOE_ERR_UNSUPPORTED;
+  if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w_router) || !aligned16(w->w_gate) || !aligned16(w->w_up) ||
+      !aligned16(w->w_down) || !aligned16(w->router_bias))
+    return MOE_ERR_ALIGNMENT;
+
+  moe_layer *L = static_cast<moe_layer *>(calloc(1, sizeof(moe_layer)));
+  if (!L) return MOE_ERR_INVALID_ARG;
+  L->cfg = c;
+  L->w = *w;
+  int major = 0;
+  if (cudaGetDevice(&L->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&L->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                             L->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, L->device) !=
+          cudaSuccess) {
+    free(L);
+    return MOE_ERR_CUDA;
+  }
+  if (major != 10) {  // the library is built for sm_100a only
+    free(L);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (c.dtype == MOE_BF16) {
+    const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
+    if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
+        !encode_bf16_2d(&L->tm_wu, w->w_up, c.d_model, G * c.d_ff, kBM) ||
+        !encode_bf16_2d(&L->tm_wd, w->w_down, c.d_ff, G * c.d_model, kBM)) {
+      free(L);
+      return MOE_ERR_CUDA;
+    }
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+moe_status moe_layer_destroy(moe_handle h) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  free(h);
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(moe_handle h, int n_tokens) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return 0;
+  return ws_layout(h->cfg, n_tokens < 1 ? 1 : n_tokens).total;
+}
+
+moe_status moe_workspace_init(moe_handle h, void *ws, size_t ws_bytes, void *stream) {
+  if (!h || !ws || ws_bytes < sizeof(DevStatus)) return MOE_ERR_INVALID_ARG;
+  return cudaMemsetAsync(ws, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream) {
+  if (!h || !ws || ws_bytes < sizeof(DevStatus)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevStatus s;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&s, ws, sizeof s, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (s.error == 0) return MOE_OK;
+  if (cudaMemset(ws, 0, sizeof(DevStatus)) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_ERR_DEVICE_TIMEOUT;
+}
+
+static moe_status route_common(moe_handle h, const void *x, const float *logits_in, int T,
+                               float *logits_out, int *idx, float *gate, int *counts,
+                               int *offsets, int *perm, int *slot_row, void *ws,
+                               size_t ws_bytes, void *stream) {
+  moe_status s = check_call(h, T, ws, ws_bytes);
+  if (s != MOE_OK || T == 0) return s;
+  if (!idx || !gate || !counts || !offsets || !perm || !slot_row) return MOE_ERR_INVALID_ARG;
+  if (!x && !logits_in) return MOE_ERR_INVALID_ARG;
+  if (x && !aligned16(x)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WsLayout W = ws_layout(h->cfg, T);
+  const float *logits = logits_in;
+  if (!logits) {
+    float *dst = logits_out ? logits_out : at<float>(ws, W.logits);
+    if ((s = launch_logits(h, x, T, dst, st)) != MOE_OK) return s;
+    logits = dst;
+  }
+  return launch_select_permute(h, logits, T, idx, gate, counts, offsets, perm, slot_row,
+                               at<int>(ws, W.chunk_hist), st);
+}
+
+moe_status moe_route(moe_handle h, const void *x, int n_tokens, float *logits_out,
+                     int *topk_idx, float *topk_gate, int *expert_counts, int *expert_offsets,
+                     int *perm, int *slot_row, void *ws, size_t ws_bytes, void *stream) {
+  if (!x) return MOE_ERR_INVALID_ARG;
+  return route_common(h, x, nullptr, n_tokens, logits_out, topk_idx, topk_gate, expert_counts,
+                      expert_offsets, perm, slot_row, ws, ws_bytes, stream);
+}
+
+moe_status moe_route_from_logits(moe_handle h, const float *logits, int n_tokens,
+                                 int *topk_idx, float *topk_gate, int *expert_counts,
+                                 int *expert_offsets, int *perm, int *slot_row, void *ws,
+                                 size_t ws_bytes, void *stream) {
+  if (!logits) return MOE_ERR_INVALID_ARG;
+  return route_common(h, nullptr, logits, n_tokens, nullptr, topk_idx, topk_gate,
+                      expert_counts, expert_offsets, perm, slot_row, ws, ws_bytes, stream);
+}
+
+static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
+                               size_t ws_bytes, void *stream, void *const *events) {
+  moe_status s = check_call(h, n_tokens, ws, ws_bytes);
+  if (s != MOE_OK || n_tokens == 0) return s;
+  if (!x || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+  const moe_config &c = h->cfg;
+  const int T = n_tokens;
+  const int Tk = T * c.top_k;
+  const int P = Tk + c.n_shared * T;
+  const WsLayout W = ws_layout(c, T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int *idx = at<int>(ws, W.idx);
+  float *gate = at<float>(ws, W.gate);
+  int *offsets = at<int>(ws, W.offsets);
+  int *perm = at<int>(ws, W.perm);
+  int *slot_row = at<int>(ws, W.slot_row);
+  float *logits = at<float>(ws, W.logits);
+  // events[i] (if given) marks the end of stage i (events[0]: the start)
+  auto mark = [&](int i) -> moe_status {
+    if (!events) return MOE_OK;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+  };
+  if ((s = mark(0)) != MOE_OK) return s;
+  if ((s = launch_logits(h, x, T, logits, st)) != MOE_OK) return s;
+  if ((s = mark(1)) != MOE_OK) return s;
+  if ((s = launch_select_permute(h, logits, T, idx, gate, at<int>(ws, W.counts), offsets, perm,
+                                 slot_row, at<int>(ws, W.chunk_hist), st, events ? 2 : 0,
+                                 events)) != MOE_OK)
+    return s;
+  if ((s = mark(3)) != MOE_OK) return s;
+
+  if (c.dtype == MOE_BF16) {
+    const int vpr = c.d_model / 8;
+    gather_rows_kernel<<<grid_for((size_t)Tk * vpr, 256, h->num_sms), 256, 0, st>>>(
+        static_cast<const uint4 *>(x), perm, c.top_k, Tk, vpr, at<uint4>(ws, W.xs));
+    if ((s = last_launch()) != MOE_OK) return s;
+    if ((s = mark(4)) != MOE_OK) return s;
+    const int bn = pick_bn(c, T);
+    __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
+    __nv_bfloat16 *ybuf = at<__nv_bfloat16>(ws, W.y);
+    GemmParams p1;
+    memset(&p1, 0, sizeof p1);
+    p1.tmA0 = h->tm_wg;
+    p1.tmA1 = h->tm_wu;
+    if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
+        !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn))
+      return MOE_ERR_CUDA;
+    p1.offsets = offsets;
+    p1.perm = perm;
+    p1.topk_gate = gate;
+    p1.out = hbuf;
+    p1.status = at<DevStatus>(ws, W.status);
+    p1.routed_scale = c.routed_scale;
+    p1.E = c.n_experts;
+    p1.n_groups = c.n_experts + c.n_shared;
+    p1.T = T;
+    p1.Tk = Tk;
+    p1.M = c.d_ff;
+    p1.K = c.d_model;
+    p1.ld_out = c.d_ff;
+    if ((s = launch_gemm<MODE_UP>(h, bn, p1, st)) != MOE_OK) return s;
+    if ((s = mark(5)) != MOE_OK) return s;
+    GemmParams p2 = p1;
+    p2.tmA0 = h->tm_wd;
+    if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn)) return MOE_ERR_CUDA;
+    p2.out = ybuf;
+    p2.M = c.d_model;
+    p2.K = c.d_ff;
+    p2.ld_out = c.d_model;
+    if ((s = launch_gemm<MODE_DOWN>(h, bn, p2, st)) != MOE_OK) return s;
+    if ((s = mark(6)) != MOE_OK) return s;
+    combine_kernel<__nv_bfloat16>
+        <<<grid_for((size_t)T * (c.d_model / 8), 256, h->num_sms), 256, 0, st>>>(
+            ybuf, slot_row, T, c.top_k, Tk, c.n_shared, c.d_model,
+            static_cast<__nv_bfloat16 *>(out));
+    if ((s = last_launch()) != MOE_OK) return s;
+    return mark(7);
+  }
+
+  float *hbuf = at<float>(ws, W.h);
+  float *ybuf = at<float>(ws, W.y);
+  if ((s = mark(4)) != MOE_OK) return s;
+  ffn_up_f32_kernel<<<grid_for((size_t)P * c.d_ff, 256, h->num_sms), 256, 0, st>>>(
+      static_cast<const float *>(x), static_cast<const float *>(h->w.w_gate),
+      static_cast<const float *>(h->w.w_up), perm, idx, Tk, c.top_k, c.n_experts, P, c.d_model,
+      c.d_ff, hbuf);
+  if ((s = last_launch()) != MOE_OK) return s;
+  if ((s = mark(5)) != MOE_OK) return s;
+  ffn_down_f32_kernel<<<grid_for((size_t)P * c.d_model, 256, h->num_sms), 256, 0, st>>>(
+      hbuf, static_cast<const float *>(h->w.w_down), perm, idx, gate, c.routed_scale, Tk,
+      c.top_k, c.n_experts, P, c.d_model, c.d_ff, ybuf);
+  if ((s = last_launch()) != MOE_OK) return s;
+  if ((s = mark(6)) != MOE_OK) return s;
+  combine_kernel<float><<<grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms), 256, 0, st>>>(
+      ybuf, slot_row, T, c.top_k, Tk, c.n_shared, c.d_model, static_cast<float *>(out));
+  if ((s = last_launch()) != MOE_OK) return s;
+  return mark(7);
+}
+
+moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
+                       size_t ws_bytes, void *stream) {
+  return forward_impl(h, x, n_tokens, out, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void *out,
+                                void *ws, size_t ws_bytes, void *stream, void *const *events,
+                                int n_events) {
+  if (!events || n_events < MOE_PROFILE_STAGES + 1) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i <= MOE_PROFILE_STAGES; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, n_tokens, out, ws, ws_bytes, stream, events);
+}
+
+}  // extern "C"

@@ -1,0 +1,344 @@
+// routing.cuh -- router logits, bias-adjusted top-k with renormalised gates, and the
+// deterministic expert-sorted permutation.
+//
+// Follows "Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active Parameters",
+// section 2.2.2 (S_t = top-K experts of token t, routing probabilities p_{t,e}) and the
+// note under the parameter table of "Step 3.5 Flash 技术论文深度解读" (architecture item 1:
+// loss-free balancing by a bias that only adjusts the selection), and section 3.2.4 of the
+// first page (fused MoE gather/scatter: tokens grouped by expert before the grouped GEMM).
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;   // E limit of the routing kernels
+constexpr int kMaxTopK = 32;        // one slot per lane
+constexpr int kChunk = 64;          // tokens per routing chunk (one CTA)
+constexpr int kRouteWarps = 8;
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// 16-byte vector of inputs -> floats.
+template <typename Tin>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&o)[8]) {
+    uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float *p, float (&o)[4]) {
+    float4 u = __ldg(reinterpret_cast<const float4 *>(p));
+    o[0] = u.x;
+    o[1] = u.y;
+    o[2] = u.z;
+    o[3] = u.w;
+  }
+};
+
+// ------------------------------------------------------------------ router logits (small T)
+// One CTA per (expert, block of TB tokens): the CTA streams W_r[e] once and reduces TB
+// dot products.  Used when the token count is small (decode), where the job is streaming
+// the 288 x d router matrix from HBM across many SMs.
+template <typename Tin, int TB>
+__global__ void __launch_bounds__(128) router_logits_rows_kernel(const Tin *__restrict__ x,
+                                                                 const Tin *__restrict__ wr,
+                                                                 int T, int d, int E,
+                                                                 float *__restrict__ logits) {
+  constexpr int V = Vec16<Tin>::N;
+  const int e = blockIdx.x;
+  const int t0 = blockIdx.y * TB;
+  const int nt = min(TB, T - t0);
+  float acc[TB];
+#pragma unroll
+  for (int t = 0; t < TB; ++t) acc[t] = 0.f;
+  for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+    float w[V];
+    Vec16<Tin>::load(wr + (size_t)e * d + i, w);
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+      if (t < nt) {
+        float xv[V];
+        Vec16<Tin>::load(x + (size_t)(t0 + t) * d + i, xv);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[t] = fmaf(xv[v], w[v], acc[t]);
+      }
+    }
+  }
+  __shared__ float red[TB][4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < TB; ++t) {
+    float v = acc[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[t][warp] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    const int t = threadIdx.x;
+    logits[(size_t)(t0 + t) * E + e] = (red[t][0] + red[t][1]) + (red[t][2] + red[t][3]);
+  }
+}
+
+// ------------------------------------------------------------------ router logits (tiled)
+// 64 tokens x 64 experts per CTA, K in steps of 32, 4 x 4 outputs per thread, fp32 FMA.
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_logits_tiled_kernel(const Tin *__restrict__ x,
+                                                                  const Tin *__restrict__ wr,
+                                                                  int T, int d, int E,
+                                                                  float *__restrict__ logits) {
+  constexpr int BT = 64, BE = 64, BK = 32;
+  __shared__ float xs[BK][BT + 4];
+  __shared__ float ws[BK][BE + 4];
+  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * BE;
+  const int tid = threadIdx.x;
+  const int tr = (tid / 16) * 4, ec = (tid % 16) * 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += BK) {
+    // 64 rows x 32 k for each operand: 2048 elements, 8 per thread
+    for (int i = tid; i < BT * BK; i += 256) {
+      const int row = i / BK, kk = i % BK;
+      const int t = t0 + row, e = e0 + row;
+      xs[kk][row] = (t < T && k0 + kk < d) ? to_f32(x[(size_t)t * d + k0 + kk]) : 0.f;
+      ws[kk][row] = (e < E && k0 + kk < d) ? to_f32(wr[(size_t)e * d + k0 + kk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < BK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = xs[kk][tr + i];
+        b[i] = ws[kk][ec + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + tr + i, e = e0 + ec + j;
+      if (t < T && e < E) logits[(size_t)t * E + e] = acc[i][j];
+    }
+}
+
+// ------------------------------------------------------------------ top-k + chunk histogram
+// Ranking: a ranks before b iff (a is a number and b is NaN) or a.s > b.s or
+// (a.s == b.s or both NaN) and a.id < b.id.  Entries past E carry id = INT_MAX, s = NaN.
+__device__ __forceinline__ bool ranks_before(float sa, int ea, float sb, int eb) {
+  const bool na = sa != sa, nb = sb != sb;
+  if (na != nb) return nb;
+  if (!na && sa != sb) return sa > sb;
+  return ea < eb;
+}
+
+// One warp per token; CTA c handles tokens [c*kChunk, (c+1)*kChunk).  Lane l holds the
+// scores of experts l, l+32, ...  k rounds of warp arg-max pick S_t in rank order; lane j
+// keeps slot j.  Gates: softmax over the selected UNBIASED logits (max-shifted, expf).
+// The CTA's per-expert selection counts go to chunk_hist[c][e] (integer, order-free).
+template <int MAXV>
+__global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
+    const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
+    int *__restrict__ topk_idx, float *__restrict__ topk_gate, int *__restrict__ chunk_hist) {
+  __shared__ int hist[kMaxExperts];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tbeg = c * kChunk, tend = min(T, tbeg + kChunk);
+  for (int t = tbeg + warp; t < tend; t += kRouteWarps) {
+    float s[MAXV], l[MAXV];
+    uint32_t used = 0;
+#pragma unroll
+    for (int v = 0; v < MAXV; ++v) {
+      const int e = lane + 32 * v;
+      if (e < E) {
+        l[v] = logits[(size_t)t * E + e];
+        s[v] = l[v] + (bias ? bias[e] : 0.f);
+      } else {
+        l[v] = 0.f;
+        s[v] = __int_as_float(0x7fc00000);
+      }
+    }
+    int my_e = 0;
+    float my_l = 0.f;
+    for (int r = 0; r < k; ++r) {
+      float bs = __int_as_float(0x7fc00000);
+      int be = 0x7fffffff;
+      float bl = 0.f;
+#pragma unroll
+      for (int v = 0; v < MAXV; ++v) {
+        const int e = lane + 32 * v;
+        const bool ok = (e < E) && !((used >> v) & 1u);
+        if (ok && ranks_before(s[v], e, bs, be)) {
+          bs = s[v];
+          be = e;
+          bl = l[v];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+        if (ranks_before(os, oe, bs, be)) {
+          bs = os;
+          be = oe;
+          bl = ol;
+        }
+      }
+      if ((be & 31) == lane) used |= 1u << (be >> 5);
+      if (lane == r) {
+        my_e = be;
+        my_l = bl;
+      }
+    }
+    // gates over lanes 0..k-1
+    float m = (lane < k) ? my_l : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = (lane < k) ? expf(my_l - m) : 0.f;
+    float z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = my_e;
+      topk_gate[(size_t)t * k + lane] = ex / z;
+      atomicAdd(&hist[my_e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)c * E + e] = hist[e];
+}
+
+// ------------------------------------------------------------------ permutation (scatter)
+// CTA c: totals and this chunk's prefix over the chunk histograms, exclusive scan over
+// experts -> offsets, then each (t, j) of the chunk gets position
+//   offsets[e] + (tokens of earlier chunks that chose e) + (earlier tokens of this chunk
+//   that chose e)
+// where the last term is a popcount over a per-expert token bitmap.  No atomics decide
+// any position, so perm and slot_row are deterministic (ascending t within an expert).
+__global__ void __launch_bounds__(256) permute_scatter_kernel(
+    const int *__restrict__ topk_idx, const int *__restrict__ chunk_hist, int T, int E, int k,
+    int n_chunks, int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
+    int *__restrict__ slot_row) {
+  __shared__ int s_tot[kMaxExperts];
+  __shared__ int s_base[kMaxExperts];
+  __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
+  __shared__ int warp_sum[32];
+  const int c = blockIdx.x;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int tot = 0, pre = 0;
+    for (int cc = 0; cc < n_chunks; ++cc) {
+      const int v = chunk_hist[(size_t)cc * E + e];
+      tot += v;
+      pre += (cc < c) ? v : 0;
+    }
+    s_tot[e] = tot;
+    s_base[e] = pre;
+#pragma unroll
+    for (int w = 0; w < kChunk / 32; ++w) bits[e][w] = 0u;
+  }
+  __syncthreads();
+  // exclusive scan of s_tot over experts: each thread owns a contiguous run
+  {
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int lo = min(E, tid * per), hi = min(E, lo + per);
+    int run = 0;
+    for (int e = lo; e < hi; ++e) run += s_tot[e];
+    // block exclusive scan of `run`
+    const int lane = tid & 31, warp = tid >> 5;
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x >> 5;
+      int v = (lane < nw) ? warp_sum[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+      }
+      if (lane < nw) warp_sum[lane] = v;  // inclusive warp totals
+    }
+    __syncthreads();
+    int excl = incl - run + (warp > 0 ? warp_sum[warp - 1] : 0);
+    for (int e = lo; e < hi; ++e) {
+      const int cnt = s_tot[e];
+      if (c == 0) {
+        counts[e] = cnt;
+        offsets[e] = excl;
+      }
+      s_base[e] += excl;
+      excl += cnt;
+    }
+    if (c == 0 && tid == 0) offsets[E] = T * k;
+  }
+  __syncthreads();
+  const int tbeg = c * kChunk, tend = min(T, tbeg + kChunk);
+  const int npair = (tend - tbeg) * k;
+  for (int q = tid; q < npair; q += blockDim.x) {
+    const int tl = q / k;
+    const int e = topk_idx[(size_t)tbeg * k + q];
+    atomicOr(&bits[e][tl >> 5], 1u << (tl & 31));
+  }
+  __syncthreads();
+  for (int q = tid; q < npair; q += blockDim.x) {
+    const int tl = q / k;
+    const int e = topk_idx[(size_t)tbeg * k + q];
+    int rank = 0;
+#pragma unroll
+    for (int w = 0; w < kChunk / 32; ++w) {
+      const uint32_t word = bits[e][w];
+      if (w < (tl >> 5)) rank += __popc(word);
+      else if (w == (tl >> 5)) rank += __popc(word & ((1u << (tl & 31)) - 1u));
+    }
+    const int p = s_base[e] + rank;
+    const int pair = tbeg * k + q;
+    perm[p] = pair;
+    slot_row[pair] = p;
+  }
+}
+
+// ------------------------------------------------------------------ row gather
+// xs[p, :] = x[perm[p] / k, :] for p < n_rows (16-byte vectors, grid-stride).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
+                                                          const int *__restrict__ perm, int k,
+                                                          int n_rows, int vec_per_row,
+                                                          uint4 *__restrict__ xs) {
+  const size_t total = (size_t)n_rows * vec_per_row;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int p = (int)(i / vec_per_row);
+    const int v = (int)(i % vec_per_row);
+    const int t = __ldg(perm + p) / k;
+    xs[i] = __ldg(x + (size_t)t * vec_per_row + v);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,66 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_layer_warp_b200 import binding
+from sparse_moe_layer_warp_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "moe_layer.h")).read()
+    return set(re.findall(r"^\S[^\n(]*?\b(moe_\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert binding.status_string(s) not in ("", "unknown status")
+    assert binding.status_string(99) == "unknown status"
+
+
+def test_init_rejects_bad_config_without_device(lib):
+    cfg = binding.moe_config(16, 4096, 288, 8, 1280, 1, binding.MOE_BF16, 1.0)
+    w = binding.moe_weights(16, 0, 32, 48, 64)
+    h = ctypes.c_void_p()
+    assert lib.moe_layer_init(None, ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+    bad = binding.moe_config(16, 4096, 288, 300, 1280, 1, binding.MOE_BF16, 1.0)  # k > E
+    assert lib.moe_layer_init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+    bad = binding.moe_config(16, 4096, 288, 8, 1280, 2, binding.MOE_BF16, 1.0)  # n_shared 2
+    assert lib.moe_layer_init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+    bad = binding.moe_config(16, 4000, 288, 8, 1280, 1, binding.MOE_BF16, 1.0)  # d % 128
+    assert lib.moe_layer_init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_UNSUPPORTED
+    bad = binding.moe_config(16, 4096, 2048, 8, 1280, 1, binding.MOE_BF16, 1.0)  # E > 1024
+    assert lib.moe_layer_init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_UNSUPPORTED
+    bad = binding.moe_config(16, 4096, 288, 40, 1280, 1, binding.MOE_BF16, 1.0)  # k > 32
+    assert lib.moe_layer_init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_UNSUPPORTED
+    wmis = binding.moe_weights(16, 0, 33, 48, 64)  # misaligned w_gate
+    assert lib.moe_layer_init(ctypes.byref(cfg), ctypes.byref(wmis), ctypes.byref(h)) == binding.MOE_ERR_ALIGNMENT
+    wnull = binding.moe_weights(16, 0, 0, 48, 64)
+    assert lib.moe_layer_init(ctypes.byref(cfg), ctypes.byref(wnull), ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+
+
+def test_null_handle_calls_rejected(lib):
+    assert lib.moe_workspace_size(None, 16) == 0
+    assert lib.moe_forward(None, None, 16, None, None, 0, None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_destroy(None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(None, None, 1, None, None, None, None, None, None, None, None, 0, None) == binding.MOE_ERR_INVALID_ARG

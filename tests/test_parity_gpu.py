@@ -1,0 +1,148 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the same
+seeded inputs.  Routing from identical fp32 logits is bit-exact; layer outputs are within
+2e-2 x RMS(out) (bf16) or 1e-5 x RMS(out) (fp32)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle_router_logits
+from sparse_moe_layer_warp_b200 import synth
+from tests.helpers import check_routing_exact, compare_layer, host_inputs, make_layer
+
+pytestmark = pytest.mark.gpu
+
+
+# --------------------------------------------------------------------------- routing
+@pytest.mark.parametrize("T,E,k,ties,zipf", [
+    (64, 16, 2, False, False), (16, 288, 8, False, False), (1, 288, 8, False, False),
+    (67, 288, 8, True, False), (256, 288, 8, False, False), (4096, 288, 8, False, True),
+    (8192, 288, 8, False, False), (33, 5, 5, True, False), (200, 40, 1, True, False),
+    (130, 1000, 32, False, False)])
+def test_route_from_logits_bit_exact(cuda_ok, T, E, k, ties, zipf):
+    w = synth.Workload("route", T=T, d=128, E=E, k=k, f=128, bias="zipf" if zipf else "uniform")
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    logits = synth.make_logits(T, E, seed=T + E, ties=ties, device="cuda")
+    check_routing_exact(layer, logits, inp.bias.cpu().numpy(), k, E)
+
+
+def test_route_nan_inf_signed_zero(cuda_ok):
+    w = synth.Workload("route", T=4, d=128, E=40, k=6, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    inp.bias.zero_()
+    layer = make_layer(inp)
+    lg = synth.make_logits(4, 40, seed=1, ties=True)
+    lg[0, 3] = float("nan")
+    lg[0, 7] = float("inf")
+    lg[1, :] = 0.0
+    lg[1, 5] = -0.0
+    lg[2, 10:20] = float("-inf")
+    check_routing_exact(layer, lg.cuda(), np.zeros(40, np.float32), 6, 40)
+
+
+@pytest.mark.parametrize("name,T", [("tiny_fp32", 64), ("decode_t16", 16), ("decode_t256", 256)])
+def test_router_logits_close(cuda_ok, name, T):
+    w = synth.WORKLOADS[name]
+    if w.d * w.E > 4096 * 288:
+        pytest.skip("size")
+    inp = synth.make_inputs(w, device="cuda", T=T)
+    layer = make_layer(inp)
+    r = layer.route(x=inp.x, want_logits=True)
+    torch.cuda.synchronize()
+    x, wr, *_ = host_inputs(inp)
+    ref = oracle_router_logits(x, wr).astype(np.float64)
+    got = r["logits"].cpu().numpy().astype(np.float64)
+    from oracle.moe_numpy import decode
+    scale = np.abs(decode(x)) @ np.abs(decode(wr)).T  # sum_i |x_i w_i|
+    # fp32 accumulation: |err| <= ~ n_chain * 2^-24 * sum|x_i w_i|; the chain is <= d terms
+    assert (np.abs(got - ref) <= w.d * 2.0**-24 * scale + 1e-30).all()
+    assert np.median(np.abs(got - ref) / np.maximum(scale, 1e-30)) < 1e-6
+
+
+# ------------------------------------------------------------------------- full layer
+SMALL = [
+    ("tiny_fp32", {}),
+    ("tiny_fp32", {"T": 1}),
+    ("tiny_fp32", {"T": 133, "E": 24, "k": 3, "seed": 2}),
+    ("tiny_fp32", {"n_shared": 0, "routed_scale": 2.5}),
+    ("tiny_fp32", {"dtype": "bf16", "d": 256, "f": 128}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 5, "d": 256, "E": 64, "k": 8, "f": 128}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 300, "d": 512, "E": 32, "k": 8, "f": 256}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 77, "d": 384, "E": 40, "k": 6, "f": 384, "seed": 3}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 513, "d": 256, "E": 8, "k": 8, "f": 128}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 200, "d": 256, "E": 48, "k": 4, "f": 128,
+                   "bias": "zipf", "n_shared": 0, "routed_scale": 1.5}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 1, "d": 256, "E": 288, "k": 8, "f": 128}),
+]
+
+
+@pytest.mark.parametrize("name,kw", SMALL)
+def test_forward_small_parity(cuda_ok, name, kw):
+    w = synth.WORKLOADS[name].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    out = layer.forward(inp.x)
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    compare_layer(inp, out, r["idx"].cpu().numpy())
+    assert layer.device_status() == 0
+
+
+def test_forward_deterministic(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=300, d=512, E=32, k=8, f=256)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    a = layer.forward(inp.x).clone()
+    b = layer.forward(inp.x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_forward_zero_tokens_is_noop(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", d=256, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    out = torch.full((1, w.d), 7.0, device="cuda", dtype=torch.bfloat16)
+    from sparse_moe_layer_warp_b200 import moe_forward
+    moe_forward(layer.handle, inp.x, 0, out, layer.workspace(1))
+    torch.cuda.synchronize()
+    assert (out == 7.0).all()
+
+
+def test_forward_rejects_too_many_tokens(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"]
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp, max_tokens=8)
+    from sparse_moe_layer_warp_b200 import MoEError
+    with pytest.raises(MoEError):
+        layer.forward(inp.x)
+
+
+# ------------------------------------------------------------ full-size workloads (sampled)
+FULL = [("decode_t16", None), ("decode_t256", 24), ("skew_t4096", 12), ("prefill_t8192", 12)]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,n_sample", FULL)
+def test_forward_full_size_sampled(cuda_ok, name, n_sample):
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    out = layer.forward(inp.x)
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    counts = r["counts"].cpu().numpy()
+    assert counts.sum() == w.T * w.k
+    rng = np.random.default_rng(7)
+    toks = None if n_sample is None else np.sort(rng.choice(w.T, n_sample, replace=False))
+    if toks is not None:
+        # always include the first and last tokens (edges of the last ragged tiles)
+        toks = np.unique(np.concatenate([[0, w.T - 1], toks]))
+    stats = compare_layer(inp, out, r["idx"].cpu().numpy(), tokens=toks)
+    print(name, stats, "empty experts:", int((counts == 0).sum()), "max load:", int(counts.max()))
+    assert layer.device_status() == 0
+    # properties that hold at any size: finite output, determinism
+    assert torch.isfinite(out.float()).all()
+    out2 = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
