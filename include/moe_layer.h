@@ -120,8 +120,9 @@ moe_status moe_route_from_logits(moe_handle h, const float *logits, int n_tokens
                                  size_t ws_bytes, void *stream);
 
 /* The whole layer: out = shared + routed_scale * sum_j g_j FFN_{S_t[j]}(x_t).  bf16 runs
- * the expert contractions on tcgen05 tensor cores with fp32 accumulation; h and the
- * per-row expert outputs are rounded to bf16 and the combine sums in fp32. */
+ * the expert contractions on tcgen05 tensor cores with fp32 accumulation; h (the operand
+ * of the down projection) is rounded to bf16, the per-row expert outputs stay fp32 and the
+ * combine sums them in a fixed order in fp32 before one rounding to the output type. */
 moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
                        size_t ws_bytes, void *stream);
 

@@ -152,6 +152,9 @@ def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
 
 def moe_forward_profiled(handle, x, n_tokens, out, ws, events, stream=None) -> None:
     """`events`: MOE_PROFILE_STAGES + 1 torch.cuda.Event(enable_timing=True) objects."""
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the CUDA event on its first record
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check("moe_forward_profiled", load_library().moe_forward_profiled(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),

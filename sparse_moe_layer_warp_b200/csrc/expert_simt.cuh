@@ -9,6 +9,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "ptx_sm100.cuh"
+
 namespace moe {
 
 // Row p of the expert-sorted space: p < Tk is pair perm[p] = t*k + j of expert
@@ -32,6 +34,8 @@ __global__ void __launch_bounds__(256) ffn_up_f32_kernel(
     const float *__restrict__ x, const float *__restrict__ wg, const float *__restrict__ wu,
     const int *__restrict__ perm, const int *__restrict__ topk_idx, int Tk, int k, int E,
     int n_rows, int d, int f, float *__restrict__ h) {
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t total = (size_t)n_rows * f;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -56,6 +60,8 @@ __global__ void __launch_bounds__(256) ffn_down_f32_kernel(
     const float *__restrict__ h, const float *__restrict__ wd, const int *__restrict__ perm,
     const int *__restrict__ topk_idx, const float *__restrict__ topk_gate, float routed_scale,
     int Tk, int k, int E, int n_rows, int d, int f, float *__restrict__ y) {
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t total = (size_t)n_rows * d;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -71,68 +77,50 @@ __global__ void __launch_bounds__(256) ffn_down_f32_kernel(
   }
 }
 
-// out[t, :] = sum_{j < k} y[slot_row[t, j], :] (+ y[Tk + t, :] if shared), summed in fp32
-// in this fixed order and rounded once.  16-byte vectors, grid-stride.
-template <typename T>
-struct CombineIO;
-template <>
-struct CombineIO<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ __forceinline__ static void add(const __nv_bfloat16 *p, float (&acc)[8]) {
-    uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 f = __bfloat1622float2(h[i]);
-      acc[2 * i] += f.x;
-      acc[2 * i + 1] += f.y;
-    }
-  }
-  __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float (&acc)[8]) {
-    uint4 u;
-    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    *reinterpret_cast<uint4 *>(p) = u;
-  }
-};
-template <>
-struct CombineIO<float> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void add(const float *p, float (&acc)[4]) {
-    float4 u = *reinterpret_cast<const float4 *>(p);
-    acc[0] += u.x;
-    acc[1] += u.y;
-    acc[2] += u.z;
-    acc[3] += u.w;
-  }
-  __device__ __forceinline__ static void store(float *p, const float (&acc)[4]) {
-    *reinterpret_cast<float4 *>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  }
-};
+// out[t, :] = sum_{j < k} y[slot_row[t, j], :] (+ y[Tk + t, :] if shared): y rows are
+// fp32, summed in this fixed order in fp32 and rounded once to the output type.  Each
+// thread owns 4 consecutive columns (16-byte loads of y), grid-stride.
+__device__ __forceinline__ void store4(float *p, const float4 &v) {
+  *reinterpret_cast<float4 *>(p) = v;
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, const float4 &v) {
+  uint2 u;
+  *reinterpret_cast<__nv_bfloat162 *>(&u.x) = __floats2bfloat162_rn(v.x, v.y);
+  *reinterpret_cast<__nv_bfloat162 *>(&u.y) = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2 *>(p) = u;
+}
 
-template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const T *__restrict__ y,
+template <typename Tout>
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y,
                                                       const int *__restrict__ slot_row,
                                                       int n_tokens, int k, int Tk,
                                                       int n_shared, int d,
-                                                      T *__restrict__ out) {
-  constexpr int V = CombineIO<T>::N;
-  const int vpr = d / V;
+                                                      Tout *__restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int vpr = d / 4;
   const size_t total = (size_t)n_tokens * vpr;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
     const int t = (int)(i / vpr);
-    const int c = (int)(i % vpr) * V;
-    float acc[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    const int c = (int)(i % vpr) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
-      const int p = slot_row[(size_t)t * k + j];
-      CombineIO<T>::add(y + (size_t)p * d + c, acc);
+      const int p = __ldg(slot_row + (size_t)t * k + j);
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)p * d + c));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
-    if (n_shared) CombineIO<T>::add(y + (size_t)(Tk + t) * d + c, acc);
-    CombineIO<T>::store(out + (size_t)t * d + c, acc);
+    if (n_shared) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)(Tk + t) * d + c));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    store4(out + (size_t)t * d + c, acc);
   }
 }
 

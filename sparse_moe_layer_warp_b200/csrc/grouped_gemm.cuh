@@ -15,8 +15,12 @@
 //
 //   MODE_UP   : A0 = W_gate, A1 = W_up (two accumulators), B = expert-sorted x rows
 //               (the shared group reads x directly); epilogue h = silu(G) * U -> bf16.
-//   MODE_DOWN : A0 = W_down, B = h rows; epilogue y = acc * scale -> bf16, scale =
-//               routed_scale * gate for routed rows and 1 for shared rows.
+//   MODE_LOGITS: router logits; one group (all T tokens), A0 = W_r (rows past E zero-filled
+//               by TMA), B = x; epilogue logits[t, e] = acc (fp32).
+//   MODE_DOWN : A0 = W_down, B = h rows; epilogue y = acc * scale -> fp32, scale =
+//               routed_scale * gate for routed rows and 1 for shared rows.  y stays fp32:
+//               rounding it to bf16 as well as h and the output would put the layer's
+//               error above 2e-2 x RMS(out) even with exact accumulation.
 //
 // Roles (192 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA issuer (warp 1
 // also owns the TMEM allocation), warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
@@ -33,7 +37,7 @@
 
 namespace moe {
 
-enum GemmMode { MODE_UP = 0, MODE_DOWN = 1 };
+enum GemmMode { MODE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
 
 struct GemmParams {
   CUtensorMap tmA0;  // UP: W_gate [G*f, d]; DOWN: W_down [G*d, f]     box {64, 128}
@@ -43,13 +47,13 @@ struct GemmParams {
   const int *offsets;       // [E + 1] expert offsets in the sorted space
   const int *perm;          // [Tk] (DOWN: gate lookup)
   const float *topk_gate;   // [Tk] (DOWN)
-  __nv_bfloat16 *out;       // UP: h [P, f]; DOWN: y [P, d]
+  void *out;                // UP: h [P, f] bf16; DOWN: y [P, d] fp32; LOGITS: [T, E] fp32
   DevStatus *status;
   float routed_scale;
   int E, n_groups, T, Tk;
-  int M;      // weight rows per group: f (UP) or d (DOWN)
-  int K;      // reduction length: d (UP) or f (DOWN)
-  int ld_out; // f (UP) or d (DOWN)
+  int M;      // weight rows per group: f (UP), d (DOWN), E (LOGITS)
+  int K;      // reduction length: d (UP, LOGITS) or f (DOWN)
+  int ld_out; // f (UP), d (DOWN), E (LOGITS)
 };
 
 constexpr int kBM = 128;         // weight rows per unit (MMA M)
@@ -79,7 +83,7 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
-           (size_t)(3 * n_groups + 1) * 4;
+           (size_t)(3 * n_groups + 1) * 4 + 2 * BN * 4 /*row scales*/;
   }
 };
 
@@ -105,10 +109,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
+  float *row_scale = reinterpret_cast<float *>(grp_row + p.n_groups);  // [2][BN] (DOWN)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups;
-  const int mtiles = p.M / kBM;
+  const int mtiles = (p.M + kBM - 1) / kBM;
   const int kblocks = p.K / kBK;
 
   if (threadIdx.x == 0) {
@@ -131,6 +136,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  // everything above overlaps the previous kernel's tail; what follows reads its outputs
+  griddep_wait();
+  griddep_launch_dependents();
   // group table: token count, first row in the sorted space, units per group
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
     int cnt, row;
@@ -311,6 +319,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row0 = grp_row[g] + nt * BN;
       const int col = mt * kBM + r;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      if (MODE == MODE_DOWN) {
+        // gate * routed_scale of each token column, staged once per unit (double-buffered
+        // by accumulator, so a fast warp never overwrites scales a slow warp still reads)
+        const int n = threadIdx.x - 64;
+        if (n < BN) {
+          float sc = 0.f;
+          if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
+          row_scale[acc * BN + n] = sc;
+        }
+        named_bar_sync(1, 128);
+      }
       for (int c0 = 0; c0 < valid; c0 += 16) {
         uint32_t v0[16];
         tmem_ld16(taddr + c0, v0);
@@ -324,18 +343,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float gv = __uint_as_float(v0[n]);
               const float uv = __uint_as_float(v1[n]);
               const float hv = gv / (1.f + expf(-gv)) * uv;
-              p.out[(size_t)(row0 + c0 + n) * p.ld_out + col] = __float2bfloat16_rn(hv);
+              static_cast<__nv_bfloat16 *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
+                  __float2bfloat16_rn(hv);
             }
           }
-        } else {
+        } else if (MODE == MODE_DOWN) {
           tmem_ld_wait();
+          const float *sc = row_scale + acc * BN + c0;
 #pragma unroll
           for (int n = 0; n < 16; ++n) {
-            if (c0 + n < valid) {
-              const int pr = row0 + c0 + n;
-              const float scale = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[pr]] : 1.f;
-              p.out[(size_t)pr * p.ld_out + col] =
-                  __float2bfloat16_rn(__uint_as_float(v0[n]) * scale);
+            if (c0 + n < valid)
+              static_cast<float *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
+                  __uint_as_float(v0[n]) * sc[n];
+          }
+        } else {  // MODE_LOGITS
+          tmem_ld_wait();
+          if (col < p.M) {
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+              if (c0 + n < valid)
+                static_cast<float *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
+                    __uint_as_float(v0[n]);
             }
           }
         }

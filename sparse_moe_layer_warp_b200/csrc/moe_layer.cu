@@ -14,6 +14,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <utility>
+
 #include "moe_layer.h"
 #include "expert_simt.cuh"
 #include "grouped_gemm.cuh"
@@ -28,7 +30,7 @@ struct moe_layer {
   int device;
   int num_sms;
   int smem_optin;
-  CUtensorMap tm_wg, tm_wu, tm_wd;
+  CUtensorMap tm_wg, tm_wu, tm_wd, tm_wr;
 };
 
 namespace {
@@ -69,6 +71,30 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t ro
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Every kernel of the library starts with griddepcontrol.wait, so each launch may use
+// programmatic stream serialisation: its CTAs can be scheduled (and run their set-up)
+// while the previous kernel drains.
+template <typename... KArgs, typename... Args>
+moe_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  Args &&...args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+int n_splits(const moe_config &c) { return (c.d_model + kSplitKSlice - 1) / kSplitKSlice; }
+
 size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 
 // Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
@@ -89,7 +115,8 @@ WsLayout ws_layout(const moe_config &c, int T) {
   const size_t P = Tk + (size_t)c.n_shared * T;
   const size_t nch = ((size_t)T + kChunk - 1) / kChunk;
   L.status = take(sizeof(DevStatus));
-  L.logits = take((size_t)T * c.n_experts * 4);
+  const size_t n_part = (T <= kSplitKTokens) ? (size_t)n_splits(c) : 1;
+  L.logits = take(n_part * T * c.n_experts * 4);  // split-K partials for small T
   L.idx = take(Tk * 4);
   L.gate = take(Tk * 4);
   L.counts = take((size_t)c.n_experts * 4);
@@ -99,7 +126,7 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.chunk_hist = take(nch * c.n_experts * 4);
   L.xs = (c.dtype == MOE_BF16) ? take(Tk * c.d_model * 2) : off;
   L.h = take(P * c.d_ff * esize(c));
-  L.y = take(P * c.d_model * esize(c));
+  L.y = take(P * c.d_model * 4);  // fp32 in both precisions
   L.total = off;
   return L;
 }
@@ -107,10 +134,6 @@ WsLayout ws_layout(const moe_config &c, int T) {
 template <typename P>
 P *at(void *ws, size_t off) {
   return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
-}
-
-moe_status last_launch() {
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int grid_for(size_t work, int per_block, int num_sms) {
@@ -130,59 +153,61 @@ int pick_bn(const moe_config &c, int T) {
 }
 
 // ------------------------------------------------------------------ routing launches
+moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
+                              cudaStream_t st);
+
+// Router logits.  Returns how many partial arrays [n][T][E] were written to `logits`
+// (split-K for small T; 1 otherwise) through *n_part.
 moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits,
-                         cudaStream_t st) {
+                         int *n_part, cudaStream_t st) {
   const moe_config &c = L->cfg;
-  constexpr int TB = 16;
-  if (T <= 32) {
-    dim3 grid(c.n_experts, (T + TB - 1) / TB);
+  *n_part = 1;
+  if (T <= kSplitKTokens) {
+    const int S = n_splits(c);
+    *n_part = S;
+    dim3 grid((c.n_experts + 31) / 32, S);
     if (c.dtype == MOE_BF16)
-      router_logits_rows_kernel<__nv_bfloat16, TB><<<grid, 128, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(x),
-          static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model, c.n_experts, logits);
-    else
-      router_logits_rows_kernel<float, TB><<<grid, 128, 0, st>>>(
-          static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
-          c.d_model, c.n_experts, logits);
-  } else {
-    dim3 grid((T + 63) / 64, (c.n_experts + 63) / 64);
-    if (c.dtype == MOE_BF16)
-      router_logits_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(x),
-          static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model, c.n_experts, logits);
-    else
-      router_logits_tiled_kernel<float><<<grid, 256, 0, st>>>(
-          static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
-          c.d_model, c.n_experts, logits);
+      return launch(router_logits_splitk_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16 *>(x),
+                    static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model,
+                    c.n_experts, logits);
+    return launch(router_logits_splitk_kernel<float>, grid, dim3(256), 0, st,
+                  static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
+                  c.d_model, c.n_experts, logits);
   }
-  return last_launch();
+  if (c.dtype == MOE_BF16) return launch_gemm_logits(L, x, T, logits, st);
+  dim3 grid((T + 63) / 64, (c.n_experts + 63) / 64);
+  return launch(router_logits_tiled_kernel<float>, grid, dim3(256), 0, st,
+                static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
+                c.d_model, c.n_experts, logits);
 }
 
-moe_status launch_select_permute(const moe_layer *L, const float *logits, int T, int *idx,
-                                 float *gate, int *counts, int *offsets, int *perm,
-                                 int *slot_row, int *chunk_hist, cudaStream_t st,
-                                 int mark_index = 0, void *const *events = nullptr) {
+moe_status launch_select_permute(const moe_layer *L, const float *logits, int n_part, int T,
+                                 float *logits_out, int *idx, float *gate, int *counts,
+                                 int *offsets, int *perm, int *slot_row, int *chunk_hist,
+                                 cudaStream_t st, void *const *events = nullptr,
+                                 int mark_index = 0) {
   const moe_config &c = L->cfg;
   const int nch = (T + kChunk - 1) / kChunk;
   const int need = (c.n_experts + 31) / 32;
   const float *bias = L->w.router_bias;
-  const int thr = kRouteWarps * 32;
-#define MOE_TOPK(V)                                                                       \
-  topk_hist_kernel<V><<<nch, thr, 0, st>>>(logits, bias, T, c.n_experts, c.top_k, idx, gate, \
-                                           chunk_hist)
-  if (need <= 1) MOE_TOPK(1);
-  else if (need <= 2) MOE_TOPK(2);
-  else if (need <= 4) MOE_TOPK(4);
-  else if (need <= 9) MOE_TOPK(9);
-  else if (need <= 16) MOE_TOPK(16);
-  else MOE_TOPK(32);
+  const dim3 thr(kRouteWarps * 32);
+  moe_status s;
+#define MOE_TOPK(V)                                                                        \
+  launch(topk_hist_kernel<V>, dim3(nch), thr, 0, st, logits, n_part, bias, T, c.n_experts, \
+         c.top_k, logits_out, idx, gate, chunk_hist)
+  if (need <= 1) s = MOE_TOPK(1);
+  else if (need <= 2) s = MOE_TOPK(2);
+  else if (need <= 4) s = MOE_TOPK(4);
+  else if (need <= 9) s = MOE_TOPK(9);
+  else if (need <= 16) s = MOE_TOPK(16);
+  else s = MOE_TOPK(32);
 #undef MOE_TOPK
-  if (last_launch() != MOE_OK) return MOE_ERR_CUDA;
+  if (s != MOE_OK) return s;
   if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  permute_scatter_kernel<<<nch, 256, 0, st>>>(idx, chunk_hist, T, c.n_experts, c.top_k, nch,
-                                              counts, offsets, perm, slot_row);
-  return last_launch();
+  return launch(permute_scatter_kernel, dim3(nch), dim3(256), 0, st, idx, chunk_hist, T,
+                c.n_experts, c.top_k, nch, counts, offsets, perm, slot_row);
 }
 
 // ------------------------------------------------------------------ grouped GEMM launch
@@ -195,8 +220,8 @@ moe_status launch_gemm_bn(const moe_layer *L, const GemmParams &p, cudaStream_t 
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  grouped_gemm_kernel<MODE, BN><<<L->num_sms, kGemmThreads, smem, st>>>(p);
-  return last_launch();
+  return launch(grouped_gemm_kernel<MODE, BN>, dim3(L->num_sms), dim3(kGemmThreads), smem, st,
+                p);
 }
 
 template <int MODE>
@@ -208,6 +233,28 @@ moe_status launch_gemm(const moe_layer *L, int bn, const GemmParams &p, cudaStre
     case 128: return launch_gemm_bn<MODE, 128>(L, p, st);
   }
   return MOE_ERR_UNSUPPORTED;
+}
+
+// Token tile of the router GEMM.
+int pick_bn_router(int T) { return T <= 256 ? 16 : (T <= 1024 ? 32 : 64); }
+
+moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
+                              cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  const int bn = pick_bn_router(T);
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.tmA0 = L->tm_wr;
+  if (!encode_bf16_2d(&p.tmB, x, c.d_model, T, bn)) return MOE_ERR_CUDA;
+  p.out = logits;
+  p.E = 0;  // one group: all T tokens, rows [0, T)
+  p.n_groups = 1;
+  p.T = T;
+  p.Tk = 0;
+  p.M = c.n_experts;
+  p.K = c.d_model;
+  p.ld_out = c.n_experts;
+  return launch_gemm<MODE_LOGITS>(L, bn, p, st);
 }
 
 moe_status check_call(const moe_layer *L, int T, void *ws, size_t ws_bytes) {
@@ -278,7 +325,8 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wu, w->w_up, c.d_model, G * c.d_ff, kBM) ||
-        !encode_bf16_2d(&L->tm_wd, w->w_down, c.d_ff, G * c.d_model, kBM)) {
+        !encode_bf16_2d(&L->tm_wd, w->w_down, c.d_ff, G * c.d_model, kBM) ||
+        !encode_bf16_2d(&L->tm_wr, w->w_router, c.d_model, c.n_experts, kBM)) {
       free(L);
       return MOE_ERR_CUDA;
     }
@@ -329,13 +377,16 @@ static moe_status route_common(moe_handle h, const void *x, const float *logits_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(h->cfg, T);
   const float *logits = logits_in;
+  int n_part = 1;
+  float *sum_out = nullptr;
   if (!logits) {
-    float *dst = logits_out ? logits_out : at<float>(ws, W.logits);
-    if ((s = launch_logits(h, x, T, dst, st)) != MOE_OK) return s;
+    float *dst = at<float>(ws, W.logits);
+    if ((s = launch_logits(h, x, T, dst, &n_part, st)) != MOE_OK) return s;
     logits = dst;
+    sum_out = logits_out;
   }
-  return launch_select_permute(h, logits, T, idx, gate, counts, offsets, perm, slot_row,
-                               at<int>(ws, W.chunk_hist), st);
+  return launch_select_permute(h, logits, n_part, T, sum_out, idx, gate, counts, offsets, perm,
+                               slot_row, at<int>(ws, W.chunk_hist), st);
 }
 
 moe_status moe_route(moe_handle h, const void *x, int n_tokens, float *logits_out,
@@ -380,23 +431,25 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                                                                                  : MOE_ERR_CUDA;
   };
   if ((s = mark(0)) != MOE_OK) return s;
-  if ((s = launch_logits(h, x, T, logits, st)) != MOE_OK) return s;
+  int n_part = 1;
+  if ((s = launch_logits(h, x, T, logits, &n_part, st)) != MOE_OK) return s;
   if ((s = mark(1)) != MOE_OK) return s;
-  if ((s = launch_select_permute(h, logits, T, idx, gate, at<int>(ws, W.counts), offsets, perm,
-                                 slot_row, at<int>(ws, W.chunk_hist), st, events ? 2 : 0,
-                                 events)) != MOE_OK)
+  if ((s = launch_select_permute(h, logits, n_part, T, nullptr, idx, gate,
+                                 at<int>(ws, W.counts), offsets, perm, slot_row,
+                                 at<int>(ws, W.chunk_hist), st, events, 2)) != MOE_OK)
     return s;
   if ((s = mark(3)) != MOE_OK) return s;
 
   if (c.dtype == MOE_BF16) {
     const int vpr = c.d_model / 8;
-    gather_rows_kernel<<<grid_for((size_t)Tk * vpr, 256, h->num_sms), 256, 0, st>>>(
-        static_cast<const uint4 *>(x), perm, c.top_k, Tk, vpr, at<uint4>(ws, W.xs));
-    if ((s = last_launch()) != MOE_OK) return s;
+    if ((s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk * vpr, 256, h->num_sms)),
+                    dim3(256), 0, st, static_cast<const uint4 *>(x), (const int *)perm,
+                    c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
+      return s;
     if ((s = mark(4)) != MOE_OK) return s;
     const int bn = pick_bn(c, T);
     __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
-    __nv_bfloat16 *ybuf = at<__nv_bfloat16>(ws, W.y);
+    float *ybuf = at<float>(ws, W.y);
     GemmParams p1;
     memset(&p1, 0, sizeof p1);
     p1.tmA0 = h->tm_wg;
@@ -428,31 +481,36 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p2.ld_out = c.d_model;
     if ((s = launch_gemm<MODE_DOWN>(h, bn, p2, st)) != MOE_OK) return s;
     if ((s = mark(6)) != MOE_OK) return s;
-    combine_kernel<__nv_bfloat16>
-        <<<grid_for((size_t)T * (c.d_model / 8), 256, h->num_sms), 256, 0, st>>>(
-            ybuf, slot_row, T, c.top_k, Tk, c.n_shared, c.d_model,
-            static_cast<__nv_bfloat16 *>(out));
-    if ((s = last_launch()) != MOE_OK) return s;
+    if ((s = launch(combine_kernel<__nv_bfloat16>,
+                    dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0,
+                    st, (const float *)ybuf, (const int *)slot_row, T, c.top_k, Tk, c.n_shared,
+                    c.d_model, static_cast<__nv_bfloat16 *>(out))) != MOE_OK)
+      return s;
     return mark(7);
   }
 
   float *hbuf = at<float>(ws, W.h);
   float *ybuf = at<float>(ws, W.y);
   if ((s = mark(4)) != MOE_OK) return s;
-  ffn_up_f32_kernel<<<grid_for((size_t)P * c.d_ff, 256, h->num_sms), 256, 0, st>>>(
-      static_cast<const float *>(x), static_cast<const float *>(h->w.w_gate),
-      static_cast<const float *>(h->w.w_up), perm, idx, Tk, c.top_k, c.n_experts, P, c.d_model,
-      c.d_ff, hbuf);
-  if ((s = last_launch()) != MOE_OK) return s;
+  if ((s = launch(ffn_up_f32_kernel, dim3(grid_for((size_t)P * c.d_ff, 256, h->num_sms)),
+                  dim3(256), 0, st, static_cast<const float *>(x),
+                  static_cast<const float *>(h->w.w_gate), static_cast<const float *>(h->w.w_up),
+                  (const int *)perm, (const int *)idx, Tk, c.top_k, c.n_experts, P, c.d_model,
+                  c.d_ff, hbuf)) != MOE_OK)
+    return s;
   if ((s = mark(5)) != MOE_OK) return s;
-  ffn_down_f32_kernel<<<grid_for((size_t)P * c.d_model, 256, h->num_sms), 256, 0, st>>>(
-      hbuf, static_cast<const float *>(h->w.w_down), perm, idx, gate, c.routed_scale, Tk,
-      c.top_k, c.n_experts, P, c.d_model, c.d_ff, ybuf);
-  if ((s = last_launch()) != MOE_OK) return s;
+  if ((s = launch(ffn_down_f32_kernel, dim3(grid_for((size_t)P * c.d_model, 256, h->num_sms)),
+                  dim3(256), 0, st, (const float *)hbuf,
+                  static_cast<const float *>(h->w.w_down), (const int *)perm, (const int *)idx,
+                  (const float *)gate, c.routed_scale, Tk, c.top_k, c.n_experts, P, c.d_model,
+                  c.d_ff, ybuf)) != MOE_OK)
+    return s;
   if ((s = mark(6)) != MOE_OK) return s;
-  combine_kernel<float><<<grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms), 256, 0, st>>>(
-      ybuf, slot_row, T, c.top_k, Tk, c.n_shared, c.d_model, static_cast<float *>(out));
-  if ((s = last_launch()) != MOE_OK) return s;
+  if ((s = launch(combine_kernel<float>,
+                  dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0, st,
+                  (const float *)ybuf, (const int *)slot_row, T, c.top_k, Tk, c.n_shared,
+                  c.d_model, static_cast<float *>(out))) != MOE_OK)
+    return s;
   return mark(7);
 }
 

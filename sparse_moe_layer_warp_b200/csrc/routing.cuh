@@ -10,12 +10,16 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "ptx_sm100.cuh"
+
 namespace moe {
 
 constexpr int kMaxExperts = 1024;   // E limit of the routing kernels
 constexpr int kMaxTopK = 32;        // one slot per lane
 constexpr int kChunk = 64;          // tokens per routing chunk (one CTA)
-constexpr int kRouteWarps = 8;
+constexpr int kRouteWarps = 16;    // top-k: one warp per token, 4 tokens per warp at most
+constexpr int kSplitKTokens = 64;   // largest T of the split-K router
+constexpr int kSplitKSlice = 256;   // d elements per split (32 lanes x 8)
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -50,47 +54,79 @@ struct Vec16<float> {
 };
 
 // ------------------------------------------------------------------ router logits (small T)
-// One CTA per (expert, block of TB tokens): the CTA streams W_r[e] once and reduces TB
-// dot products.  Used when the token count is small (decode), where the job is streaming
-// the 288 x d router matrix from HBM across many SMs.
-template <typename Tin, int TB>
-__global__ void __launch_bounds__(128) router_logits_rows_kernel(const Tin *__restrict__ x,
-                                                                 const Tin *__restrict__ wr,
-                                                                 int T, int d, int E,
-                                                                 float *__restrict__ logits) {
-  constexpr int V = Vec16<Tin>::N;
-  const int e = blockIdx.x;
-  const int t0 = blockIdx.y * TB;
-  const int nt = min(TB, T - t0);
-  float acc[TB];
+// Split-K over d: CTA (b, s) computes, for experts [32b, 32b + 32) and every token, the dot
+// product over d-slice s (kSplitKSlice elements: 8 per lane, 16-byte loads), and writes it
+// to part[s][t][e].  The top-k kernel adds the splits in increasing s, so the logits are
+// deterministic.  Decode streams the E x d router matrix from HBM across ~E/32 x d/256
+// CTAs instead of a handful.
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_logits_splitk_kernel(const Tin *__restrict__ x,
+                                                                   const Tin *__restrict__ wr,
+                                                                   int T, int d, int E,
+                                                                   float *__restrict__ part) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int V = Vec16<Tin>::N;      // elements per 16-byte load
+  constexpr int PER_LANE = 8;           // elements per lane per split
+  constexpr int TG = 16;                // tokens per register group
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * 32 + warp * 4;
+  const int s = blockIdx.y;
+  const int k0 = s * kSplitKSlice + lane * PER_LANE;
+  const bool kin = k0 < d;
+  float w[4][PER_LANE];
 #pragma unroll
-  for (int t = 0; t < TB; ++t) acc[t] = 0.f;
-  for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
-    float w[V];
-    Vec16<Tin>::load(wr + (size_t)e * d + i, w);
+  for (int i = 0; i < 4; ++i) {
+    const int e = e0 + i;
 #pragma unroll
-    for (int t = 0; t < TB; ++t) {
-      if (t < nt) {
-        float xv[V];
-        Vec16<Tin>::load(x + (size_t)(t0 + t) * d + i, xv);
+    for (int v0 = 0; v0 < PER_LANE; v0 += V) {
+      float tmp[V];
+      if (kin && e < E) Vec16<Tin>::load(wr + (size_t)e * d + k0 + v0, tmp);
+      else
 #pragma unroll
-        for (int v = 0; v < V; ++v) acc[t] = fmaf(xv[v], w[v], acc[t]);
-      }
+        for (int v = 0; v < V; ++v) tmp[v] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) w[i][v0 + v] = tmp[v];
     }
   }
-  __shared__ float red[TB][4];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int tg = 0; tg < T; tg += TG) {
+    float acc[4][TG];
 #pragma unroll
-  for (int t = 0; t < TB; ++t) {
-    float v = acc[t];
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[t][warp] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < nt) {
-    const int t = threadIdx.x;
-    logits[(size_t)(t0 + t) * E + e] = (red[t][0] + red[t][1]) + (red[t][2] + red[t][3]);
+      for (int t = 0; t < TG; ++t) acc[i][t] = 0.f;
+#pragma unroll
+    for (int t = 0; t < TG; ++t) {
+      if (tg + t < T && kin) {
+#pragma unroll
+        for (int v0 = 0; v0 < PER_LANE; v0 += V) {
+          float xv[V];
+          Vec16<Tin>::load(x + (size_t)(tg + t) * d + k0 + v0, xv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[i][t] = fmaf(xv[v], w[i][v0 + v], acc[i][t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int t = 0; t < TG; ++t) {
+        float v = acc[i][t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[i][t] = v;
+      }
+    // lane l writes (expert e0 + l / 16 * 2 + ..): spread the 64 results over the lanes
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int t = 0; t < TG; ++t) {
+        const int e = e0 + i;
+        if (lane == ((i * TG + t) & 31) && tg + t < T && e < E)
+          part[((size_t)s * T + tg + t) * E + e] = acc[i][t];
+      }
   }
 }
 
@@ -101,6 +137,8 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const Tin *__r
                                                                   const Tin *__restrict__ wr,
                                                                   int T, int d, int E,
                                                                   float *__restrict__ logits) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int BT = 64, BE = 64, BK = 32;
   __shared__ float xs[BK][BT + 4];
   __shared__ float ws[BK][BE + 4];
@@ -155,10 +193,15 @@ __device__ __forceinline__ bool ranks_before(float sa, int ea, float sb, int eb)
 // scores of experts l, l+32, ...  k rounds of warp arg-max pick S_t in rank order; lane j
 // keeps slot j.  Gates: softmax over the selected UNBIASED logits (max-shifted, expf).
 // The CTA's per-expert selection counts go to chunk_hist[c][e] (integer, order-free).
+// `logits` holds n_split partial logit arrays [n_split][T][E] that are added in increasing
+// split order (n_split = 1: plain logits); the sums are written to `logits_out` if given.
 template <int MAXV>
 __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
-    const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
-    int *__restrict__ topk_idx, float *__restrict__ topk_gate, int *__restrict__ chunk_hist) {
+    const float *__restrict__ logits, int n_split, const float *__restrict__ bias, int T,
+    int E, int k, float *__restrict__ logits_out, int *__restrict__ topk_idx,
+    float *__restrict__ topk_gate, int *__restrict__ chunk_hist) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int hist[kMaxExperts];
   const int c = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
@@ -172,7 +215,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
     for (int v = 0; v < MAXV; ++v) {
       const int e = lane + 32 * v;
       if (e < E) {
-        l[v] = logits[(size_t)t * E + e];
+        float acc = logits[(size_t)t * E + e];
+        for (int sp = 1; sp < n_split; ++sp) acc += logits[((size_t)sp * T + t) * E + e];
+        if (logits_out) logits_out[(size_t)t * E + e] = acc;
+        l[v] = acc;
         s[v] = l[v] + (bias ? bias[e] : 0.f);
       } else {
         l[v] = 0.f;
@@ -241,6 +287,8 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
     const int *__restrict__ topk_idx, const int *__restrict__ chunk_hist, int T, int E, int k,
     int n_chunks, int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
     int *__restrict__ slot_row) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int s_tot[kMaxExperts];
   __shared__ int s_base[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
@@ -331,6 +379,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
                                                           const int *__restrict__ perm, int k,
                                                           int n_rows, int vec_per_row,
                                                           uint4 *__restrict__ xs) {
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t total = (size_t)n_rows * vec_per_row;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {

@@ -14,6 +14,7 @@ decode_t16         16     4096   288  8   1280   bf16; 4 sequences x 4 MTP-3 pos
 decode_t256        256    4096   288  8   1280   bf16; batched decode
 prefill_t8192      8192   4096   288  8   1280   bf16; prefill chunk
 skew_t4096         4096   4096   288  8   1280   bf16; Zipf(1.1)-skewed expert selection
+prefill_e32_t1024  1024   4096   32   8   1280   bf16; profiler-sized prefill-like case
 =================  =====  =====  ===  ==  =====  ======================================
 
 Every workload has one shared expert with the routed experts' hidden size.  Distributions:
@@ -61,6 +62,9 @@ WORKLOADS = {
     "decode_t256": Workload("decode_t256", T=256, d=4096, E=288, k=8, f=1280),
     "prefill_t8192": Workload("prefill_t8192", T=8192, d=4096, E=288, k=8, f=1280),
     "skew_t4096": Workload("skew_t4096", T=4096, d=4096, E=288, k=8, f=1280, bias="zipf"),
+    # small case with prefill's per-expert load (~256 tokens per expert) and full-size
+    # expert matrices, ~1 GB of weights: for profiler captures that must stay small
+    "prefill_e32_t1024": Workload("prefill_e32_t1024", T=1024, d=4096, E=32, k=8, f=1280),
 }
 
 
