@@ -67,7 +67,10 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
   static constexpr int ACC_COLS = NA * BN;
-  static constexpr int TMEM_COLS_RAW = 2 * ACC_COLS;
+  // two accumulator buffers (epilogue of unit i overlaps MMAs of unit i+1) when they fit in
+  // the 512 TMEM columns; the up kernel at BN = 256 (gate + up = 512 columns) has one
+  static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
+  static constexpr int TMEM_COLS_RAW = ACC_BUFS * ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_COLS_RAW <= 32    ? 32
                                    : TMEM_COLS_RAW <= 64  ? 64
                                    : TMEM_COLS_RAW <= 128 ? 128
@@ -83,7 +86,7 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
-           (size_t)(3 * n_groups + 1) * 4 + 2 * BN * 4 /*row scales*/;
+           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * BN * 4 /*row scales*/;
   }
 };
 
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
-  float *row_scale = reinterpret_cast<float *>(grp_row + p.n_groups);  // [2][BN] (DOWN)
+  float *row_scale = reinterpret_cast<float *>(grp_row + p.n_groups);  // [ACC_BUFS][BN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups;
@@ -198,47 +201,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      // Walks the (unit, k-block) load slots of this CTA in order.
       const uint64_t pol_w = policy_evict_first();  // weights read once
       const uint64_t pol_b = policy_evict_last();   // activations: re-read per m tile
+      struct Slot {
+        int u, kb, a_row, b_row;
+        bool shared_x, single_use;
+      };
+      auto slot_set_unit = [&](Slot &c) {
+        int g, mt, nt;
+        decode(c.u, g, mt, nt);
+        c.a_row = g * p.M + mt * kBM;
+        c.shared_x = (MODE == MODE_UP) && (g >= p.E);
+        c.b_row = c.shared_x ? nt * BN : grp_row[g] + nt * BN;
+        // a weight tile read by one unit only is streamed with evict-first priority; one
+        // shared by several token tiles keeps normal priority so its neighbours hit L2
+        c.single_use = grp_count[g] <= BN;
+      };
+      auto slot_next = [&](Slot &c) {
+        if (++c.kb == kblocks) {
+          c.kb = 0;
+          c.u += gridDim.x;
+          if (c.u < total_units) slot_set_unit(c);
+        }
+      };
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        int g, mt, nt;
-        decode(u, g, mt, nt);
-        const int a_row = g * p.M + mt * kBM;
-        const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
-        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
-        const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
-        // a weight tile read by one unit only is streamed with evict-first priority; one
-        // shared by several token tiles keeps normal priority so its neighbours hit L2
-        const bool single_use = grp_count[g] <= BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          if (single_use) {
-            tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kb * kBK, a_row,
-                             pol_w);
-            if (MODE == MODE_UP)
-              tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kb * kBK,
-                               a_row, pol_w);
-          } else {
-            tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kb * kBK, a_row);
-            if (MODE == MODE_UP)
-              tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kb * kBK, a_row);
-          }
-          tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kb * kBK, b_row,
-                           pol_b);
-          ++issued;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1;
-          }
+      Slot ld{(int)blockIdx.x, 0, 0, 0, false, false};
+      if (ld.u < total_units) slot_set_unit(ld);
+      while (ld.u < total_units) {
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
+          ok = false;
+          break;
         }
+        const CUtensorMap *bmap = ld.shared_x ? &p.tmBs : &p.tmB;
+        const int kc = ld.kb * kBK;
+        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+        if (ld.single_use) {
+          tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, ld.a_row, pol_w);
+          if (MODE == MODE_UP)
+            tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, ld.a_row,
+                             pol_w);
+        } else {
+          tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, ld.a_row);
+          if (MODE == MODE_UP)
+            tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, ld.a_row);
+        }
+        tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kc, ld.b_row, pol_b);
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+        slot_next(ld);
       }
       if (!ok) {
         // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
@@ -263,8 +280,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = it % C::ACC_BUFS;
+        const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
         int g, mt, nt;
@@ -309,8 +326,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = q * 32 + lane;         // weight row within the unit
     int it = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = it % C::ACC_BUFS;
+      const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, 4)) break;
       tc_fence_after();
       int g, mt, nt;
@@ -320,10 +337,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int col = mt * kBM + r;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
       if (MODE == MODE_DOWN) {
-        // gate * routed_scale of each token column, staged once per unit (double-buffered
-        // by accumulator, so a fast warp never overwrites scales a slow warp still reads)
-        const int n = threadIdx.x - 64;
-        if (n < BN) {
+        // gate * routed_scale of each token column, staged once per unit (one copy per
+        // accumulator buffer, so a fast warp never overwrites scales a slow warp still reads)
+        for (int n = threadIdx.x - 64; n < BN; n += 128) {
           float sc = 0.f;
           if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
           row_scale[acc * BN + n] = sc;

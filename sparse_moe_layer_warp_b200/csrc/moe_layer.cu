@@ -99,8 +99,8 @@ size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 
 // Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
 struct WsLayout {
-  size_t status, logits, idx, gate, counts, offsets, perm, slot_row, chunk_hist, xs, h, y,
-      total;
+  size_t status, logits, part, idx, gate, counts, offsets, perm, slot_row, chunk_hist, xs, h,
+      y, total;
 };
 
 WsLayout ws_layout(const moe_config &c, int T) {
@@ -115,8 +115,8 @@ WsLayout ws_layout(const moe_config &c, int T) {
   const size_t P = Tk + (size_t)c.n_shared * T;
   const size_t nch = ((size_t)T + kChunk - 1) / kChunk;
   L.status = take(sizeof(DevStatus));
-  const size_t n_part = (T <= kSplitKTokens) ? (size_t)n_splits(c) : 1;
-  L.logits = take(n_part * T * c.n_experts * 4);  // split-K partials for small T
+  L.logits = take((size_t)T * c.n_experts * 4);
+  L.part = take((T <= kSplitKTokens ? (size_t)n_splits(c) : 0) * T * c.n_experts * 4);
   L.idx = take(Tk * 4);
   L.gate = take(Tk * 4);
   L.counts = take((size_t)c.n_experts * 4);
@@ -143,37 +143,38 @@ int grid_for(size_t work, int per_block, int num_sms) {
   return b < 1 ? 1 : (int)b;
 }
 
-// Token tile of the grouped GEMM from the mean tokens per routed expert.
-int pick_bn(const moe_config &c, int T) {
+// Token tile of the grouped GEMM from the mean tokens per routed expert.  Larger tiles
+// raise the tensor work per staged byte; the smallest tile that holds a typical group keeps
+// the token rows a TMA box loads mostly useful.
+// The up kernel stops at 128: at 256 its gate + up accumulators fill all 512 TMEM columns,
+// the epilogue can no longer overlap the next tile's MMAs, and it runs slower (measured).
+int pick_bn(const moe_config &c, int T, int mode) {
   const double mean = (double)T * c.top_k / c.n_experts;
   if (mean <= 4.0) return 16;
   if (mean <= 12.0) return 32;
   if (mean <= 40.0) return 64;
-  return 128;
+  if (mean <= 160.0 || mode == MODE_UP) return 128;
+  return 256;
 }
 
 // ------------------------------------------------------------------ routing launches
 moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
                               cudaStream_t st);
 
-// Router logits.  Returns how many partial arrays [n][T][E] were written to `logits`
-// (split-K for small T; 1 otherwise) through *n_part.
-moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits,
-                         int *n_part, cudaStream_t st) {
+// Router logits [T][E] into `logits`; for small T the split-K partials go to `part`.
+moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits, float *part,
+                         DevStatus *status, cudaStream_t st) {
   const moe_config &c = L->cfg;
-  *n_part = 1;
   if (T <= kSplitKTokens) {
-    const int S = n_splits(c);
-    *n_part = S;
-    dim3 grid((c.n_experts + 31) / 32, S);
+    dim3 grid((c.n_experts + 31) / 32, n_splits(c));
     if (c.dtype == MOE_BF16)
       return launch(router_logits_splitk_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
                     static_cast<const __nv_bfloat16 *>(x),
                     static_cast<const __nv_bfloat16 *>(L->w.w_router), T, c.d_model,
-                    c.n_experts, logits);
+                    c.n_experts, part, logits, status->router_ticket);
     return launch(router_logits_splitk_kernel<float>, grid, dim3(256), 0, st,
                   static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
-                  c.d_model, c.n_experts, logits);
+                  c.d_model, c.n_experts, part, logits, status->router_ticket);
   }
   if (c.dtype == MOE_BF16) return launch_gemm_logits(L, x, T, logits, st);
   dim3 grid((T + 63) / 64, (c.n_experts + 63) / 64);
@@ -182,7 +183,7 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
                 c.d_model, c.n_experts, logits);
 }
 
-moe_status launch_select_permute(const moe_layer *L, const float *logits, int n_part, int T,
+moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
                                  float *logits_out, int *idx, float *gate, int *counts,
                                  int *offsets, int *perm, int *slot_row, int *chunk_hist,
                                  cudaStream_t st, void *const *events = nullptr,
@@ -194,8 +195,8 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int n_
   const dim3 thr(kRouteWarps * 32);
   moe_status s;
 #define MOE_TOPK(V)                                                                        \
-  launch(topk_hist_kernel<V>, dim3(nch), thr, 0, st, logits, n_part, bias, T, c.n_experts, \
-         c.top_k, logits_out, idx, gate, chunk_hist)
+  launch(topk_hist_kernel<V>, dim3(nch), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
+         logits_out, idx, gate, chunk_hist)
   if (need <= 1) s = MOE_TOPK(1);
   else if (need <= 2) s = MOE_TOPK(2);
   else if (need <= 4) s = MOE_TOPK(4);
@@ -230,7 +231,12 @@ moe_status launch_gemm(const moe_layer *L, int bn, const GemmParams &p, cudaStre
     case 16: return launch_gemm_bn<MODE, 16>(L, p, st);
     case 32: return launch_gemm_bn<MODE, 32>(L, p, st);
     case 64: return launch_gemm_bn<MODE, 64>(L, p, st);
-    case 128: return launch_gemm_bn<MODE, 128>(L, p, st);
+  }
+  if constexpr (MODE != MODE_LOGITS) {
+    if (bn == 128) return launch_gemm_bn<MODE, 128>(L, p, st);
+  }
+  if constexpr (MODE == MODE_DOWN) {
+    if (bn == 256) return launch_gemm_bn<MODE, 256>(L, p, st);
   }
   return MOE_ERR_UNSUPPORTED;
 }
@@ -306,6 +312,7 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
   if (!L) return MOE_ERR_INVALID_ARG;
   L->cfg = c;
   L->w = *w;
+
   int major = 0;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
@@ -347,6 +354,7 @@ size_t moe_workspace_size(moe_handle h, int n_tokens) {
 }
 
 moe_status moe_workspace_init(moe_handle h, void *ws, size_t ws_bytes, void *stream) {
+  // zeroes the status word and the router's split-K tickets
   if (!h || !ws || ws_bytes < sizeof(DevStatus)) return MOE_ERR_INVALID_ARG;
   return cudaMemsetAsync(ws, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
@@ -377,15 +385,16 @@ static moe_status route_common(moe_handle h, const void *x, const float *logits_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(h->cfg, T);
   const float *logits = logits_in;
-  int n_part = 1;
-  float *sum_out = nullptr;
+  float *copy_out = nullptr;
   if (!logits) {
     float *dst = at<float>(ws, W.logits);
-    if ((s = launch_logits(h, x, T, dst, &n_part, st)) != MOE_OK) return s;
+    if ((s = launch_logits(h, x, T, dst, at<float>(ws, W.part), at<DevStatus>(ws, W.status),
+                           st)) != MOE_OK)
+      return s;
     logits = dst;
-    sum_out = logits_out;
+    copy_out = logits_out;
   }
-  return launch_select_permute(h, logits, n_part, T, sum_out, idx, gate, counts, offsets, perm,
+  return launch_select_permute(h, logits, T, copy_out, idx, gate, counts, offsets, perm,
                                slot_row, at<int>(ws, W.chunk_hist), st);
 }
 
@@ -431,10 +440,11 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                                                                                  : MOE_ERR_CUDA;
   };
   if ((s = mark(0)) != MOE_OK) return s;
-  int n_part = 1;
-  if ((s = launch_logits(h, x, T, logits, &n_part, st)) != MOE_OK) return s;
+  if ((s = launch_logits(h, x, T, logits, at<float>(ws, W.part), at<DevStatus>(ws, W.status),
+                         st)) != MOE_OK)
+    return s;
   if ((s = mark(1)) != MOE_OK) return s;
-  if ((s = launch_select_permute(h, logits, n_part, T, nullptr, idx, gate,
+  if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
                                  at<int>(ws, W.counts), offsets, perm, slot_row,
                                  at<int>(ws, W.chunk_hist), st, events, 2)) != MOE_OK)
     return s;
@@ -447,7 +457,8 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                     c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
       return s;
     if ((s = mark(4)) != MOE_OK) return s;
-    const int bn = pick_bn(c, T);
+    const int bn = pick_bn(c, T, MODE_UP);
+    const int bn2 = pick_bn(c, T, MODE_DOWN);
     __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
     float *ybuf = at<float>(ws, W.y);
     GemmParams p1;
@@ -474,12 +485,12 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     if ((s = mark(5)) != MOE_OK) return s;
     GemmParams p2 = p1;
     p2.tmA0 = h->tm_wd;
-    if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn)) return MOE_ERR_CUDA;
+    if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
     p2.out = ybuf;
     p2.M = c.d_model;
     p2.K = c.d_ff;
     p2.ld_out = c.d_model;
-    if ((s = launch_gemm<MODE_DOWN>(h, bn, p2, st)) != MOE_OK) return s;
+    if ((s = launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK) return s;
     if ((s = mark(6)) != MOE_OK) return s;
     if ((s = launch(combine_kernel<__nv_bfloat16>,
                     dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0,

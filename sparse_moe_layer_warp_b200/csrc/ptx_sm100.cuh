@@ -13,9 +13,10 @@ namespace moe {
 // ----------------------------------------------------------------------------- status
 // Device status word layout in the workspace header.
 struct DevStatus {
-  int error;   // 0 = ok, 1 = a bounded wait gave up
-  int where;   // which wait (kernel-specific code)
-  int pad[62];
+  int error;             // 0 = ok, 1 = a bounded wait gave up
+  int where;             // which wait (kernel-specific code)
+  int pad[30];
+  int router_ticket[32]; // split-K router: arrivals per block of 32 experts (self-resetting)
 };
 
 // Time limit of every device-side spin wait (ns of %globaltimer).

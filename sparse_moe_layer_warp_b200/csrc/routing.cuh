@@ -55,15 +55,15 @@ struct Vec16<float> {
 
 // ------------------------------------------------------------------ router logits (small T)
 // Split-K over d: CTA (b, s) computes, for experts [32b, 32b + 32) and every token, the dot
-// product over d-slice s (kSplitKSlice elements: 8 per lane, 16-byte loads), and writes it
-// to part[s][t][e].  The top-k kernel adds the splits in increasing s, so the logits are
-// deterministic.  Decode streams the E x d router matrix from HBM across ~E/32 x d/256
-// CTAs instead of a handful.
+// product over d-slice s (kSplitKSlice elements: 8 per lane, 16-byte loads) and writes it to
+// part[s][t][e].  The last CTA of block b to finish (ticket counter) adds the splits in
+// increasing s and writes logits[t][e]; the order of the sum never depends on which CTA is
+// last, so the logits are deterministic.  No CTA waits for another.  Decode streams the
+// E x d router matrix from HBM across ~E/32 x d/256 CTAs instead of a handful.
 template <typename Tin>
-__global__ void __launch_bounds__(256) router_logits_splitk_kernel(const Tin *__restrict__ x,
-                                                                   const Tin *__restrict__ wr,
-                                                                   int T, int d, int E,
-                                                                   float *__restrict__ part) {
+__global__ void __launch_bounds__(256) router_logits_splitk_kernel(
+    const Tin *__restrict__ x, const Tin *__restrict__ wr, int T, int d, int E,
+    float *__restrict__ part, float *__restrict__ logits, int *__restrict__ tickets) {
   griddep_wait();
   griddep_launch_dependents();
   constexpr int V = Vec16<Tin>::N;      // elements per 16-byte load
@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256) router_logits_splitk_kernel(const Tin *__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * 32 + warp * 4;
   const int s = blockIdx.y;
+  const int S = gridDim.y;
   const int k0 = s * kSplitKSlice + lane * PER_LANE;
   const bool kin = k0 < d;
   float w[4][PER_LANE];
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(256) router_logits_splitk_kernel(const Tin *__
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         acc[i][t] = v;
       }
-    // lane l writes (expert e0 + l / 16 * 2 + ..): spread the 64 results over the lanes
+    // spread the 64 results of the warp over its lanes for the stores
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -128,6 +129,24 @@ __global__ void __launch_bounds__(256) router_logits_splitk_kernel(const Tin *__
           part[((size_t)s * T + tg + t) * E + e] = acc[i][t];
       }
   }
+  // last arriver of this expert block reduces the splits in order
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&tickets[blockIdx.x], 1) == S - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int eb = blockIdx.x * 32;
+  const int ne = min(32, E - eb);
+  for (int i = threadIdx.x; i < T * 32; i += blockDim.x) {
+    const int t = i >> 5, e = eb + (i & 31);
+    if ((i & 31) >= ne) continue;
+    float acc = 0.f;
+    for (int sp = 0; sp < S; ++sp) acc += __ldcg(part + ((size_t)sp * T + t) * E + e);
+    logits[(size_t)t * E + e] = acc;
+  }
+  if (threadIdx.x == 0) tickets[blockIdx.x] = 0;  // ready for the next call
 }
 
 // ------------------------------------------------------------------ router logits (tiled)
@@ -180,26 +199,26 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const Tin *__r
 }
 
 // ------------------------------------------------------------------ top-k + chunk histogram
-// Ranking: a ranks before b iff (a is a number and b is NaN) or a.s > b.s or
-// (a.s == b.s or both NaN) and a.id < b.id.  Entries past E carry id = INT_MAX, s = NaN.
-__device__ __forceinline__ bool ranks_before(float sa, int ea, float sb, int eb) {
-  const bool na = sa != sa, nb = sb != sb;
-  if (na != nb) return nb;
-  if (!na && sa != sb) return sa > sb;
-  return ea < eb;
+// Ranking: a before b iff a's fp32 score is larger, or equal with the lower expert id;
+// -0.0 == +0.0; NaN below every number.  score_key maps a score to an unsigned integer with
+// the same order (NaN -> 0, every number >= 0x007FFFFF), so the warp can pick the winner
+// with two single-instruction reductions: the largest key, then the lowest id holding it.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  if (s != s) return 0u;
+  const uint32_t b = __float_as_uint(s == 0.f ? 0.f : s);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
 // One warp per token; CTA c handles tokens [c*kChunk, (c+1)*kChunk).  Lane l holds the
 // scores of experts l, l+32, ...  k rounds of warp arg-max pick S_t in rank order; lane j
 // keeps slot j.  Gates: softmax over the selected UNBIASED logits (max-shifted, expf).
 // The CTA's per-expert selection counts go to chunk_hist[c][e] (integer, order-free).
-// `logits` holds n_split partial logit arrays [n_split][T][E] that are added in increasing
-// split order (n_split = 1: plain logits); the sums are written to `logits_out` if given.
+// logits_out (optional) receives a copy of the logits read.
 template <int MAXV>
 __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
-    const float *__restrict__ logits, int n_split, const float *__restrict__ bias, int T,
-    int E, int k, float *__restrict__ logits_out, int *__restrict__ topk_idx,
-    float *__restrict__ topk_gate, int *__restrict__ chunk_hist) {
+    const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
+    float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
+    int *__restrict__ chunk_hist) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ int hist[kMaxExperts];
@@ -209,53 +228,46 @@ __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tbeg = c * kChunk, tend = min(T, tbeg + kChunk);
   for (int t = tbeg + warp; t < tend; t += kRouteWarps) {
-    float s[MAXV], l[MAXV];
-    uint32_t used = 0;
+    uint32_t key[MAXV];
+    float l[MAXV];
 #pragma unroll
     for (int v = 0; v < MAXV; ++v) {
       const int e = lane + 32 * v;
       if (e < E) {
-        float acc = logits[(size_t)t * E + e];
-        for (int sp = 1; sp < n_split; ++sp) acc += logits[((size_t)sp * T + t) * E + e];
-        if (logits_out) logits_out[(size_t)t * E + e] = acc;
-        l[v] = acc;
-        s[v] = l[v] + (bias ? bias[e] : 0.f);
+        l[v] = logits[(size_t)t * E + e];
+        if (logits_out) logits_out[(size_t)t * E + e] = l[v];
+        key[v] = score_key(l[v] + (bias ? bias[e] : 0.f));
       } else {
         l[v] = 0.f;
-        s[v] = __int_as_float(0x7fc00000);
+        key[v] = 0u;  // ties with NaN scores and loses on id (all ids here are >= E)
       }
     }
     int my_e = 0;
     float my_l = 0.f;
+    uint32_t used = 0;
     for (int r = 0; r < k; ++r) {
-      float bs = __int_as_float(0x7fc00000);
-      int be = 0x7fffffff;
+      // lane-local best among unused entries; ids grow with v, so '>' keeps the lower id
+      uint32_t bk = 0;
+      int bv = -1;
       float bl = 0.f;
 #pragma unroll
       for (int v = 0; v < MAXV; ++v) {
-        const int e = lane + 32 * v;
-        const bool ok = (e < E) && !((used >> v) & 1u);
-        if (ok && ranks_before(s[v], e, bs, be)) {
-          bs = s[v];
-          be = e;
+        const bool ok = !((used >> v) & 1u);
+        if (ok && (bv < 0 || key[v] > bk)) {
+          bk = key[v];
+          bv = v;
           bl = l[v];
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-        if (ranks_before(os, oe, bs, be)) {
-          bs = os;
-          be = oe;
-          bl = ol;
-        }
-      }
-      if ((be & 31) == lane) used |= 1u << (be >> 5);
+      const uint32_t wkey = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t cand = (bv >= 0 && bk == wkey) ? (uint32_t)(lane + 32 * bv) : 0xffffffffu;
+      const uint32_t wid = __reduce_min_sync(0xffffffffu, cand);
+      const int owner = (int)(wid & 31u);
+      if (owner == lane) used |= 1u << (wid >> 5);
+      const float wl = __shfl_sync(0xffffffffu, bl, owner);
       if (lane == r) {
-        my_e = be;
-        my_l = bl;
+        my_e = (int)wid;
+        my_l = wl;
       }
     }
     // gates over lanes 0..k-1
