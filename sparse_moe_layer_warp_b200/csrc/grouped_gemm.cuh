@@ -86,9 +86,61 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
-           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * BN * 4 /*row scales*/;
+           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * BN * 4 /*row scales*/ +
+           4 * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
   }
 };
+
+// silu(g) * u with the fast exponential and division (relative error ~1e-6, far below the
+// bf16 rounding of the result); silu(z) = z / (1 + exp(-z)) -> 0 for z -> -inf.
+__device__ __forceinline__ float swiglu(float g, float u) {
+  return __fdividef(g, 1.f + __expf(-g)) * u;
+}
+
+// Epilogue store of one 32-row x 16-token block held by a warp (lane = row, vals[n] = token
+// column c0 + n) into a row-major [token][column] output: the block is transposed through a
+// per-warp shared-memory buffer (16 x 32 fp32) so every lane writes 16-byte vectors along an
+// output row.  Rows (tokens) at or past `valid` are not written.
+__device__ __forceinline__ void store_block16_bf16(__nv_bfloat16 *out, int ld, int row0, int c0,
+                                                   int valid, int col_base, const float (&vals)[16],
+                                                   float *wbuf, int lane) {
+#pragma unroll
+  for (int n = 0; n < 16; ++n) wbuf[n * 32 + lane] = vals[n];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {  // 16 tokens x 4 chunks of 8 columns = 64 chunks
+    const int c = lane + 32 * i;
+    const int j = c >> 2, k = c & 3;
+    if (c0 + j < valid) {
+      const float4 a = *reinterpret_cast<const float4 *>(wbuf + j * 32 + 8 * k);
+      const float4 b = *reinterpret_cast<const float4 *>(wbuf + j * 32 + 8 * k + 4);
+      uint4 v;
+      *reinterpret_cast<__nv_bfloat162 *>(&v.x) = __floats2bfloat162_rn(a.x, a.y);
+      *reinterpret_cast<__nv_bfloat162 *>(&v.y) = __floats2bfloat162_rn(a.z, a.w);
+      *reinterpret_cast<__nv_bfloat162 *>(&v.z) = __floats2bfloat162_rn(b.x, b.y);
+      *reinterpret_cast<__nv_bfloat162 *>(&v.w) = __floats2bfloat162_rn(b.z, b.w);
+      *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c0 + j) * ld + col_base + 8 * k) = v;
+    }
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_block16_f32(float *out, int ld, int row0, int c0,
+                                                  int valid, int col_base, const float (&vals)[16],
+                                                  float *wbuf, int lane) {
+#pragma unroll
+  for (int n = 0; n < 16; ++n) wbuf[n * 32 + lane] = vals[n];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // 16 tokens x 8 chunks of 4 columns = 128 chunks
+    const int c = lane + 32 * i;
+    const int j = c >> 3, k = c & 7;
+    if (c0 + j < valid)
+      *reinterpret_cast<float4 *>(out + (size_t)(row0 + c0 + j) * ld + col_base + 4 * k) =
+          *reinterpret_cast<const float4 *>(wbuf + j * 32 + 4 * k);
+  }
+  __syncwarp();
+}
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -112,7 +164,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
-  float *row_scale = reinterpret_cast<float *>(grp_row + p.n_groups);  // [ACC_BUFS][BN]
+  // [ACC_BUFS][BN], 16-byte aligned: read as float4
+  float *row_scale = reinterpret_cast<float *>(
+      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+  float *xbuf = row_scale + C::ACC_BUFS * BN;  // [4 warps][16][32] epilogue transposes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups;
@@ -346,33 +401,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         named_bar_sync(1, 128);
       }
+      float *wbuf = xbuf + q * 16 * 32;
+      const int col_base = mt * kBM + q * 32;  // first output column of this warp
       for (int c0 = 0; c0 < valid; c0 += 16) {
         uint32_t v0[16];
+        float vals[16];
         tmem_ld16(taddr + c0, v0);
         if (MODE == MODE_UP) {
           uint32_t v1[16];
           tmem_ld16(taddr + BN + c0, v1);
           tmem_ld_wait();
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            if (c0 + n < valid) {
-              const float gv = __uint_as_float(v0[n]);
-              const float uv = __uint_as_float(v1[n]);
-              const float hv = gv / (1.f + expf(-gv)) * uv;
-              static_cast<__nv_bfloat16 *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
-                  __float2bfloat16_rn(hv);
-            }
-          }
+          for (int n = 0; n < 16; ++n)
+            vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
+          store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
+                             col_base, vals, wbuf, lane);
         } else if (MODE == MODE_DOWN) {
           tmem_ld_wait();
-          const float *sc = row_scale + acc * BN + c0;
+          const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            if (c0 + n < valid)
-              static_cast<float *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
-                  __uint_as_float(v0[n]) * sc[n];
+          for (int n4 = 0; n4 < 4; ++n4) {
+            const float4 s4 = sc[n4];
+            vals[4 * n4 + 0] = __uint_as_float(v0[4 * n4 + 0]) * s4.x;
+            vals[4 * n4 + 1] = __uint_as_float(v0[4 * n4 + 1]) * s4.y;
+            vals[4 * n4 + 2] = __uint_as_float(v0[4 * n4 + 2]) * s4.z;
+            vals[4 * n4 + 3] = __uint_as_float(v0[4 * n4 + 3]) * s4.w;
           }
-        } else {  // MODE_LOGITS
+          store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
+                            vals, wbuf, lane);
+        } else {  // MODE_LOGITS: E need not be a multiple of 32, so scalar masked stores
           tmem_ld_wait();
           if (col < p.M) {
 #pragma unroll

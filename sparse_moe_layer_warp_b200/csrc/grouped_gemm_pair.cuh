@@ -1,0 +1,345 @@
+// grouped_gemm_pair.cuh -- the grouped expert GEMM of grouped_gemm.cuh on CTA pairs
+// (tcgen05 cta_group::2) for large expert groups (prefill).
+//
+// Same work ("fused MoE gather/scatter with grouped GEMM", "Step 3.5 Flash: Open
+// Frontier-Level Intelligence with 11B Active Parameters", section 3.2.4; SwiGLU experts,
+// "Step 3.5 Flash 技术论文深度解读", training stability, root cause 3) and the same
+// parameters and epilogues as grouped_gemm_kernel, with a bigger tile per unit:
+// 256 weight rows x up to 256 tokens.  A cluster of two CTAs on one TPC runs it: CTA r stages
+// weight rows [128r, 128r + 128) of the unit and token rows [n0 + r*half, n0 + r*half + 128)
+// (half = the token tile split point), the leader (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, N = 2*half, and each CTA's TMEM receives its 128 rows
+// of D for all N token columns (column j = token n0 + j).  Per CTA and 64-wide K step the up
+// kernel stages 48 KB for 2 x 128 x 256 x 64 MACs -- twice the tensor work per staged byte of
+// the 1-CTA 128 x 128 tile, which is what limits that kernel at prefill sizes (it stays near
+// 70 GB/s of TMA delivery per SM).
+//
+// Barriers: full[s] lives in the leader and counts both CTAs' TMA bytes (the peer's loads
+// signal it through the .cta_group::2 load form); the leader's MMA commits arrive on empty[s]
+// and tmem_full[a] of both CTAs; tmem_empty[a] (leader) collects one arrival per epilogue
+// warp of both CTAs.  All waits are bounded as in grouped_gemm.cuh.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "grouped_gemm.cuh"
+#include "ptx_sm100.cuh"
+
+namespace moe {
+
+constexpr int kPairBM = 256;  // weight rows per unit (both CTAs)
+constexpr int kPairBN = 256;  // tokens per unit (both CTAs)
+
+template <int MODE>
+struct PairCfg {
+  static constexpr int NA = (MODE == MODE_UP) ? 2 : 1;
+  static constexpr int HALF_BN = kPairBN / 2;
+  static constexpr int A_BYTES = 128 * kBK * 2;      // this CTA's 128 weight rows
+  static constexpr int B_BYTES = HALF_BN * kBK * 2;  // this CTA's token rows
+  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = NA * kPairBN;
+  static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
+  static constexpr int TMEM_COLS = ACC_BUFS * ACC_COLS;
+  static constexpr int STAGES_RAW = (192 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation");
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC_BUFS + 1) * 8;
+  static constexpr size_t smem_bytes(int n_groups) {
+    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
+           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * kPairBN * 4 +
+           4 * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
+  }
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  using C = PairCfg<MODE>;
+  constexpr int S = C::STAGES;
+  constexpr int BN = kPairBN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA0 = smem;
+  uint8_t *sA1 = sA0 + S * C::A_BYTES;  // only used by MODE_UP
+  uint8_t *sB = sA0 + C::NA * S * C::A_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + S * C::B_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *tfull = bars + 2 * S;
+  uint64_t *tempty = bars + 2 * S + C::ACC_BUFS;
+  uint64_t *drain = bars + 2 * S + 2 * C::ACC_BUFS;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
+  int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
+  int *grp_row = grp_count + p.n_groups;                        // [G]
+  // [ACC_BUFS][BN], 16-byte aligned: read as float4
+  float *row_scale = reinterpret_cast<float *>(
+      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+  float *xbuf = row_scale + C::ACC_BUFS * BN;  // [4 warps][16][32] epilogue transposes
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int G = p.n_groups;
+  const int mtiles = p.M / kPairBM;
+  const int kblocks = p.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < C::ACC_BUFS; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmA0);
+    if (MODE == MODE_UP) {
+      tma_prefetch_desc(&p.tmA1);
+      tma_prefetch_desc(&p.tmBs);
+    }
+    tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int cnt, row;
+    if (g < p.E) {
+      row = p.offsets[g];
+      cnt = p.offsets[g + 1] - row;
+    } else {
+      row = p.Tk + (g - p.E) * p.T;
+      cnt = p.T;
+    }
+    grp_count[g] = cnt;
+    grp_row[g] = row;
+    unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of units per group (each lane a contiguous run)
+    const int per = (G + 31) / 32;
+    const int lo = min(G, lane * per), hi = min(G, lo + per);
+    int run = 0;
+    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int g = lo; g < hi; ++g) {
+      const int u = unit_prefix[g];
+      unit_prefix[g] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[G] = incl;
+  }
+  // both CTAs' barriers are initialised and TMEM allocated before any cross-CTA traffic
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = unit_prefix[G];
+
+  auto decode = [&](int u, int &g, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    g = lo;
+    const int nts = (grp_count[g] + BN - 1) / BN;
+    const int loc = u - unit_prefix[g];
+    mt = loc / nts;
+    nt = loc % nts;
+  };
+  // token split of a unit: CTA r holds tokens [n0 + r*half, n0 + (r+1)*half), N = 2*half
+  auto split = [&](int g, int nt) {
+    const int valid = min(BN, grp_count[g] - nt * BN);
+    return (((valid + 1) >> 1) + 7) & ~7;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      uint64_t pol_w_shared;
+      asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_w_shared));
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = cluster_id; u < total_units && ok; u += n_clusters) {
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const int half = split(g, nt);
+        const int a_row = g * p.M + mt * kPairBM + (int)rank * 128;
+        const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
+        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
+        const int b_row = (shared_x ? nt * BN : grp_row[g] + nt * BN) + (int)rank * half;
+        const uint64_t pw = (grp_count[g] <= BN) ? pol_w : pol_w_shared;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 11)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sA0 + stage * C::A_BYTES, &p.tmA0, fbar, kb * kBK, a_row, pw);
+          if (MODE == MODE_UP)
+            tma_load_2d_pair(sA1 + stage * C::A_BYTES, &p.tmA1, fbar, kb * kBK, a_row, pw);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, bmap, fbar, kb * kBK, b_row, pol_b);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = cluster_id; u < total_units && ok; u += n_clusters, ++it) {
+        const int acc = it % C::ACC_BUFS;
+        const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 12)) break;
+        tc_fence_after();
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const uint32_t idesc = idesc_bf16_f32(kPairBM, 2 * split(g, nt));
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, 13)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA0 + stage * C::A_BYTES);
+          const uint32_t a1 = smem_u32(sA1 + stage * C::A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t accum = (kb | kk) ? 1u : 0u;
+            const uint64_t bd = sdesc_k_sw128(b + kk * 32);
+            tc_mma_bf16_pair(d0, sdesc_k_sw128(a0 + kk * 32), bd, idesc, accum);
+            if (MODE == MODE_UP)
+              tc_mma_bf16_pair(d0 + BN, sdesc_k_sw128(a1 + kk * 32), bd, idesc, accum);
+          }
+          tc_commit_pair_both(&empty[stage]);  // slot free in both CTAs once read
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair_both(&tfull[acc]);
+      }
+      tc_commit_pair_local(drain);
+      volatile int no_abort = 0;
+      mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    int it = 0;
+    for (int u = cluster_id; u < total_units; u += n_clusters, ++it) {
+      const int acc = it % C::ACC_BUFS;
+      const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, 14)) break;
+      tc_fence_after();
+      int g, mt, nt;
+      decode(u, g, mt, nt);
+      const int valid = min(BN, grp_count[g] - nt * BN);
+      const int row0 = grp_row[g] + nt * BN;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      if (MODE == MODE_DOWN) {
+        for (int n = threadIdx.x - 64; n < BN; n += 128) {
+          float sc = 0.f;
+          if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
+          row_scale[acc * BN + n] = sc;
+        }
+        named_bar_sync(1, 128);
+      }
+      float *wbuf = xbuf + q * 16 * 32;
+      const int col_base = mt * kPairBM + (int)rank * 128 + q * 32;
+      for (int c0 = 0; c0 < valid; c0 += 16) {
+        uint32_t v0[16];
+        float vals[16];
+        tmem_ld16(taddr + c0, v0);
+        if (MODE == MODE_UP) {
+          uint32_t v1[16];
+          tmem_ld16(taddr + BN + c0, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int n = 0; n < 16; ++n)
+            vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
+          store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
+                             col_base, vals, wbuf, lane);
+        } else {
+          tmem_ld_wait();
+          const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
+#pragma unroll
+          for (int n4 = 0; n4 < 4; ++n4) {
+            const float4 s4 = sc[n4];
+            vals[4 * n4 + 0] = __uint_as_float(v0[4 * n4 + 0]) * s4.x;
+            vals[4 * n4 + 1] = __uint_as_float(v0[4 * n4 + 1]) * s4.y;
+            vals[4 * n4 + 2] = __uint_as_float(v0[4 * n4 + 2]) * s4.z;
+            vals[4 * n4 + 3] = __uint_as_float(v0[4 * n4 + 3]) * s4.w;
+          }
+          store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
+                            vals, wbuf, lane);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_leader + acc * 8);
+      }
+    }
+  }
+
+  // the pair leaves together: the leader's MMAs read the peer's shared memory, and the
+  // peer's TMA loads signal the leader's barriers
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

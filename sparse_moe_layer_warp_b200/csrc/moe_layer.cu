@@ -19,6 +19,7 @@
 #include "moe_layer.h"
 #include "expert_simt.cuh"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_pair.cuh"
 #include "ptx_sm100.cuh"
 #include "routing.cuh"
 
@@ -30,6 +31,7 @@ struct moe_layer {
   int device;
   int num_sms;
   int smem_optin;
+  int pair_grid[2];  // CTAs of the CTA-pair GEMM (up, down): 2 x co-resident clusters
   CUtensorMap tm_wg, tm_wu, tm_wd, tm_wr;
 };
 
@@ -75,22 +77,36 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // programmatic stream serialisation: its CTAs can be scheduled (and run their set-up)
 // while the previous kernel drains.
 template <typename... KArgs, typename... Args>
-moe_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                  Args &&...args) {
+moe_status launch_cl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, int cluster, Args &&...args) {
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+
+template <typename... KArgs, typename... Args>
+moe_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  Args &&...args) {
+  return launch_cl(kern, grid, block, smem, st, 1, std::forward<Args>(args)...);
 }
 
 int n_splits(const moe_config &c) { return (c.d_model + kSplitKSlice - 1) / kSplitKSlice; }
@@ -241,6 +257,59 @@ moe_status launch_gemm(const moe_layer *L, int bn, const GemmParams &p, cudaStre
   return MOE_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------------------ CTA-pair GEMM launch
+// Large expert groups (prefill) run on CTA pairs: 256 weight rows x 256 tokens per unit.
+constexpr double kPairMinMeanTokens = 96.0;
+
+bool use_pair(const moe_layer *L, int T) {
+  const moe_config &c = L->cfg;
+  const double mean = (double)T * c.top_k / c.n_experts;
+  return mean >= kPairMinMeanTokens && c.d_ff % kPairBM == 0 && c.d_model % kPairBM == 0 &&
+         L->pair_grid[0] >= 2 && L->pair_grid[1] >= 2;
+}
+
+template <int MODE>
+size_t pair_smem(const moe_config &c) {
+  return PairCfg<MODE>::smem_bytes(c.n_experts + c.n_shared);
+}
+
+// CTAs of a persistent pair-kernel grid: two per cluster that can be resident at once.
+template <int MODE>
+int pair_grid_size(const moe_layer *L) {
+  const size_t smem = pair_smem<MODE>(L->cfg);
+  if (smem > (size_t)L->smem_optin) return 0;
+  if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(L->num_sms & ~1);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<MODE>, &cfg) != cudaSuccess)
+    return 0;
+  return 2 * n;
+}
+
+template <int MODE>
+moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_t st) {
+  const size_t smem = pair_smem<MODE>(L->cfg);
+  if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = L->pair_grid[MODE == MODE_UP ? 0 : 1];
+  return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(kGemmThreads), smem, st, 2,
+                   p);
+}
+
 // Token tile of the router GEMM.
 int pick_bn_router(int T) { return T <= 256 ? 16 : (T <= 1024 ? 32 : 64); }
 
@@ -329,6 +398,9 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     return MOE_ERR_UNSUPPORTED;
   }
   if (c.dtype == MOE_BF16) {
+    L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
+    L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
+    cudaGetLastError();  // an unavailable cluster query only disables the pair path
     const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wu, w->w_up, c.d_model, G * c.d_ff, kBM) ||
@@ -457,8 +529,10 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                     c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
       return s;
     if ((s = mark(4)) != MOE_OK) return s;
-    const int bn = pick_bn(c, T, MODE_UP);
-    const int bn2 = pick_bn(c, T, MODE_DOWN);
+    const bool pair = use_pair(h, T);
+    // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
+    const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
+    const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
     __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
     float *ybuf = at<float>(ws, W.y);
     GemmParams p1;
@@ -481,7 +555,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p1.M = c.d_ff;
     p1.K = c.d_model;
     p1.ld_out = c.d_ff;
-    if ((s = launch_gemm<MODE_UP>(h, bn, p1, st)) != MOE_OK) return s;
+    if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
+        MOE_OK)
+      return s;
     if ((s = mark(5)) != MOE_OK) return s;
     GemmParams p2 = p1;
     p2.tmA0 = h->tm_wd;
@@ -490,7 +566,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p2.M = c.d_model;
     p2.K = c.d_ff;
     p2.ld_out = c.d_model;
-    if ((s = launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK) return s;
+    if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
+                  : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
+      return s;
     if ((s = mark(6)) != MOE_OK) return s;
     if ((s = launch(combine_kernel<__nv_bfloat16>,
                     dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0,

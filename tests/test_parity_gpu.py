@@ -71,6 +71,10 @@ SMALL = [
     ("tiny_fp32", {"dtype": "bf16", "T": 77, "d": 384, "E": 40, "k": 6, "f": 384, "seed": 3}),
     ("tiny_fp32", {"dtype": "bf16", "T": 513, "d": 256, "E": 8, "k": 8, "f": 128}),
     ("tiny_fp32", {"dtype": "bf16", "T": 410, "d": 512, "E": 16, "k": 8, "f": 256, "seed": 5}),
+    # large groups: the CTA-pair kernels (256 weight rows x 256 tokens per unit)
+    ("tiny_fp32", {"dtype": "bf16", "T": 700, "d": 768, "E": 8, "k": 4, "f": 512, "seed": 6}),
+    ("tiny_fp32", {"dtype": "bf16", "T": 333, "d": 256, "E": 6, "k": 2, "f": 256, "seed": 7,
+                   "n_shared": 0}),
     ("tiny_fp32", {"dtype": "bf16", "T": 200, "d": 256, "E": 48, "k": 4, "f": 128,
                    "bias": "zipf", "n_shared": 0, "routed_scale": 1.5}),
     ("tiny_fp32", {"dtype": "bf16", "T": 1, "d": 256, "E": 288, "k": 8, "f": 128}),
