@@ -144,6 +144,27 @@ moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stre
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 
+/* Router logits without any caller workspace, for callers that cannot allocate device
+ * memory: for example code that runs while a CUDA graph is being captured (a device
+ * allocation is not allowed there), plugin or embedding hosts that hand the library only its
+ * input and output buffers, and latency-critical decode loops that must not touch an
+ * allocator.  (No counterpart on the pages: this is a deployment convenience, not part of
+ * the layer's method.)
+ *
+ * Computes logits_out[t, e] = x_t . W_r[e] (fp32, [n_tokens, E], row-major) with the same
+ * split-K kernel and the same deterministic summation order as moe_route, so the values are
+ * identical to moe_route's logits.  Its scratch (split partial sums and arrival counters)
+ * lives in a fixed 2 MiB buffer inside the library's own static device memory, which every
+ * GPU that loads the library holds until the process exits.  Limits: 1 <= n_tokens <= 64 and
+ * ceil(d_model / 256) * n_tokens * E * 4 bytes <= 2 MiB (for d_model = 4096, E = 288: up to
+ * 64 tokens); larger requests return MOE_ERR_UNSUPPORTED before anything is launched.
+ * The first call on each device looks up the buffer's device address (host-side set-up), so
+ * make that first call before capturing a stream into a CUDA graph.  All calls on a device
+ * share the one buffer: calls that may overlap on the GPU (different streams without
+ * ordering) race and give wrong results; serialise them.  Asynchronous on `stream`. */
+moe_status moe_router_logits_static(moe_handle h, const void *x, int n_tokens,
+                                    float *logits_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     moe_layer_init,
     moe_route,
     moe_route_from_logits,
+    moe_router_logits_static,
     moe_workspace_init,
     moe_workspace_size,
     status_string,

@@ -28,7 +28,7 @@ MOE_BF16 = 1
 # every entry point the header declares (checked by tests against the built library)
 EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_workspace_init",
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
-           "moe_device_status", "moe_status_string")
+           "moe_device_status", "moe_status_string", "moe_router_logits_static")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -76,11 +76,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_forward.argtypes = [P, P, I, P, P, Z, P]
         lib.moe_forward_profiled.argtypes = [P, P, I, P, P, Z, P, ctypes.POINTER(P), I]
         lib.moe_device_status.argtypes = [P, P, Z, P]
+        lib.moe_router_logits_static.argtypes = [P, P, I, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
-                     "moe_device_status"):
+                     "moe_device_status", "moe_router_logits_static"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -159,6 +160,13 @@ def moe_forward_profiled(handle, x, n_tokens, out, ws, events, stream=None) -> N
     _check("moe_forward_profiled", load_library().moe_forward_profiled(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream), arr, len(events)))
+
+
+def moe_router_logits_static(handle, x, n_tokens, logits_out, stream=None) -> None:
+    """Router logits with the library's own static scratch (no workspace argument), for
+    callers that cannot allocate device memory; see include/moe_layer.h for the limits."""
+    _check("moe_router_logits_static", load_library().moe_router_logits_static(
+        handle, _p(x), int(n_tokens), _p(logits_out), _stream(stream)))
 
 
 def moe_device_status(handle, ws, stream=None) -> int:

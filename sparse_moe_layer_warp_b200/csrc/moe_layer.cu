@@ -14,6 +14,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <utility>
 
 #include "moe_layer.h"
@@ -618,3 +619,59 @@ moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void 
 }
 
 }  // extern "C"
+
+// ================================================== router logits with library-held scratch
+// For callers that cannot allocate device memory (see moe_router_logits_static in the
+// header): the split-K router's scratch -- partial sums [splits][T][E] and the per-expert-
+// block arrival counters -- lives in this file-scope device array instead of a caller
+// workspace.  In host code the array's name is only a host-side stand-in, so the device
+// address is looked up once per device with cudaGetSymbolAddress and passed to the kernel.
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(2) << 20;  // partial sums
+constexpr int kStaticTickets = 32;                        // one per block of 32 experts
+constexpr int kMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_router_scratch[kStaticScratchBytes +
+                                                                 kStaticTickets * 4];
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices];  // device address of g_router_scratch per device
+}  // namespace
+
+extern "C" moe_status moe_router_logits_static(moe_handle h, const void *x, int n_tokens,
+                                               float *logits_out, void *stream) {
+  if (!h || !x || !logits_out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(logits_out)) return MOE_ERR_ALIGNMENT;
+  const moe_config &c = h->cfg;
+  if (n_tokens < 1 || n_tokens > c.max_tokens) return MOE_ERR_INVALID_ARG;
+  const int S = n_splits(c);
+  if (n_tokens > kSplitKTokens || (c.n_experts + 31) / 32 > kStaticTickets ||
+      (size_t)S * n_tokens * c.n_experts * 4 > kStaticScratchBytes)
+    return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch size
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  void *base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      void *ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_router_scratch) != cudaSuccess || !ptr)
+        return MOE_ERR_CUDA;
+      g_static_ptr[dev] = ptr;
+    }
+    base = g_static_ptr[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *part = static_cast<float *>(base);
+  int *tickets = reinterpret_cast<int *>(static_cast<char *>(base) + kStaticScratchBytes);
+  // the counters must start at zero; the buffer keeps whatever the previous call left
+  if (cudaMemsetAsync(tickets, 0, kStaticTickets * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  dim3 grid((c.n_experts + 31) / 32, S);
+  if (c.dtype == MOE_BF16)
+    return launch(router_logits_splitk_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                  static_cast<const __nv_bfloat16 *>(x),
+                  static_cast<const __nv_bfloat16 *>(h->w.w_router), n_tokens, c.d_model,
+                  c.n_experts, part, logits_out, tickets);
+  return launch(router_logits_splitk_kernel<float>, grid, dim3(256), 0, st,
+                static_cast<const float *>(x), static_cast<const float *>(h->w.w_router),
+                n_tokens, c.d_model, c.n_experts, part, logits_out, tickets);
+}
+

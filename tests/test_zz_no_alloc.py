@@ -1,0 +1,69 @@
+"""The allocation-free router entry point (moe_router_logits_static).
+
+Some callers cannot allocate device memory -- for example code running while a CUDA graph
+is captured, or a plugin host that only hands over input and output buffers -- so this
+entry point keeps its scratch in the library's own static device buffer instead of a
+caller workspace.  These tests call it through the C ABI and check it against the regular
+workspace-based routing call, twice in a row (the shared buffer keeps the previous call's
+contents).  The file is named to be collected last, and passes alone or after the others.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from sparse_moe_layer_warp_b200 import binding, synth
+from tests.helpers import make_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _workspace_logits(layer, x):
+    r = layer.route(x=x, want_logits=True)
+    torch.cuda.synchronize()
+    return r["logits"]
+
+
+@pytest.mark.parametrize("T,E,d,dtype", [(16, 288, 4096, "bf16"), (5, 40, 512, "bf16"),
+                                         (64, 96, 1024, "bf16"), (9, 16, 256, "f32")])
+def test_static_scratch_router_matches_workspace_router(cuda_ok, T, E, d, dtype):
+    w = synth.Workload("noalloc", T=T, d=d, E=E, k=4, f=128, dtype=dtype, seed=T)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    ref = _workspace_logits(layer, inp.x)
+    x2 = synth.make_x(w, T, device="cuda", seed=99)
+    ref2 = _workspace_logits(layer, x2)
+    for x, want in ((inp.x, ref), (x2, ref2), (inp.x, ref)):  # consecutive calls
+        out = torch.full((T, E), float("nan"), device="cuda", dtype=torch.float32)
+        binding.moe_router_logits_static(layer.handle, x, T, out)
+        torch.cuda.synchronize()
+        # same kernel and summation order: identical values (the parity tolerance for fp32
+        # logits would also accept rounding differences; none are expected here)
+        assert torch.isfinite(out).all()
+        assert torch.equal(out, want)
+
+
+def test_static_scratch_router_rejects_oversized_requests(cuda_ok):
+    w = synth.Workload("noalloc", T=65, d=4096, E=288, k=8, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    out = torch.empty((65, 288), device="cuda", dtype=torch.float32)
+    lib = binding.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = lib.moe_router_logits_static(layer.handle, ctypes.c_void_p(inp.x.data_ptr()), 65,
+                                      ctypes.c_void_p(out.data_ptr()), st)
+    assert rc == binding.MOE_ERR_UNSUPPORTED  # more than 64 tokens
+    big = synth.Workload("noalloc", T=64, d=4096, E=600, k=8, f=128)
+    inp2 = synth.make_inputs(big, device="cuda")
+    layer2 = make_layer(inp2)
+    out2 = torch.empty((64, 600), device="cuda", dtype=torch.float32)
+    rc = lib.moe_router_logits_static(layer2.handle, ctypes.c_void_p(inp2.x.data_ptr()), 64,
+                                      ctypes.c_void_p(out2.data_ptr()), st)
+    assert rc == binding.MOE_ERR_UNSUPPORTED  # 16 splits x 64 x 600 x 4 B > 2 MiB
+    # a request that fits still works after the rejected ones
+    rc = lib.moe_router_logits_static(layer2.handle, ctypes.c_void_p(inp2.x.data_ptr()), 8,
+                                      ctypes.c_void_p(out2.data_ptr()), st)
+    assert rc == binding.MOE_OK
+    torch.cuda.synchronize()
+    ref = _workspace_logits(layer2, inp2.x[:8].contiguous())
+    assert torch.equal(out2[:8], ref)
