@@ -21,4 +21,6 @@ from .c_oracle import (  # noqa: F401
     oracle_expert_ffn,
     oracle_moe_forward,
     oracle_num_threads,
+    oracle_router_stats,
+    oracle_bias_update,
 )

@@ -43,6 +43,8 @@ def _load():
         lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
                                            ctypes.c_double, P, I, P, P, P, P, P]
         lib.oracle_num_threads.restype = I
+        lib.oracle_router_stats.argtypes = [P, P, I, I, I, I, P, P, P, P]
+        lib.oracle_bias_update.argtypes = [P, I, I, ctypes.c_float, P]
         _lib = lib
     return _lib
 
@@ -138,3 +140,25 @@ def oracle_moe_forward(x, w_r, bias, w_gate, w_up, w_down, k, n_shared=1, routed
                                _ptr(tokens), n, _ptr(logits_in), _ptr(out), _ptr(idx),
                                _ptr(gates), _ptr(logits))
     return out, idx, gates, logits
+
+
+def oracle_router_stats(logits, idx, n_groups):
+    """p_mean [E], f_sel [E], L_EP, routing confidence (see moe_oracle.c)."""
+    logits = np.ascontiguousarray(logits, np.float32)
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, E = logits.shape
+    k = idx.shape[1]
+    p_mean = np.empty(E, np.float32)
+    f_sel = np.empty(E, np.float32)
+    l_ep = np.empty(1, np.float32)
+    conf = np.empty(1, np.float32)
+    _load().oracle_router_stats(_ptr(logits), _ptr(idx), T, E, k, int(n_groups), _ptr(p_mean),
+                                _ptr(f_sel), _ptr(l_ep), _ptr(conf))
+    return p_mean, f_sel, float(l_ep[0]), float(conf[0])
+
+
+def oracle_bias_update(counts, Tk, gamma, bias):
+    counts = np.ascontiguousarray(counts, np.int32)
+    out = np.array(bias, np.float32, copy=True)
+    _load().oracle_bias_update(_ptr(counts), len(counts), int(Tk), float(gamma), _ptr(out))
+    return out

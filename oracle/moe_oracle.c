@@ -252,3 +252,73 @@ int oracle_num_threads(void) { return omp_get_max_threads(); }
 #else
 int oracle_num_threads(void) { return 1; }
 #endif
+
+/* ------------------------------------------------------------------------------------ */
+/* Router statistics, [P2 2.2.2] (EP-group balance loss) and [P2 5.2.3] (routing          */
+/* confidence, called Sigma_k there):                                                      */
+/*   p[t,e]   = softmax over all E unbiased logits of token t (the routing probability)    */
+/*   p_e      = (1/T) sum_t p[t,e]            f_e = (1/(T k)) sum_t s[t,e]                 */
+/*   p_g, f_g = sums over the experts of group g (G contiguous groups of E/G experts)      */
+/*   L_EP     = G sum_g f_g p_g                                                            */
+/*   conf     = (1/T) sum_t sum_{e in S_t} p[t,e]                                          */
+/* Everything in double, rounded once to fp32 at the end.                                  */
+void oracle_router_stats(const float *logits, const int *idx, int T, int E, int k, int G,
+                         float *p_mean, float *f_sel, float *l_ep, float *conf) {
+  double *pm = (double *)calloc((size_t)E, sizeof(double));
+  double *fs = (double *)calloc((size_t)E, sizeof(double));
+  double *p = (double *)malloc(sizeof(double) * (size_t)E);
+  double cf = 0.0;
+  for (int t = 0; t < T; ++t) {
+    const float *l = logits + (size_t)t * E;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e)
+      if ((double)l[e] > m) m = (double)l[e];
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) {
+      p[e] = exp((double)l[e] - m);
+      z += p[e];
+    }
+    for (int e = 0; e < E; ++e) {
+      p[e] /= z;
+      pm[e] += p[e];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      fs[e] += 1.0;
+      cf += p[e];
+    }
+  }
+  const int per = E / G;
+  double loss = 0.0;
+  for (int g = 0; g < G; ++g) {
+    double pg = 0.0, fg = 0.0;
+    for (int e = g * per; e < (g + 1) * per; ++e) {
+      pg += pm[e] / T;
+      fg += fs[e] / ((double)T * k);
+    }
+    loss += fg * pg;
+  }
+  for (int e = 0; e < E; ++e) {
+    p_mean[e] = (float)(pm[e] / T);
+    f_sel[e] = (float)(fs[e] / ((double)T * k));
+  }
+  *l_ep = (float)(G * loss);
+  *conf = (float)(cf / T);
+  free(p);
+  free(fs);
+  free(pm);
+}
+
+/* Loss-free balancing bias step ([P3 MoE] note: balance by adjusting a per-expert bias, no
+ * auxiliary loss).  The pages give no update rule; this library's reading is the plain sign
+ * step toward the mean load:  b_e <- b_e + gamma * sign(T k / E - counts[e])  (sign(0) = 0),
+ * computed in fp32 like the bias itself.  PARITY UNPINNED against the pages (no rule there);
+ * pinned only by the closed forms in the tests. */
+void oracle_bias_update(const int *counts, int E, int Tk, float gamma, float *bias) {
+  const float mean = (float)Tk / (float)E;
+  for (int e = 0; e < E; ++e) {
+    const float gap = mean - (float)counts[e];
+    const float s = (gap > 0.f) ? 1.f : ((gap < 0.f) ? -1.f : 0.f);
+    bias[e] = bias[e] + gamma * s;
+  }
+}

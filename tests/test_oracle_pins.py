@@ -213,3 +213,56 @@ def test_sampled_tokens_equal_full_run():
     part, idx2, gates2, _ = oracle_moe_forward(x, wr, b, wg, wu, wd, k=w.k, tokens=toks)
     np.testing.assert_array_equal(part, full[toks])
     np.testing.assert_array_equal(idx2, idx[toks])
+
+
+# ------------------------------------------------------------------- router statistics
+from oracle import oracle_bias_update, oracle_router_stats  # noqa: E402
+
+
+def test_router_stats_closed_forms():
+    T, E, k = 48, 12, 3
+    # equal logits -> p = 1/E; a balanced selection (each expert chosen T*k/E times) -> L_EP = 1
+    logits = np.zeros((T, E), np.float32)
+    idx = np.array([[(3 * t + j) % E for j in range(k)] for t in range(T)], np.int32)
+    for G in (1, 2, 3, 4, 6, 12):
+        pm, fs, lep, conf = oracle_router_stats(logits, idx, G)
+        np.testing.assert_allclose(pm, 1.0 / E, rtol=1e-6)
+        np.testing.assert_allclose(fs, 1.0 / E, rtol=1e-6)
+        assert abs(lep - 1.0) < 1e-6
+        assert abs(conf - k / E) < 1e-6
+    # all mass and all selections inside group 0 of G groups -> L_EP = G
+    G = 4
+    logits2 = np.full((T, E), -60.0, np.float32)
+    logits2[:, :3] = 5.0
+    idx2 = np.tile(np.arange(3, dtype=np.int32), (T, 1))
+    _, _, lep2, conf2 = oracle_router_stats(logits2, idx2, G)
+    assert abs(lep2 - G) < 1e-5
+    assert abs(conf2 - 1.0) < 1e-5
+    # G = 1: L_EP = (sum f)(sum p) = 1 for any routing
+    lg = synth.make_logits(T, E, seed=4).numpy()
+    ix, _ = oracle_route(lg, None, k)
+    assert abs(oracle_router_stats(lg, ix, 1)[2] - 1.0) < 1e-6
+    # k = E: every expert is active, confidence = 1
+    ixe, _ = oracle_route(lg, None, E)
+    assert abs(oracle_router_stats(lg, ixe, 3)[3] - 1.0) < 1e-6
+
+
+def test_router_stats_match_library_softmax_and_bincount():
+    lg = synth.make_logits(70, 40, seed=8).numpy()
+    ix, _ = oracle_route(lg, np.linspace(-0.3, 0.3, 40).astype(np.float32), 5)
+    pm, fs, lep, conf = oracle_router_stats(lg, ix, 8)
+    P = torch.softmax(torch.from_numpy(lg).double(), dim=1).numpy()
+    np.testing.assert_allclose(pm, P.mean(0), rtol=1e-6)
+    np.testing.assert_allclose(fs, np.bincount(ix.reshape(-1), minlength=40) / (70 * 5), rtol=1e-6)
+    pg = P.mean(0).reshape(8, 5).sum(1)
+    fg = (np.bincount(ix.reshape(-1), minlength=40) / (70 * 5)).reshape(8, 5).sum(1)
+    assert abs(lep - 8 * float((pg * fg).sum())) < 1e-6
+    assert abs(conf - float(np.take_along_axis(P, ix.astype(np.int64), 1).sum(1).mean())) < 1e-6
+
+
+def test_bias_update_sign_rule():
+    counts = np.array([10, 2, 6, 6], np.int32)  # T*k = 24, mean 6
+    b = oracle_bias_update(counts, 24, 0.5, np.zeros(4, np.float32))
+    assert b.tolist() == [-0.5, 0.5, 0.0, 0.0]
+    b2 = oracle_bias_update(counts, 24, 0.25, b)
+    assert b2.tolist() == [-0.75, 0.75, 0.0, 0.0]

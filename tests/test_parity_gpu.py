@@ -124,7 +124,8 @@ def test_forward_rejects_too_many_tokens(cuda_ok):
 
 
 # ------------------------------------------------------------ full-size workloads (sampled)
-FULL = [("decode_t16", None), ("decode_t256", 24), ("skew_t4096", 12), ("prefill_t8192", 12)]
+FULL = [("decode_t16", None), ("decode_t256", 24), ("skew_t4096", 12), ("prefill_t8192", 12),
+        ("dense_ffn_t4096", 8)]
 
 
 @pytest.mark.slow
