@@ -141,6 +141,29 @@ moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void 
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
 
+/* Balancing statistics of a routing result ("Step 3.5 Flash: Open Frontier-Level
+ * Intelligence with 11B Active Parameters", section 2.2.2: EP-group balance loss; section
+ * 5.2.3: routing confidence).  From fp32 logits [n_tokens, E] and topk_idx [n_tokens, k]
+ * (the outputs of moe_route):
+ *   p[t,e]     = softmax of token t's E unbiased logits (its routing probability)
+ *   p_mean[e]  = mean_t p[t,e]                       [E] fp32, device
+ *   f_sel[e]   = (selections of e) / (n_tokens * k)  [E] fp32, device
+ *   scalars[0] = L_EP = G * sum_g f_g * p_g, where f_g, p_g sum f_sel, p_mean over group g
+ *                of n_groups groups of E / n_groups consecutive experts (E % n_groups == 0)
+ *   scalars[1] = routing confidence = mean_t sum_{e in S_t} p[t,e]
+ * Deterministic; uses the workspace of moe_workspace_size(h, n_tokens). */
+moe_status moe_router_stats(moe_handle h, const float *logits, const int *topk_idx,
+                            int n_tokens, int n_groups, float *p_mean, float *f_sel,
+                            float *scalars, void *ws, size_t ws_bytes, void *stream);
+
+/* Loss-free balancing step on a bias vector (fp32 [E], device, updated in place) from the
+ * expert_counts of a routing over n_tokens tokens: bias[e] += gamma * sign(n_tokens * k / E -
+ * counts[e]) with sign(0) = 0.  The pages balance by adjusting this bias instead of an
+ * auxiliary loss ("Step 3.5 Flash 技术论文深度解读", architecture item 1) but give no rule;
+ * this sign step toward the mean load is the library's reading. */
+moe_status moe_update_router_bias(moe_handle h, const int *expert_counts, int n_tokens,
+                                  float gamma, float *bias, void *stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 

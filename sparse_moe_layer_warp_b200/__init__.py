@@ -21,6 +21,8 @@ from .binding import (  # noqa: F401
     moe_route,
     moe_route_from_logits,
     moe_router_logits_static,
+    moe_router_stats,
+    moe_update_router_bias,
     moe_workspace_init,
     moe_workspace_size,
     status_string,

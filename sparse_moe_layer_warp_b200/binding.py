@@ -28,7 +28,8 @@ MOE_BF16 = 1
 # every entry point the header declares (checked by tests against the built library)
 EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_workspace_init",
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
-           "moe_device_status", "moe_status_string", "moe_router_logits_static")
+           "moe_device_status", "moe_status_string", "moe_router_logits_static",
+           "moe_router_stats", "moe_update_router_bias")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -77,11 +78,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_forward_profiled.argtypes = [P, P, I, P, P, Z, P, ctypes.POINTER(P), I]
         lib.moe_device_status.argtypes = [P, P, Z, P]
         lib.moe_router_logits_static.argtypes = [P, P, I, P, P]
+        lib.moe_router_stats.argtypes = [P, P, P, I, I, P, P, P, P, Z, P]
+        lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
-                     "moe_device_status", "moe_router_logits_static"):
+                     "moe_device_status", "moe_router_logits_static", "moe_router_stats",
+                     "moe_update_router_bias"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -169,6 +173,18 @@ def moe_router_logits_static(handle, x, n_tokens, logits_out, stream=None) -> No
         handle, _p(x), int(n_tokens), _p(logits_out), _stream(stream)))
 
 
+def moe_router_stats(handle, logits, topk_idx, n_tokens, n_groups, p_mean, f_sel, scalars, ws,
+                     stream=None) -> None:
+    _check("moe_router_stats", load_library().moe_router_stats(
+        handle, _p(logits), _p(topk_idx), int(n_tokens), int(n_groups), _p(p_mean), _p(f_sel),
+        _p(scalars), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_update_router_bias(handle, expert_counts, n_tokens, gamma, bias, stream=None) -> None:
+    _check("moe_update_router_bias", load_library().moe_update_router_bias(
+        handle, _p(expert_counts), int(n_tokens), float(gamma), _p(bias), _stream(stream)))
+
+
 def moe_device_status(handle, ws, stream=None) -> int:
     return int(load_library().moe_device_status(handle, _p(ws), ws.numel() * ws.element_size(),
                                                  _stream(stream)))
@@ -225,6 +241,16 @@ class MoELayer:
             if lg is not None:
                 r["logits"] = lg
         return r
+
+    def router_stats(self, logits, topk_idx, n_groups, stream=None):
+        """p_mean [E], f_sel [E] and scalars [L_EP, routing confidence] (device tensors)."""
+        T = logits.shape[0]
+        p_mean = torch.empty(self.E, dtype=torch.float32, device=self.device)
+        f_sel = torch.empty(self.E, dtype=torch.float32, device=self.device)
+        scalars = torch.empty(2, dtype=torch.float32, device=self.device)
+        moe_router_stats(self.handle, logits, topk_idx, T, n_groups, p_mean, f_sel, scalars,
+                         self.workspace(T), stream)
+        return p_mean, f_sel, scalars
 
     def device_status(self, stream=None) -> int:
         return moe_device_status(self.handle, self.ws, stream)

@@ -22,6 +22,7 @@
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "ptx_sm100.cuh"
+#include "router_stats.cuh"
 #include "routing.cuh"
 
 using namespace moe;
@@ -116,8 +117,8 @@ size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 
 // Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
 struct WsLayout {
-  size_t status, logits, part, idx, gate, counts, offsets, perm, slot_row, chunk_hist, xs, h,
-      y, total;
+  size_t status, logits, part, idx, gate, counts, offsets, perm, slot_row, chunk_hist, stats,
+      xs, h, y, total;
 };
 
 WsLayout ws_layout(const moe_config &c, int T) {
@@ -141,6 +142,7 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.perm = take(Tk * 4);
   L.slot_row = take(Tk * 4);
   L.chunk_hist = take(nch * c.n_experts * 4);
+  L.stats = take(nch * (2 * (size_t)c.n_experts + 1) * 4);  // router statistics partials
   L.xs = (c.dtype == MOE_BF16) ? take(Tk * c.d_model * 2) : off;
   L.h = take(P * c.d_ff * esize(c));
   L.y = take(P * c.d_model * 4);  // fp32 in both precisions
@@ -176,7 +178,7 @@ int pick_bn(const moe_config &c, int T, int mode) {
 
 // ------------------------------------------------------------------ routing launches
 moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
-                              cudaStream_t st);
+                              DevStatus *status, cudaStream_t st);
 
 // Router logits [T][E] into `logits`; for small T the split-K partials go to `part`.
 moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits, float *part,
@@ -193,7 +195,7 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
                   static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
                   c.d_model, c.n_experts, part, logits, status->router_ticket);
   }
-  if (c.dtype == MOE_BF16) return launch_gemm_logits(L, x, T, logits, st);
+  if (c.dtype == MOE_BF16) return launch_gemm_logits(L, x, T, logits, status, st);
   dim3 grid((T + 63) / 64, (c.n_experts + 63) / 64);
   return launch(router_logits_tiled_kernel<float>, grid, dim3(256), 0, st,
                 static_cast<const float *>(x), static_cast<const float *>(L->w.w_router), T,
@@ -315,7 +317,7 @@ moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_
 int pick_bn_router(int T) { return T <= 256 ? 16 : (T <= 1024 ? 32 : 64); }
 
 moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
-                              cudaStream_t st) {
+                              DevStatus *status, cudaStream_t st) {
   const moe_config &c = L->cfg;
   const int bn = pick_bn_router(T);
   GemmParams p;
@@ -323,6 +325,7 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
   p.tmA0 = L->tm_wr;
   if (!encode_bf16_2d(&p.tmB, x, c.d_model, T, bn)) return MOE_ERR_CUDA;
   p.out = logits;
+  p.status = status;
   p.E = 0;  // one group: all T tokens, rows [0, T)
   p.n_groups = 1;
   p.T = T;
@@ -616,6 +619,51 @@ moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void 
   for (int i = 0; i <= MOE_PROFILE_STAGES; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARG;
   return forward_impl(h, x, n_tokens, out, ws, ws_bytes, stream, events);
+}
+
+moe_status moe_router_stats(moe_handle h, const float *logits, const int *topk_idx,
+                            int n_tokens, int n_groups, float *p_mean, float *f_sel,
+                            float *scalars, void *ws, size_t ws_bytes, void *stream) {
+  moe_status s = check_call(h, n_tokens, ws, ws_bytes);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0 || !logits || !topk_idx || !p_mean || !f_sel || !scalars)
+    return MOE_ERR_INVALID_ARG;
+  const moe_config &c = h->cfg;
+  if (n_groups < 1 || c.n_experts % n_groups != 0) return MOE_ERR_INVALID_ARG;
+  const WsLayout W = ws_layout(c, n_tokens);
+  const int nch = (n_tokens + kChunk - 1) / kChunk;
+  float *part_p = at<float>(ws, W.stats);
+  int *part_cnt = reinterpret_cast<int *>(part_p + (size_t)nch * c.n_experts);
+  float *part_conf = reinterpret_cast<float *>(part_cnt + (size_t)nch * c.n_experts);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t)kStatWarps * c.n_experts * 4;
+  const int need = (c.n_experts + 31) / 32;
+#define MOE_STATS(V)                                                                        \
+  (cudaFuncSetAttribute(router_stats_partial_kernel<V>,                                     \
+                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess \
+       ? MOE_ERR_CUDA                                                                       \
+       : launch(router_stats_partial_kernel<V>, dim3(nch), dim3(kStatWarps * 32), smem, st,  \
+                logits, topk_idx, n_tokens, c.n_experts, c.top_k, part_p, part_cnt, part_conf))
+  if (need <= 1) s = MOE_STATS(1);
+  else if (need <= 2) s = MOE_STATS(2);
+  else if (need <= 4) s = MOE_STATS(4);
+  else if (need <= 9) s = MOE_STATS(9);
+  else if (need <= 16) s = MOE_STATS(16);
+  else s = MOE_STATS(32);
+#undef MOE_STATS
+  if (s != MOE_OK) return s;
+  return launch(router_stats_final_kernel, dim3(1), dim3(256), 0, st, (const float *)part_p,
+                (const int *)part_cnt, (const float *)part_conf, nch, n_tokens, c.n_experts,
+                c.top_k, n_groups, p_mean, f_sel, scalars);
+}
+
+moe_status moe_update_router_bias(moe_handle h, const int *expert_counts, int n_tokens,
+                                  float gamma, float *bias, void *stream) {
+  if (!h || !expert_counts || !bias || n_tokens < 0) return MOE_ERR_INVALID_ARG;
+  const moe_config &c = h->cfg;
+  return launch(bias_update_kernel, dim3((c.n_experts + 255) / 256), dim3(256), 0,
+                static_cast<cudaStream_t>(stream), expert_counts, c.n_experts,
+                n_tokens * c.top_k, gamma, bias);
 }
 
 }  // extern "C"
