@@ -57,7 +57,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.gpu)],
+                 "-lms", "20", "-i", str(self.gpu)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
@@ -138,6 +138,25 @@ def ncu_traffic(kernel: str, workload: str):
     return ent.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------------------ multi-rank
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes, every rank gets the max."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time (weak scaling:
+    every replica runs the same per-GPU workload)."""
+    return world * steps * tokens_per_rank_step / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------------ our arm
 def run_ours(args, rank, world, local_rank):
     import numpy as np
@@ -204,12 +223,8 @@ def run_ours(args, rank, world, local_rank):
     stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(MOE_PROFILE_STAGES)]
                          for i in range(args.steps)])
     step_ms = np.array([ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)])
-    total_ms = float(step_ms.sum())
+    total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
     profiled_ms = float(np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]).mean())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     status = layer.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -233,11 +248,8 @@ def run_ours(args, rank, world, local_rank):
         hout.copy_(out, non_blocking=True)
     e1.record(st)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank != 0:
@@ -270,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
     layer_bytes = float(np.mean([a["layer_bytes"] for a in algo]))
     layer_flops = float(np.mean([a["layer_flops"] for a in algo]))
     step_s = total_ms / args.steps / 1e3
-    value = world * args.steps * T / (total_ms / 1e3)
+    value = job_throughput(T, args.steps, world, total_ms)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
@@ -287,7 +299,7 @@ def run_ours(args, rank, world, local_rank):
                            "touched_experts_mean": float(np.mean([a["touched"] for a in algo]))},
         "stages_ms": {n: round(float(v), 4) for n, v in zip(names, mean_stage)},
         "profiled_ms_per_step": round(profiled_ms, 4),
-        "e2e": {"value": round(world * args.steps * T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4)),
                 "d2h_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4))},
         "gpu_launches": int(world * args.steps * (7 if w.dtype == "bf16" else 6)),
@@ -326,7 +338,7 @@ def cpu_baseline(w, inp, x_batch, budget_s=15.0, host=None):
         done += n
         start += n
         el = time.perf_counter() - t0
-        if el >= budget_s or done >= 4 * x.shape[0]:
+        if el >= budget_s:
             break
     return {"value": round(done / el, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{done} tokens of one {w.name} batch ({el:.1f} s of plain-C fp64 oracle, "
@@ -381,7 +393,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -194,8 +194,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  // everything above overlaps the previous kernel's tail; what follows reads its outputs
-  griddep_wait();
+  // Programmatic dependent launch: this CTA may start while the previous kernel drains.
+  // The expert offsets read below come from the routing kernels, which finished before the
+  // previous kernel passed its own wait; the B operand (the previous kernel's output) is
+  // loaded only after the producer's griddep_wait; weights never depend on earlier kernels.
   griddep_launch_dependents();
   // group table: token count, first row in the sorted space, units per group
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -284,27 +286,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
+      auto load_a = [&](const Slot &c, int st) {
+        const int kc = c.kb * kBK;
+        if (c.single_use) {
+          tma_load_2d_hint(sA0 + st * C::A_BYTES, &p.tmA0, &full[st], kc, c.a_row, pol_w);
+          if (MODE == MODE_UP)
+            tma_load_2d_hint(sA1 + st * C::A_BYTES, &p.tmA1, &full[st], kc, c.a_row, pol_w);
+        } else {
+          tma_load_2d(sA0 + st * C::A_BYTES, &p.tmA0, &full[st], kc, c.a_row);
+          if (MODE == MODE_UP) tma_load_2d(sA1 + st * C::A_BYTES, &p.tmA1, &full[st], kc, c.a_row);
+        }
+      };
+      auto load_b = [&](const Slot &c, int st) {
+        tma_load_2d_hint(sB + st * C::B_BYTES, c.shared_x ? &p.tmBs : &p.tmB, &full[st],
+                         c.kb * kBK, c.b_row, pol_b);
+      };
       Slot ld{(int)blockIdx.x, 0, 0, 0, false, false};
       if (ld.u < total_units) slot_set_unit(ld);
+      // weight tiles of the first S slots go out before the wait for the previous kernel;
+      // their token rows follow once its output is complete
+      Slot pre = ld;
+      int npre = 0;
+      while (npre < S && ld.u < total_units) {
+        mbar_arrive_expect_tx(&full[npre], C::STAGE_BYTES);  // ring slots start empty
+        load_a(ld, npre);
+        ++npre;
+        slot_next(ld);
+      }
+      griddep_wait();
+      for (int i = 0; i < npre; ++i) {
+        load_b(pre, i);
+        slot_next(pre);
+      }
+      issued = npre;
+      stage = npre % S;
+      phase = (npre == S) ? 1u : 0u;
       while (ld.u < total_units) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
           ok = false;
           break;
         }
-        const CUtensorMap *bmap = ld.shared_x ? &p.tmBs : &p.tmB;
-        const int kc = ld.kb * kBK;
         mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-        if (ld.single_use) {
-          tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, ld.a_row, pol_w);
-          if (MODE == MODE_UP)
-            tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, ld.a_row,
-                             pol_w);
-        } else {
-          tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, ld.a_row);
-          if (MODE == MODE_UP)
-            tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, ld.a_row);
-        }
-        tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kc, ld.b_row, pol_b);
+        load_a(ld, stage);
+        load_b(ld, stage);
         ++issued;
         if (++stage == S) {
           stage = 0;

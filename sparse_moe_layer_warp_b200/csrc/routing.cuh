@@ -64,7 +64,6 @@ template <typename Tin>
 __global__ void __launch_bounds__(256) router_logits_splitk_kernel(
     const Tin *__restrict__ x, const Tin *__restrict__ wr, int T, int d, int E,
     float *__restrict__ part, float *__restrict__ logits, int *__restrict__ tickets) {
-  griddep_wait();
   griddep_launch_dependents();
   constexpr int V = Vec16<Tin>::N;      // elements per 16-byte load
   constexpr int PER_LANE = 8;           // elements per lane per split
@@ -90,6 +89,8 @@ __global__ void __launch_bounds__(256) router_logits_splitk_kernel(
       for (int v = 0; v < V; ++v) w[i][v0 + v] = tmp[v];
     }
   }
+  // the router weights above never depend on earlier kernels; x and the workspace do
+  griddep_wait();
   for (int tg = 0; tg < T; tg += TG) {
     float acc[4][TG];
 #pragma unroll

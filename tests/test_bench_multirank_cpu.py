@@ -1,0 +1,46 @@
+"""bench.py's multi-rank plumbing on CPU (gloo, world size 2): the slowest rank's time is
+what every rank reports, and whole-job throughput counts every replica's tokens.  The layer
+itself runs on one GPU per rank with no data-path collective ("replicas only"), so the
+timing reduction is the only cross-rank step."""
+import os
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = 10.0 + 5.0 * rank  # rank 1 is the slow one
+        got = bench.max_over_ranks(mine, world, torch.device("cpu"))
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res == {0: 15.0, 1: 15.0}
+
+
+def test_single_rank_and_throughput():
+    assert bench.max_over_ranks(3.5, 1, None) == 3.5
+    # 2 replicas x 100 steps x 16 tokens in 50 ms
+    assert bench.job_throughput(16, 100, 2, 50.0) == pytest.approx(64000.0)
