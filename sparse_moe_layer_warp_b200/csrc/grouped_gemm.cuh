@@ -194,10 +194,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  // Programmatic dependent launch: this CTA may start while the previous kernel drains.
-  // The expert offsets read below come from the routing kernels, which finished before the
-  // previous kernel passed its own wait; the B operand (the previous kernel's output) is
-  // loaded only after the producer's griddep_wait; weights never depend on earlier kernels.
+  // Programmatic dependent launch: the set-up above overlaps the previous kernel's tail;
+  // the expert offsets, the token rows and the outputs may all belong to it, so everything
+  // below waits for it to complete.
+  griddep_wait();
   griddep_launch_dependents();
   // group table: token count, first row in the sorted space, units per group
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -303,24 +303,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       };
       Slot ld{(int)blockIdx.x, 0, 0, 0, false, false};
       if (ld.u < total_units) slot_set_unit(ld);
-      // weight tiles of the first S slots go out before the wait for the previous kernel;
-      // their token rows follow once its output is complete
-      Slot pre = ld;
-      int npre = 0;
-      while (npre < S && ld.u < total_units) {
-        mbar_arrive_expect_tx(&full[npre], C::STAGE_BYTES);  // ring slots start empty
-        load_a(ld, npre);
-        ++npre;
-        slot_next(ld);
-      }
-      griddep_wait();
-      for (int i = 0; i < npre; ++i) {
-        load_b(pre, i);
-        slot_next(pre);
-      }
-      issued = npre;
-      stage = npre % S;
-      phase = (npre == S) ? 1u : 0u;
       while (ld.u < total_units) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
           ok = false;

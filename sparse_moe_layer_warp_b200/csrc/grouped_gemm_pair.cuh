@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-  // programmatic dependent launch: see grouped_gemm_kernel (weights first, B after the wait)
+  // programmatic dependent launch: everything below may read the previous kernel's output
+  griddep_wait();
   griddep_launch_dependents();
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
     int cnt, row;
@@ -181,7 +182,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      bool waited = false;  // griddep_wait done (before the first token-row load)
       for (int u = cluster_id; u < total_units && ok; u += n_clusters) {
         int g, mt, nt;
         decode(u, g, mt, nt);
@@ -191,7 +191,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
         const int b_row = (shared_x ? nt * BN : grp_row[g] + nt * BN) + (int)rank * half;
         const uint64_t pw = (grp_count[g] <= BN) ? pol_w : pol_w_shared;
-        int kb_b = 0;  // next k-block whose token rows are still to be loaded
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 11)) {
             ok = false;
@@ -202,27 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_pair(sA0 + stage * C::A_BYTES, &p.tmA0, fbar, kb * kBK, a_row, pw);
           if (MODE == MODE_UP)
             tma_load_2d_pair(sA1 + stage * C::A_BYTES, &p.tmA1, fbar, kb * kBK, a_row, pw);
-          // the weight tiles of the first ring pass go out before the wait for the previous
-          // kernel; the token rows (its output) only after it
-          if (!waited && issued + 1 < S && kb + 1 < kblocks) {
-            ++issued;
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1;
-            }
-            continue;
-          }
-          if (!waited) {
-            griddep_wait();
-            waited = true;
-            int st = (stage - (kb - kb_b) + S) % S;
-            for (; kb_b < kb; ++kb_b, st = (st + 1) % S) {
-              const uint32_t fb = mapa_shared(smem_u32(&full[st]), 0);
-              tma_load_2d_pair(sB + st * C::B_BYTES, bmap, fb, kb_b * kBK, b_row, pol_b);
-            }
-          }
           tma_load_2d_pair(sB + stage * C::B_BYTES, bmap, fbar, kb * kBK, b_row, pol_b);
-          kb_b = kb + 1;
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -230,7 +209,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (!waited) griddep_wait();
       if (!ok && leader) {
         // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
         int n = issued < S ? issued : S;

@@ -202,6 +202,32 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
                 c.d_model, c.n_experts, logits);
 }
 
+// T <= kChunk: one fused launch (selection, permutation and, if xs is given, the row
+// gather); its grid splits the gather.
+moe_status launch_route_small(const moe_layer *L, const float *logits, int T, float *logits_out,
+                              int *idx, float *gate, int *counts, int *offsets, int *perm,
+                              int *slot_row, const void *x, void *xs, cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  const int need = (c.n_experts + 31) / 32;
+  const float *bias = L->w.router_bias;
+  const dim3 thr(kRouteWarps * 32);
+  const int vpr = c.d_model * 2 / 16;  // 16-byte vectors per bf16 row
+  const size_t vecs = xs ? (size_t)T * c.top_k * vpr : 0;
+  int grid = (int)((vecs + 2047) / 2048);
+  grid = grid < 1 ? 1 : (grid > 32 ? 32 : grid);
+#define MOE_SMALL(V)                                                                           \
+  launch(route_small_kernel<V>, dim3(grid), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
+         logits_out, idx, gate, counts, offsets, perm, slot_row,                                \
+         static_cast<const uint4 *>(x), vpr, static_cast<uint4 *>(xs))
+  if (need <= 1) return MOE_SMALL(1);
+  if (need <= 2) return MOE_SMALL(2);
+  if (need <= 4) return MOE_SMALL(4);
+  if (need <= 9) return MOE_SMALL(9);
+  if (need <= 16) return MOE_SMALL(16);
+  return MOE_SMALL(32);
+#undef MOE_SMALL
+}
+
 moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
                                  float *logits_out, int *idx, float *gate, int *counts,
                                  int *offsets, int *perm, int *slot_row, int *chunk_hist,
@@ -213,6 +239,14 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   const float *bias = L->w.router_bias;
   const dim3 thr(kRouteWarps * 32);
   moe_status s;
+  if (T <= kChunk) {
+    s = launch_route_small(L, logits, T, logits_out, idx, gate, counts, offsets, perm, slot_row,
+                           nullptr, nullptr, st);
+    if (s == MOE_OK && events &&
+        cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return s;
+  }
 #define MOE_TOPK(V)                                                                        \
   launch(topk_hist_kernel<V>, dim3(nch), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
          logits_out, idx, gate, chunk_hist)
@@ -520,15 +554,24 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                          st)) != MOE_OK)
     return s;
   if ((s = mark(1)) != MOE_OK) return s;
-  if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
-                                 at<int>(ws, W.counts), offsets, perm, slot_row,
-                                 at<int>(ws, W.chunk_hist), st, events, 2)) != MOE_OK)
+  // small batches: selection, permutation and the row gather in one launch
+  const bool fused_gather = (T <= kChunk) && c.dtype == MOE_BF16;
+  if (fused_gather) {
+    if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
+                                offsets, perm, slot_row, x, at<void>(ws, W.xs), st)) != MOE_OK)
+      return s;
+    if ((s = mark(2)) != MOE_OK) return s;
+  } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
+                                        at<int>(ws, W.counts), offsets, perm, slot_row,
+                                        at<int>(ws, W.chunk_hist), st, events, 2)) != MOE_OK) {
     return s;
+  }
   if ((s = mark(3)) != MOE_OK) return s;
 
   if (c.dtype == MOE_BF16) {
     const int vpr = c.d_model / 8;
-    if ((s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk * vpr, 256, h->num_sms)),
+    if (!fused_gather &&
+        (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk * vpr, 256, h->num_sms)),
                     dim3(256), 0, st, static_cast<const uint4 *>(x), (const int *)perm,
                     c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
       return s;

@@ -215,6 +215,107 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 // keeps slot j.  Gates: softmax over the selected UNBIASED logits (max-shifted, expf).
 // The CTA's per-expert selection counts go to chunk_hist[c][e] (integer, order-free).
 // logits_out (optional) receives a copy of the logits read.
+// Selection and gates of token t by one warp.  Returns, in lane j < k, slot j's expert id
+// and gate; other lanes return (0, 0).  logits_out (optional) receives a copy of the row.
+template <int MAXV>
+__device__ __forceinline__ void topk_token(const float *__restrict__ lrow,
+                                           const float *__restrict__ bias, int E, int k,
+                                           float *__restrict__ lout, int lane, int &my_e,
+                                           float &my_gate) {
+  uint32_t key[MAXV];
+  float l[MAXV];
+#pragma unroll
+  for (int v = 0; v < MAXV; ++v) {
+    const int e = lane + 32 * v;
+    if (e < E) {
+      l[v] = lrow[e];
+      if (lout) lout[e] = l[v];
+      key[v] = score_key(l[v] + (bias ? bias[e] : 0.f));
+    } else {
+      l[v] = 0.f;
+      key[v] = 0u;  // ties with NaN scores and loses on id (all ids here are >= E)
+    }
+  }
+  my_e = 0;
+  float my_l = 0.f;
+  uint32_t used = 0;
+  for (int r = 0; r < k; ++r) {
+    // lane-local best among unused entries; ids grow with v, so '>' keeps the lower id
+    uint32_t bk = 0;
+    int bv = -1;
+    float bl = 0.f;
+#pragma unroll
+    for (int v = 0; v < MAXV; ++v) {
+      const bool ok = !((used >> v) & 1u);
+      if (ok && (bv < 0 || key[v] > bk)) {
+        bk = key[v];
+        bv = v;
+        bl = l[v];
+      }
+    }
+    const uint32_t wkey = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t cand = (bv >= 0 && bk == wkey) ? (uint32_t)(lane + 32 * bv) : 0xffffffffu;
+    const uint32_t wid = __reduce_min_sync(0xffffffffu, cand);
+    const int owner = (int)(wid & 31u);
+    if (owner == lane) used |= 1u << (wid >> 5);
+    const float wl = __shfl_sync(0xffffffffu, bl, owner);
+    if (lane == r) {
+      my_e = (int)wid;
+      my_l = wl;
+    }
+  }
+  // gates over lanes 0..k-1: softmax of the selected unbiased logits
+  float m = (lane < k) ? my_l : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float ex = (lane < k) ? expf(my_l - m) : 0.f;
+  float z = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  my_gate = (lane < k) ? ex / z : 0.f;
+  if (lane >= k) my_e = 0;
+}
+
+// Exclusive scan of cnt[0..E) into off[0..E) by the whole CTA (each thread a contiguous
+// run, warp and block scans of the run totals).  Contains __syncthreads.
+__device__ __forceinline__ void block_exclusive_scan(const int *cnt, int *off, int E,
+                                                     int *warp_sum) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int lo = min(E, tid * per), hi = min(E, lo + per);
+  int run = 0;
+  for (int e = lo; e < hi; ++e) run += cnt[e];
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int v = (lane < nw) ? warp_sum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < nw) warp_sum[lane] = v;  // inclusive warp totals
+  }
+  __syncthreads();
+  int excl = incl - run + (warp > 0 ? warp_sum[warp - 1] : 0);
+  for (int e = lo; e < hi; ++e) {
+    off[e] = excl;
+    excl += cnt[e];
+  }
+  __syncthreads();
+}
+
+// One warp per token; CTA c handles tokens [c*kChunk, (c+1)*kChunk).  Lane l holds the
+// scores of experts l, l+32, ...  k rounds of warp arg-max pick S_t in rank order; lane j
+// keeps slot j.  The CTA's per-expert selection counts go to chunk_hist[c][e] (integer,
+// order-free).
 template <int MAXV>
 __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
     const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
@@ -229,64 +330,100 @@ __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tbeg = c * kChunk, tend = min(T, tbeg + kChunk);
   for (int t = tbeg + warp; t < tend; t += kRouteWarps) {
-    uint32_t key[MAXV];
-    float l[MAXV];
-#pragma unroll
-    for (int v = 0; v < MAXV; ++v) {
-      const int e = lane + 32 * v;
-      if (e < E) {
-        l[v] = logits[(size_t)t * E + e];
-        if (logits_out) logits_out[(size_t)t * E + e] = l[v];
-        key[v] = score_key(l[v] + (bias ? bias[e] : 0.f));
-      } else {
-        l[v] = 0.f;
-        key[v] = 0u;  // ties with NaN scores and loses on id (all ids here are >= E)
-      }
-    }
-    int my_e = 0;
-    float my_l = 0.f;
-    uint32_t used = 0;
-    for (int r = 0; r < k; ++r) {
-      // lane-local best among unused entries; ids grow with v, so '>' keeps the lower id
-      uint32_t bk = 0;
-      int bv = -1;
-      float bl = 0.f;
-#pragma unroll
-      for (int v = 0; v < MAXV; ++v) {
-        const bool ok = !((used >> v) & 1u);
-        if (ok && (bv < 0 || key[v] > bk)) {
-          bk = key[v];
-          bv = v;
-          bl = l[v];
-        }
-      }
-      const uint32_t wkey = __reduce_max_sync(0xffffffffu, bk);
-      const uint32_t cand = (bv >= 0 && bk == wkey) ? (uint32_t)(lane + 32 * bv) : 0xffffffffu;
-      const uint32_t wid = __reduce_min_sync(0xffffffffu, cand);
-      const int owner = (int)(wid & 31u);
-      if (owner == lane) used |= 1u << (wid >> 5);
-      const float wl = __shfl_sync(0xffffffffu, bl, owner);
-      if (lane == r) {
-        my_e = (int)wid;
-        my_l = wl;
-      }
-    }
-    // gates over lanes 0..k-1
-    float m = (lane < k) ? my_l : -INFINITY;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float ex = (lane < k) ? expf(my_l - m) : 0.f;
-    float z = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    int my_e;
+    float my_gate;
+    topk_token<MAXV>(logits + (size_t)t * E, bias, E, k,
+                     logits_out ? logits_out + (size_t)t * E : nullptr, lane, my_e, my_gate);
     if (lane < k) {
       topk_idx[(size_t)t * k + lane] = my_e;
-      topk_gate[(size_t)t * k + lane] = ex / z;
+      topk_gate[(size_t)t * k + lane] = my_gate;
       atomicAdd(&hist[my_e], 1);
     }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)c * E + e] = hist[e];
+}
+
+// ------------------------------------------------------------------ small-T fused routing
+// T <= kChunk (decode): selection, gates, histogram, scan, permutation and (optionally) the
+// row gather in ONE launch.  Every CTA computes the selection and the permutation of all T
+// tokens (cheap, and identical in every CTA), CTA 0 writes the routing outputs, and the CTAs
+// split the gather xs[p, :] = x[perm[p] / k, :] between them.
+template <int MAXV>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
+    const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
+    float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
+    int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
+    int *__restrict__ slot_row, const uint4 *__restrict__ x, int vec_per_row,
+    uint4 *__restrict__ xs) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ int hist[kMaxExperts];
+  __shared__ int off[kMaxExperts];
+  __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
+  __shared__ int s_idx[kChunk * kMaxTopK];
+  __shared__ int s_perm[kChunk * kMaxTopK];
+  __shared__ int warp_sum[32];
+  const bool writer = blockIdx.x == 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    hist[e] = 0;
+#pragma unroll
+    for (int w = 0; w < kChunk / 32; ++w) bits[e][w] = 0u;
+  }
+  __syncthreads();
+  for (int t = warp; t < T; t += kRouteWarps) {
+    int my_e;
+    float my_gate;
+    topk_token<MAXV>(logits + (size_t)t * E, bias, E, k,
+                     (writer && logits_out) ? logits_out + (size_t)t * E : nullptr, lane, my_e,
+                     my_gate);
+    if (lane < k) {
+      s_idx[t * k + lane] = my_e;
+      atomicAdd(&hist[my_e], 1);
+      atomicOr(&bits[my_e][t >> 5], 1u << (t & 31));
+      if (writer) {
+        topk_idx[(size_t)t * k + lane] = my_e;
+        topk_gate[(size_t)t * k + lane] = my_gate;
+      }
+    }
+  }
+  __syncthreads();
+  block_exclusive_scan(hist, off, E, warp_sum);
+  if (writer) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      counts[e] = hist[e];
+      offsets[e] = off[e];
+    }
+    if (threadIdx.x == 0) offsets[E] = T * k;
+  }
+  const int npair = T * k;
+  for (int q = threadIdx.x; q < npair; q += blockDim.x) {
+    const int t = q / k;
+    const int e = s_idx[q];
+    int rank = 0;
+#pragma unroll
+    for (int w = 0; w < kChunk / 32; ++w) {
+      const uint32_t word = bits[e][w];
+      if (w < (t >> 5)) rank += __popc(word);
+      else if (w == (t >> 5)) rank += __popc(word & ((1u << (t & 31)) - 1u));
+    }
+    const int p = off[e] + rank;
+    s_perm[p] = q;
+    if (writer) {
+      perm[p] = q;
+      slot_row[q] = p;
+    }
+  }
+  if (!xs) return;
+  __syncthreads();
+  const size_t total = (size_t)npair * vec_per_row;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int p = (int)(i / vec_per_row);
+    const int v = (int)(i % vec_per_row);
+    xs[i] = __ldg(x + (size_t)(s_perm[p] / k) * vec_per_row + v);
+  }
 }
 
 // ------------------------------------------------------------------ permutation (scatter)
