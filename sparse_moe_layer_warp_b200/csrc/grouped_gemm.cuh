@@ -54,7 +54,10 @@ struct GemmParams {
   int M;      // weight rows per group: f (UP), d (DOWN), E (LOGITS)
   int K;      // reduction length: d (UP, LOGITS) or f (DOWN)
   int ld_out; // f (UP), d (DOWN), E (LOGITS)
+  int *sched;  // work counter (zero at launch) for dynamic unit claiming; null: round-robin
 };
+
+constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
 
 constexpr int kBM = 128;         // weight rows per unit (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle atom of bf16
@@ -82,8 +85,8 @@ struct GemmCfg {
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of the MMA");
   static_assert(TMEM_COLS_RAW <= 512, "TMEM has 512 columns");
-  // barriers: full[S], empty[S], tfull[2], tempty[2], drain[1]
-  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], drain[1], uq_full[Q], uq_empty[Q]
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
            (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * BN * 4 /*row scales*/ +
@@ -159,8 +162,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *tfull = bars + 2 * S;
   uint64_t *tempty = bars + 2 * S + 2;
   uint64_t *drain = bars + 2 * S + 4;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+  uint64_t *uq_full = bars + 2 * S + 5;
+  uint64_t *uq_empty = uq_full + kUnitQ;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -184,6 +190,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < kUnitQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      mbar_init(&uq_empty[q], 5);  // the MMA thread and the four epilogue warps
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA0);
@@ -255,68 +265,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     nt = loc % nts;
   };
 
+  // Work distribution: the producer claims units (from the shared counter when p.sched is
+  // set, so units that share weight or token tiles run at about the same time on different
+  // SMs and a slow unit delays nothing else; round-robin otherwise) and publishes each id
+  // through a small shared-memory queue; the MMA thread and the epilogue warps take the ids
+  // in the same order.  Id -1 ends the sequence.
+  auto claim = [&](int prev) -> int {
+    if (p.sched) return atomicAdd(p.sched, 1);
+    return prev < 0 ? (int)blockIdx.x : prev + (int)gridDim.x;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
-      // Walks the (unit, k-block) load slots of this CTA in order.
       const uint64_t pol_w = policy_evict_first();  // weights read once
       const uint64_t pol_b = policy_evict_last();   // activations: re-read per m tile
-      struct Slot {
-        int u, kb, a_row, b_row;
-        bool shared_x, single_use;
-      };
-      auto slot_set_unit = [&](Slot &c) {
-        int g, mt, nt;
-        decode(c.u, g, mt, nt);
-        c.a_row = g * p.M + mt * kBM;
-        c.shared_x = (MODE == MODE_UP) && (g >= p.E);
-        c.b_row = c.shared_x ? nt * BN : grp_row[g] + nt * BN;
-        // a weight tile read by one unit only is streamed with evict-first priority; one
-        // shared by several token tiles keeps normal priority so its neighbours hit L2
-        c.single_use = grp_count[g] <= BN;
-      };
-      auto slot_next = [&](Slot &c) {
-        if (++c.kb == kblocks) {
-          c.kb = 0;
-          c.u += gridDim.x;
-          if (c.u < total_units) slot_set_unit(c);
-        }
-      };
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      auto load_a = [&](const Slot &c, int st) {
-        const int kc = c.kb * kBK;
-        if (c.single_use) {
-          tma_load_2d_hint(sA0 + st * C::A_BYTES, &p.tmA0, &full[st], kc, c.a_row, pol_w);
-          if (MODE == MODE_UP)
-            tma_load_2d_hint(sA1 + st * C::A_BYTES, &p.tmA1, &full[st], kc, c.a_row, pol_w);
-        } else {
-          tma_load_2d(sA0 + st * C::A_BYTES, &p.tmA0, &full[st], kc, c.a_row);
-          if (MODE == MODE_UP) tma_load_2d(sA1 + st * C::A_BYTES, &p.tmA1, &full[st], kc, c.a_row);
-        }
-      };
-      auto load_b = [&](const Slot &c, int st) {
-        tma_load_2d_hint(sB + st * C::B_BYTES, c.shared_x ? &p.tmBs : &p.tmB, &full[st],
-                         c.kb * kBK, c.b_row, pol_b);
-      };
-      Slot ld{(int)blockIdx.x, 0, 0, 0, false, false};
-      if (ld.u < total_units) slot_set_unit(ld);
-      while (ld.u < total_units) {
-        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
+      int qi = 0;
+      uint32_t qph = 0;
+      for (int u = claim(-1);; u = claim(u)) {
+        const int uid = (u < total_units) ? u : -1;
+        if (!mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 5)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-        load_a(ld, stage);
-        load_b(ld, stage);
-        ++issued;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
+        uq[qi] = uid;
+        mbar_arrive(&uq_full[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
         }
-        slot_next(ld);
+        if (uid < 0) break;
+        int g, mt, nt;
+        decode(uid, g, mt, nt);
+        const int a_row = g * p.M + mt * kBM;
+        const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
+        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
+        const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
+        // a weight tile read by one unit only is streamed with evict-first priority; one
+        // shared by several token tiles keeps normal priority so its neighbours hit L2
+        const bool single_use = grp_count[g] <= BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
+            ok = false;
+            break;
+          }
+          const int kc = kb * kBK;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (single_use) {
+            tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row, pol_w);
+            if (MODE == MODE_UP)
+              tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row,
+                               pol_w);
+          } else {
+            tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row);
+            if (MODE == MODE_UP)
+              tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row);
+          }
+          tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kc, b_row, pol_b);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
       }
       if (!ok) {
         // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
@@ -340,9 +356,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++it) {
+      int qi = 0;
+      uint32_t qph = 0;
+      while (ok) {
+        if (!mbar_wait_bounded(&uq_full[qi], qph, abort_flag, p.status, 6)) break;
+        const int u = uq[qi];
+        mbar_arrive(&uq_empty[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
         const int acc = it % C::ACC_BUFS;
         const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
+        ++it;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
         int g, mt, nt;
@@ -383,13 +410,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
+    // Lane 0 of each warp polls the barriers and the warp follows it, so every lane takes
+    // the same path into the warp-wide tcgen05.ld instructions.
     const int q = warp & 3;              // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;         // weight row within the unit
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, p.status, where) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      return ok != 0;
+    };
     int it = 0;
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++it) {
+    int qi = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!warp_wait(&uq_full[qi], qph, 7)) break;
+      const int u = uq[qi];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uq_empty[qi]);
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (u < 0) break;
       const int acc = it % C::ACC_BUFS;
       const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, 4)) break;
+      ++it;
+      if (!warp_wait(&tfull[acc], acc_phase, 4)) break;
       tc_fence_after();
       int g, mt, nt;
       decode(u, g, mt, nt);

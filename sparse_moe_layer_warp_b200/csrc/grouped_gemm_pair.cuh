@@ -44,7 +44,8 @@ struct PairCfg {
   static constexpr int STAGES_RAW = (192 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation");
-  static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC_BUFS + 1) * 8;
+  // full[S], empty[S], tfull[A], tempty[A], drain, uq_full[Q], uq_empty[Q]
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC_BUFS + 1 + 2 * kUnitQ) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
            (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * kPairBN * 4 +
@@ -70,8 +71,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *tfull = bars + 2 * S;
   uint64_t *tempty = bars + 2 * S + C::ACC_BUFS;
   uint64_t *drain = bars + 2 * S + 2 * C::ACC_BUFS;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *uq_full = drain + 1;
+  uint64_t *uq_empty = uq_full + kUnitQ;  // used in the leader only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -98,6 +102,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < kUnitQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      // readers of a published unit id: the leader's MMA thread and epilogue warps, the
+      // peer's producer and epilogue warps (1 + 4 + 1 + 4)
+      mbar_init(&uq_empty[q], 10);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA0);
@@ -171,6 +181,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     return (((valid + 1) >> 1) + 7) & ~7;
   };
 
+  // unit claiming as in grouped_gemm_kernel, per CTA pair: the leader's producer claims
+  auto claim = [&](int prev) -> int {
+    if (p.sched) return atomicAdd(p.sched, 1);
+    return prev < 0 ? cluster_id : prev + n_clusters;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
@@ -182,7 +198,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int u = cluster_id; u < total_units && ok; u += n_clusters) {
+      int qi = 0;
+      uint32_t qph = 0;
+      int u = -1;
+      while (ok) {
+        // the leader claims the next unit and publishes its id to both CTAs; the peer reads it
+        if (leader) {
+          u = claim(u);
+          const int uid = (u < total_units) ? u : -1;
+          if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 15)) {
+            ok = false;
+            break;
+          }
+          uq[qi] = uid;
+          st_shared_remote(mapa_shared(smem_u32((const void *)&uq[qi]), 1), uid);
+          mbar_arrive(&uq_full[qi]);
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_full[qi]), 1));
+          u = uid;
+        } else {
+          if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 16)) {
+            ok = false;
+            break;
+          }
+          u = uq[qi];
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_empty[qi]), 0));
+        }
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
         int g, mt, nt;
         decode(u, g, mt, nt);
         const int half = split(g, nt);
@@ -208,6 +253,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             phase ^= 1;
           }
         }
+        if (u < 0) break;
       }
       if (!ok && leader) {
         // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
@@ -231,9 +277,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int u = cluster_id; u < total_units && ok; u += n_clusters, ++it) {
+      int qi = 0;
+      uint32_t qph = 0;
+      while (ok) {
+        if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 17)) break;
+        const int u = uq[qi];
+        mbar_arrive(&uq_empty[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
         const int acc = it % C::ACC_BUFS;
         const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
+        ++it;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 12)) break;
         tc_fence_after();
         int g, mt, nt;
@@ -274,11 +331,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t uq_empty_leader = mapa_shared(smem_u32(&uq_empty[0]), 0);
+    // lane 0 polls, the warp follows (uniform path into the warp-wide tcgen05.ld)
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where, bool cluster) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = (cluster ? mbar_wait_bounded<true>(bar, parity, abort_flag, p.status, where)
+                      : mbar_wait_bounded(bar, parity, abort_flag, p.status, where))
+                 ? 1
+                 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      return ok != 0;
+    };
     int it = 0;
-    for (int u = cluster_id; u < total_units; u += n_clusters, ++it) {
+    int qi = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!warp_wait(&uq_full[qi], qph, 18, true)) break;
+      const int u = uq[qi];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&uq_empty[qi]);
+        else mbar_arrive_remote(uq_empty_leader + qi * 8);
+      }
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (u < 0) break;
       const int acc = it % C::ACC_BUFS;
       const uint32_t acc_phase = (it / C::ACC_BUFS) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, 14)) break;
+      ++it;
+      if (!warp_wait(&tfull[acc], acc_phase, 14, false)) break;
       tc_fence_after();
       int g, mt, nt;
       decode(u, g, mt, nt);

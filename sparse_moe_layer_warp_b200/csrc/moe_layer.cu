@@ -206,7 +206,8 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
 // gather); its grid splits the gather.
 moe_status launch_route_small(const moe_layer *L, const float *logits, int T, float *logits_out,
                               int *idx, float *gate, int *counts, int *offsets, int *perm,
-                              int *slot_row, const void *x, void *xs, cudaStream_t st) {
+                              int *slot_row, const void *x, void *xs, int *sched_reset,
+                              cudaStream_t st) {
   const moe_config &c = L->cfg;
   const int need = (c.n_experts + 31) / 32;
   const float *bias = L->w.router_bias;
@@ -218,7 +219,7 @@ moe_status launch_route_small(const moe_layer *L, const float *logits, int T, fl
 #define MOE_SMALL(V)                                                                           \
   launch(route_small_kernel<V>, dim3(grid), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
          logits_out, idx, gate, counts, offsets, perm, slot_row,                                \
-         static_cast<const uint4 *>(x), vpr, static_cast<uint4 *>(xs))
+         static_cast<const uint4 *>(x), vpr, static_cast<uint4 *>(xs), sched_reset)
   if (need <= 1) return MOE_SMALL(1);
   if (need <= 2) return MOE_SMALL(2);
   if (need <= 4) return MOE_SMALL(4);
@@ -231,8 +232,8 @@ moe_status launch_route_small(const moe_layer *L, const float *logits, int T, fl
 moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
                                  float *logits_out, int *idx, float *gate, int *counts,
                                  int *offsets, int *perm, int *slot_row, int *chunk_hist,
-                                 cudaStream_t st, void *const *events = nullptr,
-                                 int mark_index = 0) {
+                                 int *sched_reset, cudaStream_t st,
+                                 void *const *events = nullptr, int mark_index = 0) {
   const moe_config &c = L->cfg;
   const int nch = (T + kChunk - 1) / kChunk;
   const int need = (c.n_experts + 31) / 32;
@@ -241,7 +242,7 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   moe_status s;
   if (T <= kChunk) {
     s = launch_route_small(L, logits, T, logits_out, idx, gate, counts, offsets, perm, slot_row,
-                           nullptr, nullptr, st);
+                           nullptr, nullptr, sched_reset, st);
     if (s == MOE_OK && events &&
         cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -261,7 +262,7 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch(permute_scatter_kernel, dim3(nch), dim3(256), 0, st, idx, chunk_hist, T,
-                c.n_experts, c.top_k, nch, counts, offsets, perm, slot_row);
+                c.n_experts, c.top_k, nch, counts, offsets, perm, slot_row, sched_reset);
 }
 
 // ------------------------------------------------------------------ grouped GEMM launch
@@ -505,7 +506,8 @@ static moe_status route_common(moe_handle h, const void *x, const float *logits_
     copy_out = logits_out;
   }
   return launch_select_permute(h, logits, T, copy_out, idx, gate, counts, offsets, perm,
-                               slot_row, at<int>(ws, W.chunk_hist), st);
+                               slot_row, at<int>(ws, W.chunk_hist),
+                               at<DevStatus>(ws, W.status)->sched, st);
 }
 
 moe_status moe_route(moe_handle h, const void *x, int n_tokens, float *logits_out,
@@ -558,12 +560,15 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   const bool fused_gather = (T <= kChunk) && c.dtype == MOE_BF16;
   if (fused_gather) {
     if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
-                                offsets, perm, slot_row, x, at<void>(ws, W.xs), st)) != MOE_OK)
+                                offsets, perm, slot_row, x, at<void>(ws, W.xs),
+                                at<DevStatus>(ws, W.status)->sched, st)) != MOE_OK)
       return s;
     if ((s = mark(2)) != MOE_OK) return s;
   } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
                                         at<int>(ws, W.counts), offsets, perm, slot_row,
-                                        at<int>(ws, W.chunk_hist), st, events, 2)) != MOE_OK) {
+                                        at<int>(ws, W.chunk_hist),
+                                        at<DevStatus>(ws, W.status)->sched, st, events, 2)) !=
+             MOE_OK) {
     return s;
   }
   if ((s = mark(3)) != MOE_OK) return s;
@@ -602,6 +607,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p1.M = c.d_ff;
     p1.K = c.d_model;
     p1.ld_out = c.d_ff;
+    p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
     if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
         MOE_OK)
       return s;
@@ -610,6 +616,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p2.tmA0 = h->tm_wd;
     if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
     p2.out = ybuf;
+    p2.sched = &at<DevStatus>(ws, W.status)->sched[1];
     p2.M = c.d_model;
     p2.K = c.d_ff;
     p2.ld_out = c.d_model;

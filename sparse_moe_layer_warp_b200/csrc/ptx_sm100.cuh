@@ -15,7 +15,8 @@ namespace moe {
 struct DevStatus {
   int error;             // 0 = ok, 1 = a bounded wait gave up
   int where;             // which wait (kernel-specific code)
-  int pad[30];
+  int sched[4];          // grouped-GEMM work counters (up, down), reset by the routing kernels
+  int pad[26];
   int router_ticket[32]; // split-K router: arrivals per block of 32 experts (self-resetting)
 };
 
@@ -64,16 +65,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with cluster-scope acquire: for barriers that receive arrivals (and data) from
+// the other CTA of a pair.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (after recording the
 // failure in *status and raising the CTA-wide abort flag) when the time limit passes or
 // another role of the CTA has already aborted.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag,
                                                   DevStatus *status, int where) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_wait = [&]() {
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (try_wait()) return true;
   unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_wait()) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -243,6 +262,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+
+// 32-bit store into another CTA's shared memory (shared::cluster address)
+__device__ __forceinline__ void st_shared_remote(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // arrive on an mbarrier of another CTA of the cluster (shared::cluster address)

@@ -355,9 +355,11 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
     float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
     int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
     int *__restrict__ slot_row, const uint4 *__restrict__ x, int vec_per_row,
-    uint4 *__restrict__ xs) {
+    uint4 *__restrict__ xs, int *__restrict__ sched_reset) {
   griddep_wait();
   griddep_launch_dependents();
+  // zero the grouped GEMMs' work counters for the launches that follow this one
+  if (sched_reset && blockIdx.x == 0 && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
   __shared__ int hist[kMaxExperts];
   __shared__ int off[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
@@ -436,9 +438,11 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
 __global__ void __launch_bounds__(256) permute_scatter_kernel(
     const int *__restrict__ topk_idx, const int *__restrict__ chunk_hist, int T, int E, int k,
     int n_chunks, int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
-    int *__restrict__ slot_row) {
+    int *__restrict__ slot_row, int *__restrict__ sched_reset) {
   griddep_wait();
   griddep_launch_dependents();
+  // zero the grouped GEMMs' work counters for the launches that follow this one
+  if (sched_reset && blockIdx.x == 0 && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
   __shared__ int s_tot[kMaxExperts];
   __shared__ int s_base[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
