@@ -130,8 +130,10 @@ moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, voi
  * on `stream` around its kernel stages, for per-kernel timing with no profiler attached:
  *   events[0] before the router, then one event after each of the MOE_PROFILE_STAGES
  *   stages: 1 router logits, 2 top-k + gates + chunk histograms, 3 permutation scatter,
- *   4 row gather (bf16; empty for fp32), 5 expert up + SwiGLU, 6 expert down, 7 combine.
- *   For n_tokens <= 64 stages 2-4 are one fused launch, timed as stage 2 (3 and 4 empty).
+ *   4 row gather (bf16 with more than about 12 tokens per expert; otherwise empty, the
+ *   expert-up kernel gathering the rows of x as it loads them), 5 expert up + SwiGLU,
+ *   6 expert down, 7 combine.
+ *   For n_tokens <= 64 stages 2-3 are one fused launch, timed as stage 2 (3 empty).
  * n_events must be at least MOE_PROFILE_STAGES + 1; otherwise MOE_ERR_INVALID_ARG. */
 #define MOE_PROFILE_STAGES 7
 moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void *out,

@@ -13,8 +13,13 @@
 // decode a group holds one or two tokens, so this keeps the tensor-core work tiny while
 // every SM streams weight tiles from HBM through TMA.
 //
-//   MODE_UP   : A0 = W_gate, A1 = W_up (two accumulators), B = expert-sorted x rows
-//               (the shared group reads x directly); epilogue h = silu(G) * U -> bf16.
+//   MODE_UP   : A0 = W_gate, A1 = W_up (two accumulators), B = the group's x rows;
+//               epilogue h = silu(G) * U -> bf16.  With token tiles of up to 32 rows the
+//               rows are gathered from x by token id with tile::gather4 (four rows per copy:
+//               the "gather" of section 3.2.4 fused into the operand load, no expert-sorted
+//               copy of x); larger tiles load expert-sorted rows xs written by the gather
+//               kernel, and the shared group reads x directly.  (Gathering 128-row tiles,
+//               32 gather4 copies per stage, measured 1.6x slower than the row box.)
 //   MODE_LOGITS: router logits; one group (all T tokens), A0 = W_r (rows past E zero-filled
 //               by TMA), B = x; epilogue logits[t, e] = acc (fp32).
 //   MODE_DOWN : A0 = W_down, B = h rows; epilogue y = acc * scale -> fp32, scale =
@@ -22,7 +27,8 @@
 //               rounding it to bf16 as well as h and the output would put the layer's
 //               error above 2e-2 x RMS(out) even with exact accumulation.
 //
-// Roles (192 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA issuer (warp 1
+// Roles (192 threads): warp 0 = TMA producer (lane 0 claims units and loads weight tiles;
+// in MODE_UP each lane gathers four token rows per stage), warp 1 lane 0 = MMA issuer (warp 1
 // also owns the TMEM allocation), warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
 // Pipelines: STAGES shared-memory slots (full / empty mbarriers) and two TMEM accumulator
 // buffers (tmem_full / tmem_empty) so the epilogue of unit i overlaps the MMAs of i + 1.
@@ -42,10 +48,12 @@ enum GemmMode { MODE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
 struct GemmParams {
   CUtensorMap tmA0;  // UP: W_gate [G*f, d]; DOWN: W_down [G*d, f]     box {64, 128}
   CUtensorMap tmA1;  // UP: W_up [G*f, d]                               box {64, 128}
-  CUtensorMap tmB;   // UP: xs [Tk, d]; DOWN: h [Tk + n_shared*T, f]   box {64, BN}
-  CUtensorMap tmBs;  // UP: x [T, d] (shared group)                     box {64, BN}
+  CUtensorMap tmB;   // UP, BN <= 32: x [T, d] box {64, 1} (tile::gather4 by token id);
+                     // UP, BN > 32: xs [Tk, d]; DOWN: h [Tk + n_shared*T, f]; LOGITS: x
+                     // (box {64, BN} for all but the gather map)
+  CUtensorMap tmBs;  // UP, BN > 32: x [T, d] (shared group)            box {64, BN}
   const int *offsets;       // [E + 1] expert offsets in the sorted space
-  const int *perm;          // [Tk] (DOWN: gate lookup)
+  const int *perm;          // [Tk] sorted row -> t*k + j (UP: token of a row; DOWN: gate)
   const float *topk_gate;   // [Tk] (DOWN)
   void *out;                // UP: h [P, f] bf16; DOWN: y [P, d] fp32; LOGITS: [T, E] fp32
   DevStatus *status;
@@ -55,9 +63,11 @@ struct GemmParams {
   int K;      // reduction length: d (UP, LOGITS) or f (DOWN)
   int ld_out; // f (UP), d (DOWN), E (LOGITS)
   int *sched;  // work counter (zero at launch) for dynamic unit claiming; null: round-robin
+  int topk;    // k (UP: token of routed sorted row q = perm[q] / k)
 };
 
 constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
+constexpr int kGatherMaxBN = 32;  // MODE_UP token tiles up to this size gather rows from x
 
 constexpr int kBM = 128;         // weight rows per unit (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle atom of bf16
@@ -150,6 +160,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = GemmCfg<MODE, BN>;
   constexpr int S = C::STAGES;
+  constexpr bool kGather = (MODE == MODE_UP) && (BN <= kGatherMaxBN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&p.tmA0);
     if (MODE == MODE_UP) {
       tma_prefetch_desc(&p.tmA1);
-      tma_prefetch_desc(&p.tmBs);
+      if (BN > kGatherMaxBN) tma_prefetch_desc(&p.tmBs);
     }
     tma_prefetch_desc(&p.tmB);
   }
@@ -276,76 +287,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      const uint64_t pol_w = policy_evict_first();  // weights read once
-      const uint64_t pol_b = policy_evict_last();   // activations: re-read per m tile
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      int qi = 0;
-      uint32_t qph = 0;
-      for (int u = claim(-1);; u = claim(u)) {
-        const int uid = (u < total_units) ? u : -1;
-        if (!mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 5)) {
+    // -------------------------------------------------------------- TMA producer (warp 0)
+    // Lane 0 claims units, publishes them, waits for free slots and loads the weight tiles.
+    // Gathering (MODE_UP, BN <= kGatherMaxBN): every lane then gathers four of the unit's
+    // token rows of x per stage (lane l: tile rows 4l..4l+3), n_mma rows in all; rows past
+    // the group's last token repeat its first token (their accumulator columns are never
+    // read).  Otherwise lane 0 loads the contiguous token-row box.
+    const uint64_t pol_w = policy_evict_first();  // weights read once
+    const uint64_t pol_b = policy_evict_last();   // activations: re-read per m tile
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    int qi = 0;
+    uint32_t qph = 0;
+    int u = -1;  // lane 0's claim cursor
+    for (;;) {
+      int uid = -1;
+      if (lane == 0) {
+        u = claim(u);
+        uid = (u < total_units) ? u : -1;
+        if (mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 5)) {
+          uq[qi] = uid;
+          mbar_arrive(&uq_full[qi]);
+        } else {
           ok = false;
-          break;
         }
-        uq[qi] = uid;
-        mbar_arrive(&uq_full[qi]);
-        if (++qi == kUnitQ) {
-          qi = 0;
-          qph ^= 1;
-        }
-        if (uid < 0) break;
-        int g, mt, nt;
-        decode(uid, g, mt, nt);
-        const int a_row = g * p.M + mt * kBM;
-        const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
-        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
-        const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
-        // a weight tile read by one unit only is streamed with evict-first priority; one
-        // shared by several token tiles keeps normal priority so its neighbours hit L2
-        const bool single_use = grp_count[g] <= BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1)) {
-            ok = false;
-            break;
-          }
-          const int kc = kb * kBK;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          if (single_use) {
-            tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row, pol_w);
-            if (MODE == MODE_UP)
-              tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row,
-                               pol_w);
-          } else {
-            tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row);
-            if (MODE == MODE_UP)
-              tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row);
-          }
-          tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kc, b_row, pol_b);
-          ++issued;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
       }
-      if (!ok) {
-        // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
-        int n = issued < S ? issued : S;
-        int st = stage, ph = phase;
-        for (int i = 0; i < n; ++i) {
-          if (--st < 0) {
-            st = S - 1;
-            ph ^= 1;
-          }
-          volatile int no_abort = 0;
-          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      uid = __shfl_sync(0xffffffffu, uid, 0);
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (uid < 0) break;
+      int g, mt, nt;
+      decode(uid, g, mt, nt);
+      const int a_row = g * p.M + mt * kBM;
+      const int valid = min(BN, grp_count[g] - nt * BN);
+      // the shared group of a non-gathering up kernel reads x, not the sorted rows
+      const bool shared_x = (MODE == MODE_UP) && !kGather && (g >= p.E);
+      const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
+      const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
+      // gathering: this lane's four token ids and the rows the MMA reads
+      int tok[4] = {0, 0, 0, 0};
+      int n_rows = BN;
+      if (kGather) {
+        n_rows = (valid + 15) & ~15;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pos = 4 * lane + i;
+          const int q = b_row + ((pos < valid) ? pos : 0);
+          if (4 * lane < n_rows) tok[i] = (g < p.E) ? p.perm[q] / p.topk : q - grp_row[g];
         }
+      }
+      const uint32_t stage_bytes = C::NA * C::A_BYTES + (uint32_t)n_rows * kBK * 2;
+      // a weight tile read by one unit only is streamed with evict-first priority; one
+      // shared by several token tiles keeps normal priority so its neighbours hit L2
+      const bool single_use = grp_count[g] <= BN;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int kc = kb * kBK;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 1);
+          if (ok) {
+            mbar_arrive_expect_tx(&full[stage], stage_bytes);
+            if (single_use) {
+              tma_load_2d_hint(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row,
+                               pol_w);
+              if (MODE == MODE_UP)
+                tma_load_2d_hint(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row,
+                                 pol_w);
+            } else {
+              tma_load_2d(sA0 + stage * C::A_BYTES, &p.tmA0, &full[stage], kc, a_row);
+              if (MODE == MODE_UP)
+                tma_load_2d(sA1 + stage * C::A_BYTES, &p.tmA1, &full[stage], kc, a_row);
+            }
+            if (!kGather)
+              tma_load_2d_hint(sB + stage * C::B_BYTES, bmap, &full[stage], kc, b_row, pol_b);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (kGather && 4 * lane < n_rows)
+          tma_gather4(sB + stage * C::B_BYTES + lane * 4 * kBK * 2, &p.tmB, &full[stage], kc,
+                      tok[0], tok[1], tok[2], tok[3], pol_b);
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
+      int n = issued < S ? issued : S;
+      int st = stage, ph = phase;
+      for (int i = 0; i < n; ++i) {
+        if (--st < 0) {
+          st = S - 1;
+          ph ^= 1;
+        }
+        volatile int no_abort = 0;
+        mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
       }
     }
     __syncwarp();

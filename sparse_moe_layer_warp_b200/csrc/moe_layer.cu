@@ -4,7 +4,8 @@
 //
 // One call of moe_forward launches, in stream order:
 //   router logits -> top-k + chunk histograms -> permutation scatter     (routing.cuh)
-//   bf16: row gather -> grouped GEMM up+SwiGLU -> grouped GEMM down     (grouped_gemm.cuh)
+//   bf16: [row gather] -> grouped GEMM up+SwiGLU -> grouped GEMM down   (grouped_gemm.cuh)
+//         (small token tiles: the up GEMM gathers the rows of x itself)
 //   fp32: SIMT up+SwiGLU -> SIMT down                                    (expert_simt.cuh)
 //   -> gate-weighted combine                                             (expert_simt.cuh)
 #include <cuda.h>
@@ -121,6 +122,14 @@ struct WsLayout {
       xs, h, y, total;
 };
 
+int pick_bn(const moe_config &c, int T, int mode);
+
+// The bf16 up GEMM gathers its token rows from x when its token tile is small; larger
+// tiles read an expert-sorted copy xs written by gather_rows_kernel.
+bool up_gathers_rows(const moe_config &c, int T) {
+  return pick_bn(c, T, MODE_UP) <= kGatherMaxBN;
+}
+
 WsLayout ws_layout(const moe_config &c, int T) {
   WsLayout L;
   size_t off = 0;
@@ -143,7 +152,7 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.slot_row = take(Tk * 4);
   L.chunk_hist = take(nch * c.n_experts * 4);
   L.stats = take(nch * (2 * (size_t)c.n_experts + 1) * 4);  // router statistics partials
-  L.xs = (c.dtype == MOE_BF16) ? take(Tk * c.d_model * 2) : off;
+  L.xs = (c.dtype == MOE_BF16 && !up_gathers_rows(c, T)) ? take(Tk * c.d_model * 2) : off;
   L.h = take(P * c.d_ff * esize(c));
   L.y = take(P * c.d_model * 4);  // fp32 in both precisions
   L.total = off;
@@ -202,24 +211,17 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
                 c.d_model, c.n_experts, logits);
 }
 
-// T <= kChunk: one fused launch (selection, permutation and, if xs is given, the row
-// gather); its grid splits the gather.
+// T <= kChunk: selection and permutation in one launch of one CTA.
 moe_status launch_route_small(const moe_layer *L, const float *logits, int T, float *logits_out,
                               int *idx, float *gate, int *counts, int *offsets, int *perm,
-                              int *slot_row, const void *x, void *xs, int *sched_reset,
-                              cudaStream_t st) {
+                              int *slot_row, int *sched_reset, cudaStream_t st) {
   const moe_config &c = L->cfg;
   const int need = (c.n_experts + 31) / 32;
   const float *bias = L->w.router_bias;
   const dim3 thr(kRouteWarps * 32);
-  const int vpr = c.d_model * 2 / 16;  // 16-byte vectors per bf16 row
-  const size_t vecs = xs ? (size_t)T * c.top_k * vpr : 0;
-  int grid = (int)((vecs + 2047) / 2048);
-  grid = grid < 1 ? 1 : (grid > 32 ? 32 : grid);
-#define MOE_SMALL(V)                                                                           \
-  launch(route_small_kernel<V>, dim3(grid), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
-         logits_out, idx, gate, counts, offsets, perm, slot_row,                                \
-         static_cast<const uint4 *>(x), vpr, static_cast<uint4 *>(xs), sched_reset)
+#define MOE_SMALL(V)                                                                         \
+  launch(route_small_kernel<V>, dim3(1), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
+         logits_out, idx, gate, counts, offsets, perm, slot_row, sched_reset)
   if (need <= 1) return MOE_SMALL(1);
   if (need <= 2) return MOE_SMALL(2);
   if (need <= 4) return MOE_SMALL(4);
@@ -242,7 +244,7 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   moe_status s;
   if (T <= kChunk) {
     s = launch_route_small(L, logits, T, logits_out, idx, gate, counts, offsets, perm, slot_row,
-                           nullptr, nullptr, sched_reset, st);
+                           sched_reset, st);
     if (s == MOE_OK && events &&
         cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -556,12 +558,12 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                          st)) != MOE_OK)
     return s;
   if ((s = mark(1)) != MOE_OK) return s;
-  // small batches: selection, permutation and the row gather in one launch
-  const bool fused_gather = (T <= kChunk) && c.dtype == MOE_BF16;
-  if (fused_gather) {
+  // small batches: selection and permutation in one launch
+  const bool fused_route = (T <= kChunk) && c.dtype == MOE_BF16;
+  if (fused_route) {
     if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
-                                offsets, perm, slot_row, x, at<void>(ws, W.xs),
-                                at<DevStatus>(ws, W.status)->sched, st)) != MOE_OK)
+                                offsets, perm, slot_row, at<DevStatus>(ws, W.status)->sched,
+                                st)) != MOE_OK)
       return s;
     if ((s = mark(2)) != MOE_OK) return s;
   } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
@@ -574,16 +576,18 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   if ((s = mark(3)) != MOE_OK) return s;
 
   if (c.dtype == MOE_BF16) {
+    const bool pair = use_pair(h, T);
+    // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
+    const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
+    // small token tiles: the up GEMM gathers its rows from x (no expert-sorted copy)
+    const bool gather_in_gemm = !pair && up_gathers_rows(c, T);
     const int vpr = c.d_model / 8;
-    if (!fused_gather &&
+    if (!gather_in_gemm &&
         (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk * vpr, 256, h->num_sms)),
                     dim3(256), 0, st, static_cast<const uint4 *>(x), (const int *)perm,
                     c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
       return s;
     if ((s = mark(4)) != MOE_OK) return s;
-    const bool pair = use_pair(h, T);
-    // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
-    const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
     const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
     __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
     float *ybuf = at<float>(ws, W.y);
@@ -591,9 +595,12 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     memset(&p1, 0, sizeof p1);
     p1.tmA0 = h->tm_wg;
     p1.tmA1 = h->tm_wu;
-    if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
-        !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn))
+    if (gather_in_gemm) {
+      if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
+    } else if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
+               !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
       return MOE_ERR_CUDA;
+    }
     p1.offsets = offsets;
     p1.perm = perm;
     p1.topk_gate = gate;
@@ -608,6 +615,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p1.K = c.d_model;
     p1.ld_out = c.d_ff;
     p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
+    p1.topk = c.top_k;
     if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
         MOE_OK)
       return s;

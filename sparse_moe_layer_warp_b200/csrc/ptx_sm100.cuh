@@ -150,6 +150,22 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m
       : "memory");
 }
 
+// Row gather: four rows r0..r3 of a 2-D map whose box is {box columns, 1 row}, columns
+// [c0, c0 + box columns) of each, written as four consecutive box rows at dst.  The 128-byte
+// swizzle of the map is a function of the shared-memory address, so rows written at
+// dst = tile + 4*i*128 (tile 1024-byte aligned) land exactly where a 4i..4i+3 row box
+// load would have put them.  Out-of-range coordinates read the map's fill value (zero).
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int r0, int r1, int r2, int r3,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -345,28 +345,23 @@ __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
 }
 
 // ------------------------------------------------------------------ small-T fused routing
-// T <= kChunk (decode): selection, gates, histogram, scan, permutation and (optionally) the
-// row gather in ONE launch.  Every CTA computes the selection and the permutation of all T
-// tokens (cheap, and identical in every CTA), CTA 0 writes the routing outputs, and the CTAs
-// split the gather xs[p, :] = x[perm[p] / k, :] between them.
+// T <= kChunk (decode): selection, gates, histogram, scan and permutation in ONE launch of
+// one CTA (the up GEMM gathers its token rows from x itself).
 template <int MAXV>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
     const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
     float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
     int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
-    int *__restrict__ slot_row, const uint4 *__restrict__ x, int vec_per_row,
-    uint4 *__restrict__ xs, int *__restrict__ sched_reset) {
+    int *__restrict__ slot_row, int *__restrict__ sched_reset) {
   griddep_wait();
   griddep_launch_dependents();
   // zero the grouped GEMMs' work counters for the launches that follow this one
-  if (sched_reset && blockIdx.x == 0 && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
+  if (sched_reset && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
   __shared__ int hist[kMaxExperts];
   __shared__ int off[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
   __shared__ int s_idx[kChunk * kMaxTopK];
-  __shared__ int s_perm[kChunk * kMaxTopK];
   __shared__ int warp_sum[32];
-  const bool writer = blockIdx.x == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     hist[e] = 0;
@@ -378,27 +373,22 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
     int my_e;
     float my_gate;
     topk_token<MAXV>(logits + (size_t)t * E, bias, E, k,
-                     (writer && logits_out) ? logits_out + (size_t)t * E : nullptr, lane, my_e,
-                     my_gate);
+                     logits_out ? logits_out + (size_t)t * E : nullptr, lane, my_e, my_gate);
     if (lane < k) {
       s_idx[t * k + lane] = my_e;
       atomicAdd(&hist[my_e], 1);
       atomicOr(&bits[my_e][t >> 5], 1u << (t & 31));
-      if (writer) {
-        topk_idx[(size_t)t * k + lane] = my_e;
-        topk_gate[(size_t)t * k + lane] = my_gate;
-      }
+      topk_idx[(size_t)t * k + lane] = my_e;
+      topk_gate[(size_t)t * k + lane] = my_gate;
     }
   }
   __syncthreads();
   block_exclusive_scan(hist, off, E, warp_sum);
-  if (writer) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      counts[e] = hist[e];
-      offsets[e] = off[e];
-    }
-    if (threadIdx.x == 0) offsets[E] = T * k;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    counts[e] = hist[e];
+    offsets[e] = off[e];
   }
+  if (threadIdx.x == 0) offsets[E] = T * k;
   const int npair = T * k;
   for (int q = threadIdx.x; q < npair; q += blockDim.x) {
     const int t = q / k;
@@ -411,20 +401,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
       else if (w == (t >> 5)) rank += __popc(word & ((1u << (t & 31)) - 1u));
     }
     const int p = off[e] + rank;
-    s_perm[p] = q;
-    if (writer) {
-      perm[p] = q;
-      slot_row[q] = p;
-    }
-  }
-  if (!xs) return;
-  __syncthreads();
-  const size_t total = (size_t)npair * vec_per_row;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const int p = (int)(i / vec_per_row);
-    const int v = (int)(i % vec_per_row);
-    xs[i] = __ldg(x + (size_t)(s_perm[p] / k) * vec_per_row + v);
+    perm[p] = q;
+    slot_row[q] = p;
   }
 }
 
@@ -442,7 +420,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
   griddep_wait();
   griddep_launch_dependents();
   // zero the grouped GEMMs' work counters for the launches that follow this one
-  if (sched_reset && blockIdx.x == 0 && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
+  if (sched_reset && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
   __shared__ int s_tot[kMaxExperts];
   __shared__ int s_base[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
