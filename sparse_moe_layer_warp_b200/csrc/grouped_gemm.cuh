@@ -502,21 +502,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       float *wbuf = xbuf + q * 16 * 32;
       const int col_base = mt * kBM + q * 32;  // first output column of this warp
+      // TMEM loads run one 16-column chunk ahead of their use
+      uint32_t n0[16], n1[16];
+      tmem_ld16(taddr, n0);
+      if (MODE == MODE_UP) tmem_ld16(taddr + BN, n1);
       for (int c0 = 0; c0 < valid; c0 += 16) {
-        uint32_t v0[16];
+        uint32_t v0[16], v1[16];
+        if (MODE == MODE_UP) tmem_ld_wait_regs(n0, n1);
+        else tmem_ld_wait_regs(n0);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          v0[n] = n0[n];
+          v1[n] = n1[n];
+        }
+        if (c0 + 16 < valid) {
+          tmem_ld16(taddr + c0 + 16, n0);
+          if (MODE == MODE_UP) tmem_ld16(taddr + BN + c0 + 16, n1);
+        }
         float vals[16];
-        tmem_ld16(taddr + c0, v0);
         if (MODE == MODE_UP) {
-          uint32_t v1[16];
-          tmem_ld16(taddr + BN + c0, v1);
-          tmem_ld_wait();
 #pragma unroll
           for (int n = 0; n < 16; ++n)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
           store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
                              col_base, vals, wbuf, lane);
         } else if (MODE == MODE_DOWN) {
-          tmem_ld_wait();
           const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
 #pragma unroll
           for (int n4 = 0; n4 < 4; ++n4) {
@@ -529,7 +539,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
                             vals, wbuf, lane);
         } else {  // MODE_LOGITS: E need not be a multiple of 32, so scalar masked stores
-          tmem_ld_wait();
           if (col < p.M) {
 #pragma unroll
             for (int n = 0; n < 16; ++n) {

@@ -30,6 +30,10 @@ namespace moe {
 
 constexpr int kPairBM = 256;  // weight rows per unit (both CTAs)
 constexpr int kPairBN = 256;  // tokens per unit (both CTAs)
+// warps: 0 producer, 1 MMA (leader) / TMEM owner, 2..9 epilogue -- two per TMEM lane
+// quadrant (warp % 4), splitting a unit's 16-column chunks between them
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
 
 template <int MODE>
 struct PairCfg {
@@ -49,12 +53,12 @@ struct PairCfg {
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
            (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * kPairBN * 4 +
-           4 * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
+           kPairEpiWarps * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
   }
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
   using C = PairCfg<MODE>;
   constexpr int S = C::STAGES;
@@ -82,7 +86,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // [ACC_BUFS][BN], 16-byte aligned: read as float4
   float *row_scale = reinterpret_cast<float *>(
       (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
-  float *xbuf = row_scale + C::ACC_BUFS * BN;  // [4 warps][16][32] epilogue transposes
+  float *xbuf = row_scale + C::ACC_BUFS * BN;  // [8 warps][16][32] epilogue transposes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -99,14 +103,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < C::ACC_BUFS; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&tempty[a], 2 * kPairEpiWarps);  // one per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     for (int q = 0; q < kUnitQ; ++q) {
       mbar_init(&uq_full[q], 1);
       // readers of a published unit id: the leader's MMA thread and epilogue warps, the
-      // peer's producer and epilogue warps (1 + 4 + 1 + 4)
-      mbar_init(&uq_empty[q], 10);
+      // peer's producer and epilogue warps
+      mbar_init(&uq_empty[q], 2 + 2 * kPairEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -329,7 +333,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
-    const int q = warp & 3;
+    const int q = warp & 3;         // TMEM lane quadrant
+    const int eh = (warp - 2) >> 2;  // which of the quadrant's two warps: chunks 2i + eh
     const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t uq_empty_leader = mapa_shared(smem_u32(&uq_empty[0]), 0);
     // lane 0 polls, the warp follows (uniform path into the warp-wide tcgen05.ld)
@@ -371,30 +376,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row0 = grp_row[g] + nt * BN;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
       if (MODE == MODE_DOWN) {
-        for (int n = threadIdx.x - 64; n < BN; n += 128) {
+        for (int n = threadIdx.x - 64; n < BN; n += 32 * kPairEpiWarps) {
           float sc = 0.f;
           if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
           row_scale[acc * BN + n] = sc;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kPairEpiWarps);
       }
-      float *wbuf = xbuf + q * 16 * 32;
+      float *wbuf = xbuf + (warp - 2) * 16 * 32;
       const int col_base = mt * kPairBM + (int)rank * 128 + q * 32;
-      for (int c0 = 0; c0 < valid; c0 += 16) {
-        uint32_t v0[16];
+      // TMEM loads run one 16-column chunk ahead of their use
+      uint32_t n0[16], n1[16];
+      const int c_first = 16 * eh;
+      if (c_first < valid) {
+        tmem_ld16(taddr + c_first, n0);
+        if (MODE == MODE_UP) tmem_ld16(taddr + BN + c_first, n1);
+      }
+      for (int c0 = c_first; c0 < valid; c0 += 32) {
+        uint32_t v0[16], v1[16];
+        if (MODE == MODE_UP) tmem_ld_wait_regs(n0, n1);
+        else tmem_ld_wait_regs(n0);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          v0[n] = n0[n];
+          v1[n] = n1[n];
+        }
+        if (c0 + 32 < valid) {
+          tmem_ld16(taddr + c0 + 32, n0);
+          if (MODE == MODE_UP) tmem_ld16(taddr + BN + c0 + 32, n1);
+        }
         float vals[16];
-        tmem_ld16(taddr + c0, v0);
         if (MODE == MODE_UP) {
-          uint32_t v1[16];
-          tmem_ld16(taddr + BN + c0, v1);
-          tmem_ld_wait();
 #pragma unroll
           for (int n = 0; n < 16; ++n)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
           store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
                              col_base, vals, wbuf, lane);
         } else {
-          tmem_ld_wait();
           const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
 #pragma unroll
           for (int n4 = 0; n4 < 4; ++n4) {

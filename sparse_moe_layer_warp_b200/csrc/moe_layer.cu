@@ -324,7 +324,7 @@ int pair_grid_size(const moe_layer *L) {
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3(L->num_sms & ~1);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -346,7 +346,7 @@ moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   const int grid = L->pair_grid[MODE == MODE_UP ? 0 : 1];
-  return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(kGemmThreads), smem, st, 2,
+  return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(kPairThreads), smem, st, 2,
                    p);
 }
 
@@ -583,7 +583,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     const bool gather_in_gemm = !pair && up_gathers_rows(c, T);
     const int vpr = c.d_model / 8;
     if (!gather_in_gemm &&
-        (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk * vpr, 256, h->num_sms)),
+        (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)),
                     dim3(256), 0, st, static_cast<const uint4 *>(x), (const int *)perm,
                     c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
       return s;

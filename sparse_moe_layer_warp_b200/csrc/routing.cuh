@@ -506,20 +506,22 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
 }
 
 // ------------------------------------------------------------------ row gather
-// xs[p, :] = x[perm[p] / k, :] for p < n_rows (16-byte vectors, grid-stride).
+// xs[p, :] = x[perm[p] / k, :] for p < n_rows: one warp per row (16-byte vectors, each lane
+// keeping several loads in flight), rows spread over all warps of the grid.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
                                                           const int *__restrict__ perm, int k,
                                                           int n_rows, int vec_per_row,
                                                           uint4 *__restrict__ xs) {
   griddep_wait();
   griddep_launch_dependents();
-  const size_t total = (size_t)n_rows * vec_per_row;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const int p = (int)(i / vec_per_row);
-    const int v = (int)(i % vec_per_row);
+  const int lane = threadIdx.x & 31;
+  const int n_warps = gridDim.x * (blockDim.x >> 5);
+  for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < n_rows; p += n_warps) {
     const int t = __ldg(perm + p) / k;
-    xs[i] = __ldg(x + (size_t)t * vec_per_row + v);
+    const uint4 *__restrict__ src = x + (size_t)t * vec_per_row;
+    uint4 *__restrict__ dst = xs + (size_t)p * vec_per_row;
+#pragma unroll 4
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
   }
 }
 

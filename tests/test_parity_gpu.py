@@ -78,6 +78,11 @@ SMALL = [
     ("tiny_fp32", {"dtype": "bf16", "T": 200, "d": 256, "E": 48, "k": 4, "f": 128,
                    "bias": "zipf", "n_shared": 0, "routed_scale": 1.5}),
     ("tiny_fp32", {"dtype": "bf16", "T": 1, "d": 256, "E": 288, "k": 8, "f": 128}),
+    # d = 128: one weight tile of d, half a combine segment
+    ("tiny_fp32", {"dtype": "bf16", "T": 96, "d": 128, "E": 16, "k": 4, "f": 128, "seed": 8}),
+    # a single contribution per token (dense FFN form): no averaging of rounding errors
+    ("tiny_fp32", {"dtype": "bf16", "T": 64, "d": 256, "E": 1, "k": 1, "f": 512, "seed": 9,
+                   "n_shared": 0}),
 ]
 
 
