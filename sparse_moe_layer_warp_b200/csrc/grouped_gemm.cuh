@@ -20,8 +20,10 @@
 //               copy of x); larger tiles load expert-sorted rows xs written by the gather
 //               kernel, and the shared group reads x directly.  (Gathering 128-row tiles,
 //               32 gather4 copies per stage, measured 1.6x slower than the row box.)
-//   MODE_LOGITS: router logits; one group (all T tokens), A0 = W_r (rows past E zero-filled
-//               by TMA), B = x; epilogue logits[t, e] = acc (fp32).
+//   MODE_LOGITS: router logits, fp32 out[t, e].  out_trans = 0: one group of all T tokens,
+//               A0 = W_r (rows past E zero-filled by TMA), B = x.  out_trans = 1 (many
+//               tokens): A0 = x (128 tokens per unit), one "group" of all E experts as B = W_r,
+//               so x is streamed about once and no MMA rows are spent on padding experts.
 //   MODE_DOWN : A0 = W_down, B = h rows; epilogue y = acc * scale -> fp32, scale =
 //               routed_scale * gate for routed rows and 1 for shared rows.  y stays fp32:
 //               rounding it to bf16 as well as h and the output would put the layer's
@@ -64,6 +66,7 @@ struct GemmParams {
   int ld_out; // f (UP), d (DOWN), E (LOGITS)
   int *sched;  // work counter (zero at launch) for dynamic unit claiming; null: round-robin
   int topk;    // k (UP: token of routed sorted row q = perm[q] / k)
+  int out_trans;  // LOGITS: 0 = A is W_r (experts on M), 1 = A is x (tokens on M, B = W_r)
 };
 
 constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
                             vals, wbuf, lane);
-        } else {  // MODE_LOGITS: E need not be a multiple of 32, so scalar masked stores
+        } else if (!p.out_trans) {  // MODE_LOGITS, experts on M: scalar masked stores
           if (col < p.M) {
 #pragma unroll
             for (int n = 0; n < 16; ++n) {
@@ -546,6 +549,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 static_cast<float *>(p.out)[(size_t)(row0 + c0 + n) * p.ld_out + col] =
                     __uint_as_float(v0[n]);
             }
+          }
+        } else if (col < p.M) {  // MODE_LOGITS, tokens on M: lane = token, 16 experts
+          float *dst = static_cast<float *>(p.out) + (size_t)col * p.ld_out + row0 + c0;
+          if ((p.ld_out & 3) == 0 && c0 + 16 <= valid) {
+#pragma unroll
+            for (int n4 = 0; n4 < 4; ++n4)
+              reinterpret_cast<float4 *>(dst)[n4] =
+                  make_float4(__uint_as_float(v0[4 * n4]), __uint_as_float(v0[4 * n4 + 1]),
+                              __uint_as_float(v0[4 * n4 + 2]), __uint_as_float(v0[4 * n4 + 3]));
+          } else {
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+              if (c0 + n < valid) dst[n] = __uint_as_float(v0[n]);
           }
         }
       }

@@ -288,9 +288,7 @@ moe_status launch_gemm(const moe_layer *L, int bn, const GemmParams &p, cudaStre
     case 32: return launch_gemm_bn<MODE, 32>(L, p, st);
     case 64: return launch_gemm_bn<MODE, 64>(L, p, st);
   }
-  if constexpr (MODE != MODE_LOGITS) {
-    if (bn == 128) return launch_gemm_bn<MODE, 128>(L, p, st);
-  }
+  if (bn == 128) return launch_gemm_bn<MODE, 128>(L, p, st);
   if constexpr (MODE == MODE_DOWN) {
     if (bn == 256) return launch_gemm_bn<MODE, 256>(L, p, st);
   }
@@ -353,12 +351,31 @@ moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_
 // Token tile of the router GEMM.
 int pick_bn_router(int T) { return T <= 256 ? 16 : (T <= 1024 ? 32 : 64); }
 
+// From this many tokens the router GEMM puts tokens on M (see MODE_LOGITS, out_trans).
+constexpr int kRouterTokensOnM = 1024;
+
 moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *logits,
                               DevStatus *status, cudaStream_t st) {
   const moe_config &c = L->cfg;
-  const int bn = pick_bn_router(T);
   GemmParams p;
   memset(&p, 0, sizeof p);
+  if (T >= kRouterTokensOnM) {
+    // tokens on M (128 per unit), the E experts as the N side in tiles of 128
+    if (!encode_bf16_2d(&p.tmA0, x, c.d_model, T, kBM)) return MOE_ERR_CUDA;
+    p.tmB = L->tm_wr;  // box {64, 128}: 128 experts per tile, rows past E zero-filled
+    p.out = logits;
+    p.status = status;
+    p.E = 0;  // one group of E "rows": the experts
+    p.n_groups = 1;
+    p.T = c.n_experts;
+    p.Tk = 0;
+    p.M = T;
+    p.K = c.d_model;
+    p.ld_out = c.n_experts;
+    p.out_trans = 1;
+    return launch_gemm<MODE_LOGITS>(L, 128, p, st);
+  }
+  const int bn = pick_bn_router(T);
   p.tmA0 = L->tm_wr;
   if (!encode_bf16_2d(&p.tmB, x, c.d_model, T, bn)) return MOE_ERR_CUDA;
   p.out = logits;
