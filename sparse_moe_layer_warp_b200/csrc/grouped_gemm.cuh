@@ -67,6 +67,12 @@ struct GemmParams {
   int *sched;  // work counter (zero at launch) for dynamic unit claiming; null: round-robin
   int topk;    // k (UP: token of routed sorted row q = perm[q] / k)
   int out_trans;  // LOGITS: 0 = A is W_r (experts on M), 1 = A is x (tokens on M, B = W_r)
+  // Per-group hand-over of h from the up kernel to the down kernel (null: none).  UP: each
+  // epilogue warp adds 1 to done[g] once its rows of h for group g are stored.  DOWN: the
+  // kernel does not wait for the up kernel to finish; before loading h rows of group g it
+  // waits until done[g] = 4 * done_mt * (token tiles of g at done_bn tokens).
+  int *done;
+  int done_mt, done_bn;
 };
 
 constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
@@ -220,8 +226,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   // Programmatic dependent launch: the set-up above overlaps the previous kernel's tail;
   // the expert offsets, the token rows and the outputs may all belong to it, so everything
-  // below waits for it to complete.
-  griddep_wait();
+  // below waits for it to complete.  A down kernel with the per-group hand-over (p.done)
+  // only reads what the routing kernel wrote, complete before the up kernel (its
+  // predecessor) could let it launch, and h, which it takes group by group through done[].
+  if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
   // group table: token count, first row in the sorted space, units per group
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -304,7 +312,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     int qi = 0;
     uint32_t qph = 0;
-    int u = -1;  // lane 0's claim cursor
+    int u = -1;             // lane 0's claim cursor
+    int ready_group = -1;   // lane 0, down kernel: group whose h is known to be complete
     for (;;) {
       int uid = -1;
       if (lane == 0) {
@@ -344,6 +353,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int q = b_row + ((pos < valid) ? pos : 0);
           if (4 * lane < n_rows) tok[i] = (g < p.E) ? p.perm[q] / p.topk : q - grp_row[g];
         }
+      }
+      if (MODE == MODE_DOWN && p.done) {
+        if (lane == 0 && g != ready_group) {
+          const int target = 4 * p.done_mt * ((grp_count[g] + p.done_bn - 1) / p.done_bn);
+          ok = counter_wait_bounded(p.done + g, target, abort_flag, p.status, 8);
+          fence_proxy_async_global();  // the h rows are read through TMA below
+          ready_group = g;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
       }
       const uint32_t stage_bytes = C::NA * C::A_BYTES + (uint32_t)n_rows * kBK * 2;
       // a weight tile read by one unit only is streamed with evict-first priority; one
@@ -563,6 +582,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int n = 0; n < 16; ++n)
               if (c0 + n < valid) dst[n] = __uint_as_float(v0[n]);
           }
+        }
+      }
+      if (MODE == MODE_UP && p.done) {
+        // publish this warp's rows of h for group g: stores, then a release of the count
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(p.done + g, 1);
         }
       }
       tc_fence_before();

@@ -119,7 +119,7 @@ size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 // Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
 struct WsLayout {
   size_t status, logits, part, idx, gate, counts, offsets, perm, slot_row, chunk_hist, stats,
-      xs, h, y, total;
+      xs, h, y, done, total;
 };
 
 int pick_bn(const moe_config &c, int T, int mode);
@@ -155,6 +155,7 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.xs = (c.dtype == MOE_BF16 && !up_gathers_rows(c, T)) ? take(Tk * c.d_model * 2) : off;
   L.h = take(P * c.d_ff * esize(c));
   L.y = take(P * c.d_model * 4);  // fp32 in both precisions
+  L.done = take(((size_t)c.n_experts + c.n_shared) * 4);  // per-group up completion counts
   L.total = off;
   return L;
 }
@@ -214,14 +215,14 @@ moe_status launch_logits(const moe_layer *L, const void *x, int T, float *logits
 // T <= kChunk: selection and permutation in one launch of one CTA.
 moe_status launch_route_small(const moe_layer *L, const float *logits, int T, float *logits_out,
                               int *idx, float *gate, int *counts, int *offsets, int *perm,
-                              int *slot_row, int *sched_reset, cudaStream_t st) {
+                              int *slot_row, CounterReset reset, cudaStream_t st) {
   const moe_config &c = L->cfg;
   const int need = (c.n_experts + 31) / 32;
   const float *bias = L->w.router_bias;
   const dim3 thr(kRouteWarps * 32);
 #define MOE_SMALL(V)                                                                         \
   launch(route_small_kernel<V>, dim3(1), thr, 0, st, logits, bias, T, c.n_experts, c.top_k, \
-         logits_out, idx, gate, counts, offsets, perm, slot_row, sched_reset)
+         logits_out, idx, gate, counts, offsets, perm, slot_row, reset)
   if (need <= 1) return MOE_SMALL(1);
   if (need <= 2) return MOE_SMALL(2);
   if (need <= 4) return MOE_SMALL(4);
@@ -234,7 +235,7 @@ moe_status launch_route_small(const moe_layer *L, const float *logits, int T, fl
 moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
                                  float *logits_out, int *idx, float *gate, int *counts,
                                  int *offsets, int *perm, int *slot_row, int *chunk_hist,
-                                 int *sched_reset, cudaStream_t st,
+                                 CounterReset reset, cudaStream_t st,
                                  void *const *events = nullptr, int mark_index = 0) {
   const moe_config &c = L->cfg;
   const int nch = (T + kChunk - 1) / kChunk;
@@ -244,7 +245,7 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   moe_status s;
   if (T <= kChunk) {
     s = launch_route_small(L, logits, T, logits_out, idx, gate, counts, offsets, perm, slot_row,
-                           sched_reset, st);
+                           reset, st);
     if (s == MOE_OK && events &&
         cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -264,7 +265,7 @@ moe_status launch_select_permute(const moe_layer *L, const float *logits, int T,
   if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[mark_index]), st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch(permute_scatter_kernel, dim3(nch), dim3(256), 0, st, idx, chunk_hist, T,
-                c.n_experts, c.top_k, nch, counts, offsets, perm, slot_row, sched_reset);
+                c.n_experts, c.top_k, nch, counts, offsets, perm, slot_row, reset);
 }
 
 // ------------------------------------------------------------------ grouped GEMM launch
@@ -526,7 +527,7 @@ static moe_status route_common(moe_handle h, const void *x, const float *logits_
   }
   return launch_select_permute(h, logits, T, copy_out, idx, gate, counts, offsets, perm,
                                slot_row, at<int>(ws, W.chunk_hist),
-                               at<DevStatus>(ws, W.status)->sched, st);
+                               CounterReset{at<DevStatus>(ws, W.status)->sched, nullptr, 0}, st);
 }
 
 moe_status moe_route(moe_handle h, const void *x, int n_tokens, float *logits_out,
@@ -575,18 +576,19 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                          st)) != MOE_OK)
     return s;
   if ((s = mark(1)) != MOE_OK) return s;
+  // the expert kernels' counters start from zero in every forward
+  const CounterReset reset{at<DevStatus>(ws, W.status)->sched, at<int>(ws, W.done),
+                           c.n_experts + c.n_shared};
   // small batches: selection and permutation in one launch
   const bool fused_route = (T <= kChunk) && c.dtype == MOE_BF16;
   if (fused_route) {
     if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
-                                offsets, perm, slot_row, at<DevStatus>(ws, W.status)->sched,
-                                st)) != MOE_OK)
+                                offsets, perm, slot_row, reset, st)) != MOE_OK)
       return s;
     if ((s = mark(2)) != MOE_OK) return s;
   } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
                                         at<int>(ws, W.counts), offsets, perm, slot_row,
-                                        at<int>(ws, W.chunk_hist),
-                                        at<DevStatus>(ws, W.status)->sched, st, events, 2)) !=
+                                        at<int>(ws, W.chunk_hist), reset, st, events, 2)) !=
              MOE_OK) {
     return s;
   }
@@ -633,6 +635,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p1.ld_out = c.d_ff;
     p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
     p1.topk = c.top_k;
+    // 1-CTA kernels: the down kernel starts on the SMs the up kernel leaves in its last wave
+    // and waits per expert group for that group's rows of h (see grouped_gemm_kernel)
+    if (!pair) p1.done = at<int>(ws, W.done);
     if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
         MOE_OK)
       return s;
@@ -645,6 +650,8 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p2.M = c.d_model;
     p2.K = c.d_ff;
     p2.ld_out = c.d_model;
+    p2.done_mt = c.d_ff / kBM;  // the up kernel's weight tiles per token tile
+    p2.done_bn = bn;            // and its token tile
     if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
                   : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
       return s;

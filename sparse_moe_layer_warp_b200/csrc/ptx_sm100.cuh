@@ -107,6 +107,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// Bounded wait until *ctr >= target (acquire, gpu scope).  Same limit and failure path as
+// mbar_wait_bounded.
+__device__ __forceinline__ bool counter_wait_bounded(const int *ctr, int target,
+                                                     volatile int *abort_flag,
+                                                     DevStatus *status, int where) {
+  auto load = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    return v;
+  };
+  if (load() >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (load() >= target) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        if (status) {
+          atomicExch(&status->error, 1);
+          atomicExch(&status->where, where);
+        }
+        return false;
+      }
+    }
+  }
+}
+
+// Order this thread's earlier generic-proxy view of global memory before its later
+// async-proxy (TMA) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------- programmatic dependent launch
 // Kernels of one layer call are launched with programmatic stream serialisation: a kernel
 // may start while its predecessor drains, does its set-up, then waits here before it

@@ -14,6 +14,21 @@
 
 namespace moe {
 
+// Work counters of the expert kernels that follow a routing launch, zeroed by that launch
+// (block 0) so every forward starts from zero: the grouped GEMMs' unit counters (two ints)
+// and the fused FFN's per-group completion counts.
+struct CounterReset {
+  int *sched;  // [2] or null
+  int *done;   // [n_done] or null
+  int n_done;
+  __device__ __forceinline__ void apply() const {
+    if (blockIdx.x != 0) return;
+    if (sched && threadIdx.x < 2) sched[threadIdx.x] = 0;
+    if (done)
+      for (int i = threadIdx.x; i < n_done; i += blockDim.x) done[i] = 0;
+  }
+};
+
 constexpr int kMaxExperts = 1024;   // E limit of the routing kernels
 constexpr int kMaxTopK = 32;        // one slot per lane
 constexpr int kChunk = 64;          // tokens per routing chunk (one CTA)
@@ -352,11 +367,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
     const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
     float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
     int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
-    int *__restrict__ slot_row, int *__restrict__ sched_reset) {
+    int *__restrict__ slot_row, CounterReset reset) {
   griddep_wait();
   griddep_launch_dependents();
-  // zero the grouped GEMMs' work counters for the launches that follow this one
-  if (sched_reset && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
+  reset.apply();
   __shared__ int hist[kMaxExperts];
   __shared__ int off[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
@@ -416,11 +430,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
 __global__ void __launch_bounds__(256) permute_scatter_kernel(
     const int *__restrict__ topk_idx, const int *__restrict__ chunk_hist, int T, int E, int k,
     int n_chunks, int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
-    int *__restrict__ slot_row, int *__restrict__ sched_reset) {
+    int *__restrict__ slot_row, CounterReset reset) {
   griddep_wait();
   griddep_launch_dependents();
-  // zero the grouped GEMMs' work counters for the launches that follow this one
-  if (sched_reset && threadIdx.x < 2) sched_reset[threadIdx.x] = 0;
+  reset.apply();
   __shared__ int s_tot[kMaxExperts];
   __shared__ int s_base[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
