@@ -572,25 +572,40 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                                                                                  : MOE_ERR_CUDA;
   };
   if ((s = mark(0)) != MOE_OK) return s;
-  if ((s = launch_logits(h, x, T, logits, at<float>(ws, W.part), at<DevStatus>(ws, W.status),
-                         st)) != MOE_OK)
-    return s;
-  if ((s = mark(1)) != MOE_OK) return s;
   // the expert kernels' counters start from zero in every forward
   const CounterReset reset{at<DevStatus>(ws, W.status)->sched, at<int>(ws, W.done),
                            c.n_experts + c.n_shared};
-  // small batches: selection and permutation in one launch
-  const bool fused_route = (T <= kChunk) && c.dtype == MOE_BF16;
-  if (fused_route) {
-    if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
-                                offsets, perm, slot_row, reset, st)) != MOE_OK)
+  // decode: router logits, selection and permutation in one launch
+  const bool decode_route = T <= kChunk && c.dtype == MOE_BF16 &&
+                            c.n_experts <= kDecodeMaxExperts && c.d_model % 64 == 0 &&
+                            c.d_model <= kDecodeMaxD;
+  // other small batches: selection and permutation in one launch after the router
+  const bool small_route = !decode_route && T <= kChunk && c.dtype == MOE_BF16;
+  if (decode_route) {
+    if ((s = launch(route_decode_kernel, dim3((c.n_experts + kDecodeEPC - 1) / kDecodeEPC),
+                    dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(x),
+                    static_cast<const __nv_bfloat16 *>(h->w.w_router), h->w.router_bias, T,
+                    c.d_model, c.n_experts, c.top_k, logits, idx, gate, at<int>(ws, W.counts),
+                    offsets, perm, slot_row, &at<DevStatus>(ws, W.status)->router_ticket[31],
+                    reset)) != MOE_OK)
       return s;
-    if ((s = mark(2)) != MOE_OK) return s;
-  } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
-                                        at<int>(ws, W.counts), offsets, perm, slot_row,
-                                        at<int>(ws, W.chunk_hist), reset, st, events, 2)) !=
-             MOE_OK) {
-    return s;
+    if ((s = mark(1)) != MOE_OK || (s = mark(2)) != MOE_OK) return s;
+  } else {
+    if ((s = launch_logits(h, x, T, logits, at<float>(ws, W.part), at<DevStatus>(ws, W.status),
+                           st)) != MOE_OK ||
+        (s = mark(1)) != MOE_OK)
+      return s;
+    if (small_route) {
+      if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
+                                  offsets, perm, slot_row, reset, st)) != MOE_OK ||
+          (s = mark(2)) != MOE_OK)
+        return s;
+    } else if ((s = launch_select_permute(h, logits, T, nullptr, idx, gate,
+                                          at<int>(ws, W.counts), offsets, perm, slot_row,
+                                          at<int>(ws, W.chunk_hist), reset, st, events, 2)) !=
+               MOE_OK) {
+      return s;
+    }
   }
   if ((s = mark(3)) != MOE_OK) return s;
 

@@ -17,7 +17,8 @@ struct DevStatus {
   int where;             // which wait (kernel-specific code)
   int sched[4];          // grouped-GEMM work counters (up, down), reset by the routing kernels
   int pad[26];
-  int router_ticket[32]; // split-K router: arrivals per block of 32 experts (self-resetting)
+  int router_ticket[32]; // split-K router: arrivals per block of 32 experts; [31] also the
+                         // decode router's last-CTA ticket (all self-resetting)
 };
 
 // Time limit of every device-side spin wait (ns of %globaltimer).

@@ -22,7 +22,9 @@ struct CounterReset {
   int *done;   // [n_done] or null
   int n_done;
   __device__ __forceinline__ void apply() const {
-    if (blockIdx.x != 0) return;
+    if (blockIdx.x == 0) run();
+  }
+  __device__ __forceinline__ void run() const {  // by the whole of one CTA
     if (sched && threadIdx.x < 2) sched[threadIdx.x] = 0;
     if (done)
       for (int i = threadIdx.x; i < n_done; i += blockDim.x) done[i] = 0;
@@ -238,14 +240,21 @@ __device__ __forceinline__ void topk_token(const float *__restrict__ lrow,
                                            float *__restrict__ lout, int lane, int &my_e,
                                            float &my_gate) {
   uint32_t key[MAXV];
-  float l[MAXV];
+  float l[MAXV], b[MAXV];
+  // all loads first (clamped addresses, no branches), so they are in flight together;
+  // L2-coherent logits loads: they may be this kernel's own output
+#pragma unroll
+  for (int v = 0; v < MAXV; ++v) {
+    const int e = min(lane + 32 * v, E - 1);
+    l[v] = __ldcg(lrow + e);
+    b[v] = bias ? __ldg(bias + e) : 0.f;
+  }
 #pragma unroll
   for (int v = 0; v < MAXV; ++v) {
     const int e = lane + 32 * v;
     if (e < E) {
-      l[v] = lrow[e];
       if (lout) lout[e] = l[v];
-      key[v] = score_key(l[v] + (bias ? bias[e] : 0.f));
+      key[v] = score_key(l[v] + b[v]);
     } else {
       l[v] = 0.f;
       key[v] = 0u;  // ties with NaN scores and loses on id (all ids here are >= E)
@@ -360,30 +369,28 @@ __global__ void __launch_bounds__(kRouteWarps * 32) topk_hist_kernel(
 }
 
 // ------------------------------------------------------------------ small-T fused routing
-// T <= kChunk (decode): selection, gates, histogram, scan and permutation in ONE launch of
-// one CTA (the up GEMM gathers its token rows from x itself).
+// T <= kChunk (decode): selection, gates, histogram, scan and permutation of all T tokens by
+// one CTA (any multiple of 32 threads; one warp per token).
 template <int MAXV>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
+__device__ __forceinline__ void route_small_block(
     const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
     float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
     int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
-    int *__restrict__ slot_row, CounterReset reset) {
-  griddep_wait();
-  griddep_launch_dependents();
-  reset.apply();
+    int *__restrict__ slot_row) {
   __shared__ int hist[kMaxExperts];
   __shared__ int off[kMaxExperts];
   __shared__ uint32_t bits[kMaxExperts][kChunk / 32];
   __shared__ int s_idx[kChunk * kMaxTopK];
   __shared__ int warp_sum[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_warps = blockDim.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     hist[e] = 0;
 #pragma unroll
     for (int w = 0; w < kChunk / 32; ++w) bits[e][w] = 0u;
   }
   __syncthreads();
-  for (int t = warp; t < T; t += kRouteWarps) {
+  for (int t = warp; t < T; t += n_warps) {
     int my_e;
     float my_gate;
     topk_token<MAXV>(logits + (size_t)t * E, bias, E, k,
@@ -418,6 +425,141 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
     perm[p] = q;
     slot_row[q] = p;
   }
+}
+
+template <int MAXV>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
+    const float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k,
+    float *__restrict__ logits_out, int *__restrict__ topk_idx, float *__restrict__ topk_gate,
+    int *__restrict__ counts, int *__restrict__ offsets, int *__restrict__ perm,
+    int *__restrict__ slot_row, CounterReset reset) {
+  griddep_wait();
+  griddep_launch_dependents();
+  reset.apply();
+  route_small_block<MAXV>(logits, bias, T, E, k, logits_out, topk_idx, topk_gate, counts,
+                          offsets, perm, slot_row);
+}
+
+// ------------------------------------------------------------ decode: router + routing
+// T <= kChunk tokens, bf16, E <= kDecodeMaxExperts, d a multiple of 64 and at most
+// kDecodeMaxD: the router logits and the routing in ONE launch.  CTA c computes experts
+// e0 = kDecodeEPC*c .. +kDecodeEPC over the full reduction: warp w takes the K slice
+// [w*d/8, (w+1)*d/8), each lane 16-byte chunks of it (the CTA's router rows are loaded
+// before the grid-dependency wait: they never depend on earlier kernels); per group of 16
+// tokens the 32 (expert, token) partial sums of a lane are summed across the warp by a
+// butterfly that leaves sum j in lane j (31 shuffles), then across the 8 warps in a fixed
+// order -- fp32 throughout, deterministic.  The CTA that finishes last (a ticket, reset by
+// that CTA) then runs route_small_block on all logits.
+constexpr int kDecodeEPC = 2;          // experts per CTA
+constexpr int kDecodeMaxExperts = 288; // MAXV = 9 top-k and at most 144 CTAs
+constexpr int kDecodeMaxD = 8192;      // at most 4 chunks of 8 per lane
+
+__device__ __forceinline__ float dot8_bf16(const uint4 a, const uint4 b) {
+  const __nv_bfloat162 *pa = reinterpret_cast<const __nv_bfloat162 *>(&a);
+  const __nv_bfloat162 *pb = reinterpret_cast<const __nv_bfloat162 *>(&b);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 fa = __bfloat1622float2(pa[i]);
+    const float2 fb = __bfloat1622float2(pb[i]);
+    s = fmaf(fa.x, fb.x, s);
+    s = fmaf(fa.y, fb.y, s);
+  }
+  return s;
+}
+
+__global__ void __launch_bounds__(256) route_decode_kernel(
+    const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
+    const float *__restrict__ bias, int T, int d, int E, int k, float *__restrict__ logits,
+    int *__restrict__ topk_idx, float *__restrict__ topk_gate, int *__restrict__ counts,
+    int *__restrict__ offsets, int *__restrict__ perm, int *__restrict__ slot_row,
+    int *__restrict__ ticket, CounterReset reset) {
+  constexpr int EPC = kDecodeEPC, TG = 16, MAXC = kDecodeMaxD / 64 / 32;
+  static_assert(EPC * TG == 32, "one butterfly value per lane");
+  __shared__ float red[8][32];
+  __shared__ int s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * EPC;
+  const int slice = d / 8;         // this warp's K range
+  const int chunks = slice / 8;    // 16-byte chunks in it
+  uint4 w[MAXC][EPC];
+#pragma unroll
+  for (int ci = 0; ci < MAXC; ++ci) {
+    const int c = lane + 32 * ci;
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      w[ci][e] = make_uint4(0u, 0u, 0u, 0u);
+      if (c < chunks && e0 + e < E)
+        w[ci][e] = __ldg(reinterpret_cast<const uint4 *>(wr + (size_t)(e0 + e) * d +
+                                                         warp * slice + c * 8));
+    }
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int tg = 0; tg < T; tg += TG) {
+    float a[EPC * TG];  // value j = e * TG + t
+#pragma unroll
+    for (int j = 0; j < EPC * TG; ++j) a[j] = 0.f;
+    // tokens past T read token T-1 (clamped, so the loads are unconditional and issue
+    // together); their sums are never stored
+#pragma unroll
+    for (int ci = 0; ci < MAXC; ++ci) {
+      const int c = lane + 32 * ci;
+      if (ci * 32 < chunks) {  // warp-uniform
+        const int cc = min(c, chunks - 1);
+#pragma unroll
+        for (int t0 = 0; t0 < TG; t0 += 8) {
+          uint4 xv[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            xv[t] = __ldg(reinterpret_cast<const uint4 *>(
+                x + (size_t)min(tg + t0 + t, T - 1) * d + warp * slice + cc * 8));
+          if (c < chunks) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+#pragma unroll
+              for (int e = 0; e < EPC; ++e) a[e * TG + t0 + t] += dot8_bf16(xv[t], w[ci][e]);
+          }
+        }
+      }
+    }
+    // butterfly: after the step with offset o a lane keeps the half of its 2o values whose
+    // index bit matches its lane bit, so lane j ends with the warp's sum of value j
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const float send = upper ? a[i] : a[i + o];
+        const float keep = upper ? a[i + o] : a[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    red[warp][lane] = a[0];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float v = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) v += red[ww][threadIdx.x];
+      const int e = threadIdx.x / TG, t = threadIdx.x % TG;
+      if (tg + t < T && e0 + e < E) logits[(size_t)(tg + t) * E + e0 + e] = v;
+    }
+    __syncthreads();
+  }
+  // the last CTA to finish its experts routes all tokens
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int v = atomicAdd(ticket, 1);
+    s_last = (v == (int)gridDim.x - 1);
+    if (s_last) *ticket = 0;  // ready for the next call
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  reset.run();
+  route_small_block<9>(logits, bias, T, E, k, nullptr, topk_idx, topk_gate, counts, offsets,
+                       perm, slot_row);
 }
 
 // ------------------------------------------------------------------ permutation (scatter)
