@@ -164,6 +164,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from sparse_moe_layer_warp_b200 import (MOE_PROFILE_STAGES, PROFILE_STAGE_NAMES, MoELayer,
+                                            moe_forward_launch_count,
                                             moe_forward, moe_forward_profiled, synth)
 
     torch.cuda.set_device(local_rank)
@@ -302,7 +303,8 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(job_throughput(T, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4)),
                 "d2h_bytes_per_step": int(T * w.d * (2 if w.dtype == "bf16" else 4))},
-        "gpu_launches": int(world * args.steps * (7 if w.dtype == "bf16" else 6)),
+        # kernels of the timed region: every rank's forwards, as the library plans them
+        "gpu_launches": int(world * args.steps * moe_forward_launch_count(layer.handle, T)),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -133,12 +133,18 @@ moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, voi
  *   4 row gather (bf16 with more than about 12 tokens per expert; otherwise empty, the
  *   expert-up kernel gathering the rows of x as it loads them), 5 expert up + SwiGLU,
  *   6 expert down, 7 combine.
- *   For n_tokens <= 64 stages 2-3 are one fused launch, timed as stage 2 (3 empty).
+ *   For n_tokens <= 64 (bf16) stages 2-3 are one fused launch, timed as stage 2 (3 empty);
+ *   with at most 288 experts and d_model <= 8192 stages 1-3 are one launch, timed as stage 1.
  * n_events must be at least MOE_PROFILE_STAGES + 1; otherwise MOE_ERR_INVALID_ARG. */
 #define MOE_PROFILE_STAGES 7
 moe_status moe_forward_profiled(moe_handle h, const void *x, int n_tokens, void *out,
                                 void *ws, size_t ws_bytes, void *stream, void *const *events,
                                 int n_events);
+
+/* Number of kernel launches one moe_forward of n_tokens tokens makes on the handle's
+ * configuration (the launch plan depends on n_tokens); -1 for a null handle or n_tokens
+ * outside [0, max_tokens].  No device work. */
+int moe_forward_launch_count(moe_handle h, int n_tokens);
 
 /* Waits for `stream`, then reads and clears the workspace's device status word:
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     moe_device_status,
     moe_forward,
     moe_forward_profiled,
+    moe_forward_launch_count,
     MOE_PROFILE_STAGES,
     PROFILE_STAGE_NAMES,
     moe_layer_destroy,

@@ -29,7 +29,7 @@ MOE_BF16 = 1
 EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_workspace_init",
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
            "moe_device_status", "moe_status_string", "moe_router_logits_static",
-           "moe_router_stats", "moe_update_router_bias")
+           "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -80,6 +80,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_router_logits_static.argtypes = [P, P, I, P, P]
         lib.moe_router_stats.argtypes = [P, P, P, I, I, P, P, P, P, Z, P]
         lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
+        lib.moe_forward_launch_count.argtypes = [P, I]
+        lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
@@ -153,6 +155,11 @@ def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
     _check("moe_forward", load_library().moe_forward(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_forward_launch_count(handle, n_tokens: int) -> int:
+    """Kernel launches of one moe_forward of n_tokens tokens (-1: invalid arguments)."""
+    return int(load_library().moe_forward_launch_count(handle, int(n_tokens)))
 
 
 def moe_forward_profiled(handle, x, n_tokens, out, ws, events, stream=None) -> None:

@@ -547,6 +547,44 @@ moe_status moe_route_from_logits(moe_handle h, const float *logits, int n_tokens
                       expert_counts, expert_offsets, perm, slot_row, ws, ws_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+// Which kernels a forward of T tokens runs (shared by forward_impl and the launch count).
+struct ForwardPlan {
+  bool decode_route;  // router logits + selection + permutation in one launch
+  bool small_route;   // selection + permutation in one launch after the router
+  bool pair;          // CTA-pair grouped GEMMs
+  bool gather_in_gemm;  // the up GEMM gathers x rows itself (no gather launch)
+  int launches;
+};
+
+ForwardPlan plan_forward(const moe_layer *L, int T) {
+  const moe_config &c = L->cfg;
+  ForwardPlan f;
+  f.decode_route = T <= kChunk && c.dtype == MOE_BF16 && c.n_experts <= kDecodeMaxExperts &&
+                   c.d_model % 64 == 0 && c.d_model <= kDecodeMaxD;
+  f.small_route = !f.decode_route && T <= kChunk;
+  f.pair = c.dtype == MOE_BF16 && use_pair(L, T);
+  f.gather_in_gemm = c.dtype == MOE_BF16 && !f.pair && up_gathers_rows(c, T);
+  if (T == 0) {
+    f.launches = 0;
+    return f;
+  }
+  const int routing = f.decode_route ? 1 : (f.small_route ? 2 : 3);
+  const int gather = (c.dtype == MOE_BF16 && !f.gather_in_gemm) ? 1 : 0;
+  f.launches = routing + gather + 3;  // + up, down, combine
+  return f;
+}
+}  // namespace
+
+extern "C" {
+
+int moe_forward_launch_count(moe_handle h, int n_tokens) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return -1;
+  return plan_forward(h, n_tokens).launches;
+}
+
 static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
                                size_t ws_bytes, void *stream, void *const *events) {
   moe_status s = check_call(h, n_tokens, ws, ws_bytes);
@@ -575,13 +613,8 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   // the expert kernels' counters start from zero in every forward
   const CounterReset reset{at<DevStatus>(ws, W.status)->sched, at<int>(ws, W.done),
                            c.n_experts + c.n_shared};
-  // decode: router logits, selection and permutation in one launch
-  const bool decode_route = T <= kChunk && c.dtype == MOE_BF16 &&
-                            c.n_experts <= kDecodeMaxExperts && c.d_model % 64 == 0 &&
-                            c.d_model <= kDecodeMaxD;
-  // other small batches: selection and permutation in one launch after the router
-  const bool small_route = !decode_route && T <= kChunk && c.dtype == MOE_BF16;
-  if (decode_route) {
+  const ForwardPlan plan = plan_forward(h, T);
+  if (plan.decode_route) {
     if ((s = launch(route_decode_kernel, dim3((c.n_experts + kDecodeEPC - 1) / kDecodeEPC),
                     dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(x),
                     static_cast<const __nv_bfloat16 *>(h->w.w_router), h->w.router_bias, T,
@@ -595,7 +628,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                            st)) != MOE_OK ||
         (s = mark(1)) != MOE_OK)
       return s;
-    if (small_route) {
+    if (plan.small_route) {
       if ((s = launch_route_small(h, logits, T, nullptr, idx, gate, at<int>(ws, W.counts),
                                   offsets, perm, slot_row, reset, st)) != MOE_OK ||
           (s = mark(2)) != MOE_OK)
@@ -610,11 +643,11 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   if ((s = mark(3)) != MOE_OK) return s;
 
   if (c.dtype == MOE_BF16) {
-    const bool pair = use_pair(h, T);
+    const bool pair = plan.pair;
     // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
     const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
     // small token tiles: the up GEMM gathers its rows from x (no expert-sorted copy)
-    const bool gather_in_gemm = !pair && up_gathers_rows(c, T);
+    const bool gather_in_gemm = plan.gather_in_gemm;
     const int vpr = c.d_model / 8;
     if (!gather_in_gemm &&
         (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)),

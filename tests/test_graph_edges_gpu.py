@@ -65,3 +65,46 @@ def test_forward_at_max_tokens_and_below(cuda_ok):
         r = layer.route(x=sub.x)
         torch.cuda.synchronize()
         compare_layer(sub, out, r["idx"].cpu().numpy())
+
+
+@pytest.mark.parametrize("kw,expected", [
+    # decode: routing in one launch, rows gathered by the up GEMM -> route, up, down, combine
+    ({"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 128}, 4),
+    # ~75 tokens per expert: router, top-k, scatter, row gather, up, down, combine
+    ({"dtype": "bf16", "T": 300, "d": 512, "E": 32, "k": 8, "f": 256}, 7),
+    # fp32, 64 tokens: router, small-batch routing, up, down, combine
+    ({"dtype": "f32"}, 5),
+    # fp32, 65 tokens: router, top-k, scatter, up, down, combine
+    ({"dtype": "f32", "T": 65}, 6),
+])
+def test_forward_launch_count_matches_captured_graph(cuda_ok, kw, expected):
+    from cuda.bindings import runtime as rt
+    from sparse_moe_layer_warp_b200 import moe_forward_launch_count
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    assert moe_forward_launch_count(layer.handle, w.T) == expected
+    assert moe_forward_launch_count(layer.handle, 0) == 0
+    assert moe_forward_launch_count(layer.handle, w.T + 10**6) == -1
+    x = inp.x.clone()
+    out = layer.forward(x).clone()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward(x, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        layer.forward(x, out=out)
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    assert err == rt.cudaError_t.cudaSuccess
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    assert err == rt.cudaError_t.cudaSuccess
+    kernels = 0
+    for node in nodes[:n]:
+        err, typ = rt.cudaGraphNodeGetType(node)
+        assert err == rt.cudaError_t.cudaSuccess
+        kernels += typ == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    assert kernels == expected
