@@ -150,6 +150,17 @@ int moe_forward_launch_count(moe_handle h, int n_tokens);
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
 
+/* Self-test of the failure-detection path: launches (asynchronously, on `stream`) one small
+ * kernel whose two bounded waits -- on an mbarrier that nothing arrives on and on a flag in
+ * the workspace status block that nothing sets -- give up after limit_us microseconds
+ * (1 .. 2,000,000) exactly as the layer's waits do when a pipeline stalls; the next
+ * moe_device_status() then returns MOE_ERR_DEVICE_TIMEOUT and clears the word.  Nothing
+ * faults or traps and the context stays usable.  ws: a workspace of this handle (only its
+ * status block is touched).  MOE_ERR_INVALID_ARG for a null handle/workspace or a limit out
+ * of range; MOE_ERR_ALIGNMENT if ws is not 256-byte aligned. */
+moe_status moe_selftest_wait_timeout(moe_handle h, void *ws, size_t ws_bytes, int limit_us,
+                                     void *stream);
+
 /* Balancing statistics of a routing result ("Step 3.5 Flash: Open Frontier-Level
  * Intelligence with 11B Active Parameters", section 2.2.2: EP-group balance loss; section
  * 5.2.3: routing confidence).  From fp32 logits [n_tokens, E] and topk_idx [n_tokens, k]

@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     moe_forward,
     moe_forward_profiled,
     moe_forward_launch_count,
+    moe_selftest_wait_timeout,
     MOE_PROFILE_STAGES,
     PROFILE_STAGE_NAMES,
     moe_layer_destroy,

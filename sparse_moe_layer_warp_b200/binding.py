@@ -29,7 +29,8 @@ MOE_BF16 = 1
 EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_workspace_init",
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
            "moe_device_status", "moe_status_string", "moe_router_logits_static",
-           "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count")
+           "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
+           "moe_selftest_wait_timeout")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -80,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_router_logits_static.argtypes = [P, P, I, P, P]
         lib.moe_router_stats.argtypes = [P, P, P, I, I, P, P, P, P, Z, P]
         lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
+        lib.moe_selftest_wait_timeout.argtypes = [P, P, Z, I, P]
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -87,7 +89,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
-                     "moe_update_router_bias"):
+                     "moe_update_router_bias", "moe_selftest_wait_timeout"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -155,6 +157,12 @@ def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
     _check("moe_forward", load_library().moe_forward(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_selftest_wait_timeout(handle, ws, limit_us: int, stream=None) -> None:
+    """Launch the library's timeout self-test kernel (see include/moe_layer.h)."""
+    _check("moe_selftest_wait_timeout", load_library().moe_selftest_wait_timeout(
+        handle, _p(ws), ws.numel() * ws.element_size(), int(limit_us), _stream(stream)))
 
 
 def moe_forward_launch_count(handle, n_tokens: int) -> int:

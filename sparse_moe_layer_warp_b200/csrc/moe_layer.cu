@@ -391,6 +391,24 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
   return launch_gemm<MODE_LOGITS>(L, bn, p, st);
 }
 
+// Self-test of the device timeout path: an mbarrier nobody arrives on and a workspace flag
+// nobody sets, each waited on with the library's bounded waits (limit_ns), as a stuck
+// pipeline would be.  Both give up, leaving the status word set; nothing faults or traps.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(DevStatus *status,
+                                                                   unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  abort_flag = 0;
+  mbar_wait_bounded(&bar, 0, &abort_flag, status, 101, limit_ns);
+  abort_flag = 0;
+  int *flag = &status->pad[25];
+  *flag = 0;
+  counter_wait_bounded(flag, 1, &abort_flag, status, 102, limit_ns);
+}
+
 moe_status check_call(const moe_layer *L, int T, void *ws, size_t ws_bytes) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
@@ -491,6 +509,16 @@ moe_status moe_workspace_init(moe_handle h, void *ws, size_t ws_bytes, void *str
                  cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+
+moe_status moe_selftest_wait_timeout(moe_handle h, void *ws, size_t ws_bytes, int limit_us,
+                                     void *stream) {
+  if (!h || !ws || ws_bytes < sizeof(DevStatus) || limit_us < 1 || limit_us > 2000000)
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_ALIGNMENT;
+  return launch(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0,
+                static_cast<cudaStream_t>(stream), static_cast<DevStatus *>(ws),
+                (unsigned long long)limit_us * 1000ull);
 }
 
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream) {

@@ -86,7 +86,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag,
-                                                  DevStatus *status, int where) {
+                                                  DevStatus *status, int where,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
   auto try_wait = [&]() {
     return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
@@ -96,7 +97,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     if (try_wait()) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) {
           atomicExch(&status->error, 1);
@@ -112,7 +113,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 // mbar_wait_bounded.
 __device__ __forceinline__ bool counter_wait_bounded(const int *ctr, int target,
                                                      volatile int *abort_flag,
-                                                     DevStatus *status, int where) {
+                                                     DevStatus *status, int where,
+                                                     unsigned long long limit_ns = kWaitLimitNs) {
   auto load = [&]() {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
@@ -125,7 +127,7 @@ __device__ __forceinline__ bool counter_wait_bounded(const int *ctr, int target,
     if (load() >= target) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) {
           atomicExch(&status->error, 1);

@@ -1,0 +1,109 @@
+"""Failure detection and out-of-bounds writes (GPU).
+
+* A bounded device wait that runs out (the library's self-test kernel waits on an mbarrier and
+  a flag that nothing signals) is reported by moe_device_status as MOE_ERR_DEVICE_TIMEOUT; the
+  context stays usable and the next forward is unchanged.  Nothing faults or traps.
+* Canaries: output, workspace and routing buffers are carved out of larger buffers whose
+  margins hold a fill pattern; a forward and a routing call must leave every margin intact.
+"""
+import time
+
+import pytest
+import torch
+
+from sparse_moe_layer_warp_b200 import (MoEError, moe_forward, moe_route,
+                                        moe_selftest_wait_timeout, moe_workspace_init,
+                                        moe_workspace_size, synth)
+from tests.helpers import make_layer
+
+pytestmark = pytest.mark.gpu
+
+MOE_ERR_DEVICE_TIMEOUT = 6
+
+
+def test_device_timeout_reported_and_context_survives(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=40, d=256, E=32, k=4, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    ref = layer.forward(inp.x).clone()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    t0 = time.monotonic()
+    moe_selftest_wait_timeout(layer.handle, layer.ws, 20000)  # two waits of 20 ms each
+    assert layer.device_status() == MOE_ERR_DEVICE_TIMEOUT
+    assert time.monotonic() - t0 < 5.0
+    assert layer.device_status() == 0  # reading the word clears it
+    out = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert layer.device_status() == 0
+
+
+def test_selftest_rejects_bad_limits(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=8, d=256, E=16, k=2, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    layer.workspace(w.T)
+    for bad in (0, 2_000_001):
+        with pytest.raises(MoEError):
+            moe_selftest_wait_timeout(layer.handle, layer.ws, bad)
+
+
+def _guarded(n, dtype, fill, margin=4096):
+    """A tensor of n elements inside a buffer with `margin` elements of `fill` on each side."""
+    big = torch.full((n + 2 * margin,), fill, dtype=dtype, device="cuda")
+    return big, big[margin:margin + n]
+
+
+def _margins_intact(big, n, fill, margin=4096):
+    return bool((big[:margin] == fill).all()) and bool((big[margin + n:] == fill).all())
+
+
+@pytest.mark.parametrize("kw", [
+    {"dtype": "bf16", "T": 16, "d": 512, "E": 64, "k": 8, "f": 256},     # decode routing, gather4
+    {"dtype": "bf16", "T": 300, "d": 512, "E": 32, "k": 8, "f": 256},    # row gather, 1-CTA GEMMs
+    {"dtype": "bf16", "T": 700, "d": 768, "E": 8, "k": 4, "f": 512},     # CTA-pair GEMMs
+    {"dtype": "bf16", "T": 1100, "d": 256, "E": 41, "k": 3, "f": 128},   # token-major router
+    {"dtype": "f32", "T": 100},
+])
+def test_no_writes_outside_buffers(cuda_ok, kw):
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    T, d, E, k = w.T, w.d, w.E, w.k
+    ref = layer.forward(inp.x).clone()
+    torch.cuda.synchronize()
+
+    # workspace: 256-byte aligned slice of a byte buffer filled with 0xA5
+    need = moe_workspace_size(layer.handle, T)
+    ws_big, ws = _guarded(need, torch.uint8, 0xA5)
+    assert ws.data_ptr() % 256 == 0
+    moe_workspace_init(layer.handle, ws)
+    # output: bit pattern 0x7BAD (a finite bf16 / half of an fp32 word) around the rows
+    odt = torch.int16 if w.dtype == "bf16" else torch.int32
+    out_big, out_flat = _guarded(T * d, odt, 0x7BAD)
+    out = out_flat.view(inp.x.dtype).view(T, d)
+    moe_forward(layer.handle, inp.x, T, out, ws)
+    torch.cuda.synchronize()
+    assert _margins_intact(out_big, T * d, 0x7BAD)
+    assert _margins_intact(ws_big, need, 0xA5)
+    assert torch.equal(out, ref)
+
+    # routing outputs
+    bufs = {}
+    shapes = {"logits": (T * E, torch.int32), "idx": (T * k, torch.int32),
+              "gate": (T * k, torch.int32), "counts": (E, torch.int32),
+              "offsets": (E + 1, torch.int32), "perm": (T * k, torch.int32),
+              "slot_row": (T * k, torch.int32)}
+    for name, (n, dt) in shapes.items():
+        bufs[name] = _guarded(n, dt, 0x5EED)
+    v = {name: b[1] for name, b in bufs.items()}
+    moe_route(layer.handle, inp.x, T, v["logits"].view(torch.float32), v["idx"],
+              v["gate"].view(torch.float32), v["counts"], v["offsets"], v["perm"],
+              v["slot_row"], ws)
+    torch.cuda.synchronize()
+    for name, (n, _) in shapes.items():
+        assert _margins_intact(bufs[name][0], n, 0x5EED), name
+    assert _margins_intact(ws_big, need, 0xA5)
+    assert int(v["offsets"][E]) == T * k
+    assert layer.device_status() == 0
