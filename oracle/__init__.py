@@ -23,4 +23,7 @@ from .c_oracle import (  # noqa: F401
     oracle_num_threads,
     oracle_router_stats,
     oracle_bias_update,
+    oracle_expert_act_rms,
+    oracle_expert_param_norms,
+    oracle_health_ratios,
 )

@@ -45,6 +45,8 @@ def _load():
         lib.oracle_num_threads.restype = I
         lib.oracle_router_stats.argtypes = [P, P, I, I, I, I, P, P, P, P]
         lib.oracle_bias_update.argtypes = [P, I, I, ctypes.c_float, P]
+        lib.oracle_expert_act_rms.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P]
+        lib.oracle_expert_param_norms.argtypes = [P, P, P, I, I, I, I, P]
         _lib = lib
     return _lib
 
@@ -162,3 +164,41 @@ def oracle_bias_update(counts, Tk, gamma, bias):
     out = np.array(bias, np.float32, copy=True)
     _load().oracle_bias_update(_ptr(counts), len(counts), int(Tk), float(gamma), _ptr(out))
     return out
+
+
+def oracle_expert_act_rms(x, w_gate, w_up, idx, n_experts, n_shared=1):
+    """Per-expert RMS of the SwiGLU activation over the tokens routed to it [G] (float64)."""
+    x, dt = _as_input(x)
+    w_gate, _ = _as_input(w_gate)
+    w_up, _ = _as_input(w_up)
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, d = x.shape
+    f = w_gate.shape[1]
+    k = idx.shape[1]
+    G = n_experts + n_shared
+    out = np.empty(G, np.float64)
+    _load().oracle_expert_act_rms(_ptr(x), _ptr(w_gate), _ptr(w_up), dt, T, d, f, n_experts,
+                                  n_shared, _ptr(idx), k, _ptr(out))
+    return out
+
+
+def oracle_expert_param_norms(w_gate, w_up, w_down):
+    """Frobenius norm of each expert's (W_gate, W_up, W_down) together [G] (float64)."""
+    w_gate, dt = _as_input(w_gate)
+    w_up, _ = _as_input(w_up)
+    w_down, _ = _as_input(w_down)
+    G, f, d = w_gate.shape
+    out = np.empty(G, np.float64)
+    _load().oracle_expert_param_norms(_ptr(w_gate), _ptr(w_up), _ptr(w_down), dt, d, f, G,
+                                      _ptr(out))
+    return out
+
+
+def oracle_health_ratios(act_rms, param_norms, idx, n_experts):
+    """Cross-expert ratios over the routed experts: median / max of the activation RMS of
+    the experts some token chose, and min / median of the parameter norms (NumPy median:
+    mean of the two middle values for an even count)."""
+    chosen = np.unique(np.asarray(idx).ravel())
+    a = np.asarray(act_rms, np.float64)[chosen]
+    pn = np.asarray(param_norms, np.float64)[:n_experts]
+    return float(np.median(a) / a.max()), float(pn.min() / np.median(pn))

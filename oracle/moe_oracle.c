@@ -322,3 +322,54 @@ void oracle_bias_update(const int *counts, int E, int Tk, float gamma, float *bi
     bias[e] = bias[e] + gamma * s;
   }
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Expert health signals.  [P2 4.1.2]: expert collapse shows as vanishing expert          */
+/* activations and stalling parameter norms, so per-expert activation norms and parameter */
+/* norms are to be monitored; [P3], training stability, "expert collapse": the per-expert  */
+/* activation RMS norm and the min-to-median ratio of the parameter Frobenius norms.       */
+/* Readings: the activation is the SwiGLU output h = silu(x W_g^T) * (x W_u^T) of expert g */
+/* over the tokens routed to it (all tokens for a shared expert), RMS over tokens and the f */
+/* features (0 for an expert no token chose); the parameter norm of expert g is the        */
+/* Frobenius norm of its three matrices together.  Double throughout.                      */
+void oracle_expert_act_rms(const void *x, const void *w_gate, const void *w_up, int dtype,
+                           int T, int d, int f, int E, int n_shared, const int *idx, int k,
+                           double *rms) {
+  const int G = E + n_shared;
+  for (int g = 0; g < G; ++g) {
+    double ss = 0.0;
+    long long rows = 0;
+    for (int t = 0; t < T; ++t) {
+      int chosen = g >= E;
+      for (int j = 0; j < k && !chosen; ++j) chosen = idx[(size_t)t * k + j] == g;
+      if (!chosen) continue;
+      ++rows;
+      for (int n = 0; n < f; ++n) {
+        double a = 0.0, b = 0.0;
+        for (int i = 0; i < d; ++i) {
+          const double xv = orc_elem(x, dtype, (size_t)t * d + i);
+          a += xv * orc_elem(w_gate, dtype, ((size_t)g * f + n) * d + i);
+          b += xv * orc_elem(w_up, dtype, ((size_t)g * f + n) * d + i);
+        }
+        const double h = orc_silu(a) * b;
+        ss += h * h;
+      }
+    }
+    rms[g] = rows ? sqrt(ss / ((double)rows * f)) : 0.0;
+  }
+}
+
+void oracle_expert_param_norms(const void *w_gate, const void *w_up, const void *w_down,
+                               int dtype, int d, int f, int G, double *norm) {
+  const size_t per = (size_t)f * d;
+  for (int g = 0; g < G; ++g) {
+    double ss = 0.0;
+    for (size_t i = 0; i < per; ++i) {
+      const double a = orc_elem(w_gate, dtype, (size_t)g * per + i);
+      const double b = orc_elem(w_up, dtype, (size_t)g * per + i);
+      const double c = orc_elem(w_down, dtype, (size_t)g * per + i);
+      ss += a * a + b * b + c * c;
+    }
+    norm[g] = sqrt(ss);
+  }
+}

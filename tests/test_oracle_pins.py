@@ -266,3 +266,82 @@ def test_bias_update_sign_rule():
     assert b.tolist() == [-0.5, 0.5, 0.0, 0.0]
     b2 = oracle_bias_update(counts, 24, 0.25, b)
     assert b2.tolist() == [-0.75, 0.75, 0.0, 0.0]
+
+
+# ------------------------------------------------------------------ expert health signals
+from oracle import (oracle_expert_act_rms, oracle_expert_param_norms,  # noqa: E402
+                    oracle_health_ratios)
+
+
+def _expert_inputs(T=7, d=12, f=6, E=4, k=2, seed=3):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    wg = rng.standard_normal((E + 1, f, d)).astype(np.float32) / math.sqrt(d)
+    wu = rng.standard_normal((E + 1, f, d)).astype(np.float32) / math.sqrt(d)
+    wd = rng.standard_normal((E + 1, d, f)).astype(np.float32) / math.sqrt(f)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    return x, wg, wu, wd, idx
+
+
+def test_act_rms_matches_library_swiglu():
+    # torch matmul + silu on the tokens each expert was chosen by (the shared expert: all)
+    x, wg, wu, wd, idx = _expert_inputs()
+    E = wg.shape[0] - 1
+    got = oracle_expert_act_rms(x, wg, wu, idx, E, 1)
+    X = torch.from_numpy(x).double()
+    for g in range(E + 1):
+        rows = np.arange(len(x)) if g == E else np.nonzero((idx == g).any(1))[0]
+        if len(rows) == 0:
+            assert got[g] == 0.0
+            continue
+        h = torch.nn.functional.silu(X[rows] @ torch.from_numpy(wg[g]).double().T) * \
+            (X[rows] @ torch.from_numpy(wu[g]).double().T)
+        assert abs(got[g] - float(h.pow(2).mean().sqrt())) <= 1e-12 * float(h.abs().max())
+
+
+def test_act_rms_closed_form_constant_weights_and_down_invariance():
+    # x = 1, W_g = W_u = c: every h = silu(c d) * c d; W_down plays no part
+    T, d, f, E, k, c = 5, 8, 4, 3, 1, 0.3
+    x = np.ones((T, d), np.float32)
+    wg = np.full((E + 1, f, d), c, np.float32)
+    wu = np.full((E + 1, f, d), c, np.float32)
+    idx = np.array([[0], [0], [2], [0], [2]], np.int32)  # expert 1 never chosen
+    got = oracle_expert_act_rms(x, wg, wu, idx, E, 1)
+    z = float(np.float32(c)) * d
+    want = abs(z / (1 + math.exp(-z)) * z)
+    assert got[1] == 0.0
+    for g in (0, 2, 3):
+        assert abs(got[g] - want) <= 1e-12 * want
+
+
+def test_param_norms_closed_form_and_library_norm():
+    d, f, G, c = 8, 4, 3, 0.5
+    wg = np.full((G, f, d), c, np.float32)
+    wu = np.full((G, f, d), -c, np.float32)
+    wd = np.full((G, d, f), 2 * c, np.float32)
+    got = oracle_expert_param_norms(wg, wu, wd)
+    want = math.sqrt(d * f * (c * c + c * c + 4 * c * c))  # all three matrices
+    assert np.allclose(got, want, rtol=1e-14, atol=0)
+    x, wg, wu, wd, idx = _expert_inputs()
+    got = oracle_expert_param_norms(wg, wu, wd)
+    for g in range(wg.shape[0]):
+        ref = torch.linalg.vector_norm(torch.cat([torch.from_numpy(a[g]).double().ravel()
+                                                  for a in (wg, wu, wd)]))
+        assert abs(got[g] - float(ref)) <= 1e-12 * float(ref)
+
+
+def test_health_ratios_identical_experts_and_library_median():
+    x, wg, wu, wd, idx = _expert_inputs(E=4)
+    same_g = np.repeat(wg[:1], 5, 0)
+    same_u = np.repeat(wu[:1], 5, 0)
+    same_d = np.repeat(wd[:1], 5, 0)
+    act = oracle_expert_act_rms(x, same_g, same_u, idx, 4, 1)
+    pn = oracle_expert_param_norms(same_g, same_u, same_d)
+    ra, rp = oracle_health_ratios(act, pn, idx, 4)
+    # every chosen expert sees different tokens, so only the parameter ratio is exactly 1
+    assert rp == 1.0
+    act = np.array([1.0, 4.0, 2.0, 0.0, 9.0])
+    pn = np.array([3.0, 1.0, 5.0, 2.0, 7.0])
+    ra, rp = oracle_health_ratios(act, pn, np.array([[0, 1], [2, 1]]), 4)
+    assert ra == 2.0 / 4.0  # chosen experts 0, 1, 2: median 2, max 4 (expert 3 not chosen)
+    assert rp == 1.0 / 2.5  # routed experts 0..3: min 1, median (2 + 3) / 2
