@@ -150,6 +150,24 @@ int moe_forward_launch_count(moe_handle h, int n_tokens);
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
 
+/* Expert health signals ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active
+ * Parameters", section 4.1.2: monitor per-expert activation and parameter norms; "Step 3.5
+ * Flash 技术论文深度解读", training stability, expert collapse: per-expert activation RMS
+ * norm and the min-to-median ratio of parameter Frobenius norms).  Call after moe_forward
+ * with the same workspace and n_tokens (it reads that forward's expert activations):
+ *   act_rms[g]    (g < E + n_shared) RMS of the SwiGLU activation of expert g over the
+ *                 tokens routed to it (every token for the shared expert); 0 if none
+ *   param_norm[g] Frobenius norm of W_gate[g], W_up[g] and W_down[g] together
+ *   ratios[0]     median / max of act_rms over the routed experts some token chose
+ *   ratios[1]     min / median of param_norm over the routed experts
+ *                 (median of an even count: mean of the middle two; a ratio whose
+ *                 denominator is 0 is reported as 0)
+ * Device fp32 outputs; fp64 sums, deterministic.  Reads every expert weight once (about
+ * 1.4 ms for 289 full-size experts).  Errors as moe_forward; MOE_ERR_INVALID_ARG for
+ * n_tokens == 0 or a null output. */
+moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *param_norm,
+                             float *ratios, void *ws, size_t ws_bytes, void *stream);
+
 /* Self-test of the failure-detection path: launches (asynchronously, on `stream`) one small
  * kernel whose two bounded waits -- on an mbarrier that nothing arrives on and on a flag in
  * the workspace status block that nothing sets -- give up after limit_us microseconds

@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     moe_forward_profiled,
     moe_forward_launch_count,
     moe_selftest_wait_timeout,
+    moe_expert_health,
     MOE_PROFILE_STAGES,
     PROFILE_STAGE_NAMES,
     moe_layer_destroy,

@@ -30,7 +30,7 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
            "moe_device_status", "moe_status_string", "moe_router_logits_static",
            "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
-           "moe_selftest_wait_timeout")
+           "moe_selftest_wait_timeout", "moe_expert_health")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_router_stats.argtypes = [P, P, P, I, I, P, P, P, P, Z, P]
         lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
         lib.moe_selftest_wait_timeout.argtypes = [P, P, Z, I, P]
+        lib.moe_expert_health.argtypes = [P, I, P, P, P, P, Z, P]
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -89,7 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         for name in ("moe_layer_init", "moe_layer_destroy", "moe_workspace_init", "moe_route",
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
-                     "moe_update_router_bias", "moe_selftest_wait_timeout"):
+                     "moe_update_router_bias", "moe_selftest_wait_timeout",
+                     "moe_expert_health"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -157,6 +159,13 @@ def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
     _check("moe_forward", load_library().moe_forward(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_expert_health(handle, n_tokens, act_rms, param_norm, ratios, ws, stream=None) -> None:
+    """Expert health signals of the last forward on `ws` (see include/moe_layer.h)."""
+    _check("moe_expert_health", load_library().moe_expert_health(
+        handle, int(n_tokens), _p(act_rms), _p(param_norm), _p(ratios), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_selftest_wait_timeout(handle, ws, limit_us: int, stream=None) -> None:
@@ -266,6 +275,16 @@ class MoELayer:
         moe_router_stats(self.handle, logits, topk_idx, T, n_groups, p_mean, f_sel, scalars,
                          self.workspace(T), stream)
         return p_mean, f_sel, scalars
+
+    def expert_health(self, n_tokens, stream=None):
+        """act_rms [G], param_norm [G], ratios [2] of the last forward of n_tokens tokens."""
+        G = self.E + int(self.cfg.n_shared)
+        act = torch.empty(G, dtype=torch.float32, device=self.device)
+        par = torch.empty(G, dtype=torch.float32, device=self.device)
+        ratios = torch.empty(2, dtype=torch.float32, device=self.device)
+        moe_expert_health(self.handle, n_tokens, act, par, ratios, self.workspace(n_tokens),
+                          stream)
+        return act, par, ratios
 
     def device_status(self, stream=None) -> int:
         return moe_device_status(self.handle, self.ws, stream)

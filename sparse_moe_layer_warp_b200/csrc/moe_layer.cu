@@ -20,6 +20,7 @@
 
 #include "moe_layer.h"
 #include "expert_simt.cuh"
+#include "expert_stats.cuh"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "ptx_sm100.cuh"
@@ -119,7 +120,7 @@ size_t esize(const moe_config &c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 // Workspace regions (256-byte aligned).  P = T*k + n_shared*T rows of the sorted space.
 struct WsLayout {
   size_t status, logits, part, idx, gate, counts, offsets, perm, slot_row, chunk_hist, stats,
-      xs, h, y, done, total;
+      xs, h, y, done, health, total;
 };
 
 int pick_bn(const moe_config &c, int T, int mode);
@@ -156,6 +157,8 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.h = take(P * c.d_ff * esize(c));
   L.y = take(P * c.d_model * 4);  // fp32 in both precisions
   L.done = take(((size_t)c.n_experts + c.n_shared) * 4);  // per-group up completion counts
+  // expert health: slice sums of squares, activations then parameters
+  L.health = take(2 * ((size_t)c.n_experts + c.n_shared) * kHealthSlices * 8);
   L.total = off;
   return L;
 }
@@ -521,6 +524,44 @@ moe_status moe_selftest_wait_timeout(moe_handle h, void *ws, size_t ws_bytes, in
                 (unsigned long long)limit_us * 1000ull);
 }
 
+moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *param_norm,
+                             float *ratios, void *ws, size_t ws_bytes, void *stream) {
+  moe_status s = check_call(h, n_tokens, ws, ws_bytes);
+  if (s != MOE_OK) return s;
+  if (n_tokens == 0 || !act_rms || !param_norm || !ratios) return MOE_ERR_INVALID_ARG;
+  const moe_config &c = h->cfg;
+  const int T = n_tokens, Tk = T * c.top_k, G = c.n_experts + c.n_shared;
+  const WsLayout W = ws_layout(c, T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double *act_part = at<double>(ws, W.health);
+  double *par_part = act_part + (size_t)G * kHealthSlices;
+  const int *offsets = at<int>(ws, W.offsets);
+  const dim3 grid(G, kHealthSlices);
+  const long long per = (long long)c.d_ff * c.d_model;
+  if (c.dtype == MOE_BF16) {
+    if ((s = launch(expert_act_sumsq_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                    at<const __nv_bfloat16>(ws, W.h), offsets, c.n_experts, T, Tk, c.d_ff,
+                    act_part)) != MOE_OK ||
+        (s = launch(expert_param_sumsq_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16 *>(h->w.w_gate),
+                    static_cast<const __nv_bfloat16 *>(h->w.w_up),
+                    static_cast<const __nv_bfloat16 *>(h->w.w_down), per, par_part)) != MOE_OK)
+      return s;
+  } else {
+    if ((s = launch(expert_act_sumsq_kernel<float>, grid, dim3(256), 0, st,
+                    at<const float>(ws, W.h), offsets, c.n_experts, T, Tk, c.d_ff,
+                    act_part)) != MOE_OK ||
+        (s = launch(expert_param_sumsq_kernel<float>, grid, dim3(256), 0, st,
+                    static_cast<const float *>(h->w.w_gate),
+                    static_cast<const float *>(h->w.w_up),
+                    static_cast<const float *>(h->w.w_down), per, par_part)) != MOE_OK)
+      return s;
+  }
+  return launch(expert_health_final_kernel, dim3(1), dim3(1024), 0, st, (const double *)act_part,
+                (const double *)par_part, offsets, c.n_experts, G, T, c.d_ff, act_rms,
+                param_norm, ratios);
+}
+
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream) {
   if (!h || !ws || ws_bytes < sizeof(DevStatus)) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -531,6 +572,30 @@ moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stre
   if (cudaMemset(ws, 0, sizeof(DevStatus)) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_ERR_DEVICE_TIMEOUT;
 }
+
+}  // extern "C"
+
+namespace {
+// bf16 decode batches: router logits, selection and permutation in one launch
+bool decode_route_ok(const moe_config &c, int T) {
+  return T <= kChunk && c.dtype == MOE_BF16 && c.n_experts <= kDecodeMaxExperts &&
+         c.d_model % 64 == 0 && c.d_model <= kDecodeMaxD;
+}
+
+moe_status launch_route_decode(const moe_layer *L, const void *x, int T, float *logits,
+                               int *idx, float *gate, int *counts, int *offsets, int *perm,
+                               int *slot_row, DevStatus *status, CounterReset reset,
+                               cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  return launch(route_decode_kernel, dim3((c.n_experts + kDecodeEPC - 1) / kDecodeEPC),
+                dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(x),
+                static_cast<const __nv_bfloat16 *>(L->w.w_router), L->w.router_bias, T,
+                c.d_model, c.n_experts, c.top_k, logits, idx, gate, counts, offsets, perm,
+                slot_row, &status->router_ticket[31], reset);
+}
+}  // namespace
+
+extern "C" {
 
 static moe_status route_common(moe_handle h, const void *x, const float *logits_in, int T,
                                float *logits_out, int *idx, float *gate, int *counts,
@@ -543,6 +608,13 @@ static moe_status route_common(moe_handle h, const void *x, const float *logits_
   if (x && !aligned16(x)) return MOE_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(h->cfg, T);
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  if (!logits_in && decode_route_ok(h->cfg, T)) {
+    // the forward's decode routing: logits straight into logits_out when it is given
+    float *dst = logits_out ? logits_out : at<float>(ws, W.logits);
+    return launch_route_decode(h, x, T, dst, idx, gate, counts, offsets, perm, slot_row, status,
+                               CounterReset{status->sched, nullptr, 0}, st);
+  }
   const float *logits = logits_in;
   float *copy_out = nullptr;
   if (!logits) {
@@ -590,8 +662,7 @@ struct ForwardPlan {
 ForwardPlan plan_forward(const moe_layer *L, int T) {
   const moe_config &c = L->cfg;
   ForwardPlan f;
-  f.decode_route = T <= kChunk && c.dtype == MOE_BF16 && c.n_experts <= kDecodeMaxExperts &&
-                   c.d_model % 64 == 0 && c.d_model <= kDecodeMaxD;
+  f.decode_route = decode_route_ok(c, T);
   f.small_route = !f.decode_route && T <= kChunk;
   f.pair = c.dtype == MOE_BF16 && use_pair(L, T);
   f.gather_in_gemm = c.dtype == MOE_BF16 && !f.pair && up_gathers_rows(c, T);
@@ -643,12 +714,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                            c.n_experts + c.n_shared};
   const ForwardPlan plan = plan_forward(h, T);
   if (plan.decode_route) {
-    if ((s = launch(route_decode_kernel, dim3((c.n_experts + kDecodeEPC - 1) / kDecodeEPC),
-                    dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(x),
-                    static_cast<const __nv_bfloat16 *>(h->w.w_router), h->w.router_bias, T,
-                    c.d_model, c.n_experts, c.top_k, logits, idx, gate, at<int>(ws, W.counts),
-                    offsets, perm, slot_row, &at<DevStatus>(ws, W.status)->router_ticket[31],
-                    reset)) != MOE_OK)
+    if ((s = launch_route_decode(h, x, T, logits, idx, gate, at<int>(ws, W.counts), offsets,
+                                 perm, slot_row, at<DevStatus>(ws, W.status), reset, st)) !=
+        MOE_OK)
       return s;
     if ((s = mark(1)) != MOE_OK || (s = mark(2)) != MOE_OK) return s;
   } else {

@@ -24,6 +24,15 @@ def _workspace_logits(layer, x):
     return r["logits"]
 
 
+def _assert_same_logits(out, want, x, w_router):
+    # both calls accumulate x . W_r in fp32, possibly in different orders (bf16 decode
+    # batches route through the one-launch decode router): each is within d * 2^-24 *
+    # sum_i |x_i w_i| of the exact value, so they are within twice that of each other
+    bound = 2 * x.shape[1] * 2.0**-24 * (x.double().abs() @ w_router.double().abs().T)
+    assert torch.isfinite(out).all()
+    assert ((out.double() - want.double()).abs() <= bound).all()
+
+
 @pytest.mark.parametrize("T,E,d,dtype", [(16, 288, 4096, "bf16"), (5, 40, 512, "bf16"),
                                          (64, 96, 1024, "bf16"), (9, 16, 256, "f32")])
 def test_static_scratch_router_matches_workspace_router(cuda_ok, T, E, d, dtype):
@@ -37,10 +46,7 @@ def test_static_scratch_router_matches_workspace_router(cuda_ok, T, E, d, dtype)
         out = torch.full((T, E), float("nan"), device="cuda", dtype=torch.float32)
         binding.moe_router_logits_static(layer.handle, x, T, out)
         torch.cuda.synchronize()
-        # same kernel and summation order: identical values (the parity tolerance for fp32
-        # logits would also accept rounding differences; none are expected here)
-        assert torch.isfinite(out).all()
-        assert torch.equal(out, want)
+        _assert_same_logits(out, want, x, inp.w_router)
 
 
 def test_static_scratch_router_rejects_oversized_requests(cuda_ok):
@@ -65,5 +71,6 @@ def test_static_scratch_router_rejects_oversized_requests(cuda_ok):
                                       ctypes.c_void_p(out2.data_ptr()), st)
     assert rc == binding.MOE_OK
     torch.cuda.synchronize()
-    ref = _workspace_logits(layer2, inp2.x[:8].contiguous())
-    assert torch.equal(out2[:8], ref)
+    x8 = inp2.x[:8].contiguous()
+    ref = _workspace_logits(layer2, x8)
+    _assert_same_logits(out2[:8], ref, x8, inp2.w_router)
