@@ -297,6 +297,11 @@ def run_ours(args, rank, world, local_rank):
         "layer_roofline": {"algorithmic_bytes": int(layer_bytes), "algorithmic_flops": int(layer_flops),
                            "hbm_frac": round(layer_bytes / step_s / 1e9 / peaks["hbm_gbs"], 4),
                            "tensor_frac": round(layer_flops / step_s / 1e12 / peaks["bf16_tflops"], 4),
+                           # against the measured sustained bf16 rate (the GEMM loop under the
+                           # 1 kW power cap): the regime of a long back-to-back step loop
+                           "tensor_frac_sustained": round(
+                               layer_flops / step_s / 1e12 /
+                               peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
                            "touched_experts_mean": float(np.mean([a["touched"] for a in algo]))},
         "stages_ms": {n: round(float(v), 4) for n, v in zip(names, mean_stage)},
         "profiled_ms_per_step": round(profiled_ms, 4),
