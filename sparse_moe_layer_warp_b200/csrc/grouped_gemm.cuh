@@ -70,9 +70,10 @@ struct GemmParams {
   // Per-group hand-over of h from the up kernel to the down kernel (null: none).  UP: each
   // epilogue warp adds 1 to done[g] once its rows of h for group g are stored.  DOWN: the
   // kernel does not wait for the up kernel to finish; before loading h rows of group g it
-  // waits until done[g] = 4 * done_mt * (token tiles of g at done_bn tokens).
+  // waits until done[g] = done_warps * done_mt * (token tiles of g at done_bn tokens).
   int *done;
   int done_mt, done_bn;
+  int done_warps;  // arrivals per up unit: its epilogue warps (all CTAs of the unit)
 };
 
 constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
@@ -356,7 +357,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (MODE == MODE_DOWN && p.done) {
         if (lane == 0 && g != ready_group) {
-          const int target = 4 * p.done_mt * ((grp_count[g] + p.done_bn - 1) / p.done_bn);
+          const int target =
+              p.done_warps * p.done_mt * ((grp_count[g] + p.done_bn - 1) / p.done_bn);
           ok = counter_wait_bounded(p.done + g, target, abort_flag, p.status, 8);
           fence_proxy_async_global();  // the h rows are read through TMA below
           ready_group = g;

@@ -122,8 +122,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-  // programmatic dependent launch: everything below may read the previous kernel's output
-  griddep_wait();
+  // programmatic dependent launch: everything below may read the previous kernel's output,
+  // except in a down kernel with the per-group hand-over of h (see grouped_gemm_kernel)
+  if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
     int cnt, row;
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       int qi = 0;
       uint32_t qph = 0;
       int u = -1;
+      int ready_group = -1;  // down kernel: group whose h is known to be complete
       while (ok) {
         // the leader claims the next unit and publishes its id to both CTAs; the peer reads it
         if (leader) {
@@ -240,6 +242,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
         const int b_row = (shared_x ? nt * BN : grp_row[g] + nt * BN) + (int)rank * half;
         const uint64_t pw = (grp_count[g] <= BN) ? pol_w : pol_w_shared;
+        if (MODE == MODE_DOWN && p.done && g != ready_group) {
+          // both CTAs load h rows: each waits for every up unit of the group
+          const int target =
+              p.done_warps * p.done_mt * ((grp_count[g] + p.done_bn - 1) / p.done_bn);
+          if (!counter_wait_bounded(p.done + g, target, abort_flag, p.status, 19)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // the h rows are read through TMA below
+          ready_group = g;
+        }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 11)) {
             ok = false;
@@ -424,6 +437,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
           store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
                             vals, wbuf, lane);
+        }
+      }
+      if (MODE == MODE_UP && p.done) {
+        // publish this warp's rows of h for group g: stores, then a release of the count
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(p.done + g, 1);
         }
       }
       tc_fence_before();

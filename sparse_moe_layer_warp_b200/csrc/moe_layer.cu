@@ -779,9 +779,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p1.ld_out = c.d_ff;
     p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
     p1.topk = c.top_k;
-    // 1-CTA kernels: the down kernel starts on the SMs the up kernel leaves in its last wave
-    // and waits per expert group for that group's rows of h (see grouped_gemm_kernel)
-    if (!pair) p1.done = at<int>(ws, W.done);
+    // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
+    // expert group for that group's rows of h (see grouped_gemm_kernel)
+    p1.done = at<int>(ws, W.done);
     if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
         MOE_OK)
       return s;
@@ -794,8 +794,10 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     p2.M = c.d_model;
     p2.K = c.d_ff;
     p2.ld_out = c.d_model;
-    p2.done_mt = c.d_ff / kBM;  // the up kernel's weight tiles per token tile
-    p2.done_bn = bn;            // and its token tile
+    // the up kernel's weight tiles per token tile, its token tile and its epilogue warps
+    p2.done_mt = c.d_ff / (pair ? kPairBM : kBM);
+    p2.done_bn = pair ? kPairBN : bn;
+    p2.done_warps = pair ? 2 * kPairEpiWarps : 4;
     if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
                   : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
       return s;
