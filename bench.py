@@ -116,12 +116,15 @@ def algorithmic(w, counts, T):
                 down_flops=down_flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
 
 
+# the expert GEMM kernels' own sources (their device code and the PTX wrappers they use)
+GEMM_SOURCES = ("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx_sm100.cuh")
+
+
 def kernel_source_sha():
     csrc = os.path.join(ROOT, "sparse_moe_layer_warp_b200", "csrc")
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in GEMM_SOURCES:
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
