@@ -46,6 +46,8 @@ def _load():
         lib.oracle_router_stats.argtypes = [P, P, I, I, I, I, P, P, P, P]
         lib.oracle_bias_update.argtypes = [P, I, I, ctypes.c_float, P]
         lib.oracle_expert_act_rms.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P]
+        lib.oracle_moe_backward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I,
+                                            ctypes.c_double, P, P, P, P, P, P, P]
         lib.oracle_expert_param_norms.argtypes = [P, P, P, I, I, I, I, P]
         _lib = lib
     return _lib
@@ -202,3 +204,29 @@ def oracle_health_ratios(act_rms, param_norms, idx, n_experts):
     a = np.asarray(act_rms, np.float64)[chosen]
     pn = np.asarray(param_norms, np.float64)[:n_experts]
     return float(np.median(a) / a.max()), float(pn.min() / np.median(pn))
+
+
+def oracle_moe_backward(x, dout, w_r, w_gate, w_up, w_down, idx, gates, routed_scale=1.0,
+                        n_shared=1):
+    """Gradients of the layer output for the given selection: dict of float64 arrays dx
+    [T,d], dw_router [E,d], dw_gate / dw_up [G,f,d], dw_down [G,d,f] (see moe_oracle.c)."""
+    x, dt = _as_input(x)
+    dout, dt2 = _as_input(dout)
+    assert dt == dt2
+    w_r, _ = _as_input(w_r)
+    w_gate, _ = _as_input(w_gate)
+    w_up, _ = _as_input(w_up)
+    w_down, _ = _as_input(w_down)
+    idx = np.ascontiguousarray(idx, np.int32)
+    gates = np.ascontiguousarray(gates, np.float32)
+    T, d = x.shape
+    E = w_r.shape[0]
+    G, f, _ = w_gate.shape
+    k = idx.shape[1]
+    out = dict(dx=np.empty((T, d)), dw_router=np.empty((E, d)), dw_gate=np.empty((G, f, d)),
+               dw_up=np.empty((G, f, d)), dw_down=np.empty((G, d, f)))
+    _load().oracle_moe_backward(_ptr(x), _ptr(dout), _ptr(w_r), _ptr(w_gate), _ptr(w_up),
+                                _ptr(w_down), dt, T, d, E, k, f, n_shared, float(routed_scale),
+                                _ptr(idx), _ptr(gates), _ptr(out["dx"]), _ptr(out["dw_router"]),
+                                _ptr(out["dw_gate"]), _ptr(out["dw_up"]), _ptr(out["dw_down"]))
+    return out

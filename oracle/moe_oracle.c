@@ -373,3 +373,110 @@ void oracle_expert_param_norms(const void *w_gate, const void *w_up, const void 
     norm[g] = sqrt(ss);
   }
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Backward of the layer: the chain rule through oracle_moe_forward's definition, for a     */
+/* given selection (idx) and gates -- the selection itself carries no gradient ([P3 MoE]:   */
+/* the bias only selects).  Double throughout; tokens one after another (the weight         */
+/* gradients accumulate over tokens).                                                      */
+/*   for token t and each contribution (expert e, scale s = routed_scale * g_j, or 1 for   */
+/*   the shared expert):                                                                    */
+/*     a = W_g[e] x_t,  b = W_u[e] x_t,  h = silu(a) * b,  yhat = W_d[e] h                 */
+/*     dy = s * dout_t;   dW_d[e] += dy h^T;   dh = W_d[e]^T dy                             */
+/*     da = dh * b * silu'(a),  db = dh * silu(a),  silu'(a) = sig(a) (1 + a (1 - sig(a)))  */
+/*     dW_g[e] += da x_t^T;  dW_u[e] += db x_t^T;  dx_t += W_g[e]^T da + W_u[e]^T db         */
+/*     routed: dgate_j = routed_scale * (dout_t . yhat)                                     */
+/*   router: the gates are the softmax of the selected unbiased logits, so                  */
+/*     dl[e_j] = g_j (dgate_j - sum_i g_i dgate_i), 0 for unselected experts;               */
+/*     dW_r[e] += dl[e] x_t;  dx_t += sum_e dl[e] W_r[e]                                    */
+/* Outputs: dx [T,d], dw_router [E,d], dw_gate / dw_up [G,f,d], dw_down [G,d,f] (G = E +   */
+/* n_shared), overwritten.                                                                 */
+void oracle_moe_backward(const void *x, const void *dout, const void *w_r, const void *w_gate,
+                         const void *w_up, const void *w_down, int dtype, int T, int d, int E,
+                         int k, int f, int n_shared, double routed_scale, const int *idx,
+                         const float *gates, double *dx, double *dw_router, double *dw_gate,
+                         double *dw_up, double *dw_down) {
+  const int G = E + n_shared;
+  const size_t wsz = (size_t)f * (size_t)d;
+  memset(dx, 0, sizeof(double) * (size_t)T * d);
+  memset(dw_router, 0, sizeof(double) * (size_t)E * d);
+  memset(dw_gate, 0, sizeof(double) * (size_t)G * wsz);
+  memset(dw_up, 0, sizeof(double) * (size_t)G * wsz);
+  memset(dw_down, 0, sizeof(double) * (size_t)G * wsz);
+  double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+  double *ot = (double *)malloc(sizeof(double) * (size_t)d);
+  double *a = (double *)malloc(sizeof(double) * (size_t)f);
+  double *b = (double *)malloc(sizeof(double) * (size_t)f);
+  double *h = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dh = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dy = (double *)malloc(sizeof(double) * (size_t)d);
+  double *dgate = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  for (int t = 0; t < T; ++t) {
+    for (int i = 0; i < d; ++i) {
+      xt[i] = orc_elem(x, dtype, (size_t)t * d + i);
+      ot[i] = orc_elem(dout, dtype, (size_t)t * d + i);
+    }
+    for (int c = 0; c < k + n_shared; ++c) {
+      const int routed = c < k;
+      const int e = routed ? idx[(size_t)t * k + c] : E;
+      const double s = routed ? routed_scale * (double)gates[(size_t)t * k + c] : 1.0;
+      for (int n = 0; n < f; ++n) {
+        double av = 0.0, bv = 0.0;
+        for (int i = 0; i < d; ++i) {
+          av += xt[i] * orc_elem(w_gate, dtype, (size_t)e * wsz + (size_t)n * d + i);
+          bv += xt[i] * orc_elem(w_up, dtype, (size_t)e * wsz + (size_t)n * d + i);
+        }
+        a[n] = av;
+        b[n] = bv;
+        h[n] = orc_silu(av) * bv;
+      }
+      double dot = 0.0;  /* dout_t . yhat */
+      for (int i = 0; i < d; ++i) {
+        double yh = 0.0;
+        for (int n = 0; n < f; ++n)
+          yh += orc_elem(w_down, dtype, (size_t)e * wsz + (size_t)i * f + n) * h[n];
+        dot += ot[i] * yh;
+        dy[i] = s * ot[i];
+      }
+      if (routed) dgate[c] = routed_scale * dot;
+      for (int n = 0; n < f; ++n) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) {
+          acc += orc_elem(w_down, dtype, (size_t)e * wsz + (size_t)i * f + n) * dy[i];
+          dw_down[(size_t)e * wsz + (size_t)i * f + n] += dy[i] * h[n];
+        }
+        dh[n] = acc;
+      }
+      for (int n = 0; n < f; ++n) {
+        const double sg = 1.0 / (1.0 + exp(-a[n]));
+        const double da = dh[n] * b[n] * sg * (1.0 + a[n] * (1.0 - sg));
+        const double db = dh[n] * a[n] * sg;
+        for (int i = 0; i < d; ++i) {
+          const size_t wi = (size_t)e * wsz + (size_t)n * d + i;
+          dw_gate[wi] += da * xt[i];
+          dw_up[wi] += db * xt[i];
+          dx[(size_t)t * d + i] +=
+              orc_elem(w_gate, dtype, wi) * da + orc_elem(w_up, dtype, wi) * db;
+        }
+      }
+    }
+    double sgd = 0.0;
+    for (int j = 0; j < k; ++j) sgd += (double)gates[(size_t)t * k + j] * dgate[j];
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      const double dl = (double)gates[(size_t)t * k + j] * (dgate[j] - sgd);
+      for (int i = 0; i < d; ++i) {
+        dw_router[(size_t)e * d + i] += dl * xt[i];
+        dx[(size_t)t * d + i] += dl * orc_elem(w_r, dtype, (size_t)e * d + i);
+      }
+    }
+  }
+  free(dgate);
+  free(dy);
+  free(dh);
+  free(h);
+  free(b);
+  free(a);
+  free(ot);
+  free(xt);
+}

@@ -345,3 +345,87 @@ def test_health_ratios_identical_experts_and_library_median():
     ra, rp = oracle_health_ratios(act, pn, np.array([[0, 1], [2, 1]]), 4)
     assert ra == 2.0 / 4.0  # chosen experts 0, 1, 2: median 2, max 4 (expert 3 not chosen)
     assert rp == 1.0 / 2.5  # routed experts 0..3: min 1, median (2 + 3) / 2
+
+
+# ------------------------------------------------------------------ backward
+from oracle import oracle_moe_backward  # noqa: E402
+
+
+def _torch_layer_grads(x, dout, wr, wg, wu, wd, idx, rs, n_shared):
+    """The layer in float64 torch autograd for a fixed selection: gates = softmax of the
+    selected router logits; returns the gradients of <out, dout>."""
+    X = torch.tensor(x, dtype=torch.float64, requires_grad=True)
+    WR = torch.tensor(wr, dtype=torch.float64, requires_grad=True)
+    WG = torch.tensor(wg, dtype=torch.float64, requires_grad=True)
+    WU = torch.tensor(wu, dtype=torch.float64, requires_grad=True)
+    WD = torch.tensor(wd, dtype=torch.float64, requires_grad=True)
+    E = wr.shape[0]
+    rows = []
+    for t in range(x.shape[0]):
+        sel = torch.tensor(idx[t], dtype=torch.long)
+        g = torch.softmax((X[t] @ WR.T)[sel], dim=0)
+        o = torch.zeros(x.shape[1], dtype=torch.float64)
+        for j, e in enumerate(idx[t]):
+            h = torch.nn.functional.silu(WG[e] @ X[t]) * (WU[e] @ X[t])
+            o = o + rs * g[j] * (WD[e] @ h)
+        if n_shared:
+            h = torch.nn.functional.silu(WG[E] @ X[t]) * (WU[E] @ X[t])
+            o = o + WD[E] @ h
+        rows.append(o)
+    out = torch.stack(rows)
+    (out * torch.tensor(dout, dtype=torch.float64)).sum().backward()
+    gates = np.stack([torch.softmax(torch.tensor(x[t] @ wr.T.astype(np.float64))[idx[t]], 0)
+                      .numpy() for t in range(x.shape[0])]).astype(np.float32)
+    return dict(dx=X.grad.numpy(), dw_router=WR.grad.numpy(), dw_gate=WG.grad.numpy(),
+                dw_up=WU.grad.numpy(), dw_down=WD.grad.numpy()), gates
+
+
+@pytest.mark.parametrize("n_shared,rs", [(1, 1.0), (0, 2.5)])
+def test_backward_matches_torch_autograd(n_shared, rs):
+    rng = np.random.default_rng(11)
+    T, d, f, E, k = 5, 12, 6, 5, 2
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    dout = rng.standard_normal((T, d)).astype(np.float32)
+    wr = (rng.standard_normal((E, d)) / math.sqrt(d)).astype(np.float32)
+    wg = (rng.standard_normal((E + n_shared, f, d)) / math.sqrt(d)).astype(np.float32)
+    wu = (rng.standard_normal((E + n_shared, f, d)) / math.sqrt(d)).astype(np.float32)
+    wd = (rng.standard_normal((E + n_shared, d, f)) / math.sqrt(f)).astype(np.float32)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    want, gates = _torch_layer_grads(x, dout, wr, wg, wu, wd, idx, rs, n_shared)
+    got = oracle_moe_backward(x, dout, wr, wg, wu, wd, idx, gates, rs, n_shared)
+    for name in want:
+        scale = np.abs(want[name]).max()
+        # the oracle takes the gates as fp32 (as the GPU does): relative error ~1e-7
+        assert np.abs(got[name] - want[name]).max() <= 2e-6 * scale, name
+
+
+def test_backward_matches_finite_differences():
+    # central differences of <forward(x), dout> through oracle_moe_forward itself (its own
+    # routing; the perturbation is far too small to change the selection)
+    w = synth.WORKLOADS["tiny_fp32"].replace(T=3, d=16, E=6, k=2, f=8, seed=4)
+    inp = synth.make_inputs(w)
+    x, wr, b, wg, wu, wd = [t.numpy() for t in (inp.x, inp.w_router, inp.bias, inp.w_gate,
+                                                 inp.w_up, inp.w_down)]
+    rng = np.random.default_rng(2)
+    dout = rng.standard_normal(x.shape).astype(np.float32)
+    _, idx, gates, _ = oracle_moe_forward(x, wr, b, wg, wu, wd, w.k)
+    got = oracle_moe_backward(x, dout, wr, wg, wu, wd, idx, gates)
+    eps = 1e-3
+
+    def loss(**over):
+        a = dict(x=x, wr=wr, wg=wg, wu=wu, wd=wd)
+        a.update(over)
+        out, idx2, _, _ = oracle_moe_forward(a["x"], a["wr"], b, a["wg"], a["wu"], a["wd"],
+                                             w.k)
+        assert (idx2 == idx).all()
+        return float((out * dout).sum())
+
+    for (name, arr, key, pos) in (("dx", x, "x", (1, 3)), ("dw_router", wr, "wr", (2, 5)),
+                                  ("dw_gate", wg, "wg", (6, 1, 2)),
+                                  ("dw_up", wu, "wu", (idx[0, 0], 3, 7)),
+                                  ("dw_down", wd, "wd", (idx[1, 1], 4, 5))):
+        p, m = arr.copy(), arr.copy()
+        p[pos] += eps
+        m[pos] -= eps
+        fd = (loss(**{key: p}) - loss(**{key: m})) / (2 * eps)
+        assert abs(got[name][pos] - fd) <= 2e-3 * max(1.0, abs(fd)), (name, got[name][pos], fd)
