@@ -150,6 +150,25 @@ int moe_forward_launch_count(moe_handle h, int n_tokens);
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
 
+/* Backward of moe_forward: gradients of <out, dout> with respect to x and the weights, for
+ * the forward's own selection (recomputed here with the same kernels; the selection carries
+ * no gradient -- the bias only selects, "Step 3.5 Flash 技术论文深度解读", architecture item
+ * 1 note).  Chain rule through sections 2.2 / 2.2.2 / 4.1.2 of "Step 3.5 Flash: Open
+ * Frontier-Level Intelligence with 11B Active Parameters": the gates are the softmax of the
+ * selected unbiased router logits, so the router weights receive
+ *   dl_j = g_j (dgate_j - sum_i g_i dgate_i),  dgate_j = routed_scale * (dout_t . y_j),
+ * with y_j the unscaled output of the j-th selected expert.
+ *   x, dout   [n_tokens, d] layer dtype          dx        [n_tokens, d] fp32
+ *   dw_router [E, d] fp32    dw_gate, dw_up [E + n_shared, f, d] fp32
+ *   dw_down   [E + n_shared, d, f] fp32   (all overwritten; unchosen experts get zeros)
+ * ws: at least moe_backward_workspace_size(h, n_tokens) bytes, 256-byte aligned (it holds a
+ * forward workspace at its start, which this call reuses).  fp32 accumulation on CUDA cores
+ * in a fixed order: deterministic.  Errors as moe_forward. */
+size_t moe_backward_workspace_size(moe_handle h, int n_tokens);
+moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *dout, float *dx,
+                        float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                        void *ws, size_t ws_bytes, void *stream);
+
 /* Expert health signals ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active
  * Parameters", section 4.1.2: monitor per-expert activation and parameter norms; "Step 3.5
  * Flash 技术论文深度解读", training stability, expert collapse: per-expert activation RMS

@@ -17,6 +17,8 @@ from .binding import (  # noqa: F401
     moe_forward_launch_count,
     moe_selftest_wait_timeout,
     moe_expert_health,
+    moe_backward,
+    moe_backward_workspace_size,
     MOE_PROFILE_STAGES,
     PROFILE_STAGE_NAMES,
     moe_layer_destroy,

@@ -30,7 +30,8 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_route", "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
            "moe_device_status", "moe_status_string", "moe_router_logits_static",
            "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
-           "moe_selftest_wait_timeout", "moe_expert_health")
+           "moe_selftest_wait_timeout", "moe_expert_health", "moe_backward",
+           "moe_backward_workspace_size")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -83,6 +84,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
         lib.moe_selftest_wait_timeout.argtypes = [P, P, Z, I, P]
         lib.moe_expert_health.argtypes = [P, I, P, P, P, P, Z, P]
+        lib.moe_backward.argtypes = [P, P, I, P, P, P, P, P, P, P, Z, P]
+        lib.moe_backward_workspace_size.argtypes = [P, I]
+        lib.moe_backward_workspace_size.restype = Z
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -91,7 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
                      "moe_update_router_bias", "moe_selftest_wait_timeout",
-                     "moe_expert_health"):
+                     "moe_expert_health", "moe_backward"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -159,6 +163,18 @@ def moe_forward(handle, x, n_tokens, out, ws, stream=None) -> None:
     _check("moe_forward", load_library().moe_forward(
         handle, _p(x), int(n_tokens), _p(out), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_backward_workspace_size(handle, n_tokens: int) -> int:
+    return int(load_library().moe_backward_workspace_size(handle, int(n_tokens)))
+
+
+def moe_backward(handle, x, n_tokens, dout, dx, dw_router, dw_gate, dw_up, dw_down, ws,
+                 stream=None) -> None:
+    """Gradients of <forward(x), dout> (see include/moe_layer.h); fp32 outputs."""
+    _check("moe_backward", load_library().moe_backward(
+        handle, _p(x), int(n_tokens), _p(dout), _p(dx), _p(dw_router), _p(dw_gate), _p(dw_up),
+        _p(dw_down), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_expert_health(handle, n_tokens, act_rms, param_norm, ratios, ws, stream=None) -> None:
@@ -229,6 +245,7 @@ class MoELayer:
         self.handle = moe_layer_init(self.cfg, *self.tensors)
         self.device = w_router.device
         self.ws = None
+        self.bw_ws = None
         self.E, self.k, self.d = int(E), int(top_k), int(d)
 
     def workspace(self, n_tokens: int):
@@ -275,6 +292,23 @@ class MoELayer:
         moe_router_stats(self.handle, logits, topk_idx, T, n_groups, p_mean, f_sel, scalars,
                          self.workspace(T), stream)
         return p_mean, f_sel, scalars
+
+    def backward(self, x, dout, stream=None):
+        """dict of fp32 gradients dx, dw_router, dw_gate, dw_up, dw_down (device tensors)."""
+        T = x.shape[0]
+        need = moe_backward_workspace_size(self.handle, T)
+        if self.bw_ws is None or self.bw_ws.numel() < need:
+            self.bw_ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            moe_workspace_init(self.handle, self.bw_ws)
+        G = self.E + int(self.cfg.n_shared)
+        f = int(self.cfg.d_ff)
+        kw = dict(dtype=torch.float32, device=self.device)
+        g = dict(dx=torch.empty((T, self.d), **kw), dw_router=torch.empty((self.E, self.d), **kw),
+                 dw_gate=torch.empty((G, f, self.d), **kw), dw_up=torch.empty((G, f, self.d), **kw),
+                 dw_down=torch.empty((G, self.d, f), **kw))
+        moe_backward(self.handle, x, T, dout, g["dx"], g["dw_router"], g["dw_gate"], g["dw_up"],
+                     g["dw_down"], self.bw_ws, stream)
+        return g
 
     def expert_health(self, n_tokens, stream=None):
         """act_rms [G], param_norm [G], ratios [2] of the last forward of n_tokens tokens."""

@@ -19,6 +19,7 @@
 #include <utility>
 
 #include "moe_layer.h"
+#include "backward.cuh"
 #include "expert_simt.cuh"
 #include "expert_stats.cuh"
 #include "grouped_gemm.cuh"
@@ -394,6 +395,41 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
   return launch_gemm<MODE_LOGITS>(L, bn, p, st);
 }
 
+// Backward workspace: the forward's layout, then the backward's own regions.
+struct BwLayout {
+  size_t row_token, row_group, row_scale, tile_prefix, a, b, dh, db, wide, dgate, dl, total;
+};
+
+BwLayout bw_layout(const moe_config &c, int T) {
+  BwLayout B;
+  size_t off = ws_layout(c, T).total;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~static_cast<size_t>(255);
+    return o;
+  };
+  const size_t Tk = (size_t)T * c.top_k, P = Tk + (size_t)c.n_shared * T;
+  const size_t G = (size_t)c.n_experts + c.n_shared;
+  B.row_token = take(P * 4);
+  B.row_group = take(P * 4);
+  B.row_scale = take(P * 4);
+  B.tile_prefix = take((G + 1) * 4);
+  B.a = take(P * c.d_ff * 4);
+  B.b = take(P * c.d_ff * 4);
+  B.dh = take(P * c.d_ff * 4);
+  B.db = take(P * c.d_ff * 4);
+  B.wide = take(P * c.d_model * 4);  // unscaled expert outputs, then the rows of dx
+  B.dgate = take(Tk * 4);
+  B.dl = take(Tk * 4);
+  B.total = off;
+  return B;
+}
+
+template <typename T_>
+moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
+                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                         void *ws, cudaStream_t st);
+
 // Self-test of the device timeout path: an mbarrier nobody arrives on and a workspace flag
 // nobody sets, each waited on with the library's bounded waits (limit_ns), as a stuck
 // pipeline would be.  Both give up, leaving the status word set; nothing faults or traps.
@@ -522,6 +558,31 @@ moe_status moe_selftest_wait_timeout(moe_handle h, void *ws, size_t ws_bytes, in
   return launch(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0,
                 static_cast<cudaStream_t>(stream), static_cast<DevStatus *>(ws),
                 (unsigned long long)limit_us * 1000ull);
+}
+
+size_t moe_backward_workspace_size(moe_handle h, int n_tokens) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return 0;
+  return bw_layout(h->cfg, n_tokens).total;
+}
+
+moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *dout, float *dx,
+                        float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                        void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!x || !dout || !dx || !dw_router || !dw_gate || !dw_up || !dw_down)
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < bw_layout(h->cfg, n_tokens).total) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(dout) || !aligned16(dx)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (h->cfg.dtype == MOE_BF16)
+    return backward_impl(h, static_cast<const __nv_bfloat16 *>(x),
+                         static_cast<const __nv_bfloat16 *>(dout), n_tokens, dx, dw_router,
+                         dw_gate, dw_up, dw_down, ws, st);
+  return backward_impl(h, static_cast<const float *>(x), static_cast<const float *>(dout),
+                       n_tokens, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
 
 moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *param_norm,
@@ -951,3 +1012,104 @@ extern "C" moe_status moe_router_logits_static(moe_handle h, const void *x, int 
                 n_tokens, c.d_model, c.n_experts, part, logits_out, tickets);
 }
 
+
+namespace {
+
+template <typename T_>
+moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
+                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                         void *ws, cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  const int E = c.n_experts, G = E + c.n_shared, k = c.top_k, d = c.d_model, f = c.d_ff;
+  const int Tk = T * k, P = Tk + c.n_shared * T;
+  const WsLayout W = ws_layout(c, T);
+  const BwLayout B = bw_layout(c, T);
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  int *idx = at<int>(ws, W.idx), *offsets = at<int>(ws, W.offsets), *perm = at<int>(ws, W.perm);
+  int *slot_row = at<int>(ws, W.slot_row), *counts = at<int>(ws, W.counts);
+  float *gate = at<float>(ws, W.gate), *logits = at<float>(ws, W.logits);
+  const T_ *wg = static_cast<const T_ *>(L->w.w_gate);
+  const T_ *wu = static_cast<const T_ *>(L->w.w_up);
+  const T_ *wd = static_cast<const T_ *>(L->w.w_down);
+  const T_ *wr = static_cast<const T_ *>(L->w.w_router);
+  moe_status s;
+  // 1. the forward's selection (same kernels, so the same experts and gates)
+  const ForwardPlan plan = plan_forward(L, T);
+  const CounterReset reset{status->sched, nullptr, 0};
+  if (plan.decode_route) {
+    s = launch_route_decode(L, x, T, logits, idx, gate, counts, offsets, perm, slot_row, status,
+                            reset, st);
+  } else {
+    s = launch_logits(L, x, T, logits, at<float>(ws, W.part), status, st);
+    if (s == MOE_OK)
+      s = plan.small_route
+              ? launch_route_small(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
+                                   slot_row, reset, st)
+              : launch_select_permute(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
+                                      slot_row, at<int>(ws, W.chunk_hist), reset, st);
+  }
+  if (s != MOE_OK) return s;
+  // 2. row bookkeeping
+  int *row_token = at<int>(ws, B.row_token), *row_group = at<int>(ws, B.row_group);
+  float *row_scale = at<float>(ws, B.row_scale);
+  int *tile_prefix = at<int>(ws, B.tile_prefix);
+  float *a = at<float>(ws, B.a), *b = at<float>(ws, B.b), *dh = at<float>(ws, B.dh);
+  float *db = at<float>(ws, B.db), *wide = at<float>(ws, B.wide);
+  float *dgate = at<float>(ws, B.dgate), *dl = at<float>(ws, B.dl);
+  if ((s = launch(bw_rows_kernel, dim3(grid_for(P, 256, L->num_sms)), dim3(256), 0, st,
+                  (const int *)perm, (const int *)idx, (const float *)gate, T, k, E, c.n_shared,
+                  c.routed_scale, row_token, row_group, row_scale)) != MOE_OK ||
+      (s = launch(bw_tiles_kernel, dim3(1), dim3(32), 0, st, (const int *)offsets, E, G, T,
+                  tile_prefix)) != MOE_OK)
+    return s;
+  const int n_tiles = P / kBwRows + G;  // upper bound of the row-tile list
+  auto cdiv = [](int n, int m) { return (n + m - 1) / m; };
+  const SrcX<T_> src_x{x, row_token, d};
+  const SrcDy<T_> src_dy{dout, row_token, row_scale, d};
+  const SrcH src_h{a, b, f};
+  const SrcRow src_da{dh, f}, src_db{db, f};
+  // 3. pre-activations a, b; unscaled expert outputs; dgate
+  if ((s = launch(bw_nt_kernel<2, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256), 0, st,
+                  wg, wu, f, d, src_x, (const int *)tile_prefix, (const int *)offsets, E, G, T,
+                  Tk, a, b)) != MOE_OK ||
+      (s = launch(bw_nt_kernel<1, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
+                  wd, d, f, src_h, (const int *)tile_prefix, (const int *)offsets, E, G, T, Tk,
+                  wide, wide)) != MOE_OK ||
+      (s = launch(bw_dgate_kernel<T_>, dim3(grid_for(Tk, 8, L->num_sms)), dim3(256), 0, st,
+                  dout, (const float *)wide, (const int *)row_token, (const int *)perm, Tk, d,
+                  c.routed_scale, dgate)) != MOE_OK)
+    return s;
+  // 4. dh, dW_d, then da (over dh) and db
+  if ((s = launch(bw_nn_kernel<1, T_, SrcDy<T_>, SrcDy<T_>>, dim3(n_tiles, cdiv(f, 64)),
+                  dim3(256), 0, st, wd, wd, d, f, src_dy, src_dy, (const int *)tile_prefix,
+                  (const int *)offsets, E, G, T, Tk, dh)) != MOE_OK ||
+      (s = launch(bw_wgrad_kernel<SrcDy<T_>, SrcH>, dim3(G, cdiv(d, 32), cdiv(f, 64)),
+                  dim3(256), 0, st, src_dy, src_h, d, f, (const int *)offsets, E, T, Tk,
+                  dw_down)) != MOE_OK ||
+      (s = launch(bw_swiglu_kernel, dim3(grid_for((size_t)P * f, 256, L->num_sms)), dim3(256),
+                  0, st, (const float *)a, (const float *)b, dh, db, (size_t)P * f)) != MOE_OK)
+    return s;
+  // 5. rows of dx (over the unscaled outputs, no longer needed), dW_g, dW_u
+  if ((s = launch(bw_nn_kernel<2, T_, SrcRow, SrcRow>, dim3(n_tiles, cdiv(d, 64)), dim3(256),
+                  0, st, wg, wu, f, d, src_da, src_db, (const int *)tile_prefix,
+                  (const int *)offsets, E, G, T, Tk, wide)) != MOE_OK ||
+      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 32), cdiv(d, 64)),
+                  dim3(256), 0, st, src_da, src_x, f, d, (const int *)offsets, E, T, Tk,
+                  dw_gate)) != MOE_OK ||
+      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 32), cdiv(d, 64)),
+                  dim3(256), 0, st, src_db, src_x, f, d, (const int *)offsets, E, T, Tk,
+                  dw_up)) != MOE_OK)
+    return s;
+  // 6. router and dx
+  if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
+                  (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
+      (s = launch(bw_router_dw_kernel<T_>, dim3(E, cdiv(d, 256)), dim3(256), 0, st, x,
+                  (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
+                  dw_router)) != MOE_OK)
+    return s;
+  return launch(bw_dx_kernel<T_>, dim3(grid_for((size_t)T * d, 256, L->num_sms)), dim3(256), 0,
+                st, (const float *)wide, (const int *)slot_row, (const int *)idx,
+                (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
+}
+
+}  // namespace

@@ -1,0 +1,65 @@
+"""GPU parity for the layer backward (moe_backward) against the CPU oracle's chain rule, on
+the GPU's own selection (the oracle takes the same idx and gates)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle_moe_backward
+from sparse_moe_layer_warp_b200 import synth
+from tests.helpers import host_inputs, make_layer
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 128},             # decode routing
+    {"dtype": "bf16", "T": 40, "d": 256, "E": 16, "k": 4, "f": 128, "routed_scale": 2.0},
+    {"dtype": "bf16", "T": 150, "d": 256, "E": 8, "k": 4, "f": 256, "seed": 3},  # 75 per expert
+    {"dtype": "bf16", "T": 90, "d": 128, "E": 24, "k": 3, "f": 128, "bias": "zipf",
+     "n_shared": 0},                                                               # empty experts
+    {"dtype": "f32"},
+]
+
+
+@pytest.mark.parametrize("kw", CASES)
+def test_backward_matches_oracle(cuda_ok, kw):
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    dout = synth.make_x(w, w.T, device="cuda", seed=77)
+    g = layer.backward(inp.x, dout)
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    x, wr, _, wg, wu, wd = host_inputs(inp)
+    ref = oracle_moe_backward(x, synth.to_numpy_bits(dout), wr, wg, wu, wd,
+                              r["idx"].cpu().numpy(), r["gates"].cpu().numpy(),
+                              w.routed_scale, w.n_shared)
+    counts = r["counts"].cpu().numpy()
+    for name, want in ref.items():
+        got = g[name].cpu().numpy().astype(np.float64)
+        assert got.shape == want.shape, name
+        scale = np.abs(want).max()
+        # fp32 sums of products of exactly decoded inputs: far inside 2e-4 of the largest
+        # entry (the sums run over at most d = 4096 / f terms)
+        err = np.abs(got - want).max()
+        assert err <= 2e-4 * scale, (name, err, scale)
+    # experts no token chose get exactly zero weight gradients
+    unchosen = np.nonzero(counts == 0)[0]
+    for name in ("dw_gate", "dw_up", "dw_down"):
+        assert (g[name][unchosen] == 0).all()
+    assert (g["dw_router"][unchosen] == 0).all()
+    # deterministic
+    g2 = layer.backward(inp.x, dout)
+    torch.cuda.synchronize()
+    for name in g:
+        assert torch.equal(g[name], g2[name]), name
+    assert layer.device_status() == 0
+
+
+def test_backward_of_zero_dout_is_zero(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=20, d=128, E=8, k=2, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    g = layer.backward(inp.x, torch.zeros_like(inp.x))
+    torch.cuda.synchronize()
+    for name, t in g.items():
+        assert (t == 0).all(), name
