@@ -400,6 +400,102 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------- backward arm
+# fp32 CUDA-core peak of the backward kernels: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x
+# the 1965 MHz maximum SM clock
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args, rank, world, local_rank):
+    """Times moe_backward (gradients of <forward(x), dout>) on the workload: a separate
+    measurement, not the forward's headline line."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from sparse_moe_layer_warp_b200 import MoELayer, synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    T = w.T
+    inp = synth.make_inputs(w, device=dev)
+    layer = MoELayer(inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down, top_k=w.k,
+                     max_tokens=T, n_shared=w.n_shared, routed_scale=w.routed_scale)
+    nb = args.steps + args.warmup
+    xs = [synth.make_x(w, T, device=dev, seed=1000 * (rank + 1) + i) for i in range(nb)]
+    douts = [synth.make_x(w, T, device=dev, seed=5000 * (rank + 1) + i) for i in range(nb)]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    touched = []
+    for i in range(args.warmup, nb):
+        touched.append(int((layer.route(x=xs[i])["counts"] > 0).sum().item()) + w.n_shared)
+    # weight-gradient buffers allocated once; every step accumulates into them
+    grads = layer.backward(xs[0], douts[0])
+    for i in range(args.warmup):
+        flush.zero_()
+        layer.backward(xs[i], douts[i], grads=grads)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local_rank] if visible else local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(st)
+        layer.backward(xs[args.warmup + i], douts[args.warmup + i], grads=grads)
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    step_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
+    if layer.device_status() != 0:
+        raise RuntimeError("device status after the timed region")
+    if rank != 0:
+        return None
+    P = T * w.k + w.n_shared * T
+    es = 2 if w.dtype == "bf16" else 4
+    # recompute a and b, unscaled outputs, dh, rows of dx (two products), three weight
+    # gradients: 18 P f d flops; the router adds 4 T k d
+    flops = 18.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
+    # weights of the touched experts read four times (gate/up twice, down twice); their
+    # three fp32 weight gradients and the router's read and written (they accumulate)
+    tm = float(np.mean(touched))
+    nbytes = tm * 6 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+    step_s = total_ms / args.steps / 1e3
+    peaks, _ = load_peaks()
+    alu = flops / step_s / 1e12
+    hbm = nbytes / step_s / 1e9
+    ridge = FP32_ALU_TFLOPS * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / nbytes > ridge:
+        roof = {"bound": "alu", "achieved": round(alu, 2), "peak": round(FP32_ALU_TFLOPS, 1),
+                "unit": "TFLOP/s", "frac": round(alu / FP32_ALU_TFLOPS, 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(hbm, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(hbm / peaks["hbm_gbs"], 4)}
+    roof.update({"traffic": None, "kernel": "moe_backward (all kernels)",
+                 "algorithmic_flops_per_step": int(flops), "algorithmic_bytes_per_step": int(nbytes),
+                 "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; HBM measured"})
+    return {
+        "metric": "MoE-layer backward tokens/s on 1 B200 (fp32 CUDA-core kernels)",
+        "pass": "backward",
+        "value": round(job_throughput(T, args.steps, world, total_ms), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; fresh x and dout every step; random-init weights)",
+        "config": {"workload": w.name, "tokens": T, "d_model": w.d, "n_experts": w.E,
+                   "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared,
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)"},
+        "roofline": roof, "clocks": clocks,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -409,6 +505,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time moe_backward instead (a separate measurement)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -431,7 +529,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=None)
     try:
-        res = run_ours(args, rank, world, local_rank)
+        res = (run_backward if args.which == "backward" else run_ours)(args, rank, world,
+                                                                       local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()

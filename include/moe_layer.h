@@ -158,9 +158,11 @@ moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stre
  * selected unbiased router logits, so the router weights receive
  *   dl_j = g_j (dgate_j - sum_i g_i dgate_i),  dgate_j = routed_scale * (dout_t . y_j),
  * with y_j the unscaled output of the j-th selected expert.
- *   x, dout   [n_tokens, d] layer dtype          dx        [n_tokens, d] fp32
+ *   x, dout   [n_tokens, d] layer dtype          dx        [n_tokens, d] fp32 (overwritten)
  *   dw_router [E, d] fp32    dw_gate, dw_up [E + n_shared, f, d] fp32
- *   dw_down   [E + n_shared, d, f] fp32   (all overwritten; unchosen experts get zeros)
+ *   dw_down   [E + n_shared, d, f] fp32
+ * The weight gradients ACCUMULATE (+=) into the caller's buffers, as over micro-batches;
+ * rows of experts no token chose are not touched (zero the buffers before the first call).
  * ws: at least moe_backward_workspace_size(h, n_tokens) bytes, 256-byte aligned (it holds a
  * forward workspace at its start, which this call reuses).  fp32 accumulation on CUDA cores
  * in a fixed order: deterministic.  Errors as moe_forward. */

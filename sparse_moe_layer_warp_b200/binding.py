@@ -293,8 +293,9 @@ class MoELayer:
                          self.workspace(T), stream)
         return p_mean, f_sel, scalars
 
-    def backward(self, x, dout, stream=None):
-        """dict of fp32 gradients dx, dw_router, dw_gate, dw_up, dw_down (device tensors)."""
+    def backward(self, x, dout, stream=None, grads=None):
+        """dict of fp32 gradients dx, dw_router, dw_gate, dw_up, dw_down (device tensors); the
+        weight gradients are added to `grads`' tensors when given (new zeroed ones if not)."""
         T = x.shape[0]
         need = moe_backward_workspace_size(self.handle, T)
         if self.bw_ws is None or self.bw_ws.numel() < need:
@@ -303,9 +304,15 @@ class MoELayer:
         G = self.E + int(self.cfg.n_shared)
         f = int(self.cfg.d_ff)
         kw = dict(dtype=torch.float32, device=self.device)
-        g = dict(dx=torch.empty((T, self.d), **kw), dw_router=torch.empty((self.E, self.d), **kw),
-                 dw_gate=torch.empty((G, f, self.d), **kw), dw_up=torch.empty((G, f, self.d), **kw),
-                 dw_down=torch.empty((G, self.d, f), **kw))
+        if grads is not None:
+            g = dict(grads)
+            g["dx"] = torch.empty((T, self.d), **kw)
+        else:  # the weight gradients accumulate: start them at zero
+            g = dict(dx=torch.empty((T, self.d), **kw),
+                     dw_router=torch.zeros((self.E, self.d), **kw),
+                     dw_gate=torch.zeros((G, f, self.d), **kw),
+                     dw_up=torch.zeros((G, f, self.d), **kw),
+                     dw_down=torch.zeros((G, self.d, f), **kw))
         moe_backward(self.handle, x, T, dout, g["dx"], g["dw_router"], g["dw_gate"], g["dw_up"],
                      g["dw_down"], self.bw_ws, stream)
         return g

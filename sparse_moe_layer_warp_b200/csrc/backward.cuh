@@ -9,7 +9,9 @@
 //   a = W_g[g] x_t,  b = W_u[g] x_t,  h = silu(a) b,  yhat = W_d[g] h
 //   dy = s dout_t,  dh = W_d[g]^T dy,  da = dh b silu'(a),  db = dh silu(a)
 //   dX_p = W_g[g]^T da + W_u[g]^T db
-//   dW_d[g] = sum_p dy h^T,  dW_g[g] = sum_p da x_t^T,  dW_u[g] = sum_p db x_t^T
+//   dW_d[g] += sum_p dy h^T,  dW_g[g] += sum_p da x_t^T,  dW_u[g] += sum_p db x_t^T
+//   (weight gradients accumulate into the caller's buffers, as over micro-batches; experts
+//   no token chose are not touched)
 //   routed rows: dgate = routed_scale * (dout_t . yhat)
 // and for the router (gates = softmax of the selected unbiased logits):
 //   dl_j = g_j (dgate_j - sum_i g_i dgate_i),  dW_r[e] = sum dl x_t,  dx_t += sum dl W_r[e]
@@ -19,7 +21,7 @@
 // Three grouped row kernels do the matrix work (tiles of 16 rows of one group):
 //   bw_nt_kernel   out[p][m] = sum_k W[g][m][k] v_p[k]      (W row-major [M, K])
 //   bw_nn_kernel   out[p][n] = sum_k W[g][k][n] v_p[k]      (W row-major [K, N])
-//   bw_wgrad_kernel dW[g][m][n] = sum_{p in g} u_p[m] v_p[n]
+//   bw_wgrad_kernel dW[g][m][n] += sum_{p in g} u_p[m] v_p[n]
 // with the row vectors v_p, u_p produced on the fly by small source functors.
 #pragma once
 #include <cuda_bf16.h>
@@ -250,9 +252,9 @@ __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
 }
 
 // ------------------------------------------------------------------------- WGRAD
-// Block (g, m block of 32, n block of 64): dW[g][m][n] = sum over the group's rows p of
+// Block (g, m block of 32, n block of 64): dW[g][m][n] += sum over the group's rows p of
 // u_p[m] v_p[n], rows in order, 16 at a time.  Thread (mi = tid / 16, ni = tid % 16) owns
-// m = m0 + 2 mi + {0, 1}, n = n0 + ni + 16 j.  Groups with no rows get zeros.
+// m = m0 + 2 mi + {0, 1}, n = n0 + ni + 16 j.  Groups with no rows are left untouched.
 template <typename SrcU, typename SrcV>
 __global__ void __launch_bounds__(256) bw_wgrad_kernel(SrcU u, SrcV v, int M, int N,
                                                        const int *__restrict__ offsets, int E,
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(256) bw_wgrad_kernel(SrcU u, SrcV v, int M, in
   const int m0 = blockIdx.y * 32, n0 = blockIdx.z * 64;
   const int base = (g < E) ? offsets[g] : Tk + (g - E) * T;
   const int cnt = (g < E) ? offsets[g + 1] - offsets[g] : T;
+  if (cnt == 0) return;
   const int mi = threadIdx.x >> 4, ni = threadIdx.x & 15;
   float acc[2][4];
 #pragma unroll
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(256) bw_wgrad_kernel(SrcU u, SrcV v, int M, in
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + ni + 16 * j;
-      if (n < N) dW[((size_t)g * M + m) * N + n] = acc[a][j];
+      if (n < N) dW[((size_t)g * M + m) * N + n] += acc[a][j];
     }
   }
 }
@@ -357,7 +360,8 @@ __global__ void __launch_bounds__(256) bw_router_dl_kernel(const float *__restri
   }
 }
 
-// dW_r[e][i] = sum over the rows of routed group e (ascending token) of dl x_t[i].
+// dW_r[e][i] += sum over the rows of routed group e (ascending token) of dl x_t[i]; experts
+// no token chose are left untouched.
 template <typename Tin>
 __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict__ x,
                                                            const float *__restrict__ dl,
@@ -368,13 +372,13 @@ __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict
   griddep_launch_dependents();
   const int e = blockIdx.x;
   const int i = blockIdx.y * blockDim.x + threadIdx.x;
-  if (i >= d) return;
+  if (i >= d || offsets[e] == offsets[e + 1]) return;
   float acc = 0.f;
   for (int p = offsets[e]; p < offsets[e + 1]; ++p) {
     const int q = perm[p];
     acc = fmaf(dl[q], bw_f32(x[(size_t)(q / k) * d + i]), acc);
   }
-  dw_r[(size_t)e * d + i] = acc;
+  dw_r[(size_t)e * d + i] += acc;
 }
 
 // dx[t][i] = sum_j dX[slot_row[t,j]][i] + dX[shared row][i] + sum_j dl[t,j] W_r[e_j][i].

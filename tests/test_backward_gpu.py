@@ -42,7 +42,7 @@ def test_backward_matches_oracle(cuda_ok, kw):
         # entry (the sums run over at most d = 4096 / f terms)
         err = np.abs(got - want).max()
         assert err <= 2e-4 * scale, (name, err, scale)
-    # experts no token chose get exactly zero weight gradients
+    # experts no token chose keep their (zero) weight gradients
     unchosen = np.nonzero(counts == 0)[0]
     for name in ("dw_gate", "dw_up", "dw_down"):
         assert (g[name][unchosen] == 0).all()
@@ -52,6 +52,12 @@ def test_backward_matches_oracle(cuda_ok, kw):
     torch.cuda.synchronize()
     for name in g:
         assert torch.equal(g[name], g2[name]), name
+    # weight gradients accumulate: a second call into the same buffers adds the same amount
+    once = {n: g[n].clone() for n in g}
+    g3 = layer.backward(inp.x, dout, grads=g)
+    torch.cuda.synchronize()
+    for name in ("dw_router", "dw_gate", "dw_up", "dw_down"):
+        assert torch.equal(g3[name], 2 * once[name]), name
     assert layer.device_status() == 0
 
 
