@@ -640,7 +640,7 @@ namespace {
 // bf16 decode batches: router logits, selection and permutation in one launch
 bool decode_route_ok(const moe_config &c, int T) {
   return T <= kChunk && c.dtype == MOE_BF16 && c.n_experts <= kDecodeMaxExperts &&
-         c.d_model % 64 == 0 && c.d_model <= kDecodeMaxD;
+         c.d_model % (kDecodeWarps * 8) == 0 && c.d_model <= kDecodeMaxD;
 }
 
 moe_status launch_route_decode(const moe_layer *L, const void *x, int T, float *logits,
@@ -649,7 +649,7 @@ moe_status launch_route_decode(const moe_layer *L, const void *x, int T, float *
                                cudaStream_t st) {
   const moe_config &c = L->cfg;
   return launch(route_decode_kernel, dim3((c.n_experts + kDecodeEPC - 1) / kDecodeEPC),
-                dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(x),
+                dim3(kDecodeWarps * 32), 0, st, static_cast<const __nv_bfloat16 *>(x),
                 static_cast<const __nv_bfloat16 *>(L->w.w_router), L->w.router_bias, T,
                 c.d_model, c.n_experts, c.top_k, logits, idx, gate, counts, offsets, perm,
                 slot_row, &status->router_ticket[31], reset);

@@ -441,18 +441,19 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_small_kernel(
 }
 
 // ------------------------------------------------------------ decode: router + routing
-// T <= kChunk tokens, bf16, E <= kDecodeMaxExperts, d a multiple of 64 and at most
-// kDecodeMaxD: the router logits and the routing in ONE launch.  CTA c computes experts
-// e0 = kDecodeEPC*c .. +kDecodeEPC over the full reduction: warp w takes the K slice
-// [w*d/8, (w+1)*d/8), each lane 16-byte chunks of it (the CTA's router rows are loaded
+// T <= kChunk tokens, bf16, E <= kDecodeMaxExperts, d a multiple of 128 and at most
+// kDecodeMaxD: the router logits and the routing in ONE launch.  CTA c (kDecodeWarps warps)
+// computes experts e0 = kDecodeEPC*c .. +kDecodeEPC over the full reduction: warp w takes
+// the K slice [w*d/16, (w+1)*d/16), each lane 16-byte chunks of it (the CTA's router rows are loaded
 // before the grid-dependency wait: they never depend on earlier kernels); per group of 16
 // tokens the 32 (expert, token) partial sums of a lane are summed across the warp by a
-// butterfly that leaves sum j in lane j (31 shuffles), then across the 8 warps in a fixed
+// butterfly that leaves sum j in lane j (31 shuffles), then across the warps in a fixed
 // order -- fp32 throughout, deterministic.  The CTA that finishes last (a ticket, reset by
-// that CTA) then runs route_small_block on all logits.
+// that CTA) then runs route_small_block on all logits, one token per warp.
 constexpr int kDecodeEPC = 2;          // experts per CTA
 constexpr int kDecodeMaxExperts = 288; // MAXV = 9 top-k and at most 144 CTAs
-constexpr int kDecodeMaxD = 8192;      // at most 4 chunks of 8 per lane
+constexpr int kDecodeMaxD = 8192;      // at most 2 chunks of 8 per lane
+constexpr int kDecodeWarps = 16;
 
 __device__ __forceinline__ float dot8_bf16(const uint4 a, const uint4 b) {
   const __nv_bfloat162 *pa = reinterpret_cast<const __nv_bfloat162 *>(&a);
@@ -468,19 +469,20 @@ __device__ __forceinline__ float dot8_bf16(const uint4 a, const uint4 b) {
   return s;
 }
 
-__global__ void __launch_bounds__(256) route_decode_kernel(
+__global__ void __launch_bounds__(kDecodeWarps * 32) route_decode_kernel(
     const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
     const float *__restrict__ bias, int T, int d, int E, int k, float *__restrict__ logits,
     int *__restrict__ topk_idx, float *__restrict__ topk_gate, int *__restrict__ counts,
     int *__restrict__ offsets, int *__restrict__ perm, int *__restrict__ slot_row,
     int *__restrict__ ticket, CounterReset reset) {
-  constexpr int EPC = kDecodeEPC, TG = 16, MAXC = kDecodeMaxD / 64 / 32;
+  constexpr int EPC = kDecodeEPC, TG = 16, NW = kDecodeWarps;
+  constexpr int MAXC = kDecodeMaxD / (NW * 8) / 32;
   static_assert(EPC * TG == 32, "one butterfly value per lane");
-  __shared__ float red[8][32];
+  __shared__ float red[NW][32];
   __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * EPC;
-  const int slice = d / 8;         // this warp's K range
+  const int slice = d / NW;        // this warp's K range
   const int chunks = slice / 8;    // 16-byte chunks in it
   uint4 w[MAXC][EPC];
 #pragma unroll
@@ -540,7 +542,7 @@ __global__ void __launch_bounds__(256) route_decode_kernel(
     if (threadIdx.x < 32) {
       float v = 0.f;
 #pragma unroll
-      for (int ww = 0; ww < 8; ++ww) v += red[ww][threadIdx.x];
+      for (int ww = 0; ww < NW; ++ww) v += red[ww][threadIdx.x];
       const int e = threadIdx.x / TG, t = threadIdx.x % TG;
       if (tg + t < T && e0 + e < E) logits[(size_t)(tg + t) * E + e0 + e] = v;
     }
