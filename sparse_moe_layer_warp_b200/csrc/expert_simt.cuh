@@ -105,13 +105,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     const int t = (int)(i / vpr);
     const int c = (int)(i % vpr) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const int p = __ldg(slot_row + (size_t)t * k + j);
-      const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)p * d + c));
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+    // eight slots at a time: their row indices, then their rows, are loaded before the
+    // first add, so the loads are in flight together; the sum keeps slot order
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int p[8];
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        p[j] = (j0 + j < k) ? __ldg(slot_row + (size_t)t * k + j0 + j) : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = (j0 + j < k) ? __ldg(reinterpret_cast<const float4 *>(y + (size_t)p[j] * d + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j0 + j < k) {
+          acc.x += v[j].x;
+          acc.y += v[j].y;
+          acc.z += v[j].z;
+          acc.w += v[j].w;
+        }
+      }
     }
     if (n_shared) {
       const float4 v = __ldg(reinterpret_cast<const float4 *>(y + (size_t)(Tk + t) * d + c));
