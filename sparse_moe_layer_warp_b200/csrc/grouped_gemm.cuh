@@ -14,7 +14,8 @@
 // every SM streams weight tiles from HBM through TMA.
 //
 //   MODE_UP   : A0 = W_gate, A1 = W_up (two accumulators), B = the group's x rows;
-//               epilogue h = silu(G) * U -> bf16.  With token tiles of up to 32 rows the
+//               epilogue h = silu(G) * U -> bf16 (with out2 set: G and U in fp32, for the
+//               backward's recompute).  With token tiles of up to 32 rows the
 //               rows are gathered from x by token id with tile::gather4 (four rows per copy:
 //               the "gather" of section 3.2.4 fused into the operand load, no expert-sorted
 //               copy of x); larger tiles load expert-sorted rows xs written by the gather
@@ -58,6 +59,8 @@ struct GemmParams {
   const int *perm;          // [Tk] sorted row -> t*k + j (UP: token of a row; DOWN: gate)
   const float *topk_gate;   // [Tk] (DOWN)
   void *out;                // UP: h [P, f] bf16; DOWN: y [P, d] fp32; LOGITS: [T, E] fp32
+  float *out2;              // UP with out2 set: out = fp32 pre-activation x W_g^T, out2 =
+                            // x W_u^T, [P, f] each, instead of h (for the backward)
   DevStatus *status;
   float routed_scale;
   int E, n_groups, T, Tk;
@@ -544,7 +547,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (MODE == MODE_UP) tmem_ld16(taddr + BN + c0 + 16, n1);
         }
         float vals[16];
-        if (MODE == MODE_UP) {
+        if (MODE == MODE_UP && p.out2) {  // the pre-activations themselves (backward)
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v0[n]);
+          store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
+                            vals, wbuf, lane);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v1[n]);
+          store_block16_f32(p.out2, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+        } else if (MODE == MODE_UP) {
 #pragma unroll
           for (int n = 0; n < 16; ++n)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));

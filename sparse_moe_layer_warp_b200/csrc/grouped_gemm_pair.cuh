@@ -419,7 +419,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (MODE == MODE_UP) tmem_ld16(taddr + BN + c0 + 32, n1);
         }
         float vals[16];
-        if (MODE == MODE_UP) {
+        if (MODE == MODE_UP && p.out2) {  // the pre-activations themselves (backward)
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v0[n]);
+          store_block16_f32(static_cast<float *>(p.out), p.ld_out, row0, c0, valid, col_base,
+                            vals, wbuf, lane);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v1[n]);
+          store_block16_f32(p.out2, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+        } else if (MODE == MODE_UP) {
 #pragma unroll
           for (int n = 0; n < 16; ++n)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));

@@ -736,6 +736,57 @@ ForwardPlan plan_forward(const moe_layer *L, int T) {
   f.launches = routing + gather + 3;  // + up, down, combine
   return f;
 }
+
+// bf16: the expert-sorted copy of x rows, unless the up GEMM gathers them itself.
+moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
+                             const WsLayout &W, const ForwardPlan &plan, cudaStream_t st) {
+  if (plan.gather_in_gemm) return MOE_OK;
+  const moe_config &c = h->cfg;
+  const int Tk = T * c.top_k;
+  return launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)), dim3(256), 0, st,
+                static_cast<const uint4 *>(x), (const int *)at<int>(ws, W.perm), c.top_k, Tk,
+                c.d_model / 8, at<uint4>(ws, W.xs));
+}
+
+// bf16 expert up GEMM over the routing in `ws`: h (bf16, `out`) -- or, with out2 set, the
+// fp32 pre-activations x W_g^T (`out`) and x W_u^T (`out2`).  done: the per-group h
+// hand-over counts (null: none).  *used receives the parameters (the down GEMM's start).
+moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
+                            const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
+                            int *done, cudaStream_t st, GemmParams *used) {
+  const moe_config &c = h->cfg;
+  const int Tk = T * c.top_k;
+  // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
+  const int bn = plan.pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
+  GemmParams &p1 = *used;
+  memset(&p1, 0, sizeof p1);
+  p1.tmA0 = h->tm_wg;
+  p1.tmA1 = h->tm_wu;
+  if (plan.gather_in_gemm) {
+    if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
+  } else if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
+             !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
+    return MOE_ERR_CUDA;
+  }
+  p1.offsets = at<int>(ws, W.offsets);
+  p1.perm = at<int>(ws, W.perm);
+  p1.topk_gate = at<float>(ws, W.gate);
+  p1.out = out;
+  p1.out2 = out2;
+  p1.status = at<DevStatus>(ws, W.status);
+  p1.routed_scale = c.routed_scale;
+  p1.E = c.n_experts;
+  p1.n_groups = c.n_experts + c.n_shared;
+  p1.T = T;
+  p1.Tk = Tk;
+  p1.M = c.d_ff;
+  p1.K = c.d_model;
+  p1.ld_out = c.d_ff;
+  p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
+  p1.topk = c.top_k;
+  p1.done = done;
+  return plan.pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st);
+}
 }  // namespace
 
 extern "C" {
@@ -801,50 +852,17 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
 
   if (c.dtype == MOE_BF16) {
     const bool pair = plan.pair;
-    // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
     const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
-    // small token tiles: the up GEMM gathers its rows from x (no expert-sorted copy)
-    const bool gather_in_gemm = plan.gather_in_gemm;
-    const int vpr = c.d_model / 8;
-    if (!gather_in_gemm &&
-        (s = launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)),
-                    dim3(256), 0, st, static_cast<const uint4 *>(x), (const int *)perm,
-                    c.top_k, Tk, vpr, at<uint4>(ws, W.xs))) != MOE_OK)
+    if ((s = launch_row_gather(h, x, T, ws, W, plan, st)) != MOE_OK || (s = mark(4)) != MOE_OK)
       return s;
-    if ((s = mark(4)) != MOE_OK) return s;
     const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
     __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
     float *ybuf = at<float>(ws, W.y);
-    GemmParams p1;
-    memset(&p1, 0, sizeof p1);
-    p1.tmA0 = h->tm_wg;
-    p1.tmA1 = h->tm_wu;
-    if (gather_in_gemm) {
-      if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
-    } else if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
-               !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
-      return MOE_ERR_CUDA;
-    }
-    p1.offsets = offsets;
-    p1.perm = perm;
-    p1.topk_gate = gate;
-    p1.out = hbuf;
-    p1.status = at<DevStatus>(ws, W.status);
-    p1.routed_scale = c.routed_scale;
-    p1.E = c.n_experts;
-    p1.n_groups = c.n_experts + c.n_shared;
-    p1.T = T;
-    p1.Tk = Tk;
-    p1.M = c.d_ff;
-    p1.K = c.d_model;
-    p1.ld_out = c.d_ff;
-    p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
-    p1.topk = c.top_k;
     // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
     // expert group for that group's rows of h (see grouped_gemm_kernel)
-    p1.done = at<int>(ws, W.done);
-    if ((s = pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st)) !=
-        MOE_OK)
+    GemmParams p1;
+    if ((s = launch_expert_up(h, x, T, ws, W, plan, hbuf, nullptr, at<int>(ws, W.done), st,
+                              &p1)) != MOE_OK)
       return s;
     if ((s = mark(5)) != MOE_OK) return s;
     GemmParams p2 = p1;
@@ -1068,11 +1086,19 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   const SrcDy<T_> src_dy{dout, row_token, row_scale, d};
   const SrcH src_h{a, b, f};
   const SrcRow src_da{dh, f}, src_db{db, f};
-  // 3. pre-activations a, b; unscaled expert outputs; dgate
-  if ((s = launch(bw_nt_kernel<2, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256), 0, st,
-                  wg, wu, f, d, src_x, (const int *)tile_prefix, (const int *)offsets, E, G, T,
-                  Tk, a, b)) != MOE_OK ||
-      (s = launch(bw_nt_kernel<1, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
+  // 3. pre-activations a, b (bf16: the forward's tcgen05 up GEMM storing them in fp32);
+  //    unscaled expert outputs; dgate
+  if (c.dtype == MOE_BF16) {
+    GemmParams pu;
+    if ((s = launch_row_gather(L, x, T, ws, W, plan, st)) != MOE_OK ||
+        (s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu)) != MOE_OK)
+      return s;
+  } else if ((s = launch(bw_nt_kernel<2, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256),
+                         0, st, wg, wu, f, d, src_x, (const int *)tile_prefix,
+                         (const int *)offsets, E, G, T, Tk, a, b)) != MOE_OK) {
+    return s;
+  }
+  if ((s = launch(bw_nt_kernel<1, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
                   wd, d, f, src_h, (const int *)tile_prefix, (const int *)offsets, E, G, T, Tk,
                   wide, wide)) != MOE_OK ||
       (s = launch(bw_dgate_kernel<T_>, dim3(grid_for(Tk, 8, L->num_sms)), dim3(256), 0, st,
