@@ -355,6 +355,38 @@ def cpu_baseline(w, inp, x_batch, budget_s=15.0, host=None):
                       f"OpenMP over tokens)"}
 
 
+def cpu_baseline_backward(w, inp, x_batch, dout_batch, idx, gates, budget_s=10.0):
+    """The oracle's backward, as it stands (single-threaded, fp64), on tokens of one batch
+    taken one at a time until the budget is spent (tokens/s)."""
+    from oracle import oracle_moe_backward
+    from sparse_moe_layer_warp_b200 import synth
+
+    import numpy as np
+
+    wr, _, wg, wu, wd = _host_weights(inp)
+    x = synth.to_numpy_bits(x_batch)
+    o = synth.to_numpy_bits(dout_batch)
+    E = w.E
+    done, el = 0, 0.0
+    while el < budget_s:
+        t = done % x.shape[0]
+        # the token's own experts (and the shared one) only: the oracle's dense fp64
+        # gradients of all experts would not fit in host memory at full size
+        sel = np.concatenate([idx[t], np.arange(E, E + w.n_shared)]).astype(np.int64)
+        args = (x[t:t + 1], o[t:t + 1], np.ascontiguousarray(wr[idx[t]]),
+                np.ascontiguousarray(wg[sel]), np.ascontiguousarray(wu[sel]),
+                np.ascontiguousarray(wd[sel]), np.arange(w.k, dtype=np.int32)[None],
+                gates[t:t + 1])
+        t0 = time.perf_counter()
+        oracle_moe_backward(*args, w.routed_scale, w.n_shared)
+        el += time.perf_counter() - t0
+        done += 1
+    return {"value": round(done / el, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} tokens of one {w.name} batch, one at a time ({el:.1f} s of the "
+                      f"plain-C fp64 oracle backward, single-threaded, on each token's "
+                      f"{w.k} + {w.n_shared} experts)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -493,7 +525,14 @@ def run_backward(args, rank, world, local_rank):
                    "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared,
                    "l2": "flushed between timed steps (256 MiB write, outside the events)"},
         "roofline": roof, "clocks": clocks,
-    }
+    } | ({} if args.no_cpu_baseline else {"cpu_baseline": cpu_baseline_backward(
+        w, inp, xs[args.warmup], douts[args.warmup], *_routing_np(layer, xs[args.warmup]),
+        budget_s=min(args.cpu_budget, 10.0))})
+
+
+def _routing_np(layer, x):
+    r = layer.route(x=x)
+    return r["idx"].cpu().numpy(), r["gates"].cpu().numpy()
 
 
 def main():
