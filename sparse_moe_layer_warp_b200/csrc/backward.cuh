@@ -137,9 +137,29 @@ __device__ __forceinline__ bool bw_tile(int b, const int *tile_prefix, const int
   return true;
 }
 
+// 8 consecutive weights as floats (16 bytes of bf16, or 32 of fp32).
+__device__ __forceinline__ void bw_load8(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 r = __ldg(reinterpret_cast<const uint4 *>(p));
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void bw_load8(const float *p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4 *>(p + 4));
+  v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+  v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+
 // ---------------------------------------------------------------------------- NT
 // Block (tile, m block of 64): out_j[p][m] = sum_k W_j[g][m][k] v_p[k] for j < NW (the
-// matrices share v).  Thread (r = tid / 16, c = tid % 16) owns row r and m = c + 16 i.
+// matrices share v).  K and M are multiples of 8 (the weight tile is staged with one
+// 16-byte load per thread and matrix).  Thread (r = tid / 16, c = tid % 16) owns row r
+// and m = c + 16 i.
 template <int NW, typename Tw, typename Src>
 __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
                                                     const Tw *__restrict__ W1, int M, int K,
@@ -161,15 +181,21 @@ __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
   const Tw *Wj[2] = {W0, W1};
+  // weight tile staging: thread -> (row mm = tid / 4, 8 columns at kq = 8 (tid % 4))
+  const int mm = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 8;
   for (int k0 = 0; k0 < K; k0 += kBwK) {
 #pragma unroll
-    for (int j = 0; j < NW; ++j)
-      for (int e = threadIdx.x; e < 64 * kBwK; e += blockDim.x) {
-        const int mm = e / kBwK, kk = e % kBwK;
-        const int m = m0 + mm, kx = k0 + kk;
-        ws[j][mm][kk] =
-            (m < M && kx < K) ? bw_f32(Wj[j][((size_t)g * M + m) * K + kx]) : 0.f;
+    for (int j = 0; j < NW; ++j) {
+      float w8[8];
+      if (m0 + mm < M && k0 + kq < K) {
+        bw_load8(Wj[j] + ((size_t)g * M + m0 + mm) * K + k0 + kq, w8);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w8[i] = 0.f;
       }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ws[j][mm][kq + i] = w8[i];
+    }
     for (int e = threadIdx.x; e < kBwRows * kBwK; e += blockDim.x) {
       const int rr = e / kBwK, kk = e % kBwK;
       vs[rr][kk] = (rr < rows && k0 + kk < K) ? src(row0 + rr, k0 + kk) : 0.f;
@@ -198,7 +224,8 @@ __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
 }
 
 // ---------------------------------------------------------------------------- NN
-// Block (tile, n block of 64): out[p][n] = sum_j sum_k W_j[g][k][n] v_j,p[k].
+// Block (tile, n block of 64): out[p][n] = sum_j sum_k W_j[g][k][n] v_j,p[k]; N a multiple
+// of 8 (one 16-byte weight load per thread and matrix per stage).
 template <int NW, typename Tw, typename Src0, typename Src1>
 __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
                                                     const Tw *__restrict__ W1, int K, int N,
@@ -216,15 +243,21 @@ __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
   const int r = threadIdx.x >> 4, c = threadIdx.x & 15;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const Tw *Wj[2] = {W0, W1};
+  // weight tile staging: thread -> (row kk = tid / 8, 8 columns at nq = 8 (tid % 8))
+  const int kr = threadIdx.x >> 3, nq = (threadIdx.x & 7) * 8;
   for (int k0 = 0; k0 < K; k0 += kBwK) {
 #pragma unroll
-    for (int j = 0; j < NW; ++j)
-      for (int e = threadIdx.x; e < kBwK * 64; e += blockDim.x) {
-        const int kk = e / 64, nn = e % 64;
-        const int kx = k0 + kk, n = n0 + nn;
-        ws[j][kk][nn] =
-            (kx < K && n < N) ? bw_f32(Wj[j][((size_t)g * K + kx) * N + n]) : 0.f;
+    for (int j = 0; j < NW; ++j) {
+      float w8[8];
+      if (k0 + kr < K && n0 + nq < N) {
+        bw_load8(Wj[j] + ((size_t)g * K + k0 + kr) * N + n0 + nq, w8);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w8[i] = 0.f;
       }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ws[j][kr][nq + i] = w8[i];
+    }
     for (int e = threadIdx.x; e < kBwRows * kBwK; e += blockDim.x) {
       const int rr = e / kBwK, kk = e % kBwK;
       const bool in = rr < rows && k0 + kk < K;
@@ -252,59 +285,65 @@ __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
 }
 
 // ------------------------------------------------------------------------- WGRAD
-// Block (g, m block of 32, n block of 64): dW[g][m][n] += sum over the group's rows p of
+// Block (g, m block of 64, n block of 128): dW[g][m][n] += sum over the group's rows p of
 // u_p[m] v_p[n], rows in order, 16 at a time.  Thread (mi = tid / 16, ni = tid % 16) owns
-// m = m0 + 2 mi + {0, 1}, n = n0 + ni + 16 j.  Groups with no rows are left untouched.
+// m = m0 + 4 mi + {0..3} and n = n0 + 8 ni + {0..7} (N a multiple of 8: the gradient is
+// read and written as float4).  Groups with no rows are left untouched.
 template <typename SrcU, typename SrcV>
 __global__ void __launch_bounds__(256) bw_wgrad_kernel(SrcU u, SrcV v, int M, int N,
                                                        const int *__restrict__ offsets, int E,
                                                        int T, int Tk, float *dW) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ float us[kBwRows][32 + 1];
-  __shared__ float vsm[kBwRows][64 + 1];
+  __shared__ float us[kBwRows][64 + 4];
+  __shared__ float vsm[kBwRows][128 + 4];
   const int g = blockIdx.x;
-  const int m0 = blockIdx.y * 32, n0 = blockIdx.z * 64;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.z * 128;
   const int base = (g < E) ? offsets[g] : Tk + (g - E) * T;
   const int cnt = (g < E) ? offsets[g + 1] - offsets[g] : T;
   if (cnt == 0) return;
   const int mi = threadIdx.x >> 4, ni = threadIdx.x & 15;
-  float acc[2][4];
+  float acc[4][8];
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[a][j] = 0.f;
+    for (int j = 0; j < 8; ++j) acc[a][j] = 0.f;
   for (int r0 = 0; r0 < cnt; r0 += kBwRows) {
     const int rows = min(kBwRows, cnt - r0);
-    for (int e = threadIdx.x; e < kBwRows * 32; e += blockDim.x) {
-      const int rr = e / 32, mm = e % 32;
+    for (int e = threadIdx.x; e < kBwRows * 64; e += blockDim.x) {
+      const int rr = e / 64, mm = e % 64;
       us[rr][mm] = (rr < rows && m0 + mm < M) ? u(base + r0 + rr, m0 + mm) : 0.f;
     }
-    for (int e = threadIdx.x; e < kBwRows * 64; e += blockDim.x) {
-      const int rr = e / 64, nn = e % 64;
+    for (int e = threadIdx.x; e < kBwRows * 128; e += blockDim.x) {
+      const int rr = e / 128, nn = e % 128;
       vsm[rr][nn] = (rr < rows && n0 + nn < N) ? v(base + r0 + rr, n0 + nn) : 0.f;
     }
     __syncthreads();
     for (int rr = 0; rr < rows; ++rr) {
-      const float u0 = us[rr][2 * mi], u1 = us[rr][2 * mi + 1];
+      const float4 ua = *reinterpret_cast<const float4 *>(&us[rr][4 * mi]);
+      const float4 v0 = *reinterpret_cast<const float4 *>(&vsm[rr][8 * ni]);
+      const float4 v1 = *reinterpret_cast<const float4 *>(&vsm[rr][8 * ni + 4]);
+      const float uu[4] = {ua.x, ua.y, ua.z, ua.w};
+      const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float vv = vsm[rr][ni + 16 * j];
-        acc[0][j] = fmaf(u0, vv, acc[0][j]);
-        acc[1][j] = fmaf(u1, vv, acc[1][j]);
-      }
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[a][j] = fmaf(uu[a], vv[j], acc[a][j]);
     }
     __syncthreads();
   }
+  const int n = n0 + 8 * ni;
+  if (n >= N) return;
 #pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    const int m = m0 + 2 * mi + a;
+  for (int a = 0; a < 4; ++a) {
+    const int m = m0 + 4 * mi + a;
     if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + ni + 16 * j;
-      if (n < N) dW[((size_t)g * M + m) * N + n] += acc[a][j];
-    }
+    float4 *dst = reinterpret_cast<float4 *>(dW + ((size_t)g * M + m) * N + n);
+    float4 x0 = dst[0], x1 = dst[1];
+    x0.x += acc[a][0], x0.y += acc[a][1], x0.z += acc[a][2], x0.w += acc[a][3];
+    x1.x += acc[a][4], x1.y += acc[a][5], x1.z += acc[a][6], x1.w += acc[a][7];
+    dst[0] = x0;
+    dst[1] = x1;
   }
 }
 

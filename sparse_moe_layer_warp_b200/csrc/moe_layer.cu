@@ -575,7 +575,10 @@ moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *d
     return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < bw_layout(h->cfg, n_tokens).total) return MOE_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_ALIGNMENT;
-  if (!aligned16(x) || !aligned16(dout) || !aligned16(dx)) return MOE_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(dout) || !aligned16(dx) || !aligned16(dw_router) ||
+      !aligned16(dw_gate) || !aligned16(dw_up) || !aligned16(dw_down))
+    return MOE_ERR_ALIGNMENT;
+  if (h->cfg.d_ff % 8 != 0) return MOE_ERR_UNSUPPORTED;  // 8-wide weight and gradient rows
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (h->cfg.dtype == MOE_BF16)
     return backward_impl(h, static_cast<const __nv_bfloat16 *>(x),
@@ -1109,7 +1112,7 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   if ((s = launch(bw_nn_kernel<1, T_, SrcDy<T_>, SrcDy<T_>>, dim3(n_tiles, cdiv(f, 64)),
                   dim3(256), 0, st, wd, wd, d, f, src_dy, src_dy, (const int *)tile_prefix,
                   (const int *)offsets, E, G, T, Tk, dh)) != MOE_OK ||
-      (s = launch(bw_wgrad_kernel<SrcDy<T_>, SrcH>, dim3(G, cdiv(d, 32), cdiv(f, 64)),
+      (s = launch(bw_wgrad_kernel<SrcDy<T_>, SrcH>, dim3(G, cdiv(d, 64), cdiv(f, 128)),
                   dim3(256), 0, st, src_dy, src_h, d, f, (const int *)offsets, E, T, Tk,
                   dw_down)) != MOE_OK ||
       (s = launch(bw_swiglu_kernel, dim3(grid_for((size_t)P * f, 256, L->num_sms)), dim3(256),
@@ -1119,10 +1122,10 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   if ((s = launch(bw_nn_kernel<2, T_, SrcRow, SrcRow>, dim3(n_tiles, cdiv(d, 64)), dim3(256),
                   0, st, wg, wu, f, d, src_da, src_db, (const int *)tile_prefix,
                   (const int *)offsets, E, G, T, Tk, wide)) != MOE_OK ||
-      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 32), cdiv(d, 64)),
+      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 64), cdiv(d, 128)),
                   dim3(256), 0, st, src_da, src_x, f, d, (const int *)offsets, E, T, Tk,
                   dw_gate)) != MOE_OK ||
-      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 32), cdiv(d, 64)),
+      (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 64), cdiv(d, 128)),
                   dim3(256), 0, st, src_db, src_x, f, d, (const int *)offsets, E, T, Tk,
                   dw_up)) != MOE_OK)
     return s;
