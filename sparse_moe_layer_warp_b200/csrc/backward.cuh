@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256) bw_rows_kernel(const int *__restrict__ pe
 }
 
 __global__ void __launch_bounds__(32) bw_tiles_kernel(const int *__restrict__ offsets, int E,
-                                                      int G, int T, int *tile_prefix) {
+                                                      int G, int T, int R, int *tile_prefix) {
   griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x != 0) return;
@@ -112,12 +112,14 @@ __global__ void __launch_bounds__(32) bw_tiles_kernel(const int *__restrict__ of
   for (int g = 0; g < G; ++g) {
     tile_prefix[g] = acc;
     const int cnt = (g < E) ? offsets[g + 1] - offsets[g] : T;
-    acc += (cnt + kBwRows - 1) / kBwRows;
+    acc += (cnt + R - 1) / R;
   }
   tile_prefix[G] = acc;
 }
 
-// Tile b of the row-tile list -> group, first row, rows.  Returns false past the list.
+// Tile b of the row-tile list (tiles of R rows) -> group, first row, rows.  Returns false
+// past the list.
+template <int R>
 __device__ __forceinline__ bool bw_tile(int b, const int *tile_prefix, const int *offsets,
                                         int E, int G, int T, int Tk, int &g, int &row0,
                                         int &rows) {
@@ -132,8 +134,8 @@ __device__ __forceinline__ bool bw_tile(int b, const int *tile_prefix, const int
   const int base = (g < E) ? offsets[g] : Tk + (g - E) * T;
   const int cnt = (g < E) ? offsets[g + 1] - offsets[g] : T;
   const int i = b - tile_prefix[g];
-  row0 = base + i * kBwRows;
-  rows = min(kBwRows, cnt - i * kBwRows);
+  row0 = base + i * R;
+  rows = min(R, cnt - i * R);
   return true;
 }
 
@@ -156,11 +158,11 @@ __device__ __forceinline__ void bw_load8(const float *p, float (&v)[8]) {
 }
 
 // ---------------------------------------------------------------------------- NT
-// Block (tile, m block of 64): out_j[p][m] = sum_k W_j[g][m][k] v_p[k] for j < NW (the
-// matrices share v).  K and M are multiples of 8 (the weight tile is staged with one
-// 16-byte load per thread and matrix).  Thread (r = tid / 16, c = tid % 16) owns row r
-// and m = c + 16 i.
-template <int NW, typename Tw, typename Src>
+// Block (tile of R rows, m block of 64): out_j[p][m] = sum_k W_j[g][m][k] v_p[k] for j < NW
+// (the matrices share v).  K and M are multiples of 8 (the weight tile is staged with one
+// 16-byte load per thread and matrix).  Thread (r = tid / 16, c = tid % 16) owns rows
+// r + 16 a (a < R / 16) and m = c + 16 i: R / 16 x 4 outputs.
+template <int NW, int R, typename Tw, typename Src>
 __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
                                                     const Tw *__restrict__ W1, int M, int K,
                                                     Src src, const int *__restrict__ tile_prefix,
@@ -169,17 +171,20 @@ __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
                                                     float *out1) {
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int RA = R / 16;
   __shared__ float ws[NW][64][kBwK + 1];
-  __shared__ float vs[kBwRows][kBwK + 1];
+  __shared__ float vs[R][kBwK + 1];
   int g, row0, rows;
-  if (!bw_tile(blockIdx.x, tile_prefix, offsets, E, G, T, Tk, g, row0, rows)) return;
+  if (!bw_tile<R>(blockIdx.x, tile_prefix, offsets, E, G, T, Tk, g, row0, rows)) return;
   const int m0 = blockIdx.y * 64;
   const int r = threadIdx.x >> 4, c = threadIdx.x & 15;
-  float acc[NW][4];
+  float acc[NW][RA][4];
 #pragma unroll
   for (int j = 0; j < NW; ++j)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+    for (int a = 0; a < RA; ++a)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[j][a][i] = 0.f;
   const Tw *Wj[2] = {W0, W1};
   // weight tile staging: thread -> (row mm = tid / 4, 8 columns at kq = 8 (tid % 4))
   const int mm = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 8;
@@ -196,37 +201,48 @@ __global__ void __launch_bounds__(256) bw_nt_kernel(const Tw *__restrict__ W0,
 #pragma unroll
       for (int i = 0; i < 8; ++i) ws[j][mm][kq + i] = w8[i];
     }
-    for (int e = threadIdx.x; e < kBwRows * kBwK; e += blockDim.x) {
+    for (int e = threadIdx.x; e < R * kBwK; e += blockDim.x) {
       const int rr = e / kBwK, kk = e % kBwK;
       vs[rr][kk] = (rr < rows && k0 + kk < K) ? src(row0 + rr, k0 + kk) : 0.f;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int kk = 0; kk < kBwK; ++kk) {
-      const float v = vs[r][kk];
+      float v[RA], w[NW][4];
+#pragma unroll
+      for (int a = 0; a < RA; ++a) v[a] = vs[r + 16 * a][kk];
 #pragma unroll
       for (int j = 0; j < NW; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[j][i] = fmaf(ws[j][c + 16 * i][kk], v, acc[j][i]);
+        for (int i = 0; i < 4; ++i) w[j][i] = ws[j][c + 16 * i][kk];
+#pragma unroll
+      for (int j = 0; j < NW; ++j)
+#pragma unroll
+        for (int a = 0; a < RA; ++a)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[j][a][i] = fmaf(w[j][i], v[a], acc[j][a][i]);
     }
     __syncthreads();
   }
-  if (r < rows) {
-    float *outs[2] = {out0, out1};
+  float *outs[2] = {out0, out1};
+#pragma unroll
+  for (int a = 0; a < RA; ++a) {
+    if (r + 16 * a >= rows) continue;
 #pragma unroll
     for (int j = 0; j < NW; ++j)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = m0 + c + 16 * i;
-        if (m < M) outs[j][(size_t)(row0 + r) * M + m] = acc[j][i];
+        if (m < M) outs[j][(size_t)(row0 + r + 16 * a) * M + m] = acc[j][a][i];
       }
   }
 }
 
 // ---------------------------------------------------------------------------- NN
-// Block (tile, n block of 64): out[p][n] = sum_j sum_k W_j[g][k][n] v_j,p[k]; N a multiple
-// of 8 (one 16-byte weight load per thread and matrix per stage).
-template <int NW, typename Tw, typename Src0, typename Src1>
+// Block (tile of R rows, n block of 64): out[p][n] = sum_j sum_k W_j[g][k][n] v_j,p[k]; N a
+// multiple of 8 (one 16-byte weight load per thread and matrix per stage).  Thread
+// (r, c) owns rows r + 16 a and n = c + 16 i.
+template <int NW, int R, typename Tw, typename Src0, typename Src1>
 __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
                                                     const Tw *__restrict__ W1, int K, int N,
                                                     Src0 src0, Src1 src1,
@@ -235,13 +251,18 @@ __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
                                                     int G, int T, int Tk, float *out) {
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int RA = R / 16;
   __shared__ float ws[NW][kBwK][64 + 1];
-  __shared__ float vs[NW][kBwRows][kBwK + 1];
+  __shared__ float vs[NW][R][kBwK + 1];
   int g, row0, rows;
-  if (!bw_tile(blockIdx.x, tile_prefix, offsets, E, G, T, Tk, g, row0, rows)) return;
+  if (!bw_tile<R>(blockIdx.x, tile_prefix, offsets, E, G, T, Tk, g, row0, rows)) return;
   const int n0 = blockIdx.y * 64;
   const int r = threadIdx.x >> 4, c = threadIdx.x & 15;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[RA][4];
+#pragma unroll
+  for (int a = 0; a < RA; ++a)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[a][i] = 0.f;
   const Tw *Wj[2] = {W0, W1};
   // weight tile staging: thread -> (row kk = tid / 8, 8 columns at nq = 8 (tid % 8))
   const int kr = threadIdx.x >> 3, nq = (threadIdx.x & 7) * 8;
@@ -258,28 +279,36 @@ __global__ void __launch_bounds__(256) bw_nn_kernel(const Tw *__restrict__ W0,
 #pragma unroll
       for (int i = 0; i < 8; ++i) ws[j][kr][nq + i] = w8[i];
     }
-    for (int e = threadIdx.x; e < kBwRows * kBwK; e += blockDim.x) {
+    for (int e = threadIdx.x; e < R * kBwK; e += blockDim.x) {
       const int rr = e / kBwK, kk = e % kBwK;
       const bool in = rr < rows && k0 + kk < K;
       vs[0][rr][kk] = in ? src0(row0 + rr, k0 + kk) : 0.f;
       if (NW > 1) vs[NW - 1][rr][kk] = in ? src1(row0 + rr, k0 + kk) : 0.f;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int kk = 0; kk < kBwK; ++kk)
 #pragma unroll
       for (int j = 0; j < NW; ++j) {
-        const float v = vs[j][r][kk];
+        float v[RA], w[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = fmaf(ws[j][kk][c + 16 * i], v, acc[i]);
+        for (int a = 0; a < RA; ++a) v[a] = vs[j][r + 16 * a][kk];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = ws[j][kk][c + 16 * i];
+#pragma unroll
+        for (int a = 0; a < RA; ++a)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[a][i] = fmaf(w[i], v[a], acc[a][i]);
       }
     __syncthreads();
   }
-  if (r < rows) {
+#pragma unroll
+  for (int a = 0; a < RA; ++a) {
+    if (r + 16 * a >= rows) continue;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int n = n0 + c + 16 * i;
-      if (n < N) out[(size_t)(row0 + r) * N + n] = acc[i];
+      if (n < N) out[(size_t)(row0 + r + 16 * a) * N + n] = acc[a][i];
     }
   }
 }

@@ -1036,8 +1036,10 @@ extern "C" moe_status moe_router_logits_static(moe_handle h, const void *x, int 
 
 namespace {
 
-template <typename T_>
-moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
+// R: rows of one expert group per tile of the row kernels (16 for decode-sized groups, 64
+// when groups average 32 rows or more)
+template <typename T_, int R>
+moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
                          float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
                          void *ws, cudaStream_t st) {
   const moe_config &c = L->cfg;
@@ -1080,10 +1082,10 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   if ((s = launch(bw_rows_kernel, dim3(grid_for(P, 256, L->num_sms)), dim3(256), 0, st,
                   (const int *)perm, (const int *)idx, (const float *)gate, T, k, E, c.n_shared,
                   c.routed_scale, row_token, row_group, row_scale)) != MOE_OK ||
-      (s = launch(bw_tiles_kernel, dim3(1), dim3(32), 0, st, (const int *)offsets, E, G, T,
+      (s = launch(bw_tiles_kernel, dim3(1), dim3(32), 0, st, (const int *)offsets, E, G, T, R,
                   tile_prefix)) != MOE_OK)
     return s;
-  const int n_tiles = P / kBwRows + G;  // upper bound of the row-tile list
+  const int n_tiles = P / R + G;  // upper bound of the row-tile list
   auto cdiv = [](int n, int m) { return (n + m - 1) / m; };
   const SrcX<T_> src_x{x, row_token, d};
   const SrcDy<T_> src_dy{dout, row_token, row_scale, d};
@@ -1096,12 +1098,12 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
     if ((s = launch_row_gather(L, x, T, ws, W, plan, st)) != MOE_OK ||
         (s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu)) != MOE_OK)
       return s;
-  } else if ((s = launch(bw_nt_kernel<2, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256),
+  } else if ((s = launch(bw_nt_kernel<2, R, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256),
                          0, st, wg, wu, f, d, src_x, (const int *)tile_prefix,
                          (const int *)offsets, E, G, T, Tk, a, b)) != MOE_OK) {
     return s;
   }
-  if ((s = launch(bw_nt_kernel<1, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
+  if ((s = launch(bw_nt_kernel<1, R, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
                   wd, d, f, src_h, (const int *)tile_prefix, (const int *)offsets, E, G, T, Tk,
                   wide, wide)) != MOE_OK ||
       (s = launch(bw_dgate_kernel<T_>, dim3(grid_for(Tk, 8, L->num_sms)), dim3(256), 0, st,
@@ -1109,7 +1111,7 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
                   c.routed_scale, dgate)) != MOE_OK)
     return s;
   // 4. dh, dW_d, then da (over dh) and db
-  if ((s = launch(bw_nn_kernel<1, T_, SrcDy<T_>, SrcDy<T_>>, dim3(n_tiles, cdiv(f, 64)),
+  if ((s = launch(bw_nn_kernel<1, R, T_, SrcDy<T_>, SrcDy<T_>>, dim3(n_tiles, cdiv(f, 64)),
                   dim3(256), 0, st, wd, wd, d, f, src_dy, src_dy, (const int *)tile_prefix,
                   (const int *)offsets, E, G, T, Tk, dh)) != MOE_OK ||
       (s = launch(bw_wgrad_kernel<SrcDy<T_>, SrcH>, dim3(G, cdiv(d, 64), cdiv(f, 128)),
@@ -1119,7 +1121,7 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
                   0, st, (const float *)a, (const float *)b, dh, db, (size_t)P * f)) != MOE_OK)
     return s;
   // 5. rows of dx (over the unscaled outputs, no longer needed), dW_g, dW_u
-  if ((s = launch(bw_nn_kernel<2, T_, SrcRow, SrcRow>, dim3(n_tiles, cdiv(d, 64)), dim3(256),
+  if ((s = launch(bw_nn_kernel<2, R, T_, SrcRow, SrcRow>, dim3(n_tiles, cdiv(d, 64)), dim3(256),
                   0, st, wg, wu, f, d, src_da, src_db, (const int *)tile_prefix,
                   (const int *)offsets, E, G, T, Tk, wide)) != MOE_OK ||
       (s = launch(bw_wgrad_kernel<SrcRow, SrcX<T_>>, dim3(G, cdiv(f, 64), cdiv(d, 128)),
@@ -1139,6 +1141,18 @@ moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   return launch(bw_dx_kernel<T_>, dim3(grid_for((size_t)T * d, 256, L->num_sms)), dim3(256), 0,
                 st, (const float *)wide, (const int *)slot_row, (const int *)idx,
                 (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
+}
+
+template <typename T_>
+moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
+                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                         void *ws, cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  const long long P = (long long)T * (c.top_k + c.n_shared);
+  const long long G = c.n_experts + c.n_shared;
+  if (P >= 32 * G)
+    return backward_rows<T_, 64>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
+  return backward_rows<T_, 16>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
 
 }  // namespace
