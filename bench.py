@@ -492,34 +492,47 @@ def run_backward(args, rank, world, local_rank):
         return None
     P = T * w.k + w.n_shared * T
     es = 2 if w.dtype == "bf16" else 4
-    # recompute a and b, unscaled outputs, dh, rows of dx (two products), three weight
-    # gradients: 18 P f d flops; the router adds 4 T k d
-    flops = 18.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
-    # weights of the touched experts read four times (gate/up twice, down twice); their
-    # three fp32 weight gradients and the router's read and written (they accumulate)
     tm = float(np.mean(touched))
-    nbytes = tm * 6 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+    peaks, src = load_peaks()
     step_s = total_ms / args.steps / 1e3
-    peaks, _ = load_peaks()
-    alu = flops / step_s / 1e12
+    if w.dtype == "bf16":
+        # tensor cores: recompute a and b (4 P f d), dh (2), rows of dx (4), three weight
+        # gradients (6): 16 P f d flops; the router adds 4 T k d.  Weights of the touched
+        # experts read five times (gate and up twice, down once); their three fp32 weight
+        # gradients and the router's read and written (they accumulate).
+        flops = 16.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
+        nbytes = tm * 5 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+        peak_c = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        peak_name = f"bf16 dense, sustained ({src})"
+        unit_c, kind = "TFLOP/s", "tensor"
+        label = "tcgen05 grouped GEMMs"
+    else:
+        # CUDA cores: recompute a and b, unscaled outputs, dh, rows of dx (two products),
+        # three weight gradients: 18 P f d flops; weights read six times
+        flops = 18.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
+        nbytes = tm * 6 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+        peak_c, peak_name = FP32_ALU_TFLOPS, "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
+        unit_c, kind = "TFLOP/s", "alu"
+        label = "fp32 CUDA-core kernels"
+    comp = flops / step_s / 1e12
     hbm = nbytes / step_s / 1e9
-    ridge = FP32_ALU_TFLOPS * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    ridge = peak_c * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if flops / nbytes > ridge:
-        roof = {"bound": "alu", "achieved": round(alu, 2), "peak": round(FP32_ALU_TFLOPS, 1),
-                "unit": "TFLOP/s", "frac": round(alu / FP32_ALU_TFLOPS, 4)}
+        roof = {"bound": kind, "achieved": round(comp, 2), "peak": round(peak_c, 1),
+                "unit": unit_c, "frac": round(comp / peak_c, 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(hbm, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(hbm / peaks["hbm_gbs"], 4)}
     roof.update({"traffic": None, "kernel": "moe_backward (all kernels)",
                  "algorithmic_flops_per_step": int(flops), "algorithmic_bytes_per_step": int(nbytes),
-                 "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz; HBM measured"})
+                 "peak_source": f"{peak_name}; HBM {src}"})
     return {
-        "metric": "MoE-layer backward tokens/s on 1 B200 (fp32 CUDA-core kernels)",
+        "metric": f"MoE-layer backward tokens/s on 1 B200 ({label})",
         "pass": "backward",
         "value": round(job_throughput(T, args.steps, world, total_ms), 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; fresh x and dout every step; random-init weights)",
         "config": {"workload": w.name, "tokens": T, "d_model": w.d, "n_experts": w.E,
                    "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared,

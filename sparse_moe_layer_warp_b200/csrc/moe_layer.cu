@@ -23,6 +23,7 @@
 #include "expert_simt.cuh"
 #include "expert_stats.cuh"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_bw.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "ptx_sm100.cuh"
 #include "router_stats.cuh"
@@ -38,6 +39,9 @@ struct moe_layer {
   int smem_optin;
   int pair_grid[2];  // CTAs of the CTA-pair GEMM (up, down): 2 x co-resident clusters
   CUtensorMap tm_wg, tm_wu, tm_wd, tm_wr;
+  // the same weights as MN-major operands of the backward (box {64, 64}): W_gate and W_up
+  // as [G*f, d], W_down as [G*d, f]
+  CUtensorMap tm_wg_mn, tm_wu_mn, tm_wd_mn;
 };
 
 namespace {
@@ -72,6 +76,21 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t ro
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Row-major fp32 matrix [rows, cols] -> tiled map with box {32 columns, 32 rows} and
+// 128-byte swizzle (the staging tiles of the weight-gradient reductions).
+bool encode_f32_2d(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
@@ -395,9 +414,17 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
   return launch_gemm<MODE_LOGITS>(L, bn, p, st);
 }
 
+// The bf16 backward runs its matrix products on the tensor cores (its weight dimensions are
+// multiples of the 128-row tile, as the forward requires); the fp32 one on CUDA cores.
+bool backward_on_tensor_cores(const moe_config &c) { return c.dtype == MOE_BF16; }
+
 // Backward workspace: the forward's layout, then the backward's own regions.
 struct BwLayout {
-  size_t row_token, row_group, row_scale, tile_prefix, a, b, dh, db, wide, dgate, dl, total;
+  size_t row_token, row_group, row_scale, tile_prefix, a, b, dh, db, wide, dgate, dl;
+  // tensor-core path: expert-sorted bf16 rows of x, dout, da, db, s*h ([P + 1] rows each,
+  // the last all zero) and the partial sums of dgate
+  size_t xs16, dys16, da16, db16, hs16, dgate_part;
+  size_t total;
 };
 
 BwLayout bw_layout(const moe_config &c, int T) {
@@ -408,6 +435,7 @@ BwLayout bw_layout(const moe_config &c, int T) {
     off += (bytes + 255) & ~static_cast<size_t>(255);
     return o;
   };
+  const bool tc = backward_on_tensor_cores(c);
   const size_t Tk = (size_t)T * c.top_k, P = Tk + (size_t)c.n_shared * T;
   const size_t G = (size_t)c.n_experts + c.n_shared;
   B.row_token = take(P * 4);
@@ -416,19 +444,27 @@ BwLayout bw_layout(const moe_config &c, int T) {
   B.tile_prefix = take((G + 1) * 4);
   B.a = take(P * c.d_ff * 4);
   B.b = take(P * c.d_ff * 4);
-  B.dh = take(P * c.d_ff * 4);
-  B.db = take(P * c.d_ff * 4);
+  B.dh = take(tc ? 0 : P * c.d_ff * 4);
+  B.db = take(tc ? 0 : P * c.d_ff * 4);
   B.wide = take(P * c.d_model * 4);  // unscaled expert outputs, then the rows of dx
   B.dgate = take(Tk * 4);
   B.dl = take(Tk * 4);
+  B.xs16 = take(tc ? (P + 1) * c.d_model * 2 : 0);
+  B.dys16 = take(tc ? (P + 1) * c.d_model * 2 : 0);
+  B.da16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
+  B.db16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
+  B.hs16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
+  B.dgate_part = take(tc ? Tk * (c.d_ff / 32) * 4 : 0);
   B.total = off;
   return B;
 }
 
-template <typename T_>
-moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
-                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
-                         void *ws, cudaStream_t st);
+moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
+                       int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
+                       float *dw_down, void *ws, cudaStream_t st);
+moe_status backward_f32(const moe_layer *L, const float *x, const float *dout, int T, float *dx,
+                        float *dw_router, float *dw_gate, float *dw_up, float *dw_down, void *ws,
+                        cudaStream_t st);
 
 // Self-test of the device timeout path: an mbarrier nobody arrives on and a workspace flag
 // nobody sets, each waited on with the library's bounded waits (limit_ns), as a stuck
@@ -521,7 +557,10 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wu, w->w_up, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wd, w->w_down, c.d_ff, G * c.d_model, kBM) ||
-        !encode_bf16_2d(&L->tm_wr, w->w_router, c.d_model, c.n_experts, kBM)) {
+        !encode_bf16_2d(&L->tm_wr, w->w_router, c.d_model, c.n_experts, kBM) ||
+        !encode_bf16_2d(&L->tm_wg_mn, w->w_gate, c.d_model, G * c.d_ff, 64) ||
+        !encode_bf16_2d(&L->tm_wu_mn, w->w_up, c.d_model, G * c.d_ff, 64) ||
+        !encode_bf16_2d(&L->tm_wd_mn, w->w_down, c.d_ff, G * c.d_model, 64)) {
       free(L);
       return MOE_ERR_CUDA;
     }
@@ -581,11 +620,11 @@ moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *d
   if (h->cfg.d_ff % 8 != 0) return MOE_ERR_UNSUPPORTED;  // 8-wide weight and gradient rows
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (h->cfg.dtype == MOE_BF16)
-    return backward_impl(h, static_cast<const __nv_bfloat16 *>(x),
-                         static_cast<const __nv_bfloat16 *>(dout), n_tokens, dx, dw_router,
-                         dw_gate, dw_up, dw_down, ws, st);
-  return backward_impl(h, static_cast<const float *>(x), static_cast<const float *>(dout),
-                       n_tokens, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
+    return backward_tc(h, static_cast<const __nv_bfloat16 *>(x),
+                       static_cast<const __nv_bfloat16 *>(dout), n_tokens, dx, dw_router, dw_gate,
+                       dw_up, dw_down, ws, st);
+  return backward_f32(h, static_cast<const float *>(x), static_cast<const float *>(dout),
+                      n_tokens, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
 
 moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *param_norm,
@@ -756,7 +795,8 @@ moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
 // hand-over counts (null: none).  *used receives the parameters (the down GEMM's start).
 moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
                             const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
-                            int *done, cudaStream_t st, GemmParams *used) {
+                            int *done, cudaStream_t st, GemmParams *used,
+                            const void *xs = nullptr) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
@@ -767,7 +807,7 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
   p1.tmA1 = h->tm_wu;
   if (plan.gather_in_gemm) {
     if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
-  } else if (!encode_bf16_2d(&p1.tmB, at<void>(ws, W.xs), c.d_model, Tk, bn) ||
+  } else if (!encode_bf16_2d(&p1.tmB, xs ? xs : at<void>(ws, W.xs), c.d_model, Tk, bn) ||
              !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
     return MOE_ERR_CUDA;
   }
@@ -1036,6 +1076,28 @@ extern "C" moe_status moe_router_logits_static(moe_handle h, const void *x, int 
 
 namespace {
 
+// The forward's routing kernels over x (same experts, gates and sorted order), with the
+// grouped GEMMs' work counters reset.
+moe_status backward_select(const moe_layer *L, const void *x, int T, void *ws, cudaStream_t st) {
+  const WsLayout W = ws_layout(L->cfg, T);
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  int *idx = at<int>(ws, W.idx), *offsets = at<int>(ws, W.offsets), *perm = at<int>(ws, W.perm);
+  int *slot_row = at<int>(ws, W.slot_row), *counts = at<int>(ws, W.counts);
+  float *gate = at<float>(ws, W.gate), *logits = at<float>(ws, W.logits);
+  const ForwardPlan plan = plan_forward(L, T);
+  const CounterReset reset{status->sched, nullptr, 0};
+  if (plan.decode_route)
+    return launch_route_decode(L, x, T, logits, idx, gate, counts, offsets, perm, slot_row,
+                               status, reset, st);
+  moe_status s = launch_logits(L, x, T, logits, at<float>(ws, W.part), status, st);
+  if (s != MOE_OK) return s;
+  return plan.small_route
+             ? launch_route_small(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
+                                  slot_row, reset, st)
+             : launch_select_permute(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
+                                     slot_row, at<int>(ws, W.chunk_hist), reset, st);
+}
+
 // R: rows of one expert group per tile of the row kernels (16 for decode-sized groups, 64
 // when groups average 32 rows or more)
 template <typename T_, int R>
@@ -1047,31 +1109,16 @@ moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   const int Tk = T * k, P = Tk + c.n_shared * T;
   const WsLayout W = ws_layout(c, T);
   const BwLayout B = bw_layout(c, T);
-  DevStatus *status = at<DevStatus>(ws, W.status);
   int *idx = at<int>(ws, W.idx), *offsets = at<int>(ws, W.offsets), *perm = at<int>(ws, W.perm);
-  int *slot_row = at<int>(ws, W.slot_row), *counts = at<int>(ws, W.counts);
-  float *gate = at<float>(ws, W.gate), *logits = at<float>(ws, W.logits);
+  int *slot_row = at<int>(ws, W.slot_row);
+  float *gate = at<float>(ws, W.gate);
   const T_ *wg = static_cast<const T_ *>(L->w.w_gate);
   const T_ *wu = static_cast<const T_ *>(L->w.w_up);
   const T_ *wd = static_cast<const T_ *>(L->w.w_down);
   const T_ *wr = static_cast<const T_ *>(L->w.w_router);
   moe_status s;
   // 1. the forward's selection (same kernels, so the same experts and gates)
-  const ForwardPlan plan = plan_forward(L, T);
-  const CounterReset reset{status->sched, nullptr, 0};
-  if (plan.decode_route) {
-    s = launch_route_decode(L, x, T, logits, idx, gate, counts, offsets, perm, slot_row, status,
-                            reset, st);
-  } else {
-    s = launch_logits(L, x, T, logits, at<float>(ws, W.part), status, st);
-    if (s == MOE_OK)
-      s = plan.small_route
-              ? launch_route_small(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
-                                   slot_row, reset, st)
-              : launch_select_permute(L, logits, T, nullptr, idx, gate, counts, offsets, perm,
-                                      slot_row, at<int>(ws, W.chunk_hist), reset, st);
-  }
-  if (s != MOE_OK) return s;
+  if ((s = backward_select(L, x, T, ws, st)) != MOE_OK) return s;
   // 2. row bookkeeping
   int *row_token = at<int>(ws, B.row_token), *row_group = at<int>(ws, B.row_group);
   float *row_scale = at<float>(ws, B.row_scale);
@@ -1091,18 +1138,11 @@ moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   const SrcDy<T_> src_dy{dout, row_token, row_scale, d};
   const SrcH src_h{a, b, f};
   const SrcRow src_da{dh, f}, src_db{db, f};
-  // 3. pre-activations a, b (bf16: the forward's tcgen05 up GEMM storing them in fp32);
-  //    unscaled expert outputs; dgate
-  if (c.dtype == MOE_BF16) {
-    GemmParams pu;
-    if ((s = launch_row_gather(L, x, T, ws, W, plan, st)) != MOE_OK ||
-        (s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu)) != MOE_OK)
-      return s;
-  } else if ((s = launch(bw_nt_kernel<2, R, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256),
-                         0, st, wg, wu, f, d, src_x, (const int *)tile_prefix,
-                         (const int *)offsets, E, G, T, Tk, a, b)) != MOE_OK) {
+  // 3. pre-activations a, b; unscaled expert outputs; dgate
+  if ((s = launch(bw_nt_kernel<2, R, T_, SrcX<T_>>, dim3(n_tiles, cdiv(f, 64)), dim3(256), 0, st,
+                  wg, wu, f, d, src_x, (const int *)tile_prefix, (const int *)offsets, E, G, T,
+                  Tk, a, b)) != MOE_OK)
     return s;
-  }
   if ((s = launch(bw_nt_kernel<1, R, T_, SrcH>, dim3(n_tiles, cdiv(d, 64)), dim3(256), 0, st, wd,
                   wd, d, f, src_h, (const int *)tile_prefix, (const int *)offsets, E, G, T, Tk,
                   wide, wide)) != MOE_OK ||
@@ -1143,16 +1183,179 @@ moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T,
                 (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
 }
 
-template <typename T_>
-moe_status backward_impl(const moe_layer *L, const T_ *x, const T_ *dout, int T, float *dx,
-                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
-                         void *ws, cudaStream_t st) {
+// ------------------------------------------------------- tensor-core backward launches
+template <int MODE, int BN>
+moe_status launch_bw_dgrad_bn(const moe_layer *L, const BwDgradParams &p, cudaStream_t st) {
+  using C = BwDgradCfg<BN>;
+  const size_t smem = C::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bw_dgrad_kernel<MODE, BN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch(bw_dgrad_kernel<MODE, BN>, dim3(L->num_sms), dim3(kGemmThreads), smem, st, p);
+}
+
+template <int MODE>
+moe_status launch_bw_dgrad(const moe_layer *L, int bn, const BwDgradParams &p, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_bw_dgrad_bn<MODE, 16>(L, p, st);
+    case 32: return launch_bw_dgrad_bn<MODE, 32>(L, p, st);
+    case 64: return launch_bw_dgrad_bn<MODE, 64>(L, p, st);
+    case 128: return launch_bw_dgrad_bn<MODE, 128>(L, p, st);
+    case 256: return launch_bw_dgrad_bn<MODE, 256>(L, p, st);
+  }
+  return MOE_ERR_UNSUPPORTED;
+}
+
+template <int BNW>
+moe_status launch_bw_wgrad(const moe_layer *L, const BwWgradParams &p, cudaStream_t st) {
+  using C = BwWgradCfg<BNW>;
+  const size_t smem = C::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bw_wgrad_kernel<BNW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch(bw_wgrad_kernel<BNW>, dim3(L->num_sms), dim3(kGemmThreads), smem, st, p);
+}
+
+// bf16 backward with every matrix product on the tensor cores (grouped_gemm_bw.cuh):
+//   selection -> row bookkeeping -> sorted bf16 rows of x and dout -> a, b (the forward's
+//   up GEMM) -> DH (dh, SwiGLU backward, dgate partials) -> dgate -> DX (rows of dx) ->
+//   the three weight gradients in one launch -> router terms and dx.
+moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
+                       int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
+                       float *dw_down, void *ws, cudaStream_t st) {
+  const moe_config &c = L->cfg;
+  const int E = c.n_experts, G = E + c.n_shared, k = c.top_k, d = c.d_model, f = c.d_ff;
+  const int Tk = T * k, P = Tk + c.n_shared * T;
+  const WsLayout W = ws_layout(c, T);
+  const BwLayout B = bw_layout(c, T);
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  int *idx = at<int>(ws, W.idx), *offsets = at<int>(ws, W.offsets), *perm = at<int>(ws, W.perm);
+  int *slot_row = at<int>(ws, W.slot_row);
+  float *gate = at<float>(ws, W.gate);
+  int *row_token = at<int>(ws, B.row_token), *row_group = at<int>(ws, B.row_group);
+  float *row_scale = at<float>(ws, B.row_scale);
+  float *a = at<float>(ws, B.a), *b = at<float>(ws, B.b), *wide = at<float>(ws, B.wide);
+  float *dgate = at<float>(ws, B.dgate), *dl = at<float>(ws, B.dl);
+  __nv_bfloat16 *xs = at<__nv_bfloat16>(ws, B.xs16), *dys = at<__nv_bfloat16>(ws, B.dys16);
+  __nv_bfloat16 *da = at<__nv_bfloat16>(ws, B.da16), *db = at<__nv_bfloat16>(ws, B.db16);
+  __nv_bfloat16 *hs = at<__nv_bfloat16>(ws, B.hs16);
+  float *dgate_part = at<float>(ws, B.dgate_part);
+  const __nv_bfloat16 *wr = static_cast<const __nv_bfloat16 *>(L->w.w_router);
+  moe_status s;
+  if ((s = backward_select(L, x, T, ws, st)) != MOE_OK) return s;
+  if ((s = launch(bw_rows_kernel, dim3(grid_for(P, 256, L->num_sms)), dim3(256), 0, st,
+                  (const int *)perm, (const int *)idx, (const float *)gate, T, k, E, c.n_shared,
+                  c.routed_scale, row_token, row_group, row_scale)) != MOE_OK ||
+      (s = launch(bw_sorted_rows_kernel, dim3(grid_for((size_t)P + 1, 8, L->num_sms)),
+                  dim3(256), 0, st, x, dout, (const int *)row_token, P, d, f, xs, dys, da, db,
+                  hs)) != MOE_OK)
+    return s;
+  // pre-activations a, b: the forward's up GEMM, token rows from the sorted copy
+  const ForwardPlan plan = plan_forward(L, T);
+  GemmParams pu;
+  if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, xs)) != MOE_OK)
+    return s;
+  // DH
+  const int bn = pick_bn(c, T, MODE_DOWN);
+  BwDgradParams pd;
+  memset(&pd, 0, sizeof pd);
+  pd.tmA0 = L->tm_wd_mn;
+  if (!encode_bf16_2d(&pd.tmB0, dys, d, (uint64_t)P + 1, bn)) return MOE_ERR_CUDA;
+  pd.offsets = offsets;
+  pd.row_scale = row_scale;
+  pd.pre_a = a;
+  pd.pre_b = b;
+  pd.da = da;
+  pd.db = db;
+  pd.hs = hs;
+  pd.dgate_part = dgate_part;
+  pd.status = status;
+  pd.E = E;
+  pd.n_groups = G;
+  pd.T = T;
+  pd.Tk = Tk;
+  pd.M = f;
+  pd.K = d;
+  pd.n_pairs = 1;
+  pd.n_part = f / 32;
+  pd.sched = &status->sched[1];
+  if ((s = launch_bw_dgrad<BW_DH>(L, bn, pd, st)) != MOE_OK ||
+      (s = launch(bw_dgate_reduce_kernel, dim3(grid_for(Tk, 256, L->num_sms)), dim3(256), 0, st,
+                  (const float *)dgate_part, f / 32, (const int *)perm, Tk, c.routed_scale,
+                  dgate)) != MOE_OK)
+    return s;
+  // DX: rows of dx = W_gate^T da + W_up^T db
+  BwDgradParams px = pd;
+  px.tmA0 = L->tm_wg_mn;
+  px.tmA1 = L->tm_wu_mn;
+  if (!encode_bf16_2d(&px.tmB0, da, f, (uint64_t)P + 1, bn) ||
+      !encode_bf16_2d(&px.tmB1, db, f, (uint64_t)P + 1, bn))
+    return MOE_ERR_CUDA;
+  px.out = wide;
+  px.M = d;
+  px.K = f;
+  px.n_pairs = 2;
+  px.sched = &status->sched[2];
+  if ((s = launch_bw_dgrad<BW_DX>(L, bn, px, st)) != MOE_OK) return s;
+  // weight gradients: dW_down += dout^T (s h), dW_gate += da^T x, dW_up += db^T x
+  BwWgradParams pw;
+  memset(&pw, 0, sizeof pw);
+  __nv_bfloat16 *ops[kWgOps] = {dys, hs, da, db, xs};
+  const int widths[kWgOps] = {d, f, f, f, d};
+  for (int i = 0; i < kWgOps; ++i)
+    if (!encode_bf16_2d(&pw.box[i], ops[i], widths[i], (uint64_t)P + 1, 64) ||
+        !encode_bf16_2d(&pw.gat[i], ops[i], widths[i], (uint64_t)P + 1, 1))
+      return MOE_ERR_CUDA;
+  if (!encode_f32_2d(&pw.out[0], dw_down, f, (uint64_t)G * d) ||
+      !encode_f32_2d(&pw.out[1], dw_gate, d, (uint64_t)G * f) ||
+      !encode_f32_2d(&pw.out[2], dw_up, d, (uint64_t)G * f))
+    return MOE_ERR_CUDA;
+  const int a_op[kWgProbs] = {0, 2, 3}, b_op[kWgProbs] = {1, 4, 4};
+  const int Ms[kWgProbs] = {d, f, f}, Ns[kWgProbs] = {f, d, d};
+  for (int i = 0; i < kWgProbs; ++i) {
+    pw.a_op[i] = a_op[i];
+    pw.b_op[i] = b_op[i];
+    pw.M[i] = Ms[i];
+    pw.N[i] = Ns[i];
+  }
+  pw.n_prob = kWgProbs;
+  pw.offsets = offsets;
+  pw.status = status;
+  pw.E = E;
+  pw.n_groups = G;
+  pw.T = T;
+  pw.Tk = Tk;
+  pw.zero_row = P;
+  pw.sched = &status->sched[3];
+  s = (d % 256 == 0 && f % 256 == 0) ? launch_bw_wgrad<256>(L, pw, st)
+                                     : launch_bw_wgrad<128>(L, pw, st);
+  if (s != MOE_OK) return s;
+  // router and dx
+  if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
+                  (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
+      (s = launch(bw_router_dw_kernel<__nv_bfloat16>, dim3(E, (d + 255) / 256), dim3(256), 0,
+                  st, x, (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
+                  dw_router)) != MOE_OK)
+    return s;
+  return launch(bw_dx_kernel<__nv_bfloat16>, dim3(grid_for((size_t)T * d, 256, L->num_sms)),
+                dim3(256), 0, st, (const float *)wide, (const int *)slot_row, (const int *)idx,
+                (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
+}
+
+// fp32 layer: CUDA-core row kernels (64-row tiles when groups average 32 rows or more)
+moe_status backward_f32(const moe_layer *L, const float *x, const float *dout, int T, float *dx,
+                        float *dw_router, float *dw_gate, float *dw_up, float *dw_down, void *ws,
+                        cudaStream_t st) {
   const moe_config &c = L->cfg;
   const long long P = (long long)T * (c.top_k + c.n_shared);
   const long long G = c.n_experts + c.n_shared;
   if (P >= 32 * G)
-    return backward_rows<T_, 64>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
-  return backward_rows<T_, 16>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
+    return backward_rows<float, 64>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws,
+                                    st);
+  return backward_rows<float, 16>(L, x, dout, T, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
 
 }  // namespace

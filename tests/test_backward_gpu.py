@@ -16,8 +16,22 @@ CASES = [
     {"dtype": "bf16", "T": 150, "d": 256, "E": 8, "k": 4, "f": 256, "seed": 3},  # 75 per expert
     {"dtype": "bf16", "T": 90, "d": 128, "E": 24, "k": 3, "f": 128, "bias": "zipf",
      "n_shared": 0},                                                               # empty experts
+    {"dtype": "bf16", "T": 400, "d": 128, "E": 8, "k": 4, "f": 128, "seed": 5},   # 256-row tiles
     {"dtype": "f32"},
 ]
+
+
+def tolerance(dtype):
+    """Largest |error| allowed, relative to the largest |reference| entry of a gradient.
+
+    fp32 layer: fp32 sums of products of exactly decoded inputs, far inside 2e-4.
+    bf16 layer (tensor cores): the second-stage products take da, db and s*h rounded to bf16
+    (unit roundoff u = 2^-8), each product with one rounded operand, so every term of a
+    weight-gradient or dx sum carries a relative error of at most u; with independent rounding
+    signs the largest error stays below u * max|ref| (a float64 simulation of exactly these
+    roundings at the sizes below gives 1.4e-3 .. 2.4e-3).  The bound is 2u = 2^-7; dgate and
+    the router terms are computed from fp32 values and sit far inside it."""
+    return 2.0 ** -7 if dtype == "bf16" else 2e-4
 
 
 @pytest.mark.parametrize("kw", CASES)
@@ -38,10 +52,8 @@ def test_backward_matches_oracle(cuda_ok, kw):
         got = g[name].cpu().numpy().astype(np.float64)
         assert got.shape == want.shape, name
         scale = np.abs(want).max()
-        # fp32 sums of products of exactly decoded inputs: far inside 2e-4 of the largest
-        # entry (the sums run over at most d = 4096 / f terms)
         err = np.abs(got - want).max()
-        assert err <= 2e-4 * scale, (name, err, scale)
+        assert err <= tolerance(kw["dtype"]) * scale, (name, err, scale)
     # experts no token chose keep their (zero) weight gradients
     unchosen = np.nonzero(counts == 0)[0]
     for name in ("dw_gate", "dw_up", "dw_down"):
