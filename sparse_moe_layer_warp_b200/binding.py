@@ -328,7 +328,13 @@ class MoELayer:
         return act, par, ratios
 
     def device_status(self, stream=None) -> int:
-        return moe_device_status(self.handle, self.ws, stream)
+        """Device status of the forward's and the backward's workspaces (0: no bounded wait
+        gave up in either)."""
+        st = 0
+        for ws in (self.ws, self.bw_ws):
+            if ws is not None:
+                st = st or moe_device_status(self.handle, ws, stream)
+        return st
 
     def close(self):
         if self.handle is not None:

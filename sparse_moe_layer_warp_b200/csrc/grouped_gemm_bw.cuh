@@ -526,10 +526,17 @@ struct BwWgradCfg {
   static constexpr int ACC_COLS = BNW;
   static constexpr int TMEM_COLS = 2 * BNW;
   static constexpr int STG_BYTES = 32 * 32 * 4;   // one 32 x 32 fp32 reduction tile
-  static constexpr int STG_TOTAL = 4 * 2 * STG_BYTES;  // per epilogue warp, double-buffered
+#ifndef MOE_WG_STG_BUFS
+#define MOE_WG_STG_BUFS 2
+#endif
+#ifndef MOE_WG_MAX_STAGES
+#define MOE_WG_MAX_STAGES 8
+#endif
+  static constexpr int STG_BUFS = MOE_WG_STG_BUFS;  // staging tiles per epilogue warp
+  static constexpr int STG_TOTAL = 4 * STG_BUFS * STG_BYTES;
   static constexpr int SMEM_BUDGET = 220 * 1024 - STG_TOTAL;
   static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int STAGES = STAGES_RAW > MOE_WG_MAX_STAGES ? MOE_WG_MAX_STAGES : STAGES_RAW;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(BNW == 128 || BNW == 256, "N tile");
   static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
@@ -823,7 +830,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       return ok != 0;
     };
-    uint8_t *my_stg = stg + q * 2 * C::STG_BYTES;
+    uint8_t *my_stg = stg + q * C::STG_BUFS * C::STG_BYTES;
     int it = 0, n_red = 0;
     int qi = 0;
     uint32_t qph = 0;
@@ -852,9 +859,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld16(taddr + 32 * c, v0);
         tmem_ld16(taddr + 32 * c + 16, v1);
         tmem_ld_wait_regs(v0, v1);
-        uint8_t *buf = my_stg + (n_red & 1) * C::STG_BYTES;
-        if (n_red >= 2) {  // the reduction that last read this tile has finished reading
-          if (lane == 0) bulk_wait_group_read<1>();
+        uint8_t *buf = my_stg + (n_red % C::STG_BUFS) * C::STG_BYTES;
+        if (n_red >= C::STG_BUFS) {  // the reduction that last read this tile is done reading
+          if (lane == 0) bulk_wait_group_read<C::STG_BUFS - 1>();
           __syncwarp();
         }
         // row `lane`, 16-byte chunk j of the row at position j ^ (lane & 7) (128-byte swizzle)
