@@ -27,4 +27,5 @@ from .c_oracle import (  # noqa: F401
     oracle_expert_param_norms,
     oracle_health_ratios,
     oracle_moe_backward,
+    oracle_moe_backward_sampled,
 )

@@ -49,6 +49,9 @@ def _load():
         lib.oracle_moe_backward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I,
                                             ctypes.c_double, P, P, P, P, P, P, P]
         lib.oracle_expert_param_norms.argtypes = [P, P, P, I, I, I, I, P]
+        lib.oracle_moe_backward_sampled.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I,
+                                                    ctypes.c_double, P, P, I, P, P, I, P, P, P,
+                                                    P, I, P, P]
         _lib = lib
     return _lib
 
@@ -229,4 +232,38 @@ def oracle_moe_backward(x, dout, w_r, w_gate, w_up, w_down, idx, gates, routed_s
                                 _ptr(w_down), dt, T, d, E, k, f, n_shared, float(routed_scale),
                                 _ptr(idx), _ptr(gates), _ptr(out["dx"]), _ptr(out["dw_router"]),
                                 _ptr(out["dw_gate"]), _ptr(out["dw_up"]), _ptr(out["dw_down"]))
+    return out
+
+
+def oracle_moe_backward_sampled(x, dout, w_r, w_gate, w_up, w_down, idx, gates, toks, exps,
+                                rexps, routed_scale=1.0, n_shared=1):
+    """Selected parts of oracle_moe_backward's result, for sizes whose full weight gradients
+    do not fit in memory: dict of float64 arrays dx [len(toks), d] (those tokens' rows),
+    dw_gate / dw_up [len(exps), f, d], dw_down [len(exps), d, f] (those experts; the shared
+    expert is index E), dw_router [len(rexps), d] (those routed experts)."""
+    x, dt = _as_input(x)
+    dout, dt2 = _as_input(dout)
+    assert dt == dt2
+    w_r, _ = _as_input(w_r)
+    w_gate, _ = _as_input(w_gate)
+    w_up, _ = _as_input(w_up)
+    w_down, _ = _as_input(w_down)
+    idx = np.ascontiguousarray(idx, np.int32)
+    gates = np.ascontiguousarray(gates, np.float32)
+    toks = np.ascontiguousarray(toks, np.int32)
+    exps = np.ascontiguousarray(exps, np.int32)
+    rexps = np.ascontiguousarray(rexps, np.int32)
+    T, d = x.shape
+    E = w_r.shape[0]
+    G, f, _ = w_gate.shape
+    k = idx.shape[1]
+    ne = len(exps)
+    out = dict(dx=np.empty((len(toks), d)), dw_gate=np.empty((ne, f, d)),
+               dw_up=np.empty((ne, f, d)), dw_down=np.empty((ne, d, f)),
+               dw_router=np.empty((len(rexps), d)))
+    _load().oracle_moe_backward_sampled(
+        _ptr(x), _ptr(dout), _ptr(w_r), _ptr(w_gate), _ptr(w_up), _ptr(w_down), dt, T, d, E,
+        k, f, n_shared, float(routed_scale), _ptr(idx), _ptr(gates), len(toks), _ptr(toks),
+        _ptr(out["dx"]), ne, _ptr(exps), _ptr(out["dw_gate"]), _ptr(out["dw_up"]),
+        _ptr(out["dw_down"]), len(rexps), _ptr(rexps), _ptr(out["dw_router"]))
     return out

@@ -480,3 +480,127 @@ void oracle_moe_backward(const void *x, const void *dout, const void *w_r, const
   free(ot);
   free(xt);
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Sampled backward for layer sizes whose full weight gradients do not fit in memory: the  */
+/* same chain rule as oracle_moe_backward, restricted to                                    */
+/*   dx of the tokens toks[0..n_tok)                        -> dx_s  [n_tok, d]             */
+/*   dW_gate, dW_up, dW_down of the experts exps[0..n_exp)  -> dwg_s, dwu_s [n_exp, f, d],  */
+/*                                                             dwd_s [n_exp, d, f]          */
+/*   dW_router rows of the routed experts rexps[0..n_rexp)  -> dwr_s [n_rexp, d]            */
+/* A contribution (token t, expert e) is evaluated when e is in exps or the token's dx or   */
+/* router terms are needed (t in toks, or one of its routed experts in rexps: those need    */
+/* dgate of all of its slots).  Tokens in increasing order, as in oracle_moe_backward.      */
+static int orc_in(const int *list, int n, int v) {
+  for (int i = 0; i < n; ++i)
+    if (list[i] == v) return i;
+  return -1;
+}
+
+void oracle_moe_backward_sampled(const void *x, const void *dout, const void *w_r,
+                                 const void *w_gate, const void *w_up, const void *w_down,
+                                 int dtype, int T, int d, int E, int k, int f, int n_shared,
+                                 double routed_scale, const int *idx, const float *gates,
+                                 int n_tok, const int *toks, double *dx_s, int n_exp,
+                                 const int *exps, double *dwg_s, double *dwu_s, double *dwd_s,
+                                 int n_rexp, const int *rexps, double *dwr_s) {
+  const size_t wsz = (size_t)f * (size_t)d;
+  memset(dx_s, 0, sizeof(double) * (size_t)n_tok * d);
+  memset(dwg_s, 0, sizeof(double) * (size_t)n_exp * wsz);
+  memset(dwu_s, 0, sizeof(double) * (size_t)n_exp * wsz);
+  memset(dwd_s, 0, sizeof(double) * (size_t)n_exp * wsz);
+  memset(dwr_s, 0, sizeof(double) * (size_t)n_rexp * d);
+  double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+  double *ot = (double *)malloc(sizeof(double) * (size_t)d);
+  double *a = (double *)malloc(sizeof(double) * (size_t)f);
+  double *b = (double *)malloc(sizeof(double) * (size_t)f);
+  double *h = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dh = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dy = (double *)malloc(sizeof(double) * (size_t)d);
+  double *dgate = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  for (int t = 0; t < T; ++t) {
+    const int ti = orc_in(toks, n_tok, t);
+    int whole = ti >= 0;  /* every contribution of the token is needed */
+    for (int j = 0; j < k; ++j)
+      if (orc_in(rexps, n_rexp, idx[(size_t)t * k + j]) >= 0) whole = 1;
+    int any = whole;
+    for (int c = 0; c < k + n_shared && !any; ++c) {
+      const int e = c < k ? idx[(size_t)t * k + c] : E;
+      if (orc_in(exps, n_exp, e) >= 0) any = 1;
+    }
+    if (!any) continue;
+    for (int i = 0; i < d; ++i) {
+      xt[i] = orc_elem(x, dtype, (size_t)t * d + i);
+      ot[i] = orc_elem(dout, dtype, (size_t)t * d + i);
+    }
+    for (int c = 0; c < k + n_shared; ++c) {
+      const int routed = c < k;
+      const int e = routed ? idx[(size_t)t * k + c] : E;
+      const int ei = orc_in(exps, n_exp, e);
+      if (!whole && ei < 0) continue;
+      const double s = routed ? routed_scale * (double)gates[(size_t)t * k + c] : 1.0;
+      for (int n = 0; n < f; ++n) {
+        double av = 0.0, bv = 0.0;
+        for (int i = 0; i < d; ++i) {
+          av += xt[i] * orc_elem(w_gate, dtype, (size_t)e * wsz + (size_t)n * d + i);
+          bv += xt[i] * orc_elem(w_up, dtype, (size_t)e * wsz + (size_t)n * d + i);
+        }
+        a[n] = av;
+        b[n] = bv;
+        h[n] = orc_silu(av) * bv;
+      }
+      double dot = 0.0;  /* dout_t . yhat */
+      for (int i = 0; i < d; ++i) {
+        double yh = 0.0;
+        for (int n = 0; n < f; ++n)
+          yh += orc_elem(w_down, dtype, (size_t)e * wsz + (size_t)i * f + n) * h[n];
+        dot += ot[i] * yh;
+        dy[i] = s * ot[i];
+      }
+      if (routed) dgate[c] = routed_scale * dot;
+      for (int n = 0; n < f; ++n) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) {
+          acc += orc_elem(w_down, dtype, (size_t)e * wsz + (size_t)i * f + n) * dy[i];
+          if (ei >= 0) dwd_s[(size_t)ei * wsz + (size_t)i * f + n] += dy[i] * h[n];
+        }
+        dh[n] = acc;
+      }
+      for (int n = 0; n < f; ++n) {
+        const double sg = 1.0 / (1.0 + exp(-a[n]));
+        const double da = dh[n] * b[n] * sg * (1.0 + a[n] * (1.0 - sg));
+        const double db = dh[n] * a[n] * sg;
+        for (int i = 0; i < d; ++i) {
+          const size_t wi = (size_t)e * wsz + (size_t)n * d + i;
+          if (ei >= 0) {
+            dwg_s[(size_t)ei * wsz + (size_t)n * d + i] += da * xt[i];
+            dwu_s[(size_t)ei * wsz + (size_t)n * d + i] += db * xt[i];
+          }
+          if (ti >= 0)
+            dx_s[(size_t)ti * d + i] +=
+                orc_elem(w_gate, dtype, wi) * da + orc_elem(w_up, dtype, wi) * db;
+        }
+      }
+    }
+    if (!whole) continue;
+    double sgd = 0.0;
+    for (int j = 0; j < k; ++j) sgd += (double)gates[(size_t)t * k + j] * dgate[j];
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      const double dl = (double)gates[(size_t)t * k + j] * (dgate[j] - sgd);
+      const int ri = orc_in(rexps, n_rexp, e);
+      for (int i = 0; i < d; ++i) {
+        if (ri >= 0) dwr_s[(size_t)ri * d + i] += dl * xt[i];
+        if (ti >= 0) dx_s[(size_t)ti * d + i] += dl * orc_elem(w_r, dtype, (size_t)e * d + i);
+      }
+    }
+  }
+  free(dgate);
+  free(dy);
+  free(dh);
+  free(h);
+  free(b);
+  free(a);
+  free(ot);
+  free(xt);
+}

@@ -23,12 +23,15 @@
 // stride byte offset steps between 8-row K groups (the canonical MN-major layout of the
 // tcgen05 shared-memory descriptor), with the instruction descriptor's A/B major bits set.
 //
-// Ragged groups.  The dgrad GEMMs tile a group's rows on N as the forward does (columns
-// past the group's rows are computed from neighbouring rows and never stored).  The weight
-// gradients take a group's rows as K in blocks of 64: full blocks are box loads; the last,
-// partial block is gathered four rows at a time (tile::gather4) with the rows past the
-// group pointing at an all-zero row kept after the sorted rows, so no row of a neighbouring
-// group enters the sum.  Each dW tile is owned by one unit, which adds its finished
+// Row layout.  The backward keeps its expert-sorted rows (x, dout, da, db, s*h and the
+// recomputed a, b) with every group padded to a multiple of 16 rows: routed group g starts at
+// poff[g] (an exclusive scan of the padded counts, computed on the device), the shared group
+// at a fixed row s0 = T*k + 15*E past any possible routed end, and the padding rows of the
+// bf16 operands are zero.  The dgrad GEMMs tile a group's rows on N as the forward does
+// (columns past the group's rows are never stored).  The weight gradients take a group's
+// rows as K in blocks of 64 box-loaded rows and issue only the 16-row MMA steps that reach
+// the group's padded end, so rows of a neighbouring group are loaded but never multiplied and
+// the padding adds zeros.  Each dW tile is owned by one unit, which adds its finished
 // accumulator into the caller's fp32 gradient with TMA reductions (cp.reduce.async.bulk
 // .tensor add): one addition per element and call, so the result is deterministic.
 //
@@ -93,22 +96,42 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// -------------------------------------------------------------------- row layout
+struct BwRows {
+  const int *offsets;  // [E + 1] group starts in the unpadded sorted rows
+  const int *poff;     // [E + 1] starts of the routed groups in the padded rows
+  int E, T, Tk;
+  int s0;              // padded start of the shared group (n_shared is 0 or 1)
+  // group g: first padded row, first unpadded row, rows
+  __device__ __forceinline__ void group(int g, int &rowp, int &rowu, int &cnt) const {
+    if (g < E) {
+      rowu = offsets[g];
+      cnt = offsets[g + 1] - rowu;
+      rowp = poff[g];
+    } else {
+      rowu = Tk;
+      cnt = T;
+      rowp = s0;
+    }
+  }
+};
+
 // --------------------------------------------------------------------- dgrad GEMMs
 enum BwDgradMode { BW_DH = 0, BW_DX = 1 };
 
 struct BwDgradParams {
   CUtensorMap tmA0;  // DH: W_down as [G*d, f]; DX: W_gate as [G*f, d]      box {64, 64}
   CUtensorMap tmA1;  // DX: W_up as [G*f, d]                                box {64, 64}
-  CUtensorMap tmB0;  // DH: dout rows [P+1, d]; DX: da [P+1, f] (sorted)    box {64, BN}
-  CUtensorMap tmB1;  // DX: db [P+1, f]                                     box {64, BN}
-  const int *offsets;          // [E + 1]
-  const float *row_scale;      // [P] s_p (DH)
-  const float *pre_a, *pre_b;  // [P, f] fp32 pre-activations (DH)
-  __nv_bfloat16 *da, *db, *hs; // [P + 1, f] (DH)
-  float *dgate_part;           // [P, n_part] (DH): partial sums of dhu . h
-  float *out;                  // DX: dX rows [P, d] fp32
+  CUtensorMap tmB0;  // DH: dout rows [R, d]; DX: da [R, f] (padded rows)  box {64, BN}
+  CUtensorMap tmB1;  // DX: db [R, f]                                      box {64, BN}
+  BwRows rows;
+  const float *row_scale;      // [P] s_p by unpadded row (DH)
+  const float *pre_a, *pre_b;  // [R, f] fp32 pre-activations, padded rows (DH)
+  __nv_bfloat16 *da, *db, *hs; // [R, f] padded rows (DH)
+  float *dgate_part;           // [Tk, n_part] by unpadded row (DH): partial sums of dhu . h
+  float *out;                  // DX: dX rows [P, d] fp32, unpadded rows
   DevStatus *status;
-  int E, n_groups, T, Tk;
+  int n_groups;
   int M;       // weight rows per group on M: f (DH), d (DX)
   int K;       // reduction length per operand pair: d (DH), f (DX)
   int n_pairs; // 1 (DH) or 2 (DX: W_gate with da, then W_up with db)
@@ -136,7 +159,7 @@ struct BwDgradCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N of the MMA");
   static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
-    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 + (size_t)(3 * n_groups + 1) * 4 +
+    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 + (size_t)(4 * n_groups + 1) * 4 +
            ACC_BUFS * BN * 4 /*row scales*/ + 4 * 16 * 32 * 4 /*store transposes*/ +
            4 * 16 * 33 * 4 /*dgate reductions*/ + 16;
   }
@@ -165,9 +188,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);        // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                     // [G]
-  int *grp_row = grp_count + p.n_groups;                             // [G]
+  int *grp_row = grp_count + p.n_groups;                             // [G] padded
+  int *grp_rowu = grp_row + p.n_groups;                              // [G] unpadded
   float *row_scale = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+      (reinterpret_cast<uintptr_t>(grp_rowu + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
   float *xbuf = row_scale + C::ACC_BUFS * BN;  // [4 warps][16][32] store transposes
   float *rbuf = xbuf + 4 * 16 * 32;            // [4 warps][16][33] dgate reductions
 
@@ -204,16 +228,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    int cnt, row;
-    if (g < p.E) {
-      row = p.offsets[g];
-      cnt = p.offsets[g + 1] - row;
-    } else {
-      row = p.Tk + (g - p.E) * p.T;
-      cnt = p.T;
-    }
+    int rowp, rowu, cnt;
+    p.rows.group(g, rowp, rowu, cnt);
     grp_count[g] = cnt;
-    grp_row[g] = row;
+    grp_row[g] = rowp;
+    grp_rowu[g] = rowu;
     unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
   }
   __syncthreads();
@@ -415,13 +434,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int g, mt, nt;
       decode(u, g, mt, nt);
       const int valid = min(BN, grp_count[g] - nt * BN);
-      const int row0 = grp_row[g] + nt * BN;
+      const int row0 = grp_row[g] + nt * BN;    // padded
+      const int rowu0 = grp_rowu[g] + nt * BN;  // unpadded
       const int col_base = mt * kBM + q * 32;  // first output column (M index) of this warp
       const int col = col_base + lane;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
       if (MODE == BW_DH) {
         for (int n = threadIdx.x - 64; n < BN; n += 128)
-          row_scale[acc * BN + n] = (n < valid) ? p.row_scale[row0 + n] : 0.f;
+          row_scale[acc * BN + n] = (n < valid) ? p.row_scale[rowu0 + n] : 0.f;
         named_bar_sync(1, 128);
       }
       uint32_t nx[16];
@@ -436,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (MODE == BW_DX) {
 #pragma unroll
           for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v[n]);
-          store_block16_f32(p.out, p.M, row0, c0, valid, col_base, vals, wbuf, lane);
+          store_block16_f32(p.out, p.M, rowu0, c0, valid, col_base, vals, wbuf, lane);
         } else {
           // pre-activations of the chunk's rows (coalesced: lanes read consecutive columns)
           float av[16], bv[16];
@@ -476,11 +496,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int n = 0; n < 16; ++n) red[n * 33 + lane] = vals[n];
           __syncwarp();
-          if (lane < 16 && c0 + lane < valid && g < p.E) {
+          if (lane < 16 && c0 + lane < valid && g < p.rows.E) {
             float sum = 0.f;
 #pragma unroll 8
             for (int i = 0; i < 32; ++i) sum += red[lane * 33 + i];
-            p.dgate_part[(size_t)(row0 + c0 + lane) * p.n_part + mt * 4 + q] = sum;
+            p.dgate_part[(size_t)(rowu0 + c0 + lane) * p.n_part + mt * 4 + q] = sum;
           }
           __syncwarp();
         }
@@ -498,45 +518,148 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------- wgrad GEMM
-constexpr int kWgOps = 5;    // sorted operands: dout, hs, da, db, x
+// ---------------------------------------------------------------------- wgrad GEMMs
+constexpr int kWgOps = 5;    // sorted operands: dout, s*h, da, db, x
 constexpr int kWgProbs = 3;  // dW_down, dW_gate, dW_up
 
 struct BwWgradParams {
-  CUtensorMap box[kWgOps];   // sorted rows [P + 1, width] bf16, box {64, 64}
-  CUtensorMap gat[kWgOps];   // the same rows, box {64, 1} (tile::gather4)
+  CUtensorMap box[kWgOps];   // padded sorted rows [R, width] bf16, box {64, 64}
   CUtensorMap out[kWgProbs]; // dW as [G * M, N] fp32, box {32, 32}, 128-byte swizzle
+  float *dw[kWgProbs];       // the same gradients as plain pointers
   int a_op[kWgProbs], b_op[kWgProbs];  // operand of the M side and of the N side
-  int M[kWgProbs], N[kWgProbs];        // dW[g] is [M, N]; M % 128 == 0, N % BNW == 0
+  int M[kWgProbs], N[kWgProbs];        // dW[g] is [M, N]; M, N multiples of the unit tile
   int n_prob;
-  const int *offsets;
+  BwRows rows;
   DevStatus *status;
-  int E, n_groups, T, Tk;
-  int zero_row;  // P: the all-zero row after the sorted rows
-  int *sched;
+  int n_groups;
+  int *sched;  // work counter (zero at launch)
 };
+
+constexpr int kWgStgBytes = 32 * 32 * 4;  // one 32 x 32 fp32 reduction tile
+
+// Warp-wide epilogue of one weight-gradient unit: the warp's 32 accumulator rows (TMEM lane
+// quadrant at `taddr`), 32-column chunks c = c_first, c_first + c_step, ... < n_cols, each
+// registers -> swizzled staging tile -> TMA reduction into dW at (col0 + 32 c, row).  The
+// warp cycles through NBUF staging tiles; lane 0 issues and tracks the reductions.  TMEM
+// loads run one chunk ahead.
+template <int NBUF>
+__device__ __forceinline__ void wgrad_epilogue(uint32_t taddr, int c_first, int c_step, int n_cols,
+                                               const CUtensorMap *omap, int col0, int row,
+                                               uint8_t *stg, int &n_red, int lane) {
+  uint32_t n0[16], n1[16];
+  if (32 * c_first < n_cols) {
+    tmem_ld16(taddr + 32 * c_first, n0);
+    tmem_ld16(taddr + 32 * c_first + 16, n1);
+  }
+  for (int c = c_first; 32 * c < n_cols; c += c_step) {
+    uint32_t v0[16], v1[16];
+    tmem_ld_wait_regs(n0, n1);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      v0[i] = n0[i];
+      v1[i] = n1[i];
+    }
+    if (32 * (c + c_step) < n_cols) {
+      tmem_ld16(taddr + 32 * (c + c_step), n0);
+      tmem_ld16(taddr + 32 * (c + c_step) + 16, n1);
+    }
+    uint8_t *buf = stg + (n_red % NBUF) * kWgStgBytes;
+    if (n_red >= NBUF) {  // the reduction that last read this tile is done reading it
+      if (lane == 0) bulk_wait_group_read<NBUF - 1>();
+      __syncwarp();
+    }
+    // row `lane`, 16-byte chunk j of the row at position j ^ (lane & 7) (128-byte swizzle)
+    uint8_t *r = buf + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<float4 *>(r + ((j ^ (lane & 7)) << 4)) =
+          make_float4(__uint_as_float(v0[4 * j]), __uint_as_float(v0[4 * j + 1]),
+                      __uint_as_float(v0[4 * j + 2]), __uint_as_float(v0[4 * j + 3]));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<float4 *>(r + (((j + 4) ^ (lane & 7)) << 4)) =
+          make_float4(__uint_as_float(v1[4 * j]), __uint_as_float(v1[4 * j + 1]),
+                      __uint_as_float(v1[4 * j + 2]), __uint_as_float(v1[4 * j + 3]));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(omap, buf, col0 + 32 * c, row);
+      bulk_commit_group();
+    }
+    ++n_red;
+  }
+}
+
+// Group table and unit scan shared by both weight-gradient kernels: units of (problem,
+// group) with rows, mtiles(pr) x ntiles(pr) each; exclusive prefix in unit_prefix.
+template <int BMW, int BNW>
+__device__ __forceinline__ void wgrad_unit_table(const BwWgradParams &p, int *unit_prefix,
+                                                 int *grp_count, int *grp_row) {
+  const int G = p.n_groups, NP = p.n_prob;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int rowp, rowu, cnt;
+    p.rows.group(g, rowp, rowu, cnt);
+    grp_count[g] = cnt;
+    grp_row[g] = rowp;
+    for (int pr = 0; pr < NP; ++pr)
+      unit_prefix[pr * G + g] = cnt > 0 ? (p.M[pr] / BMW) * (p.N[pr] / BNW) : 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int n = NP * G;
+    const int per = (n + 31) / 32;
+    const int lo = min(n, lane * per), hi = min(n, lo + per);
+    int run = 0;
+    for (int i = lo; i < hi; ++i) run += unit_prefix[i];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int i = lo; i < hi; ++i) {
+      const int u = unit_prefix[i];
+      unit_prefix[i] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[n] = incl;
+  }
+}
+
+// unit -> (problem, group, m tile, n tile), n tile innermost
+template <int BNW>
+__device__ __forceinline__ void wgrad_decode(const BwWgradParams &p, const int *unit_prefix, int u,
+                                             int &pr, int &g, int &mt, int &nt) {
+  const int G = p.n_groups;
+  int lo = 0, hi = p.n_prob * G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (unit_prefix[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  pr = lo / G;
+  g = lo - pr * G;
+  const int nts = p.N[pr] / BNW;
+  const int loc = u - unit_prefix[lo];
+  mt = loc / nts;
+  nt = loc % nts;
+}
 
 template <int BNW>
 struct BwWgradCfg {
   static constexpr int NB = BNW / 64;             // 64-element boxes on the N side
-  static constexpr int A_BYTES = kBM * kBK * 2;   // 2 boxes of 64 M x 64 rows
-  static constexpr int B_BYTES = BNW * kBK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BOX_BYTES = 64 * kBK * 2;  // 8 KB
+  static constexpr int A_BYTES = 2 * BOX_BYTES;   // 128 M x 64 rows
+  static constexpr int B_BYTES = NB * BOX_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int ACC_COLS = BNW;
   static constexpr int TMEM_COLS = 2 * BNW;
-  static constexpr int STG_BYTES = 32 * 32 * 4;   // one 32 x 32 fp32 reduction tile
-#ifndef MOE_WG_STG_BUFS
-#define MOE_WG_STG_BUFS 2
-#endif
-#ifndef MOE_WG_MAX_STAGES
-#define MOE_WG_MAX_STAGES 8
-#endif
-  static constexpr int STG_BUFS = MOE_WG_STG_BUFS;  // staging tiles per epilogue warp
-  static constexpr int STG_TOTAL = 4 * STG_BUFS * STG_BYTES;
-  static constexpr int SMEM_BUDGET = 220 * 1024 - STG_TOTAL;
-  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > MOE_WG_MAX_STAGES ? MOE_WG_MAX_STAGES : STAGES_RAW;
+  static constexpr int STG_BUFS = 2;
+  static constexpr int STG_TOTAL = 4 * STG_BUFS * kWgStgBytes;
+  static constexpr int STAGES_RAW = (220 * 1024 - STG_TOTAL) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(BNW == 128 || BNW == 256, "N tile");
   static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
@@ -546,6 +669,7 @@ struct BwWgradCfg {
   }
 };
 
+// One CTA per unit: 128 x BNW tile of dW[g].
 template <int BNW>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     bw_wgrad_kernel(const __grid_constant__ BwWgradParams p) {
@@ -569,10 +693,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
   const int G = p.n_groups;
-  const int NP = p.n_prob;
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [NP * G + 1]
-  int *grp_count = unit_prefix + NP * G + 1;                    // [G]
-  int *grp_row = grp_count + G;                                 // [G]
+  int *grp_count = unit_prefix + p.n_prob * G + 1;              // [G]
+  int *grp_row = grp_count + G;                                 // [G] padded
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -596,168 +719,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   griddep_wait();
   griddep_launch_dependents();
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    int cnt, row;
-    if (g < p.E) {
-      row = p.offsets[g];
-      cnt = p.offsets[g + 1] - row;
-    } else {
-      row = p.Tk + (g - p.E) * p.T;
-      cnt = p.T;
-    }
-    grp_count[g] = cnt;
-    grp_row[g] = row;
-    for (int pr = 0; pr < NP; ++pr)
-      unit_prefix[pr * G + g] = cnt > 0 ? (p.M[pr] / kBM) * (p.N[pr] / BNW) : 0;
-  }
-  __syncthreads();
-  if (warp == 0) {  // exclusive scan over (problem, group)
-    const int n = NP * G;
-    const int per = (n + 31) / 32;
-    const int lo = min(n, lane * per), hi = min(n, lo + per);
-    int run = 0;
-    for (int i = lo; i < hi; ++i) run += unit_prefix[i];
-    int incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int excl = incl - run;
-    for (int i = lo; i < hi; ++i) {
-      const int u = unit_prefix[i];
-      unit_prefix[i] = excl;
-      excl += u;
-    }
-    if (lane == 31) unit_prefix[n] = incl;
-  }
+  wgrad_unit_table<kBM, BNW>(p, unit_prefix, grp_count, grp_row);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_units = unit_prefix[NP * G];
-
-  // unit -> (problem, group, m tile, n tile), n tile innermost
-  auto decode = [&](int u, int &pr, int &g, int &mt, int &nt) {
-    int lo = 0, hi = NP * G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (unit_prefix[mid] <= u) lo = mid;
-      else hi = mid - 1;
-    }
-    pr = lo / G;
-    g = lo - pr * G;
-    const int nts = p.N[pr] / BNW;
-    const int loc = u - unit_prefix[lo];
-    mt = loc / nts;
-    nt = loc % nts;
-  };
+  const int total_units = unit_prefix[p.n_prob * G];
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    // Lane 0 claims units and loads full 64-row blocks as boxes; the last partial block of
-    // a group is gathered by the whole warp, rows past the group read from the zero row.
-    int stage = 0;
-    uint32_t phase = 0;
-    int issued = 0;
-    bool ok = true;
-    int qi = 0;
-    uint32_t qph = 0;
-    for (;;) {
-      int uid = -1;
-      if (lane == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      for (;;) {
         const int u = atomicAdd(p.sched, 1);
-        uid = (u < total_units) ? u : -1;
-        if (mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 31)) {
-          uq[qi] = uid;
-          mbar_arrive(&uq_full[qi]);
-        } else {
+        const int uid = (u < total_units) ? u : -1;
+        if (!mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 31)) {
           ok = false;
+          break;
         }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      uid = __shfl_sync(0xffffffffu, uid, 0);
-      if (++qi == kUnitQ) {
-        qi = 0;
-        qph ^= 1;
-      }
-      if (uid < 0) break;
-      int pr, g, mt, nt;
-      decode(uid, pr, g, mt, nt);
-      const CUtensorMap *abox = &p.box[p.a_op[pr]], *bbox = &p.box[p.b_op[pr]];
-      const CUtensorMap *agat = &p.gat[p.a_op[pr]], *bgat = &p.gat[p.b_op[pr]];
-      const int m0 = mt * kBM, n0 = nt * BNW;
-      const int cnt = grp_count[g], start = grp_row[g];
-      const int kbs = (cnt + kBK - 1) / kBK;
-      for (int kb = 0; kb < kbs; ++kb) {
-        const int r0 = start + kb * kBK;
-        const int rows_in = min(kBK, cnt - kb * kBK);
-        const int n_rows = (rows_in + 15) & ~15;
-        if (lane == 0) {
-          ok = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 32);
-          if (ok) {
-            mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 + C::NB) * n_rows * 128);
-            if (rows_in == kBK) {
-              uint8_t *a_dst = sA + stage * C::A_BYTES;
-              uint8_t *b_dst = sB + stage * C::B_BYTES;
-              tma_load_2d(a_dst, abox, &full[stage], m0, r0);
-              tma_load_2d(a_dst + C::BOX_BYTES, abox, &full[stage], m0 + 64, r0);
+        uq[qi] = uid;
+        mbar_arrive(&uq_full[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (uid < 0) break;
+        int pr, g, mt, nt;
+        wgrad_decode<BNW>(p, unit_prefix, uid, pr, g, mt, nt);
+        const CUtensorMap *abox = &p.box[p.a_op[pr]], *bbox = &p.box[p.b_op[pr]];
+        const int m0 = mt * kBM, n0 = nt * BNW;
+        const int kbs = (grp_count[g] + kBK - 1) / kBK;
+        for (int kb = 0; kb < kbs; ++kb) {
+          const int r0 = grp_row[g] + kb * kBK;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 32)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          uint8_t *a_dst = sA + stage * C::A_BYTES;
+          uint8_t *b_dst = sB + stage * C::B_BYTES;
+          tma_load_2d(a_dst, abox, &full[stage], m0, r0);
+          tma_load_2d(a_dst + C::BOX_BYTES, abox, &full[stage], m0 + 64, r0);
 #pragma unroll
-              for (int h = 0; h < C::NB; ++h)
-                tma_load_2d(b_dst + h * C::BOX_BYTES, bbox, &full[stage], n0 + 64 * h, r0);
-            }
+          for (int h = 0; h < C::NB; ++h)
+            tma_load_2d(b_dst + h * C::BOX_BYTES, bbox, &full[stage], n0 + 64 * h, r0);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        if (rows_in < kBK) {
-          // (2 + NB) boxes x n_rows / 4 gathers, spread over the lanes
-          const int quads = n_rows / 4;
-          const int total = (2 + C::NB) * quads;
-          const uint64_t pol = policy_evict_last();
-          for (int i = lane; i < total; i += 32) {
-            const int bx = i / quads, qd = i - bx * quads;
-            int rr[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = 4 * qd + e;
-              rr[e] = (r < rows_in) ? r0 + r : p.zero_row;
-            }
-            uint8_t *dst;
-            const CUtensorMap *map;
-            int x;
-            if (bx < 2) {
-              dst = sA + stage * C::A_BYTES + bx * C::BOX_BYTES;
-              map = agat;
-              x = m0 + 64 * bx;
-            } else {
-              dst = sB + stage * C::B_BYTES + (bx - 2) * C::BOX_BYTES;
-              map = bgat;
-              x = n0 + 64 * (bx - 2);
-            }
-            tma_gather4(dst + qd * 4 * 128, map, &full[stage], x, rr[0], rr[1], rr[2], rr[3],
-                        pol);
-          }
-        }
-        ++issued;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
       }
-      if (!ok) break;
-    }
-    if (!ok && lane == 0) {
-      int n = issued < S ? issued : S;
-      int st = stage, ph = phase;
-      for (int i = 0; i < n; ++i) {
-        if (--st < 0) {
-          st = S - 1;
-          ph ^= 1;
+      if (!ok) {
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
         }
-        volatile int no_abort = 0;
-        mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
       }
     }
     __syncwarp();
@@ -786,7 +815,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 34)) break;
         tc_fence_after();
         int pr, g, mt, nt;
-        decode(u, pr, g, mt, nt);
+        wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
         const int cnt = grp_count[g];
         const int kbs = (cnt + kBK - 1) / kBK;
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -796,8 +825,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const int rows_in = min(kBK, cnt - kb * kBK);
-          const int k16 = (rows_in + 15) >> 4;
+          // 16-row steps up to the group's padded end (padding rows are zero)
+          const int k16 = (min(kBK, cnt - kb * kBK) + 15) >> 4;
           const uint32_t a = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
           for (int kk = 0; kk < k16; ++kk)
@@ -819,9 +848,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // --------------------------------------------------------------------- epilogue
-    // Warp q owns accumulator rows 32q..32q+31 (its TMEM lane quadrant).  Each 32-column
-    // chunk goes registers -> swizzled staging tile -> TMA reduction into dW; two staging
-    // tiles per warp, so the next chunk is written while the previous reduction reads.
     const int q = warp & 3;
     auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
       int ok = 1;
@@ -830,7 +856,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       return ok != 0;
     };
-    uint8_t *my_stg = stg + q * C::STG_BUFS * C::STG_BYTES;
+    uint8_t *my_stg = stg + q * C::STG_BUFS * kWgStgBytes;
     int it = 0, n_red = 0;
     int qi = 0;
     uint32_t qph = 0;
@@ -850,40 +876,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!warp_wait(&tfull[acc], acc_phase, 37)) break;
       tc_fence_after();
       int pr, g, mt, nt;
-      decode(u, pr, g, mt, nt);
+      wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
-      const int out_row = g * p.M[pr] + mt * kBM + q * 32;
-      const CUtensorMap *omap = &p.out[pr];
-      for (int c = 0; c < BNW / 32; ++c) {
-        uint32_t v0[16], v1[16];
-        tmem_ld16(taddr + 32 * c, v0);
-        tmem_ld16(taddr + 32 * c + 16, v1);
-        tmem_ld_wait_regs(v0, v1);
-        uint8_t *buf = my_stg + (n_red % C::STG_BUFS) * C::STG_BYTES;
-        if (n_red >= C::STG_BUFS) {  // the reduction that last read this tile is done reading
-          if (lane == 0) bulk_wait_group_read<C::STG_BUFS - 1>();
-          __syncwarp();
-        }
-        // row `lane`, 16-byte chunk j of the row at position j ^ (lane & 7) (128-byte swizzle)
-        uint8_t *row = buf + lane * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<float4 *>(row + ((j ^ (lane & 7)) << 4)) =
-              make_float4(__uint_as_float(v0[4 * j]), __uint_as_float(v0[4 * j + 1]),
-                          __uint_as_float(v0[4 * j + 2]), __uint_as_float(v0[4 * j + 3]));
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<float4 *>(row + (((j + 4) ^ (lane & 7)) << 4)) =
-              make_float4(__uint_as_float(v1[4 * j]), __uint_as_float(v1[4 * j + 1]),
-                          __uint_as_float(v1[4 * j + 2]), __uint_as_float(v1[4 * j + 3]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_2d(omap, buf, nt * BNW + 32 * c, out_row);
-          bulk_commit_group();
-        }
-        ++n_red;
-      }
+      wgrad_epilogue<C::STG_BUFS>(taddr, 0, 1, BNW, &p.out[pr], nt * BNW,
+                                  g * p.M[pr] + mt * kBM + q * 32, my_stg, n_red, lane);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -899,23 +895,364 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// CTA-pair weight-gradient kernel: 256 x 256 tiles of dW[g] on a cluster of two CTAs
+// (tcgen05 cta_group::2).  CTA r stages rows [128 r, 128 r + 128) of the unit's M range and
+// columns [128 r, 128 r + 128) of its N range for every 64-row K block (32 KB), the leader
+// issues M = 256, N = 256 MMAs, and each CTA's TMEM receives its 128 rows for all 256
+// columns.  Per staged byte this is 1.5x the MMA work of the one-CTA 128 x 256 tile, which
+// matters because the K loops are short (a group's rows) and the tiles are re-read from L2
+// for every output tile.  Barriers and unit publication as in grouped_gemm_pair.cuh: full[s]
+// lives in the leader and counts both CTAs' bytes, the MMA commits arrive in both CTAs, and
+// tempty / uq_empty (leader) collect the arrivals of both CTAs' warps.
+constexpr int kWgPairEpiWarps = 8;  // two per TMEM lane quadrant, alternating 32-column chunks
+constexpr int kWgPairThreads = 32 * (2 + kWgPairEpiWarps);
+
+struct BwWgradPairCfg {
+  static constexpr int BOX_BYTES = 64 * kBK * 2;  // 8 KB
+  static constexpr int A_BYTES = 2 * BOX_BYTES;   // this CTA's 128 M x 64 rows
+  static constexpr int B_BYTES = 2 * BOX_BYTES;   // this CTA's 128 N x 64 rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int STG_BUFS = 2;
+  static constexpr int STG_TOTAL = kWgPairEpiWarps * STG_BUFS * kWgStgBytes;
+  static constexpr int STAGES_RAW = (220 * 1024 - STG_TOTAL) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "pipeline too shallow");
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
+  static constexpr size_t smem_bytes(int n_groups) {
+    return 1024 + (size_t)STAGES * STAGE_BYTES + STG_TOTAL + BAR_BYTES + 64 +
+           (size_t)(kWgProbs * n_groups + 1) * 4 + (size_t)n_groups * 2 * 4 + 16;
+  }
+};
+
+__global__ void __launch_bounds__(kWgPairThreads, 1)
+    bw_wgrad_pair_kernel(const __grid_constant__ BwWgradParams p) {
+  using C = BwWgradPairCfg;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + S * C::A_BYTES;
+  uint8_t *stg = sB + S * C::B_BYTES;  // 1024-byte aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(stg + C::STG_TOTAL);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *tfull = bars + 2 * S;
+  uint64_t *tempty = bars + 2 * S + 2;
+  uint64_t *drain = bars + 2 * S + 4;
+  uint64_t *uq_full = bars + 2 * S + 5;
+  uint64_t *uq_empty = uq_full + kUnitQ;  // used in the leader only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
+  const int G = p.n_groups;
+  int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [NP * G + 1]
+  int *grp_count = unit_prefix + p.n_prob * G + 1;              // [G]
+  int *grp_row = grp_count + G;                                 // [G] padded
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kWgPairEpiWarps);  // one per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    for (int q = 0; q < kUnitQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      // readers of a published unit id: the leader's MMA thread and epilogue warps, the
+      // peer's producer and epilogue warps
+      mbar_init(&uq_empty[q], 2 + 2 * kWgPairEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  griddep_wait();
+  griddep_launch_dependents();
+  wgrad_unit_table<2 * kBM, 256>(p, unit_prefix, grp_count, grp_row);
+  // both CTAs' barriers are initialised and TMEM allocated before any cross-CTA traffic
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = unit_prefix[p.n_prob * G];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      int u = -1;
+      while (ok) {
+        if (leader) {
+          const int c = atomicAdd(p.sched, 1);
+          const int uid = (c < total_units) ? c : -1;
+          if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 41)) {
+            ok = false;
+            break;
+          }
+          uq[qi] = uid;
+          st_shared_remote(mapa_shared(smem_u32((const void *)&uq[qi]), 1), uid);
+          mbar_arrive(&uq_full[qi]);
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_full[qi]), 1));
+          u = uid;
+        } else {
+          if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 42)) {
+            ok = false;
+            break;
+          }
+          u = uq[qi];
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_empty[qi]), 0));
+        }
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        int pr, g, mt, nt;
+        wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
+        const CUtensorMap *abox = &p.box[p.a_op[pr]], *bbox = &p.box[p.b_op[pr]];
+        const int ma = mt * 256 + (int)rank * 128, nb = nt * 256 + (int)rank * 128;
+        const int kbs = (grp_count[g] + kBK - 1) / kBK;
+        for (int kb = 0; kb < kbs; ++kb) {
+          const int r0 = grp_row[g] + kb * kBK;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 43)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          uint8_t *a_dst = sA + stage * C::A_BYTES;
+          uint8_t *b_dst = sB + stage * C::B_BYTES;
+          tma_load_2d_pair(a_dst, abox, fbar, ma, r0, pol);
+          tma_load_2d_pair(a_dst + C::BOX_BYTES, abox, fbar, ma + 64, r0, pol);
+          tma_load_2d_pair(b_dst, bbox, fbar, nb, r0, pol);
+          tma_load_2d_pair(b_dst + C::BOX_BYTES, bbox, fbar, nb + 64, r0, pol);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // drain: wait (time-bounded, ignoring the abort flag) for the copies still in flight
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      constexpr uint32_t idesc = idesc_bf16_f32_major(2 * kBM, 256, true, true);
+      while (ok) {
+        if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 44)) break;
+        const int u = uq[qi];
+        mbar_arrive(&uq_empty[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        ++it;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 45)) break;
+        tc_fence_after();
+        int pr, g, mt, nt;
+        wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
+        const int cnt = grp_count[g];
+        const int kbs = (cnt + kBK - 1) / kBK;
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, 46)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int k16 = (min(kBK, cnt - kb * kBK) + 15) >> 4;
+          const uint32_t a = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+          for (int kk = 0; kk < k16; ++kk)
+            tc_mma_bf16_pair(d0, sdesc_mn_sw128(a + kk * 16 * 128, C::BOX_BYTES),
+                             sdesc_mn_sw128(b + kk * 16 * 128, C::BOX_BYTES), idesc,
+                             (kb | kk) ? 1u : 0u);
+          tc_commit_pair_both(&empty[stage]);  // slot free in both CTAs once read
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair_both(&tfull[acc]);
+      }
+      tc_commit_pair_local(drain);
+      volatile int no_abort = 0;
+      mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;          // TMEM lane quadrant
+    const int eh = (warp - 2) >> 2;  // which of the quadrant's two warps: chunks eh, eh + 2, ..
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t uq_empty_leader = mapa_shared(smem_u32(&uq_empty[0]), 0);
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where, bool cluster) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = (cluster ? mbar_wait_bounded<true>(bar, parity, abort_flag, p.status, where)
+                      : mbar_wait_bounded(bar, parity, abort_flag, p.status, where))
+                 ? 1
+                 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      return ok != 0;
+    };
+    uint8_t *my_stg = stg + (warp - 2) * C::STG_BUFS * kWgStgBytes;
+    int it = 0, n_red = 0;
+    int qi = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!warp_wait(&uq_full[qi], qph, 47, true)) break;
+      const int u = uq[qi];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&uq_empty[qi]);
+        else mbar_arrive_remote(uq_empty_leader + qi * 8);
+      }
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (u < 0) break;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      ++it;
+      if (!warp_wait(&tfull[acc], acc_phase, 48, false)) break;
+      tc_fence_after();
+      int pr, g, mt, nt;
+      wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      wgrad_epilogue<C::STG_BUFS>(taddr, eh, 2, 256, &p.out[pr], nt * 256,
+                                  g * p.M[pr] + mt * 256 + (int)rank * 128 + q * 32, my_stg,
+                                  n_red, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_leader + acc * 8);
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
+  // the pair leaves together: the leader's MMAs read the peer's shared memory, and the
+  // peer's TMA loads signal the leader's barriers
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // --------------------------------------------------------------- small backward kernels
-// Sorted rows of x and dout (row p of group g: token row_token[p]) with the all-zero row P
-// after them; the zero row of da, db and hs as well.  One warp per row, 16-byte copies.
+// poff[g] = sum over routed groups g' < g of their row counts rounded up to 16 (g <= E).
+// One warp: each lane scans a contiguous run of groups.
+__global__ void __launch_bounds__(32) bw_pad_offsets_kernel(const int *__restrict__ offsets,
+                                                            int E, int *poff) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x;
+  const int per = (E + 31) / 32;
+  const int lo = min(E, lane * per), hi = min(E, lo + per);
+  int run = 0;
+  for (int g = lo; g < hi; ++g) run += (offsets[g + 1] - offsets[g] + 15) & ~15;
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int excl = incl - run;
+  for (int g = lo; g < hi; ++g) {
+    poff[g] = excl;
+    excl += (offsets[g + 1] - offsets[g] + 15) & ~15;
+  }
+  if (lane == 31) poff[E] = incl;
+}
+
+// Padded expert-sorted rows [0, R): x and dout of the row's token into xs, dys; zero rows of
+// xs, dys, da, db, hs at the padding; perm_pad[r] = the (token, slot) pair of routed row r
+// (padding rows repeat their group's first pair).  Rows between the routed end and the
+// shared group belong to no group and are not written.  One warp per row, 16-byte copies.
 __global__ void __launch_bounds__(256) bw_sorted_rows_kernel(
     const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ dout,
-    const int *__restrict__ row_token, int P, int d, int f, __nv_bfloat16 *xs,
-    __nv_bfloat16 *dys, __nv_bfloat16 *da, __nv_bfloat16 *db, __nv_bfloat16 *hs) {
+    const int *__restrict__ perm, int k, BwRows rows, int n_shared, int R, int d, int f,
+    __nv_bfloat16 *xs, __nv_bfloat16 *dys, __nv_bfloat16 *da, __nv_bfloat16 *db,
+    __nv_bfloat16 *hs, int *perm_pad) {
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int vec_d = d / 8, vec_f = f / 8;
-  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p <= P; p += nw) {
-    uint4 *xo = reinterpret_cast<uint4 *>(xs + (size_t)p * d);
-    uint4 *yo = reinterpret_cast<uint4 *>(dys + (size_t)p * d);
-    if (p < P) {
-      const int t = row_token[p];
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  const int routed_end = rows.poff[rows.E];
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < R; r += nw) {
+    int t = -1;  // token of the row; -1: padding
+    if (r >= rows.s0) {
+      if (n_shared == 0) continue;
+      const int i = r - rows.s0;
+      if (i < rows.T) t = i;
+    } else {
+      if (r >= routed_end) continue;  // between the groups: unused
+      int lo = 0, hi = rows.E - 1;    // last g with poff[g] <= r
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rows.poff[mid] <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      const int g = lo;
+      const int base = rows.offsets[g], cnt = rows.offsets[g + 1] - base;
+      const int i = r - rows.poff[g];
+      const int q = perm[base + (i < cnt ? i : 0)];
+      if (lane == 0) perm_pad[r] = q;
+      if (i < cnt) t = q / k;
+    }
+    uint4 *xo = reinterpret_cast<uint4 *>(xs + (size_t)r * d);
+    uint4 *yo = reinterpret_cast<uint4 *>(dys + (size_t)r * d);
+    if (t >= 0) {
       const uint4 *xi = reinterpret_cast<const uint4 *>(x + (size_t)t * d);
       const uint4 *yi = reinterpret_cast<const uint4 *>(dout + (size_t)t * d);
       for (int i = lane; i < vec_d; i += 32) {
@@ -923,15 +1260,14 @@ __global__ void __launch_bounds__(256) bw_sorted_rows_kernel(
         yo[i] = __ldg(yi + i);
       }
     } else {
-      const uint4 z = make_uint4(0, 0, 0, 0);
       for (int i = lane; i < vec_d; i += 32) {
         xo[i] = z;
         yo[i] = z;
       }
       for (int i = lane; i < vec_f; i += 32) {
-        reinterpret_cast<uint4 *>(da + (size_t)P * f)[i] = z;
-        reinterpret_cast<uint4 *>(db + (size_t)P * f)[i] = z;
-        reinterpret_cast<uint4 *>(hs + (size_t)P * f)[i] = z;
+        reinterpret_cast<uint4 *>(da + (size_t)r * f)[i] = z;
+        reinterpret_cast<uint4 *>(db + (size_t)r * f)[i] = z;
+        reinterpret_cast<uint4 *>(hs + (size_t)r * f)[i] = z;
       }
     }
   }

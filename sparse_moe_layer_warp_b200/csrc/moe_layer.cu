@@ -42,6 +42,7 @@ struct moe_layer {
   // the same weights as MN-major operands of the backward (box {64, 64}): W_gate and W_up
   // as [G*f, d], W_down as [G*d, f]
   CUtensorMap tm_wg_mn, tm_wu_mn, tm_wd_mn;
+  int wg_pair_grid;  // CTAs of the CTA-pair weight-gradient kernel (0: not available)
 };
 
 namespace {
@@ -361,6 +362,30 @@ int pair_grid_size(const moe_layer *L) {
   return 2 * n;
 }
 
+// CTAs of the persistent CTA-pair weight-gradient kernel (two per co-resident cluster).
+int wgrad_pair_grid_size(const moe_layer *L) {
+  const size_t smem = BwWgradPairCfg::smem_bytes(L->cfg.n_experts + L->cfg.n_shared);
+  if (smem > (size_t)L->smem_optin) return 0;
+  if (cudaFuncSetAttribute(bw_wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(L->num_sms & ~1);
+  cfg.blockDim = dim3(kWgPairThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, bw_wgrad_pair_kernel, &cfg) != cudaSuccess) return 0;
+  return 2 * n;
+}
+
 template <int MODE>
 moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_t st) {
   const size_t smem = pair_smem<MODE>(L->cfg);
@@ -421,11 +446,19 @@ bool backward_on_tensor_cores(const moe_config &c) { return c.dtype == MOE_BF16;
 // Backward workspace: the forward's layout, then the backward's own regions.
 struct BwLayout {
   size_t row_token, row_group, row_scale, tile_prefix, a, b, dh, db, wide, dgate, dl;
-  // tensor-core path: expert-sorted bf16 rows of x, dout, da, db, s*h ([P + 1] rows each,
-  // the last all zero) and the partial sums of dgate
-  size_t xs16, dys16, da16, db16, hs16, dgate_part;
+  // tensor-core path: padded expert-sorted rows (bw_rows() of them) of x, dout, da, db,
+  // s*h (bf16), the routed groups' padded starts, the (token, slot) pair of each padded
+  // row, and the partial sums of dgate
+  size_t xs16, dys16, da16, db16, hs16, poff, perm_pad, dgate_part;
   size_t total;
 };
+
+// Padded sorted rows of the tensor-core backward: routed groups rounded up to 16 rows
+// (at most T*k + 15*E rows), then the shared group at s0 = T*k + 15*E.
+int bw_s0(const moe_config &c, int T) { return T * c.top_k + 15 * c.n_experts; }
+int bw_rows(const moe_config &c, int T) {
+  return bw_s0(c, T) + (c.n_shared ? (T + 15) / 16 * 16 : 0);
+}
 
 BwLayout bw_layout(const moe_config &c, int T) {
   BwLayout B;
@@ -438,22 +471,26 @@ BwLayout bw_layout(const moe_config &c, int T) {
   const bool tc = backward_on_tensor_cores(c);
   const size_t Tk = (size_t)T * c.top_k, P = Tk + (size_t)c.n_shared * T;
   const size_t G = (size_t)c.n_experts + c.n_shared;
+  const size_t R = tc ? (size_t)bw_rows(c, T) : P;  // rows of a and b
   B.row_token = take(P * 4);
   B.row_group = take(P * 4);
   B.row_scale = take(P * 4);
   B.tile_prefix = take((G + 1) * 4);
-  B.a = take(P * c.d_ff * 4);
-  B.b = take(P * c.d_ff * 4);
+  B.a = take(R * c.d_ff * 4);
+  B.b = take(R * c.d_ff * 4);
   B.dh = take(tc ? 0 : P * c.d_ff * 4);
   B.db = take(tc ? 0 : P * c.d_ff * 4);
   B.wide = take(P * c.d_model * 4);  // unscaled expert outputs, then the rows of dx
   B.dgate = take(Tk * 4);
   B.dl = take(Tk * 4);
-  B.xs16 = take(tc ? (P + 1) * c.d_model * 2 : 0);
-  B.dys16 = take(tc ? (P + 1) * c.d_model * 2 : 0);
-  B.da16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
-  B.db16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
-  B.hs16 = take(tc ? (P + 1) * c.d_ff * 2 : 0);
+  const size_t Rt = tc ? R : 0;
+  B.xs16 = take(Rt * c.d_model * 2);
+  B.dys16 = take(Rt * c.d_model * 2);
+  B.da16 = take(Rt * c.d_ff * 2);
+  B.db16 = take(Rt * c.d_ff * 2);
+  B.hs16 = take(Rt * c.d_ff * 2);
+  B.poff = take(tc ? ((size_t)c.n_experts + 1) * 4 : 0);
+  B.perm_pad = take(Rt * 4);
   B.dgate_part = take(tc ? Tk * (c.d_ff / 32) * 4 : 0);
   B.total = off;
   return B;
@@ -552,6 +589,7 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
   if (c.dtype == MOE_BF16) {
     L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
+    L->wg_pair_grid = wgrad_pair_grid_size(L);
     cudaGetLastError();  // an unavailable cluster query only disables the pair path
     const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
@@ -793,10 +831,21 @@ moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
 // bf16 expert up GEMM over the routing in `ws`: h (bf16, `out`) -- or, with out2 set, the
 // fp32 pre-activations x W_g^T (`out`) and x W_u^T (`out2`).  done: the per-group h
 // hand-over counts (null: none).  *used receives the parameters (the down GEMM's start).
+// Row layout of an up GEMM that does not use the forward's (the backward's padded rows):
+// group starts (routed groups; counts from consecutive starts), the (token, slot) pair of
+// each row, the shared group's first row, and the sorted copy of x with its row count.
+struct UpRows {
+  const int *offsets;
+  const int *perm;
+  int shared_row;
+  const void *xs;
+  int xs_rows;
+};
+
 moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
                             const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
                             int *done, cudaStream_t st, GemmParams *used,
-                            const void *xs = nullptr) {
+                            const UpRows *rows = nullptr) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
@@ -807,7 +856,8 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
   p1.tmA1 = h->tm_wu;
   if (plan.gather_in_gemm) {
     if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
-  } else if (!encode_bf16_2d(&p1.tmB, xs ? xs : at<void>(ws, W.xs), c.d_model, Tk, bn) ||
+  } else if (!encode_bf16_2d(&p1.tmB, rows ? rows->xs : at<void>(ws, W.xs), c.d_model,
+                             rows ? rows->xs_rows : Tk, bn) ||
              !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
     return MOE_ERR_CUDA;
   }
@@ -828,6 +878,11 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
   p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
   p1.topk = c.top_k;
   p1.done = done;
+  if (rows) {
+    p1.offsets = rows->offsets;
+    p1.perm = rows->perm;
+    p1.Tk = rows->shared_row;
+  }
   return plan.pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st);
 }
 }  // namespace
@@ -1219,16 +1274,31 @@ moe_status launch_bw_wgrad(const moe_layer *L, const BwWgradParams &p, cudaStrea
   return launch(bw_wgrad_kernel<BNW>, dim3(L->num_sms), dim3(kGemmThreads), smem, st, p);
 }
 
+// Mean routed rows per expert from which the weight gradients run on CTA pairs.
+constexpr double kWgradPairMinRows = 16.0;
+
+moe_status launch_bw_wgrad_pair(const moe_layer *L, const BwWgradParams &p, cudaStream_t st) {
+  const size_t smem = BwWgradPairCfg::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bw_wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_cl(bw_wgrad_pair_kernel, dim3(L->wg_pair_grid), dim3(kWgPairThreads), smem, st,
+                   2, p);
+}
+
 // bf16 backward with every matrix product on the tensor cores (grouped_gemm_bw.cuh):
-//   selection -> row bookkeeping -> sorted bf16 rows of x and dout -> a, b (the forward's
-//   up GEMM) -> DH (dh, SwiGLU backward, dgate partials) -> dgate -> DX (rows of dx) ->
-//   the three weight gradients in one launch -> router terms and dx.
+//   selection -> row bookkeeping -> padded sorted bf16 rows of x and dout -> a, b (the
+//   forward's up GEMM on the padded rows) -> DH (dh, SwiGLU backward, dgate partials) ->
+//   dgate -> DX (rows of dx) -> the three weight gradients in one launch -> router terms
+//   and dx.
 moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
                        int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
                        float *dw_down, void *ws, cudaStream_t st) {
   const moe_config &c = L->cfg;
   const int E = c.n_experts, G = E + c.n_shared, k = c.top_k, d = c.d_model, f = c.d_ff;
   const int Tk = T * k, P = Tk + c.n_shared * T;
+  const int R = bw_rows(c, T);
   const WsLayout W = ws_layout(c, T);
   const BwLayout B = bw_layout(c, T);
   DevStatus *status = at<DevStatus>(ws, W.status);
@@ -1242,29 +1312,34 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   __nv_bfloat16 *xs = at<__nv_bfloat16>(ws, B.xs16), *dys = at<__nv_bfloat16>(ws, B.dys16);
   __nv_bfloat16 *da = at<__nv_bfloat16>(ws, B.da16), *db = at<__nv_bfloat16>(ws, B.db16);
   __nv_bfloat16 *hs = at<__nv_bfloat16>(ws, B.hs16);
+  int *poff = at<int>(ws, B.poff), *perm_pad = at<int>(ws, B.perm_pad);
   float *dgate_part = at<float>(ws, B.dgate_part);
   const __nv_bfloat16 *wr = static_cast<const __nv_bfloat16 *>(L->w.w_router);
+  const BwRows rows{offsets, poff, E, T, Tk, bw_s0(c, T)};
   moe_status s;
   if ((s = backward_select(L, x, T, ws, st)) != MOE_OK) return s;
   if ((s = launch(bw_rows_kernel, dim3(grid_for(P, 256, L->num_sms)), dim3(256), 0, st,
                   (const int *)perm, (const int *)idx, (const float *)gate, T, k, E, c.n_shared,
                   c.routed_scale, row_token, row_group, row_scale)) != MOE_OK ||
-      (s = launch(bw_sorted_rows_kernel, dim3(grid_for((size_t)P + 1, 8, L->num_sms)),
-                  dim3(256), 0, st, x, dout, (const int *)row_token, P, d, f, xs, dys, da, db,
-                  hs)) != MOE_OK)
+      (s = launch(bw_pad_offsets_kernel, dim3(1), dim3(32), 0, st, (const int *)offsets, E,
+                  poff)) != MOE_OK ||
+      (s = launch(bw_sorted_rows_kernel, dim3(grid_for((size_t)R, 8, L->num_sms)), dim3(256), 0,
+                  st, x, dout, (const int *)perm, k, rows, c.n_shared, R, d, f, xs, dys, da, db,
+                  hs, perm_pad)) != MOE_OK)
     return s;
-  // pre-activations a, b: the forward's up GEMM, token rows from the sorted copy
+  // pre-activations a, b: the forward's up GEMM over the padded rows
   const ForwardPlan plan = plan_forward(L, T);
+  const UpRows up_rows{poff, perm_pad, rows.s0, xs, R};
   GemmParams pu;
-  if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, xs)) != MOE_OK)
+  if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, &up_rows)) != MOE_OK)
     return s;
   // DH
   const int bn = pick_bn(c, T, MODE_DOWN);
   BwDgradParams pd;
   memset(&pd, 0, sizeof pd);
   pd.tmA0 = L->tm_wd_mn;
-  if (!encode_bf16_2d(&pd.tmB0, dys, d, (uint64_t)P + 1, bn)) return MOE_ERR_CUDA;
-  pd.offsets = offsets;
+  if (!encode_bf16_2d(&pd.tmB0, dys, d, (uint64_t)R, bn)) return MOE_ERR_CUDA;
+  pd.rows = rows;
   pd.row_scale = row_scale;
   pd.pre_a = a;
   pd.pre_b = b;
@@ -1273,10 +1348,7 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   pd.hs = hs;
   pd.dgate_part = dgate_part;
   pd.status = status;
-  pd.E = E;
   pd.n_groups = G;
-  pd.T = T;
-  pd.Tk = Tk;
   pd.M = f;
   pd.K = d;
   pd.n_pairs = 1;
@@ -1291,8 +1363,8 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   BwDgradParams px = pd;
   px.tmA0 = L->tm_wg_mn;
   px.tmA1 = L->tm_wu_mn;
-  if (!encode_bf16_2d(&px.tmB0, da, f, (uint64_t)P + 1, bn) ||
-      !encode_bf16_2d(&px.tmB1, db, f, (uint64_t)P + 1, bn))
+  if (!encode_bf16_2d(&px.tmB0, da, f, (uint64_t)R, bn) ||
+      !encode_bf16_2d(&px.tmB1, db, f, (uint64_t)R, bn))
     return MOE_ERR_CUDA;
   px.out = wide;
   px.M = d;
@@ -1306,13 +1378,14 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   __nv_bfloat16 *ops[kWgOps] = {dys, hs, da, db, xs};
   const int widths[kWgOps] = {d, f, f, f, d};
   for (int i = 0; i < kWgOps; ++i)
-    if (!encode_bf16_2d(&pw.box[i], ops[i], widths[i], (uint64_t)P + 1, 64) ||
-        !encode_bf16_2d(&pw.gat[i], ops[i], widths[i], (uint64_t)P + 1, 1))
-      return MOE_ERR_CUDA;
+    if (!encode_bf16_2d(&pw.box[i], ops[i], widths[i], (uint64_t)R, 64)) return MOE_ERR_CUDA;
   if (!encode_f32_2d(&pw.out[0], dw_down, f, (uint64_t)G * d) ||
       !encode_f32_2d(&pw.out[1], dw_gate, d, (uint64_t)G * f) ||
       !encode_f32_2d(&pw.out[2], dw_up, d, (uint64_t)G * f))
     return MOE_ERR_CUDA;
+  pw.dw[0] = dw_down;
+  pw.dw[1] = dw_gate;
+  pw.dw[2] = dw_up;
   const int a_op[kWgProbs] = {0, 2, 3}, b_op[kWgProbs] = {1, 4, 4};
   const int Ms[kWgProbs] = {d, f, f}, Ns[kWgProbs] = {f, d, d};
   for (int i = 0; i < kWgProbs; ++i) {
@@ -1322,16 +1395,19 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
     pw.N[i] = Ns[i];
   }
   pw.n_prob = kWgProbs;
-  pw.offsets = offsets;
+  pw.rows = rows;
   pw.status = status;
-  pw.E = E;
   pw.n_groups = G;
-  pw.T = T;
-  pw.Tk = Tk;
-  pw.zero_row = P;
   pw.sched = &status->sched[3];
-  s = (d % 256 == 0 && f % 256 == 0) ? launch_bw_wgrad<256>(L, pw, st)
-                                     : launch_bw_wgrad<128>(L, pw, st);
+  // CTA pairs (256 x 256 tiles) when the groups' K loops are long enough for their operand
+  // traffic to matter; decode-sized groups (a row or two each) are bound by the gradient
+  // read-modify-write, where the one-CTA kernel's shorter per-unit path is faster
+  const bool pair_wg = (double)T * k / E >= kWgradPairMinRows;
+  if (pair_wg && d % 256 == 0 && f % 256 == 0 && L->wg_pair_grid >= 2)
+    s = launch_bw_wgrad_pair(L, pw, st);
+  else
+    s = (d % 256 == 0 && f % 256 == 0) ? launch_bw_wgrad<256>(L, pw, st)
+                                       : launch_bw_wgrad<128>(L, pw, st);
   if (s != MOE_OK) return s;
   // router and dx
   if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,

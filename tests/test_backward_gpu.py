@@ -17,6 +17,11 @@ CASES = [
     {"dtype": "bf16", "T": 90, "d": 128, "E": 24, "k": 3, "f": 128, "bias": "zipf",
      "n_shared": 0},                                                               # empty experts
     {"dtype": "bf16", "T": 400, "d": 128, "E": 8, "k": 4, "f": 128, "seed": 5},   # 256-row tiles
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 256, "seed": 6},   # pair wgrad,
+    {"dtype": "bf16", "T": 75, "d": 512, "E": 12, "k": 2, "f": 256, "seed": 7,    # small groups
+     "routed_scale": 0.5},                                                       # ragged 16-row pads
+    {"dtype": "bf16", "T": 200, "d": 256, "E": 16, "k": 4, "f": 256, "seed": 8,   # pair wgrad,
+     "bias": "zipf"},                                                               # skewed groups
     {"dtype": "f32"},
 ]
 

@@ -429,3 +429,33 @@ def test_backward_matches_finite_differences():
         m[pos] -= eps
         fd = (loss(**{key: p}) - loss(**{key: m})) / (2 * eps)
         assert abs(got[name][pos] - fd) <= 2e-3 * max(1.0, abs(fd)), (name, got[name][pos], fd)
+
+
+# ------------------------------------------------------------ sampled backward
+from oracle import oracle_moe_backward_sampled  # noqa: E402
+
+
+@pytest.mark.parametrize("n_shared,rs,dtype", [(1, 1.0, "f32"), (0, 1.5, "f32"), (1, 1.0, "bf16")])
+def test_sampled_backward_equals_full_backward(n_shared, rs, dtype):
+    """The sampled entry point returns exactly the selected rows / experts of the full
+    (autograd- and finite-difference-pinned) oracle backward."""
+    w = synth.WORKLOADS["tiny_fp32"].replace(T=9, d=16, E=6, k=2, f=8, seed=12, dtype=dtype,
+                                             n_shared=n_shared)
+    inp = synth.make_inputs(w)
+    x, wr, b, wg, wu, wd = [synth.to_numpy_bits(t) for t in (inp.x, inp.w_router, inp.bias,
+                                                             inp.w_gate, inp.w_up, inp.w_down)]
+    dout = synth.to_numpy_bits(synth.make_x(w, w.T, seed=21))
+    _, idx, gates, _ = oracle_moe_forward(x, wr, b, wg, wu, wd, w.k, n_shared=n_shared,
+                                          routed_scale=rs)
+    full = oracle_moe_backward(x, dout, wr, wg, wu, wd, idx, gates, rs, n_shared)
+    toks = [0, 4, 8]
+    exps = sorted({int(idx[1, 0]), int(idx[5, 1])} | ({w.E} if n_shared else set()))
+    unchosen = [e for e in range(w.E) if e not in set(idx.ravel().tolist())]
+    exps = exps + unchosen[:1]
+    rexps = sorted({int(idx[2, 1]), int(idx[7, 0])})
+    got = oracle_moe_backward_sampled(x, dout, wr, wg, wu, wd, idx, gates, toks, exps, rexps,
+                                      rs, n_shared)
+    assert np.array_equal(got["dx"], full["dx"][toks])
+    for name in ("dw_gate", "dw_up", "dw_down"):
+        assert np.array_equal(got[name], full[name][exps]), name
+    assert np.array_equal(got["dw_router"], full["dw_router"][rexps])
