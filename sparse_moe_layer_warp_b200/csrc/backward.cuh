@@ -428,8 +428,26 @@ __global__ void __launch_bounds__(256) bw_router_dl_kernel(const float *__restri
   }
 }
 
+// Two consecutive inputs as floats (4 bytes of bf16, 8 of fp32); four (8 / 16 bytes).
+__device__ __forceinline__ float2 bw_load2(const __nv_bfloat16 *p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ float2 bw_load2(const float *p) {
+  return *reinterpret_cast<const float2 *>(p);
+}
+__device__ __forceinline__ float4 bw_load4(const __nv_bfloat16 *p) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2 *>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float4 bw_load4(const float *p) {
+  return __ldg(reinterpret_cast<const float4 *>(p));
+}
+
 // dW_r[e][i] += sum over the rows of routed group e (ascending token) of dl x_t[i]; experts
-// no token chose are left untouched.
+// no token chose are left untouched.  Block (e, 512 columns): each thread two columns, the
+// rows four at a time (their loads issued together, the sums still in row order).
 template <typename Tin>
 __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict__ x,
                                                            const float *__restrict__ dl,
@@ -439,17 +457,42 @@ __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict
   griddep_wait();
   griddep_launch_dependents();
   const int e = blockIdx.x;
-  const int i = blockIdx.y * blockDim.x + threadIdx.x;
-  if (i >= d || offsets[e] == offsets[e + 1]) return;
-  float acc = 0.f;
-  for (int p = offsets[e]; p < offsets[e + 1]; ++p) {
-    const int q = perm[p];
-    acc = fmaf(dl[q], bw_f32(x[(size_t)(q / k) * d + i]), acc);
+  const int i = 2 * (blockIdx.y * blockDim.x + threadIdx.x);
+  const int lo = offsets[e], hi = offsets[e + 1];
+  if (i >= d || lo == hi) return;
+  float2 acc = make_float2(0.f, 0.f);
+  int p = lo;
+  for (; p + 4 <= hi; p += 4) {
+    int q[4];
+    float w[4];
+    float2 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) q[u] = perm[p + u];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      w[u] = dl[q[u]];
+      v[u] = bw_load2(x + (size_t)(q[u] / k) * d + i);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc.x = fmaf(w[u], v[u].x, acc.x);
+      acc.y = fmaf(w[u], v[u].y, acc.y);
+    }
   }
-  dw_r[(size_t)e * d + i] += acc;
+  for (; p < hi; ++p) {
+    const int q = perm[p];
+    const float w = dl[q];
+    const float2 v = bw_load2(x + (size_t)(q / k) * d + i);
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+  }
+  float2 *o = reinterpret_cast<float2 *>(dw_r + (size_t)e * d + i);
+  const float2 old = *o;
+  *o = make_float2(old.x + acc.x, old.y + acc.y);
 }
 
-// dx[t][i] = sum_j dX[slot_row[t,j]][i] + dX[shared row][i] + sum_j dl[t,j] W_r[e_j][i].
+// dx[t][i] = sum_j dX[slot_row[t,j]][i] + dX[shared row][i] + sum_j dl[t,j] W_r[e_j][i],
+// four consecutive columns per thread (16-byte rows of dX, d a multiple of 4).
 template <typename Tw>
 __global__ void __launch_bounds__(256) bw_dx_kernel(const float *__restrict__ dX,
                                                     const int *__restrict__ slot_row,
@@ -459,16 +502,36 @@ __global__ void __launch_bounds__(256) bw_dx_kernel(const float *__restrict__ dX
                                                     int Tk, int n_shared, int d, float *dx) {
   griddep_wait();
   griddep_launch_dependents();
-  const size_t total = (size_t)T * d;
+  const int d4 = d / 4;
+  const size_t total = (size_t)T * d4;
   for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
        id += (size_t)gridDim.x * blockDim.x) {
-    const int t = (int)(id / d), i = (int)(id % d);
-    float s = 0.f;
-    for (int j = 0; j < k; ++j) s += dX[(size_t)slot_row[t * k + j] * d + i];
-    if (n_shared) s += dX[(size_t)(Tk + t) * d + i];
-    for (int j = 0; j < k; ++j)
-      s = fmaf(dl[t * k + j], bw_f32(w_r[(size_t)topk_idx[t * k + j] * d + i]), s);
-    dx[id] = s;
+    const int t = (int)(id / d4), i = 4 * (int)(id % d4);
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(
+          dX + (size_t)slot_row[t * k + j] * d + i));
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    if (n_shared) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(dX + (size_t)(Tk + t) * d + i));
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    for (int j = 0; j < k; ++j) {
+      const float g = dl[t * k + j];
+      const float4 w = bw_load4(w_r + (size_t)topk_idx[t * k + j] * d + i);
+      s.x = fmaf(g, w.x, s.x);
+      s.y = fmaf(g, w.y, s.y);
+      s.z = fmaf(g, w.z, s.z);
+      s.w = fmaf(g, w.w, s.w);
+    }
+    *reinterpret_cast<float4 *>(dx + (size_t)t * d + i) = s;
   }
 }
 

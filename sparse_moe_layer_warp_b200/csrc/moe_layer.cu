@@ -1229,12 +1229,12 @@ moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   // 6. router and dx
   if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
                   (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
-      (s = launch(bw_router_dw_kernel<T_>, dim3(E, cdiv(d, 256)), dim3(256), 0, st, x,
+      (s = launch(bw_router_dw_kernel<T_>, dim3(E, cdiv(d, 512)), dim3(256), 0, st, x,
                   (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
                   dw_router)) != MOE_OK)
     return s;
-  return launch(bw_dx_kernel<T_>, dim3(grid_for((size_t)T * d, 256, L->num_sms)), dim3(256), 0,
-                st, (const float *)wide, (const int *)slot_row, (const int *)idx,
+  return launch(bw_dx_kernel<T_>, dim3(grid_for((size_t)T * d / 4, 256, L->num_sms)), dim3(256),
+                0, st, (const float *)wide, (const int *)slot_row, (const int *)idx,
                 (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
 }
 
@@ -1412,11 +1412,11 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   // router and dx
   if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
                   (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
-      (s = launch(bw_router_dw_kernel<__nv_bfloat16>, dim3(E, (d + 255) / 256), dim3(256), 0,
+      (s = launch(bw_router_dw_kernel<__nv_bfloat16>, dim3(E, (d + 511) / 512), dim3(256), 0,
                   st, x, (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
                   dw_router)) != MOE_OK)
     return s;
-  return launch(bw_dx_kernel<__nv_bfloat16>, dim3(grid_for((size_t)T * d, 256, L->num_sms)),
+  return launch(bw_dx_kernel<__nv_bfloat16>, dim3(grid_for((size_t)T * d / 4, 256, L->num_sms)),
                 dim3(256), 0, st, (const float *)wide, (const int *)slot_row, (const int *)idx,
                 (const float *)dl, wr, T, k, Tk, c.n_shared, d, dx);
 }
