@@ -518,6 +518,408 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// CTA-pair dgrad kernel for large groups: 256 weight rows x up to 256 tokens per unit on a
+// cluster of two CTAs (tcgen05 cta_group::2), the layout of grouped_gemm_pair.cuh with the
+// weight tile MN-major.  CTA r stages weight rows [128 r, 128 r + 128) of the unit (two
+// 64-wide MN-major boxes) and token rows [n0 + r*half, n0 + (r+1)*half) (half the token
+// tile, K-major), so each CTA loads half the token tile of the one-CTA kernel per MMA.
+constexpr int kBwPairEpiWarps = 8;
+constexpr int kBwPairThreads = 32 * (2 + kBwPairEpiWarps);
+
+struct BwDgradPairCfg {
+  static constexpr int BN = 256;
+  static constexpr int HALF_BN = BN / 2;
+  static constexpr int A_BYTES = 128 * kBK * 2;       // this CTA's 128 weight rows
+  static constexpr int B_BYTES = HALF_BN * kBK * 2;   // this CTA's token rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int STAGES_RAW = (160 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
+  static constexpr size_t smem_bytes(int n_groups) {
+    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
+           (size_t)(4 * n_groups + 1) * 4 + 2 * BN * 4 /*row scales*/ +
+           kBwPairEpiWarps * 16 * 32 * 4 /*store transposes*/ +
+           kBwPairEpiWarps * 16 * 33 * 4 /*dgate reductions*/ + 16;
+  }
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kBwPairThreads, 1)
+    bw_dgrad_pair_kernel(const __grid_constant__ BwDgradParams p) {
+  using C = BwDgradPairCfg;
+  constexpr int S = C::STAGES;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + S * C::A_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + S * C::B_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *tfull = bars + 2 * S;
+  uint64_t *tempty = bars + 2 * S + 2;
+  uint64_t *drain = bars + 2 * S + 4;
+  uint64_t *uq_full = bars + 2 * S + 5;
+  uint64_t *uq_empty = uq_full + kUnitQ;  // used in the leader only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
+  int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);        // [G + 1]
+  int *grp_count = unit_prefix + p.n_groups + 1;                     // [G]
+  int *grp_row = grp_count + p.n_groups;                             // [G] padded
+  int *grp_rowu = grp_row + p.n_groups;                              // [G] unpadded
+  float *row_scale = reinterpret_cast<float *>(
+      (reinterpret_cast<uintptr_t>(grp_rowu + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+  float *xbuf = row_scale + 2 * BN;             // [8 warps][16][32] store transposes
+  float *rbuf = xbuf + kBwPairEpiWarps * 16 * 32;  // [8 warps][16][33] dgate reductions
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int G = p.n_groups;
+  const int mtiles = p.M / 256;
+  const int kpp = p.K / kBK;
+  const int kblocks = p.n_pairs * kpp;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kBwPairEpiWarps);
+    }
+    mbar_init(drain, 1);
+    for (int q = 0; q < kUnitQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      mbar_init(&uq_empty[q], 2 + 2 * kBwPairEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int rowp, rowu, cnt;
+    p.rows.group(g, rowp, rowu, cnt);
+    grp_count[g] = cnt;
+    grp_row[g] = rowp;
+    grp_rowu[g] = rowu;
+    unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int lo = min(G, lane * per), hi = min(G, lo + per);
+    int run = 0;
+    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int g = lo; g < hi; ++g) {
+      const int u = unit_prefix[g];
+      unit_prefix[g] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = unit_prefix[G];
+
+  auto decode = [&](int u, int &g, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    g = lo;
+    const int nts = (grp_count[g] + BN - 1) / BN;
+    const int loc = u - unit_prefix[g];
+    mt = loc / nts;
+    nt = loc % nts;
+  };
+  // token split: CTA r holds tokens [n0 + r*half, n0 + (r+1)*half), N = 2*half
+  auto split = [&](int g, int nt) {
+    const int valid = min(BN, grp_count[g] - nt * BN);
+    return (((valid + 1) >> 1) + 7) & ~7;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      int u = -1;
+      while (ok) {
+        if (leader) {
+          const int c = atomicAdd(p.sched, 1);
+          const int uid = (c < total_units) ? c : -1;
+          if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 51)) {
+            ok = false;
+            break;
+          }
+          uq[qi] = uid;
+          st_shared_remote(mapa_shared(smem_u32((const void *)&uq[qi]), 1), uid);
+          mbar_arrive(&uq_full[qi]);
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_full[qi]), 1));
+          u = uid;
+        } else {
+          if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 52)) {
+            ok = false;
+            break;
+          }
+          u = uq[qi];
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_empty[qi]), 0));
+        }
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const int half = split(g, nt);
+        const int a_x = mt * 256 + (int)rank * 128;
+        const int b_row = grp_row[g] + nt * BN + (int)rank * half;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          const int pair = kb / kpp;
+          const int kc = (kb - pair * kpp) * kBK;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 53)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const CUtensorMap *amap = pair ? &p.tmA1 : &p.tmA0;
+          const CUtensorMap *bmap = pair ? &p.tmB1 : &p.tmB0;
+          uint8_t *a_dst = sA + stage * C::A_BYTES;
+          const int a_row = g * p.K + kc;
+          tma_load_2d_pair(a_dst, amap, fbar, a_x, a_row, pol_w);
+          tma_load_2d_pair(a_dst + C::A_BYTES / 2, amap, fbar, a_x + 64, a_row, pol_w);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, bmap, fbar, kc, b_row, pol_b);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      while (ok) {
+        if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, p.status, 54)) break;
+        const int u = uq[qi];
+        mbar_arrive(&uq_empty[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        ++it;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 55)) break;
+        tc_fence_after();
+        int g, mt, nt;
+        decode(u, g, mt, nt);
+        const uint32_t idesc = idesc_bf16_f32_major(256, 2 * split(g, nt), true, false);
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, 56)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            tc_mma_bf16_pair(d0, sdesc_mn_sw128(a + kk * 16 * 128, C::A_BYTES / 2),
+                             sdesc_k_sw128(b + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+          tc_commit_pair_both(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair_both(&tfull[acc]);
+      }
+      tc_commit_pair_local(drain);
+      volatile int no_abort = 0;
+      mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int eh = (warp - 2) >> 2;  // chunks 2i + eh of the quadrant's token columns
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t uq_empty_leader = mapa_shared(smem_u32(&uq_empty[0]), 0);
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where, bool cluster) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = (cluster ? mbar_wait_bounded<true>(bar, parity, abort_flag, p.status, where)
+                      : mbar_wait_bounded(bar, parity, abort_flag, p.status, where))
+                 ? 1
+                 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      return ok != 0;
+    };
+    float *wbuf = xbuf + (warp - 2) * 16 * 32;
+    float *red = rbuf + (warp - 2) * 16 * 33;
+    int it = 0;
+    int qi = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!warp_wait(&uq_full[qi], qph, 57, true)) break;
+      const int u = uq[qi];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&uq_empty[qi]);
+        else mbar_arrive_remote(uq_empty_leader + qi * 8);
+      }
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (u < 0) break;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      ++it;
+      if (!warp_wait(&tfull[acc], acc_phase, 58, false)) break;
+      tc_fence_after();
+      int g, mt, nt;
+      decode(u, g, mt, nt);
+      const int valid = min(BN, grp_count[g] - nt * BN);
+      const int row0 = grp_row[g] + nt * BN;    // padded
+      const int rowu0 = grp_rowu[g] + nt * BN;  // unpadded
+      const int col_base = mt * 256 + (int)rank * 128 + q * 32;
+      const int col = col_base + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      if (MODE == BW_DH) {
+        for (int n = threadIdx.x - 64; n < BN; n += 32 * kBwPairEpiWarps)
+          row_scale[acc * BN + n] = (n < valid) ? p.row_scale[rowu0 + n] : 0.f;
+        named_bar_sync(1, 32 * kBwPairEpiWarps);
+      }
+      uint32_t nx[16];
+      const int c_first = 16 * eh;
+      if (c_first < valid) tmem_ld16(taddr + c_first, nx);
+      for (int c0 = c_first; c0 < valid; c0 += 32) {
+        uint32_t v[16];
+        tmem_ld_wait_regs(nx);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) v[n] = nx[n];
+        if (c0 + 32 < valid) tmem_ld16(taddr + c0 + 32, nx);
+        float vals[16];
+        if (MODE == BW_DX) {
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v[n]);
+          store_block16_f32(p.out, p.M, rowu0, c0, valid, col_base, vals, wbuf, lane);
+        } else {
+          float av[16], bv[16];
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            const bool in = c0 + n < valid;
+            const size_t i = (size_t)(row0 + c0 + n) * p.M + col;
+            av[n] = in ? p.pre_a[i] : 0.f;
+            bv[n] = in ? p.pre_b[i] : 0.f;
+          }
+          float dav[16], dbv[16], hsv[16];
+          const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
+#pragma unroll
+          for (int n4 = 0; n4 < 4; ++n4) {
+            const float4 s4 = sc[n4];
+            const float ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int n = 4 * n4 + e;
+              const float a = av[n], b = bv[n], s = ss[e];
+              const float dhu = __uint_as_float(v[n]);
+              const float sig = __fdividef(1.f, 1.f + __expf(-a));
+              const float silu = a * sig;
+              const float h = silu * b;
+              const float dh = s * dhu;
+              vals[n] = dhu * h;
+              dav[n] = dh * b * sig * (1.f + a * (1.f - sig));
+              dbv[n] = dh * silu;
+              hsv[n] = s * h;
+            }
+          }
+          store_block16_bf16(p.da, p.M, row0, c0, valid, col_base, dav, wbuf, lane);
+          store_block16_bf16(p.db, p.M, row0, c0, valid, col_base, dbv, wbuf, lane);
+          store_block16_bf16(p.hs, p.M, row0, c0, valid, col_base, hsv, wbuf, lane);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) red[n * 33 + lane] = vals[n];
+          __syncwarp();
+          if (lane < 16 && c0 + lane < valid && g < p.rows.E) {
+            float sum = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) sum += red[lane * 33 + i];
+            p.dgate_part[(size_t)(rowu0 + c0 + lane) * p.n_part + col_base / 32] = sum;
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_leader + acc * 8);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------------- wgrad GEMMs
 constexpr int kWgOps = 5;    // sorted operands: dout, s*h, da, db, x
 constexpr int kWgProbs = 3;  // dW_down, dW_gate, dW_up

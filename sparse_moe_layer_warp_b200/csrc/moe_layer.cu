@@ -43,6 +43,7 @@ struct moe_layer {
   // as [G*f, d], W_down as [G*d, f]
   CUtensorMap tm_wg_mn, tm_wu_mn, tm_wd_mn;
   int wg_pair_grid;  // CTAs of the CTA-pair weight-gradient kernel (0: not available)
+  int bw_pair_grid;  // CTAs of the CTA-pair dgrad kernels (0: not available)
 };
 
 namespace {
@@ -386,6 +387,33 @@ int wgrad_pair_grid_size(const moe_layer *L) {
   return 2 * n;
 }
 
+// CTAs of the persistent CTA-pair dgrad kernels (both modes share the configuration).
+int dgrad_pair_grid_size(const moe_layer *L) {
+  const size_t smem = BwDgradPairCfg::smem_bytes(L->cfg.n_experts + L->cfg.n_shared);
+  if (smem > (size_t)L->smem_optin) return 0;
+  int n[2] = {0, 0};
+  void (*kern[2])(BwDgradParams) = {bw_dgrad_pair_kernel<BW_DH>, bw_dgrad_pair_kernel<BW_DX>};
+  for (int i = 0; i < 2; ++i) {
+    if (cudaFuncSetAttribute(kern[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return 0;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(L->num_sms & ~1);
+    cfg.blockDim = dim3(kBwPairThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n[i], kern[i], &cfg) != cudaSuccess) return 0;
+  }
+  return 2 * (n[0] < n[1] ? n[0] : n[1]);
+}
+
 template <int MODE>
 moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_t st) {
   const size_t smem = pair_smem<MODE>(L->cfg);
@@ -590,6 +618,7 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
     L->wg_pair_grid = wgrad_pair_grid_size(L);
+    L->bw_pair_grid = dgrad_pair_grid_size(L);
     cudaGetLastError();  // an unavailable cluster query only disables the pair path
     const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
@@ -1274,6 +1303,17 @@ moe_status launch_bw_wgrad(const moe_layer *L, const BwWgradParams &p, cudaStrea
   return launch(bw_wgrad_kernel<BNW>, dim3(L->num_sms), dim3(kGemmThreads), smem, st, p);
 }
 
+template <int MODE>
+moe_status launch_bw_dgrad_pair(const moe_layer *L, const BwDgradParams &p, cudaStream_t st) {
+  const size_t smem = BwDgradPairCfg::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bw_dgrad_pair_kernel<MODE>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_cl(bw_dgrad_pair_kernel<MODE>, dim3(L->bw_pair_grid), dim3(kBwPairThreads), smem,
+                   st, 2, p);
+}
+
 // Mean routed rows per expert from which the weight gradients run on CTA pairs.
 constexpr double kWgradPairMinRows = 16.0;
 
@@ -1333,8 +1373,9 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   GemmParams pu;
   if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, &up_rows)) != MOE_OK)
     return s;
-  // DH
-  const int bn = pick_bn(c, T, MODE_DOWN);
+  // DH (CTA pairs for groups as large as the forward's pair threshold)
+  const bool pair_dg = plan.pair && d % 256 == 0 && f % 256 == 0 && L->bw_pair_grid >= 2;
+  const int bn = pair_dg ? BwDgradPairCfg::HALF_BN : pick_bn(c, T, MODE_DOWN);
   BwDgradParams pd;
   memset(&pd, 0, sizeof pd);
   pd.tmA0 = L->tm_wd_mn;
@@ -1354,7 +1395,8 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   pd.n_pairs = 1;
   pd.n_part = f / 32;
   pd.sched = &status->sched[1];
-  if ((s = launch_bw_dgrad<BW_DH>(L, bn, pd, st)) != MOE_OK ||
+  if ((s = pair_dg ? launch_bw_dgrad_pair<BW_DH>(L, pd, st)
+                   : launch_bw_dgrad<BW_DH>(L, bn, pd, st)) != MOE_OK ||
       (s = launch(bw_dgate_reduce_kernel, dim3(grid_for(Tk, 256, L->num_sms)), dim3(256), 0, st,
                   (const float *)dgate_part, f / 32, (const int *)perm, Tk, c.routed_scale,
                   dgate)) != MOE_OK)
@@ -1371,7 +1413,9 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   px.K = f;
   px.n_pairs = 2;
   px.sched = &status->sched[2];
-  if ((s = launch_bw_dgrad<BW_DX>(L, bn, px, st)) != MOE_OK) return s;
+  if ((s = pair_dg ? launch_bw_dgrad_pair<BW_DX>(L, px, st)
+                   : launch_bw_dgrad<BW_DX>(L, bn, px, st)) != MOE_OK)
+    return s;
   // weight gradients: dW_down += dout^T (s h), dW_gate += da^T x, dW_up += db^T x
   BwWgradParams pw;
   memset(&pw, 0, sizeof pw);

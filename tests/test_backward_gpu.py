@@ -22,6 +22,9 @@ CASES = [
      "routed_scale": 0.5},                                                       # ragged 16-row pads
     {"dtype": "bf16", "T": 200, "d": 256, "E": 16, "k": 4, "f": 256, "seed": 8,   # pair wgrad,
      "bias": "zipf"},                                                               # skewed groups
+    {"dtype": "bf16", "T": 256, "d": 256, "E": 8, "k": 4, "f": 256, "seed": 9},   # pair dgrad
+    {"dtype": "bf16", "T": 300, "d": 256, "E": 8, "k": 4, "f": 512, "seed": 10,   # pair dgrad,
+     "bias": "zipf", "routed_scale": 1.5},                                          # skewed
     {"dtype": "f32"},
 ]
 
