@@ -164,8 +164,13 @@ moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stre
  * The weight gradients ACCUMULATE (+=) into the caller's buffers, as over micro-batches;
  * rows of experts no token chose are not touched (zero the buffers before the first call).
  * ws: at least moe_backward_workspace_size(h, n_tokens) bytes, 256-byte aligned (it holds a
- * forward workspace at its start, which this call reuses).  fp32 accumulation on CUDA cores
- * in a fixed order: deterministic.  Errors as moe_forward. */
+ * forward workspace at its start, which this call reuses).
+ * bf16 layer: the matrix products run on the tensor cores with fp32 accumulation; da, db and
+ * routed_scale * gate * h enter the second-stage products rounded to bf16 (each weight
+ * gradient and dx term has one rounded operand), dgate and the router terms are computed
+ * from fp32 values.  fp32 layer: fp32 throughout on CUDA cores.  Every sum runs in a fixed
+ * order and each weight-gradient element receives one addition per call: deterministic.
+ * Errors as moe_forward. */
 size_t moe_backward_workspace_size(moe_handle h, int n_tokens);
 moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *dout, float *dx,
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
