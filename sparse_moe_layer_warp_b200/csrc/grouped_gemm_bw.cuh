@@ -927,7 +927,6 @@ constexpr int kWgProbs = 3;  // dW_down, dW_gate, dW_up
 struct BwWgradParams {
   CUtensorMap box[kWgOps];   // padded sorted rows [R, width] bf16, box {64, 64}
   CUtensorMap out[kWgProbs]; // dW as [G * M, N] fp32, box {32, 32}, 128-byte swizzle
-  float *dw[kWgProbs];       // the same gradients as plain pointers
   int a_op[kWgProbs], b_op[kWgProbs];  // operand of the M side and of the N side
   int M[kWgProbs], N[kWgProbs];        // dW[g] is [M, N]; M, N multiples of the unit tile
   int n_prob;
@@ -1580,6 +1579,409 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
 
   // the pair leaves together: the leader's MMAs read the peer's shared memory, and the
   // peer's TMA loads signal the leader's barriers
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ dx rows + weight gradients
+// One persistent CTA-pair kernel for the two steps that follow DH: the dgrad units of DX
+// (256 d rows x up to 256 tokens, K = 2 f, bound by moving weight and activation tiles into
+// the SMs) and the weight-gradient units (256 x 256 tiles of dW, K = the group's rows, bound
+// by the fp32 gradient read-modify-write in HBM).  Units are listed group by group, each
+// group's DX units first, so the pairs claiming consecutive units run both kinds at once and
+// the two bottlenecks overlap.  Stage layout (32 KB per CTA: a 128-row MN-major A tile and a
+// 128-row B tile), barriers and unit publication are those of the two pair kernels above.
+struct BwTailParams {
+  BwDgradParams dx;  // DX: tmA0/tmA1 = W_gate/W_up (MN-major), tmB0/tmB1 = da/db (box {64, 128})
+  BwWgradParams wg;  // weight gradients (256 x 256 tiles)
+};
+
+struct BwTailPairCfg {
+  static constexpr int BOX_BYTES = 64 * kBK * 2;  // 8 KB
+  static constexpr int A_BYTES = 2 * BOX_BYTES;   // this CTA's 128 M rows x 64 K
+  static constexpr int B_BYTES = 2 * BOX_BYTES;   // 128 N columns (wgrad) / tokens (dx) x 64 K
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int STG_BUFS = 2;
+  static constexpr int STG_TOTAL = kWgPairEpiWarps * STG_BUFS * kWgStgBytes;
+  static constexpr int XBUF_BYTES = kWgPairEpiWarps * 16 * 32 * 4;
+  static constexpr int STAGES_RAW = (212 * 1024 - STG_TOTAL - XBUF_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "pipeline too shallow");
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
+  static constexpr size_t smem_bytes(int n_groups) {
+    return 1024 + (size_t)STAGES * STAGE_BYTES + STG_TOTAL + XBUF_BYTES + BAR_BYTES + 64 +
+           (size_t)(4 * n_groups + 1) * 4 + 16;
+  }
+};
+
+__global__ void __launch_bounds__(kWgPairThreads, 1)
+    bw_tail_pair_kernel(const __grid_constant__ BwTailParams P) {
+  using C = BwTailPairCfg;
+  constexpr int S = C::STAGES;
+  const BwDgradParams &px = P.dx;
+  const BwWgradParams &pw = P.wg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + S * C::A_BYTES;
+  uint8_t *stg = sB + S * C::B_BYTES;  // 1024-byte aligned
+  float *xbuf = reinterpret_cast<float *>(stg + C::STG_TOTAL);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(stg + C::STG_TOTAL + C::XBUF_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *tfull = bars + 2 * S;
+  uint64_t *tempty = bars + 2 * S + 2;
+  uint64_t *drain = bars + 2 * S + 4;
+  uint64_t *uq_full = bars + 2 * S + 5;
+  uint64_t *uq_empty = uq_full + kUnitQ;  // used in the leader only
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
+  const int G = pw.n_groups;
+  int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
+  int *grp_count = unit_prefix + G + 1;                         // [G]
+  int *grp_row = grp_count + G;                                 // [G] padded
+  int *grp_rowu = grp_row + G;                                  // [G] unpadded
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int dx_mtiles = px.M / 256;
+  const int dx_kpp = px.K / kBK;
+  const int dx_kblocks = 2 * dx_kpp;
+  int wg_units_per_group = 0;  // the same for every group with rows
+  for (int pr = 0; pr < pw.n_prob; ++pr) wg_units_per_group += (pw.M[pr] / 256) * (pw.N[pr] / 256);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kWgPairEpiWarps);
+    }
+    mbar_init(drain, 1);
+    for (int q = 0; q < kUnitQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      mbar_init(&uq_empty[q], 2 + 2 * kWgPairEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int rowp, rowu, cnt;
+    pw.rows.group(g, rowp, rowu, cnt);
+    grp_count[g] = cnt;
+    grp_row[g] = rowp;
+    grp_rowu[g] = rowu;
+    unit_prefix[g] = cnt > 0 ? dx_mtiles * ((cnt + 255) / 256) + wg_units_per_group : 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int lo = min(G, lane * per), hi = min(G, lo + per);
+    int run = 0;
+    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int g = lo; g < hi; ++g) {
+      const int u = unit_prefix[g];
+      unit_prefix[g] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = unit_prefix[G];
+
+  // unit -> group and kind: dx (pr = -1; mt, nt over d rows / tokens) or weight gradient
+  // (problem pr; mt, nt over the 256 x 256 tiles of dW, n innermost)
+  auto decode = [&](int u, int &g, int &pr, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    g = lo;
+    int loc = u - unit_prefix[g];
+    const int nts = (grp_count[g] + 255) / 256;
+    if (loc < dx_mtiles * nts) {
+      pr = -1;
+      mt = loc / nts;
+      nt = loc % nts;
+      return;
+    }
+    loc -= dx_mtiles * nts;
+    for (pr = 0; pr < pw.n_prob; ++pr) {
+      const int n_here = (pw.M[pr] / 256) * (pw.N[pr] / 256);
+      if (loc < n_here) break;
+      loc -= n_here;
+    }
+    const int ntw = pw.N[pr] / 256;
+    mt = loc / ntw;
+    nt = loc % ntw;
+  };
+  // dx token split: CTA r holds tokens [n0 + r*half, n0 + (r+1)*half), N = 2*half
+  auto split = [&](int g, int nt) {
+    const int valid = min(256, grp_count[g] - nt * 256);
+    return (((valid + 1) >> 1) + 7) & ~7;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      int u = -1;
+      while (ok) {
+        if (leader) {
+          const int c = atomicAdd(pw.sched, 1);
+          const int uid = (c < total_units) ? c : -1;
+          if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, pw.status, 61)) {
+            ok = false;
+            break;
+          }
+          uq[qi] = uid;
+          st_shared_remote(mapa_shared(smem_u32((const void *)&uq[qi]), 1), uid);
+          mbar_arrive(&uq_full[qi]);
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_full[qi]), 1));
+          u = uid;
+        } else {
+          if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, pw.status, 62)) {
+            ok = false;
+            break;
+          }
+          u = uq[qi];
+          mbar_arrive_remote(mapa_shared(smem_u32(&uq_empty[qi]), 0));
+        }
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        int g, pr, mt, nt;
+        decode(u, g, pr, mt, nt);
+        const int kbs = (pr < 0) ? dx_kblocks : (grp_count[g] + kBK - 1) / kBK;
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, pw.status, 63)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          uint8_t *a_dst = sA + stage * C::A_BYTES;
+          uint8_t *b_dst = sB + stage * C::B_BYTES;
+          if (pr < 0) {
+            const int pair = kb / dx_kpp;
+            const int kc = (kb - pair * dx_kpp) * kBK;
+            const CUtensorMap *amap = pair ? &px.tmA1 : &px.tmA0;
+            const CUtensorMap *bmap = pair ? &px.tmB1 : &px.tmB0;
+            const int a_x = mt * 256 + (int)rank * 128;
+            const int a_row = g * px.K + kc;
+            tma_load_2d_pair(a_dst, amap, fbar, a_x, a_row, pol_w);
+            tma_load_2d_pair(a_dst + C::BOX_BYTES, amap, fbar, a_x + 64, a_row, pol_w);
+            tma_load_2d_pair(b_dst, bmap, fbar, kc,
+                             grp_row[g] + nt * 256 + (int)rank * split(g, nt), pol_b);
+          } else {
+            const CUtensorMap *abox = &pw.box[pw.a_op[pr]], *bbox = &pw.box[pw.b_op[pr]];
+            const int ma = mt * 256 + (int)rank * 128, nb = nt * 256 + (int)rank * 128;
+            const int r0 = grp_row[g] + kb * kBK;
+            tma_load_2d_pair(a_dst, abox, fbar, ma, r0, pol_b);
+            tma_load_2d_pair(a_dst + C::BOX_BYTES, abox, fbar, ma + 64, r0, pol_b);
+            tma_load_2d_pair(b_dst, bbox, fbar, nb, r0, pol_b);
+            tma_load_2d_pair(b_dst + C::BOX_BYTES, bbox, fbar, nb + 64, r0, pol_b);
+          }
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {
+        int n = issued < S ? issued : S;
+        int st = stage, ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            ph ^= 1;
+          }
+          volatile int no_abort = 0;
+          mbar_wait_bounded(&full[st], ph, &no_abort, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      int qi = 0;
+      uint32_t qph = 0;
+      while (ok) {
+        if (!mbar_wait_bounded<true>(&uq_full[qi], qph, abort_flag, pw.status, 64)) break;
+        const int u = uq[qi];
+        mbar_arrive(&uq_empty[qi]);
+        if (++qi == kUnitQ) {
+          qi = 0;
+          qph ^= 1;
+        }
+        if (u < 0) break;
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        ++it;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, pw.status, 65)) break;
+        tc_fence_after();
+        int g, pr, mt, nt;
+        decode(u, g, pr, mt, nt);
+        const int cnt = grp_count[g];
+        const int kbs = (pr < 0) ? dx_kblocks : (cnt + kBK - 1) / kBK;
+        const uint32_t idesc = (pr < 0)
+                                   ? idesc_bf16_f32_major(256, 2 * split(g, nt), true, false)
+                                   : idesc_bf16_f32_major(256, 256, true, true);
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, pw.status, 66)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+          if (pr < 0) {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              tc_mma_bf16_pair(d0, sdesc_mn_sw128(a + kk * 16 * 128, C::BOX_BYTES),
+                               sdesc_k_sw128(b + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+          } else {
+            const int k16 = (min(kBK, cnt - kb * kBK) + 15) >> 4;
+            for (int kk = 0; kk < k16; ++kk)
+              tc_mma_bf16_pair(d0, sdesc_mn_sw128(a + kk * 16 * 128, C::BOX_BYTES),
+                               sdesc_mn_sw128(b + kk * 16 * 128, C::BOX_BYTES), idesc,
+                               (kb | kk) ? 1u : 0u);
+          }
+          tc_commit_pair_both(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair_both(&tfull[acc]);
+      }
+      tc_commit_pair_local(drain);
+      volatile int no_abort = 0;
+      mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int eh = (warp - 2) >> 2;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t uq_empty_leader = mapa_shared(smem_u32(&uq_empty[0]), 0);
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int where, bool cluster) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = (cluster ? mbar_wait_bounded<true>(bar, parity, abort_flag, pw.status, where)
+                      : mbar_wait_bounded(bar, parity, abort_flag, pw.status, where))
+                 ? 1
+                 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      return ok != 0;
+    };
+    uint8_t *my_stg = stg + (warp - 2) * C::STG_BUFS * kWgStgBytes;
+    float *wbuf = xbuf + (warp - 2) * 16 * 32;
+    int it = 0, n_red = 0;
+    int qi = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!warp_wait(&uq_full[qi], qph, 67, true)) break;
+      const int u = uq[qi];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&uq_empty[qi]);
+        else mbar_arrive_remote(uq_empty_leader + qi * 8);
+      }
+      if (++qi == kUnitQ) {
+        qi = 0;
+        qph ^= 1;
+      }
+      if (u < 0) break;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      ++it;
+      if (!warp_wait(&tfull[acc], acc_phase, 68, false)) break;
+      tc_fence_after();
+      int g, pr, mt, nt;
+      decode(u, g, pr, mt, nt);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      if (pr < 0) {
+        // rows of dx: fp32, tokens of this unit at unpadded rows
+        const int valid = min(256, grp_count[g] - nt * 256);
+        const int rowu0 = grp_rowu[g] + nt * 256;
+        const int col_base = mt * 256 + (int)rank * 128 + q * 32;
+        uint32_t nx[16];
+        const int c_first = 16 * eh;
+        if (c_first < valid) tmem_ld16(taddr + c_first, nx);
+        for (int c0 = c_first; c0 < valid; c0 += 32) {
+          uint32_t v[16];
+          tmem_ld_wait_regs(nx);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) v[n] = nx[n];
+          if (c0 + 32 < valid) tmem_ld16(taddr + c0 + 32, nx);
+          float vals[16];
+#pragma unroll
+          for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v[n]);
+          store_block16_f32(px.out, px.M, rowu0, c0, valid, col_base, vals, wbuf, lane);
+        }
+      } else {
+        wgrad_epilogue<C::STG_BUFS>(taddr, eh, 2, 256, &pw.out[pr], nt * 256,
+                                    g * pw.M[pr] + mt * 256 + (int)rank * 128 + q * 32, my_stg,
+                                    n_red, lane);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_leader + acc * 8);
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
   tc_fence_before();
   __syncthreads();
   cluster_sync();

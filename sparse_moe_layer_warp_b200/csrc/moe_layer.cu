@@ -44,6 +44,7 @@ struct moe_layer {
   CUtensorMap tm_wg_mn, tm_wu_mn, tm_wd_mn;
   int wg_pair_grid;  // CTAs of the CTA-pair weight-gradient kernel (0: not available)
   int bw_pair_grid;  // CTAs of the CTA-pair dgrad kernels (0: not available)
+  int tail_pair_grid;  // CTAs of the CTA-pair dx + weight-gradient kernel (0: not available)
 };
 
 namespace {
@@ -387,6 +388,30 @@ int wgrad_pair_grid_size(const moe_layer *L) {
   return 2 * n;
 }
 
+// CTAs of a persistent cluster-of-two kernel: two per cluster that can be resident at once.
+template <typename KP>
+int cluster_grid_size(void (*kern)(KP), size_t smem, int threads, const moe_layer *L) {
+  if (smem > (size_t)L->smem_optin) return 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(L->num_sms & ~1);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return 0;
+  return 2 * n;
+}
+
 // CTAs of the persistent CTA-pair dgrad kernels (both modes share the configuration).
 int dgrad_pair_grid_size(const moe_layer *L) {
   const size_t smem = BwDgradPairCfg::smem_bytes(L->cfg.n_experts + L->cfg.n_shared);
@@ -619,6 +644,9 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
     L->wg_pair_grid = wgrad_pair_grid_size(L);
     L->bw_pair_grid = dgrad_pair_grid_size(L);
+    L->tail_pair_grid = cluster_grid_size(bw_tail_pair_kernel,
+                                          BwTailPairCfg::smem_bytes(c.n_experts + c.n_shared),
+                                          kWgPairThreads, L);
     cudaGetLastError();  // an unavailable cluster query only disables the pair path
     const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
@@ -1314,6 +1342,16 @@ moe_status launch_bw_dgrad_pair(const moe_layer *L, const BwDgradParams &p, cuda
                    st, 2, p);
 }
 
+moe_status launch_bw_tail_pair(const moe_layer *L, const BwTailParams &p, cudaStream_t st) {
+  const size_t smem = BwTailPairCfg::smem_bytes(p.wg.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bw_tail_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_cl(bw_tail_pair_kernel, dim3(L->tail_pair_grid), dim3(kWgPairThreads), smem, st,
+                   2, p);
+}
+
 // Mean routed rows per expert from which the weight gradients run on CTA pairs.
 constexpr double kWgradPairMinRows = 16.0;
 
@@ -1413,9 +1451,6 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   px.K = f;
   px.n_pairs = 2;
   px.sched = &status->sched[2];
-  if ((s = pair_dg ? launch_bw_dgrad_pair<BW_DX>(L, px, st)
-                   : launch_bw_dgrad<BW_DX>(L, bn, px, st)) != MOE_OK)
-    return s;
   // weight gradients: dW_down += dout^T (s h), dW_gate += da^T x, dW_up += db^T x
   BwWgradParams pw;
   memset(&pw, 0, sizeof pw);
@@ -1427,9 +1462,6 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
       !encode_f32_2d(&pw.out[1], dw_gate, d, (uint64_t)G * f) ||
       !encode_f32_2d(&pw.out[2], dw_up, d, (uint64_t)G * f))
     return MOE_ERR_CUDA;
-  pw.dw[0] = dw_down;
-  pw.dw[1] = dw_gate;
-  pw.dw[2] = dw_up;
   const int a_op[kWgProbs] = {0, 2, 3}, b_op[kWgProbs] = {1, 4, 4};
   const int Ms[kWgProbs] = {d, f, f}, Ns[kWgProbs] = {f, d, d};
   for (int i = 0; i < kWgProbs; ++i) {
@@ -1447,11 +1479,21 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   // traffic to matter; decode-sized groups (a row or two each) are bound by the gradient
   // read-modify-write, where the one-CTA kernel's shorter per-unit path is faster
   const bool pair_wg = (double)T * k / E >= kWgradPairMinRows;
-  if (pair_wg && d % 256 == 0 && f % 256 == 0 && L->wg_pair_grid >= 2)
-    s = launch_bw_wgrad_pair(L, pw, st);
-  else
-    s = (d % 256 == 0 && f % 256 == 0) ? launch_bw_wgrad<256>(L, pw, st)
-                                       : launch_bw_wgrad<128>(L, pw, st);
+  if (pair_dg && pair_wg && L->tail_pair_grid >= 2) {
+    // dx rows and weight gradients in one launch, their units interleaved
+    BwTailParams pt;
+    pt.dx = px;
+    pt.wg = pw;
+    s = launch_bw_tail_pair(L, pt, st);
+  } else {
+    s = pair_dg ? launch_bw_dgrad_pair<BW_DX>(L, px, st) : launch_bw_dgrad<BW_DX>(L, bn, px, st);
+    if (s != MOE_OK) return s;
+    if (pair_wg && d % 256 == 0 && f % 256 == 0 && L->wg_pair_grid >= 2)
+      s = launch_bw_wgrad_pair(L, pw, st);
+    else
+      s = (d % 256 == 0 && f % 256 == 0) ? launch_bw_wgrad<256>(L, pw, st)
+                                         : launch_bw_wgrad<128>(L, pw, st);
+  }
   if (s != MOE_OK) return s;
   // router and dx
   if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
