@@ -107,3 +107,80 @@ def test_no_writes_outside_buffers(cuda_ok, kw):
     assert _margins_intact(ws_big, need, 0xA5)
     assert int(v["offsets"][E]) == T * k
     assert layer.device_status() == 0
+
+
+@pytest.mark.parametrize("kw", [
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 256},     # decode routing, 1-CTA
+    {"dtype": "bf16", "T": 200, "d": 256, "E": 16, "k": 4, "f": 256,     # pair weight gradients
+     "bias": "zipf"},
+    {"dtype": "bf16", "T": 300, "d": 256, "E": 8, "k": 4, "f": 512},     # pair dgrad + fused tail
+    {"dtype": "f32", "T": 40},
+])
+def test_backward_no_writes_outside_buffers(cuda_ok, kw):
+    """moe_backward writes only inside dx, the four gradient buffers and its workspace; the
+    gradient rows of experts no token chose keep their previous contents."""
+    from sparse_moe_layer_warp_b200 import moe_backward, moe_backward_workspace_size
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    dout = synth.make_x(w, w.T, device="cuda", seed=5)
+    ref = layer.backward(inp.x, dout)
+    counts = layer.route(x=inp.x)["counts"]
+    torch.cuda.synchronize()
+    T, d, E, f = w.T, w.d, w.E, w.f
+    G = E + w.n_shared
+    need = moe_backward_workspace_size(layer.handle, T)
+    ws_big, ws = _guarded(need, torch.uint8, 0xA5)
+    moe_workspace_init(layer.handle, ws)
+    sizes = {"dx": T * d, "dw_router": E * d, "dw_gate": G * f * d, "dw_up": G * f * d,
+             "dw_down": G * d * f}
+    fill = 0x3F800000  # 1.0f: the gradients accumulate onto ones
+    bufs = {n: _guarded(m, torch.int32, fill) for n, m in sizes.items()}
+    v = {n: b[1].view(torch.float32) for n, b in bufs.items()}
+    moe_backward(layer.handle, inp.x, T, dout, v["dx"], v["dw_router"], v["dw_gate"], v["dw_up"],
+                 v["dw_down"], ws)
+    torch.cuda.synchronize()
+    assert _margins_intact(ws_big, need, 0xA5)
+    for n, m in sizes.items():
+        assert _margins_intact(bufs[n][0], m, fill), n
+    # dx is overwritten; the weight gradients are added to the ones
+    assert torch.equal(v["dx"].view(T, d), ref["dx"])
+    unchosen = torch.nonzero(counts == 0).flatten()
+    for n in ("dw_router", "dw_gate", "dw_up", "dw_down"):
+        got = v[n].view(ref[n].shape)
+        # one fp32 addition onto 1.0: |(1 + r) - 1 - r| <= 2^-24 (1 + |r|)
+        tol = 1.2e-7 * (1.0 + ref[n].abs().max().item())
+        assert torch.allclose(got - 1.0, ref[n], rtol=0, atol=tol), n
+        if len(unchosen):
+            assert (got[unchosen] == 1.0).all(), n
+
+
+def test_backward_rejects_bad_arguments(cuda_ok):
+    from sparse_moe_layer_warp_b200 import moe_backward, moe_backward_workspace_size
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=16, d=256, E=16, k=2, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    T, d, E, f, G = w.T, w.d, w.E, w.f, w.E + 1
+    ws = torch.zeros(moe_backward_workspace_size(layer.handle, T), dtype=torch.uint8,
+                     device="cuda")
+    moe_workspace_init(layer.handle, ws)
+    dout = synth.make_x(w, T, device="cuda", seed=6)
+    g = {"dx": torch.zeros(T, d, device="cuda"), "dwr": torch.zeros(E, d, device="cuda"),
+         "dwg": torch.zeros(G, f, d, device="cuda"), "dwu": torch.zeros(G, f, d, device="cuda"),
+         "dwd": torch.zeros(G, d, f, device="cuda")}
+
+    def call(x=inp.x, n=T, dx=g["dx"], wsb=ws):
+        moe_backward(layer.handle, x, n, dout, dx, g["dwr"], g["dwg"], g["dwu"], g["dwd"], wsb)
+
+    with pytest.raises(MoEError):
+        call(n=T + 1)                               # more tokens than max_tokens
+    with pytest.raises(MoEError):
+        call(wsb=ws[:-256])                          # workspace too small
+    with pytest.raises(MoEError):
+        call(wsb=ws[16:])                            # workspace not 256-byte aligned
+    dx_big = torch.zeros(T * d + 4, device="cuda")
+    with pytest.raises(MoEError):
+        call(dx=dx_big[1:1 + T * d].view(T, d))      # dx not 16-byte aligned
+    call()                                          # the valid call still works
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
