@@ -461,11 +461,17 @@ def run_backward(args, rank, world, local_rank):
     touched = []
     for i in range(args.warmup, nb):
         touched.append(int((layer.route(x=xs[i])["counts"] > 0).sum().item()) + w.n_shared)
+    # --saved: each step's pre-activations kept by a training forward (moe_forward_save) of
+    # its x, run before the timed region; the timed call then skips their recompute
+    saved = [None] * nb
+    if args.saved:
+        for i in range(nb):
+            saved[i] = layer.forward_save(xs[i])[1]
     # weight-gradient buffers allocated once; every step accumulates into them
-    grads = layer.backward(xs[0], douts[0])
+    grads = layer.backward(xs[0], douts[0], saved=saved[0])
     for i in range(args.warmup):
         flush.zero_()
-        layer.backward(xs[i], douts[i], grads=grads)
+        layer.backward(xs[i], douts[i], grads=grads, saved=saved[i])
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -480,7 +486,8 @@ def run_backward(args, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(st)
-        layer.backward(xs[args.warmup + i], douts[args.warmup + i], grads=grads)
+        layer.backward(xs[args.warmup + i], douts[args.warmup + i], grads=grads,
+                       saved=saved[args.warmup + i])
         ev[i][1].record(st)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -502,10 +509,17 @@ def run_backward(args, rank, world, local_rank):
         # gradients and the router's read and written (they accumulate).
         flops = 16.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
         nbytes = tm * 5 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+        label = "tcgen05 grouped GEMMs"
+        if args.saved:
+            # a and b kept by the training forward: no recompute (12 P f d flops, weights read
+            # three times), the kept fp32 a, b read once
+            flops = 12.0 * P * w.f * w.d + 4.0 * T * w.k * w.d
+            nbytes = (tm * 3 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
+                      + 8.0 * P * w.f)
+            label += ", pre-activations kept by the training forward"
         peak_c = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         peak_name = f"bf16 dense, sustained ({src})"
         unit_c, kind = "TFLOP/s", "tensor"
-        label = "tcgen05 grouped GEMMs"
     else:
         # CUDA cores: recompute a and b, unscaled outputs, dh, rows of dx (two products),
         # three weight gradients: 18 P f d flops; weights read six times
@@ -557,6 +571,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--saved", action="store_true",
+                    help="with --pass backward: time moe_backward_saved on pre-activations "
+                         "kept by a training forward (moe_forward_save) instead")
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
                     help="backward: time moe_backward instead (a separate measurement)")
     args = ap.parse_args()

@@ -176,6 +176,27 @@ moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *d
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
                         void *ws, size_t ws_bytes, void *stream);
 
+/* Training pair (bf16 layer): a forward that keeps what the backward would otherwise
+ * recompute, and the backward that uses it.
+ * moe_forward_save is moe_forward (same out, same workspace use) that also writes the fp32
+ * pre-activations a = x W_gate^T and b = x W_up^T of every expert-sorted row to `saved`:
+ *   saved  [2, P, f] fp32, a then b, P = n_tokens * (top_k + n_shared) rows: the routed rows
+ *          in the routing's sorted order (expert-major, ascending token), then the shared
+ *          expert's n_tokens rows; at least moe_saved_size(h, n_tokens) bytes, 16-byte aligned
+ * moe_backward_saved is moe_backward for a moe_forward_save of the same x and n_tokens (and
+ * unchanged weights and router bias, so the routing it recomputes is the same): it reads a
+ * and b from `saved` instead of recomputing them (one grouped GEMM over the gate and up
+ * weights less); its results are those of moe_backward.
+ * MOE_ERR_UNSUPPORTED for the fp32 layer; MOE_ERR_INVALID_ARG for a null or short `saved`,
+ * MOE_ERR_ALIGNMENT for a misaligned one; otherwise errors as moe_forward / moe_backward. */
+size_t moe_saved_size(moe_handle h, int n_tokens);
+moe_status moe_forward_save(moe_handle h, const void *x, int n_tokens, void *out, float *saved,
+                            size_t saved_bytes, void *ws, size_t ws_bytes, void *stream);
+moe_status moe_backward_saved(moe_handle h, const void *x, int n_tokens, const void *dout,
+                              const float *saved, size_t saved_bytes, float *dx,
+                              float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                              void *ws, size_t ws_bytes, void *stream);
+
 /* Expert health signals ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active
  * Parameters", section 4.1.2: monitor per-expert activation and parameter norms; "Step 3.5
  * Flash 技术论文深度解读", training stability, expert collapse: per-expert activation RMS

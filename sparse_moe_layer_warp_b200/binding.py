@@ -31,7 +31,8 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_device_status", "moe_status_string", "moe_router_logits_static",
            "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
            "moe_selftest_wait_timeout", "moe_expert_health", "moe_backward",
-           "moe_backward_workspace_size")
+           "moe_backward_workspace_size", "moe_saved_size", "moe_forward_save",
+           "moe_backward_saved")
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -87,6 +88,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_backward.argtypes = [P, P, I, P, P, P, P, P, P, P, Z, P]
         lib.moe_backward_workspace_size.argtypes = [P, I]
         lib.moe_backward_workspace_size.restype = Z
+        lib.moe_saved_size.argtypes = [P, I]
+        lib.moe_saved_size.restype = Z
+        lib.moe_forward_save.argtypes = [P, P, I, P, P, Z, P, Z, P]
+        lib.moe_backward_saved.argtypes = [P, P, I, P, P, Z, P, P, P, P, P, P, Z, P]
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -95,7 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                      "moe_route_from_logits", "moe_forward", "moe_forward_profiled",
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
                      "moe_update_router_bias", "moe_selftest_wait_timeout",
-                     "moe_expert_health", "moe_backward"):
+                     "moe_expert_health", "moe_backward", "moe_forward_save",
+                     "moe_backward_saved"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -175,6 +181,26 @@ def moe_backward(handle, x, n_tokens, dout, dx, dw_router, dw_gate, dw_up, dw_do
     _check("moe_backward", load_library().moe_backward(
         handle, _p(x), int(n_tokens), _p(dout), _p(dx), _p(dw_router), _p(dw_gate), _p(dw_up),
         _p(dw_down), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_saved_size(handle, n_tokens: int) -> int:
+    return int(load_library().moe_saved_size(handle, int(n_tokens)))
+
+
+def moe_forward_save(handle, x, n_tokens, out, saved, ws, stream=None) -> None:
+    """moe_forward that also keeps the fp32 pre-activations for moe_backward_saved."""
+    _check("moe_forward_save", load_library().moe_forward_save(
+        handle, _p(x), int(n_tokens), _p(out), _p(saved), saved.numel() * saved.element_size(),
+        _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_backward_saved(handle, x, n_tokens, dout, saved, dx, dw_router, dw_gate, dw_up, dw_down,
+                       ws, stream=None) -> None:
+    """moe_backward reading the pre-activations kept by moe_forward_save."""
+    _check("moe_backward_saved", load_library().moe_backward_saved(
+        handle, _p(x), int(n_tokens), _p(dout), _p(saved), saved.numel() * saved.element_size(),
+        _p(dx), _p(dw_router), _p(dw_gate), _p(dw_up), _p(dw_down), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_expert_health(handle, n_tokens, act_rms, param_norm, ratios, ws, stream=None) -> None:
@@ -293,9 +319,24 @@ class MoELayer:
                          self.workspace(T), stream)
         return p_mean, f_sel, scalars
 
-    def backward(self, x, dout, stream=None, grads=None):
+    def forward_save(self, x, out=None, saved=None, stream=None):
+        """Training forward (bf16): (out, saved) with `saved` the fp32 pre-activations that
+        backward(..., saved=saved) reads instead of recomputing them."""
+        T = x.shape[0]
+        ws = self.workspace(T)
+        if out is None:
+            out = torch.empty_like(x)
+        if saved is None:
+            saved = torch.empty(moe_saved_size(self.handle, T) // 4, dtype=torch.float32,
+                                device=self.device)
+        moe_forward_save(self.handle, x, T, out, saved, ws, stream)
+        return out, saved
+
+    def backward(self, x, dout, stream=None, grads=None, saved=None):
         """dict of fp32 gradients dx, dw_router, dw_gate, dw_up, dw_down (device tensors); the
-        weight gradients are added to `grads`' tensors when given (new zeroed ones if not)."""
+        weight gradients are added to `grads`' tensors when given (new zeroed ones if not).
+        With `saved` (from forward_save of the same x) the pre-activations are not
+        recomputed."""
         T = x.shape[0]
         need = moe_backward_workspace_size(self.handle, T)
         if self.bw_ws is None or self.bw_ws.numel() < need:
@@ -313,8 +354,12 @@ class MoELayer:
                      dw_gate=torch.zeros((G, f, self.d), **kw),
                      dw_up=torch.zeros((G, f, self.d), **kw),
                      dw_down=torch.zeros((G, self.d, f), **kw))
-        moe_backward(self.handle, x, T, dout, g["dx"], g["dw_router"], g["dw_gate"], g["dw_up"],
-                     g["dw_down"], self.bw_ws, stream)
+        if saved is not None:
+            moe_backward_saved(self.handle, x, T, dout, saved, g["dx"], g["dw_router"],
+                               g["dw_gate"], g["dw_up"], g["dw_down"], self.bw_ws, stream)
+        else:
+            moe_backward(self.handle, x, T, dout, g["dx"], g["dw_router"], g["dw_gate"],
+                         g["dw_up"], g["dw_down"], self.bw_ws, stream)
         return g
 
     def expert_health(self, n_tokens, stream=None):

@@ -61,6 +61,8 @@ struct GemmParams {
   void *out;                // UP: h [P, f] bf16; DOWN: y [P, d] fp32; LOGITS: [T, E] fp32
   float *out2;              // UP with out2 set: out = fp32 pre-activation x W_g^T, out2 =
                             // x W_u^T, [P, f] each, instead of h (for the backward)
+  float *save_a, *save_b;   // UP, training forward: h to out as usual and, in addition, the
+                            // fp32 pre-activations x W_g^T, x W_u^T [P, f] (null: not kept)
   DevStatus *status;
   float routed_scale;
   int E, n_groups, T, Tk;
@@ -561,6 +563,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
           store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
                              col_base, vals, wbuf, lane);
+          if (p.save_a) {  // training forward: keep the pre-activations for the backward
+#pragma unroll
+            for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v0[n]);
+            store_block16_f32(p.save_a, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+#pragma unroll
+            for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v1[n]);
+            store_block16_f32(p.save_b, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+          }
         } else if (MODE == MODE_DOWN) {
           const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
 #pragma unroll

@@ -126,7 +126,10 @@ struct BwDgradParams {
   CUtensorMap tmB1;  // DX: db [R, f]                                      box {64, BN}
   BwRows rows;
   const float *row_scale;      // [P] s_p by unpadded row (DH)
-  const float *pre_a, *pre_b;  // [R, f] fp32 pre-activations, padded rows (DH)
+  const float *pre_a, *pre_b;  // fp32 pre-activations (DH): [R, f] at the padded rows, or
+                               // [P, f] at the unpadded rows when pre_unpadded is set (kept
+                               // by a training forward)
+  int pre_unpadded;
   __nv_bfloat16 *da, *db, *hs; // [R, f] padded rows (DH)
   float *dgate_part;           // [Tk, n_part] by unpadded row (DH): partial sums of dhu . h
   float *out;                  // DX: dX rows [P, d] fp32, unpadded rows
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int n = 0; n < 16; ++n) {
             const bool in = c0 + n < valid;
-            const size_t i = (size_t)(row0 + c0 + n) * p.M + col;
+            const size_t i = (size_t)((p.pre_unpadded ? rowu0 : row0) + c0 + n) * p.M + col;
             av[n] = in ? p.pre_a[i] : 0.f;
             bv[n] = in ? p.pre_b[i] : 0.f;
           }
@@ -862,7 +865,7 @@ __global__ void __launch_bounds__(kBwPairThreads, 1)
 #pragma unroll
           for (int n = 0; n < 16; ++n) {
             const bool in = c0 + n < valid;
-            const size_t i = (size_t)(row0 + c0 + n) * p.M + col;
+            const size_t i = (size_t)((p.pre_unpadded ? rowu0 : row0) + c0 + n) * p.M + col;
             av[n] = in ? p.pre_a[i] : 0.f;
             bv[n] = in ? p.pre_b[i] : 0.f;
           }

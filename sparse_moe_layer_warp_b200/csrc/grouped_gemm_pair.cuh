@@ -433,6 +433,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             vals[n] = swiglu(__uint_as_float(v0[n]), __uint_as_float(v1[n]));
           store_block16_bf16(static_cast<__nv_bfloat16 *>(p.out), p.ld_out, row0, c0, valid,
                              col_base, vals, wbuf, lane);
+          if (p.save_a) {  // training forward: keep the pre-activations for the backward
+#pragma unroll
+            for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v0[n]);
+            store_block16_f32(p.save_a, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+#pragma unroll
+            for (int n = 0; n < 16; ++n) vals[n] = __uint_as_float(v1[n]);
+            store_block16_f32(p.save_b, p.ld_out, row0, c0, valid, col_base, vals, wbuf, lane);
+          }
         } else {
           const float4 *sc = reinterpret_cast<const float4 *>(row_scale + acc * BN + c0);
 #pragma unroll

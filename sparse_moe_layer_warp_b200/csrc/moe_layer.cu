@@ -551,7 +551,7 @@ BwLayout bw_layout(const moe_config &c, int T) {
 
 moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
                        int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
-                       float *dw_down, void *ws, cudaStream_t st);
+                       float *dw_down, void *ws, cudaStream_t st, const float *saved);
 moe_status backward_f32(const moe_layer *L, const float *x, const float *dout, int T, float *dx,
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down, void *ws,
                         cudaStream_t st);
@@ -699,9 +699,35 @@ size_t moe_backward_workspace_size(moe_handle h, int n_tokens) {
   return bw_layout(h->cfg, n_tokens).total;
 }
 
+static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, const void *dout,
+                                 const float *saved, float *dx, float *dw_router,
+                                 float *dw_gate, float *dw_up, float *dw_down, void *ws,
+                                 size_t ws_bytes, void *stream);
+
 moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *dout, float *dx,
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
                         void *ws, size_t ws_bytes, void *stream) {
+  return backward_entry(h, x, n_tokens, dout, nullptr, dx, dw_router, dw_gate, dw_up, dw_down,
+                        ws, ws_bytes, stream);
+}
+
+moe_status moe_backward_saved(moe_handle h, const void *x, int n_tokens, const void *dout,
+                              const float *saved, size_t saved_bytes, float *dx,
+                              float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                              void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (n_tokens > 0 && (!saved || saved_bytes < moe_saved_size(h, n_tokens)))
+    return MOE_ERR_INVALID_ARG;
+  if (saved && !aligned16(saved)) return MOE_ERR_ALIGNMENT;
+  return backward_entry(h, x, n_tokens, dout, saved, dx, dw_router, dw_gate, dw_up, dw_down, ws,
+                        ws_bytes, stream);
+}
+
+static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, const void *dout,
+                                 const float *saved, float *dx, float *dw_router,
+                                 float *dw_gate, float *dw_up, float *dw_down, void *ws,
+                                 size_t ws_bytes, void *stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
   if (n_tokens == 0) return MOE_OK;
@@ -717,7 +743,7 @@ moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *d
   if (h->cfg.dtype == MOE_BF16)
     return backward_tc(h, static_cast<const __nv_bfloat16 *>(x),
                        static_cast<const __nv_bfloat16 *>(dout), n_tokens, dx, dw_router, dw_gate,
-                       dw_up, dw_down, ws, st);
+                       dw_up, dw_down, ws, st, saved);
   return backward_f32(h, static_cast<const float *>(x), static_cast<const float *>(dout),
                       n_tokens, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
@@ -902,7 +928,8 @@ struct UpRows {
 moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
                             const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
                             int *done, cudaStream_t st, GemmParams *used,
-                            const UpRows *rows = nullptr) {
+                            const UpRows *rows = nullptr, float *save_a = nullptr,
+                            float *save_b = nullptr) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
@@ -935,6 +962,8 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
   p1.sched = &at<DevStatus>(ws, W.status)->sched[0];  // dynamic unit claiming
   p1.topk = c.top_k;
   p1.done = done;
+  p1.save_a = save_a;
+  p1.save_b = save_b;
   if (rows) {
     p1.offsets = rows->offsets;
     p1.perm = rows->perm;
@@ -952,7 +981,8 @@ int moe_forward_launch_count(moe_handle h, int n_tokens) {
 }
 
 static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
-                               size_t ws_bytes, void *stream, void *const *events) {
+                               size_t ws_bytes, void *stream, void *const *events,
+                               float *saved = nullptr) {
   moe_status s = check_call(h, n_tokens, ws, ws_bytes);
   if (s != MOE_OK || n_tokens == 0) return s;
   if (!x || !out) return MOE_ERR_INVALID_ARG;
@@ -1017,7 +1047,8 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
     // expert group for that group's rows of h (see grouped_gemm_kernel)
     GemmParams p1;
     if ((s = launch_expert_up(h, x, T, ws, W, plan, hbuf, nullptr, at<int>(ws, W.done), st,
-                              &p1)) != MOE_OK)
+                              &p1, nullptr, saved, saved ? saved + (size_t)P * c.d_ff : nullptr)) !=
+        MOE_OK)
       return s;
     if ((s = mark(5)) != MOE_OK) return s;
     GemmParams p2 = p1;
@@ -1067,6 +1098,23 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                   c.d_model, static_cast<float *>(out))) != MOE_OK)
     return s;
   return mark(7);
+}
+
+size_t moe_saved_size(moe_handle h, int n_tokens) {
+  if (!h || n_tokens < 0 || n_tokens > h->cfg.max_tokens) return 0;
+  const moe_config &c = h->cfg;
+  return 2 * (size_t)n_tokens * (c.top_k + c.n_shared) * c.d_ff * sizeof(float);
+}
+
+moe_status moe_forward_save(moe_handle h, const void *x, int n_tokens, void *out, float *saved,
+                            size_t saved_bytes, void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!saved || saved_bytes < moe_saved_size(h, n_tokens)))
+    return MOE_ERR_INVALID_ARG;
+  if (saved && !aligned16(saved)) return MOE_ERR_ALIGNMENT;
+  return forward_impl(h, x, n_tokens, out, ws, ws_bytes, stream, nullptr, saved);
 }
 
 moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, void *ws,
@@ -1372,7 +1420,7 @@ moe_status launch_bw_wgrad_pair(const moe_layer *L, const BwWgradParams &p, cuda
 //   and dx.
 moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
                        int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
-                       float *dw_down, void *ws, cudaStream_t st) {
+                       float *dw_down, void *ws, cudaStream_t st, const float *saved) {
   const moe_config &c = L->cfg;
   const int E = c.n_experts, G = E + c.n_shared, k = c.top_k, d = c.d_model, f = c.d_ff;
   const int Tk = T * k, P = Tk + c.n_shared * T;
@@ -1405,12 +1453,15 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
                   st, x, dout, (const int *)perm, k, rows, c.n_shared, R, d, f, xs, dys, da, db,
                   hs, perm_pad)) != MOE_OK)
     return s;
-  // pre-activations a, b: the forward's up GEMM over the padded rows
+  // pre-activations a, b: kept by a training forward (unpadded rows), or recomputed by the
+  // forward's up GEMM over the padded rows
   const ForwardPlan plan = plan_forward(L, T);
-  const UpRows up_rows{poff, perm_pad, rows.s0, xs, R};
-  GemmParams pu;
-  if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, &up_rows)) != MOE_OK)
-    return s;
+  if (!saved) {
+    const UpRows up_rows{poff, perm_pad, rows.s0, xs, R};
+    GemmParams pu;
+    if ((s = launch_expert_up(L, x, T, ws, W, plan, a, b, nullptr, st, &pu, &up_rows)) != MOE_OK)
+      return s;
+  }
   // DH (CTA pairs for groups as large as the forward's pair threshold)
   const bool pair_dg = plan.pair && d % 256 == 0 && f % 256 == 0 && L->bw_pair_grid >= 2;
   const int bn = pair_dg ? BwDgradPairCfg::HALF_BN : pick_bn(c, T, MODE_DOWN);
@@ -1420,8 +1471,9 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   if (!encode_bf16_2d(&pd.tmB0, dys, d, (uint64_t)R, bn)) return MOE_ERR_CUDA;
   pd.rows = rows;
   pd.row_scale = row_scale;
-  pd.pre_a = a;
-  pd.pre_b = b;
+  pd.pre_a = saved ? saved : a;
+  pd.pre_b = saved ? saved + (size_t)P * f : b;
+  pd.pre_unpadded = saved ? 1 : 0;
   pd.da = da;
   pd.db = db;
   pd.hs = hs;

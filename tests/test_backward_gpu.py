@@ -89,3 +89,31 @@ def test_backward_of_zero_dout_is_zero(cuda_ok):
     torch.cuda.synchronize()
     for name, t in g.items():
         assert (t == 0).all(), name
+
+
+@pytest.mark.parametrize("kw", [
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 128},             # decode path
+    {"dtype": "bf16", "T": 150, "d": 256, "E": 8, "k": 4, "f": 256, "seed": 3},  # 1-CTA / pair wgrad
+    {"dtype": "bf16", "T": 300, "d": 256, "E": 8, "k": 4, "f": 512, "seed": 10,  # CTA pairs
+     "bias": "zipf"},
+])
+def test_training_pair_matches_forward_and_backward(cuda_ok, kw):
+    """forward_save returns moe_forward's output; backward from its saved pre-activations
+    returns moe_backward's gradients (the kept a, b are the recompute's values)."""
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    dout = synth.make_x(w, w.T, device="cuda", seed=78)
+    out_ref = layer.forward(inp.x).clone()
+    g_ref = layer.backward(inp.x, dout)
+    out, saved = layer.forward_save(inp.x)
+    g = layer.backward(inp.x, dout, saved=saved)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_ref)
+    for name in g_ref:
+        ref = g_ref[name]
+        # same arithmetic on the same values: equal up to the MMA accumulation order of a
+        # and b in the two token tilings (the forward's rows are not padded)
+        err = (g[name] - ref).abs().max().item()
+        assert err <= 1e-5 * ref.abs().max().item() + 1e-30, (name, err)
+    assert layer.device_status() == 0
