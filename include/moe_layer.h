@@ -177,7 +177,10 @@ moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *d
                         void *ws, size_t ws_bytes, void *stream);
 
 /* Training pair (bf16 layer): a forward that keeps what the backward would otherwise
- * recompute, and the backward that uses it.
+ * recompute, and the backward that uses it -- the per-submodule choice between recomputing
+ * activations and keeping them ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B
+ * Active Parameters", section 3.2.5, fine-grained selective checkpointing): moe_backward
+ * recomputes the expert pre-activations, this pair keeps them.
  * moe_forward_save is moe_forward (same out, same workspace use) that also writes the fp32
  * pre-activations a = x W_gate^T and b = x W_up^T of every expert-sorted row to `saved`:
  *   saved  [2, P, f] fp32, a then b, P = n_tokens * (top_k + n_shared) rows: the routed rows
