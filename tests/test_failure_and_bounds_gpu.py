@@ -184,3 +184,49 @@ def test_backward_rejects_bad_arguments(cuda_ok):
     call()                                          # the valid call still works
     torch.cuda.synchronize()
     assert layer.device_status() == 0
+
+
+def test_training_pair_bounds_and_arguments(cuda_ok):
+    """moe_forward_save writes inside `saved` only; short, misaligned or fp32-layer calls
+    of the training pair are rejected before any launch."""
+    from sparse_moe_layer_warp_b200 import (moe_backward_saved, moe_backward_workspace_size,
+                                            moe_forward_save, moe_saved_size)
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", T=50, d=256, E=16, k=4, f=128)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    T, d = w.T, w.d
+    n = moe_saved_size(layer.handle, T) // 4
+    assert n == 2 * T * (w.k + w.n_shared) * w.f
+    big, saved_i = _guarded(n, torch.int32, 0x5EED)
+    saved = saved_i.view(torch.float32)
+    out = torch.empty_like(inp.x)
+    ws = layer.workspace(T)
+    moe_forward_save(layer.handle, inp.x, T, out, saved, ws)
+    torch.cuda.synchronize()
+    assert _margins_intact(big, n, 0x5EED)
+    assert torch.equal(out, layer.forward(inp.x))
+    with pytest.raises(MoEError):
+        moe_forward_save(layer.handle, inp.x, T, out, saved[:-4], ws)      # too short
+    with pytest.raises(MoEError):
+        moe_forward_save(layer.handle, inp.x, T, out, big.view(torch.float32)[1:1 + n], ws)
+    bws = torch.empty(moe_backward_workspace_size(layer.handle, T), dtype=torch.uint8,
+                      device="cuda")
+    moe_workspace_init(layer.handle, bws)
+    G = w.E + 1
+    gr = [torch.zeros(T, d, device="cuda"), torch.zeros(w.E, d, device="cuda"),
+          torch.zeros(G, w.f, d, device="cuda"), torch.zeros(G, w.f, d, device="cuda"),
+          torch.zeros(G, d, w.f, device="cuda")]
+    dout = synth.make_x(w, T, device="cuda", seed=9)
+    with pytest.raises(MoEError):
+        moe_backward_saved(layer.handle, inp.x, T, dout, saved[:-4], *gr, bws)
+    moe_backward_saved(layer.handle, inp.x, T, dout, saved, *gr, bws)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    # the fp32 layer has no training pair
+    w32 = synth.WORKLOADS["tiny_fp32"]
+    inp32 = synth.make_inputs(w32, device="cuda")
+    layer32 = make_layer(inp32)
+    s32 = torch.empty(moe_saved_size(layer32.handle, w32.T) // 4, device="cuda")
+    with pytest.raises(MoEError):
+        moe_forward_save(layer32.handle, inp32.x, w32.T, torch.empty_like(inp32.x), s32,
+                         layer32.workspace(w32.T))
