@@ -5,7 +5,8 @@
 // 技术论文深度解读", training stability, root cause 3) as grouped GEMMs over the
 // expert-sorted rows ("fused MoE gather/scatter with grouped GEMM", first page, section
 // 3.2.4).  Per sorted row p of group g (token t, scale s_p = routed_scale * gate, 1 for the
-// shared expert), with a = W_g[g] x_t and b = W_u[g] x_t recomputed by the forward's up GEMM:
+// shared expert), with a = W_g[g] x_t and b = W_u[g] x_t recomputed by the forward's up GEMM
+// (or kept by a training forward):
 //
 //   DH    dhu_p = W_d[g]^T dout_t                (weights on M: f rows; K = d)
 //         epilogue: h = silu(a) b, dgate partial sum dhu . h, dh = s_p dhu,
@@ -35,10 +36,15 @@
 // accumulator into the caller's fp32 gradient with TMA reductions (cp.reduce.async.bulk
 // .tensor add): one addition per element and call, so the result is deterministic.
 //
-// Roles, pipelines and bounded waits are those of grouped_gemm.cuh: warp 0 produces (lane 0
-// claims units), warp 1 lane 0 issues the MMAs, warps 2..5 run the epilogue, STAGES
-// shared-memory slots and two TMEM accumulators; every wait gives up after the time limit,
-// drains its in-flight copies and MMAs, frees TMEM and reports through the status word.
+// Kernels: bw_dgrad_kernel (one CTA per unit, DH or DX), bw_dgrad_pair_kernel (the same on a
+// CTA pair, 256 weight rows per unit), bw_wgrad_kernel / bw_wgrad_pair_kernel (weight
+// gradients, 128 x 256 or 256 x 256 tiles), bw_tail_pair_kernel (DX and the weight gradients
+// in one persistent launch with interleaved units), and the small row-layout kernels.
+// Roles, pipelines and bounded waits are those of grouped_gemm.cuh and grouped_gemm_pair.cuh:
+// warp 0 produces (lane 0 claims units; on a pair the leader claims and publishes), warp 1
+// lane 0 issues the MMAs, warps 2..5 (2..9 on a pair) run the epilogue, STAGES shared-memory
+// slots and two TMEM accumulators; every wait gives up after the time limit, drains its
+// in-flight copies and MMAs, frees TMEM and reports through the status word.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
