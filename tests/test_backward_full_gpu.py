@@ -19,6 +19,8 @@ U_BF16 = 2.0 ** -8   # bf16 unit roundoff; bound 2u * max |ref| (see test_backwa
 @pytest.mark.parametrize("name,toks,n_routed,router", [
     ("decode_t16", [0, 9, 15], 2, True),
     ("prefill_t8192", [0, 4097], 1, False),   # router rows would need ~228 whole tokens
+    ("skew_t4096", [0, 2047], 2, False),      # Zipf-skewed groups (the two smallest)
+    ("dense_ffn_t4096", [0, 4095], 0, False),  # one 4096-row expert: dx rows only
 ])
 def test_backward_full_size_sampled(cuda_ok, name, toks, n_routed, router):
     w = synth.WORKLOADS[name]
