@@ -471,7 +471,7 @@ def run_backward(args, rank, world, local_rank):
     grads = layer.backward(xs[0], douts[0], saved=saved[0])
     for i in range(args.warmup):
         flush.zero_()
-        layer.backward(xs[i], douts[i], grads=grads, saved=saved[i])
+        layer.backward(xs[i], douts[i], grads=grads, saved=saved[i], overwrite=args.overwrite)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -487,7 +487,7 @@ def run_backward(args, rank, world, local_rank):
         flush.zero_()
         ev[i][0].record(st)
         layer.backward(xs[args.warmup + i], douts[args.warmup + i], grads=grads,
-                       saved=saved[args.warmup + i])
+                       saved=saved[args.warmup + i], overwrite=args.overwrite)
         ev[i][1].record(st)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -517,6 +517,11 @@ def run_backward(args, rank, world, local_rank):
             nbytes = (tm * 3 * w.f * w.d * es + tm * 3 * w.f * w.d * 8 + w.E * w.d * 8
                       + 8.0 * P * w.f)
             label += ", pre-activations kept by the training forward"
+        if args.overwrite:
+            # gradients written, not read: every expert's (zeros for the untouched ones)
+            G = w.E + w.n_shared
+            nbytes += G * 3 * w.f * w.d * 4 - tm * 3 * w.f * w.d * 8 - w.E * w.d * 4
+            label += ", weight gradients overwritten"
         peak_c = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         peak_name = f"bf16 dense, sustained ({src})"
         unit_c, kind = "TFLOP/s", "tensor"
@@ -571,6 +576,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--overwrite", action="store_true",
+                    help="with --pass backward: the weight gradients are set, not accumulated "
+                         "(MOE_BACKWARD_OVERWRITE)")
     ap.add_argument("--saved", action="store_true",
                     help="with --pass backward: time moe_backward_saved on pre-activations "
                          "kept by a training forward (moe_forward_save) instead")

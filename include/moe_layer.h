@@ -200,6 +200,19 @@ moe_status moe_backward_saved(moe_handle h, const void *x, int n_tokens, const v
                               float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* Backward with options: `saved` as in moe_backward_saved (null: recompute, as moe_backward;
+ * non-null needs the bf16 layer), and `flags`:
+ *   MOE_BACKWARD_OVERWRITE  the weight gradients are SET to this call's gradients instead of
+ *                           added (rows of experts no token chose are set to zero), so the
+ *                           first micro-batch needs no zeroed buffers and, in the bf16 layer,
+ *                           the gradient tiles are stored instead of read, added and written.
+ * Results otherwise as moe_backward; MOE_ERR_INVALID_ARG for unknown flags. */
+#define MOE_BACKWARD_OVERWRITE 1u
+moe_status moe_backward_ex(moe_handle h, const void *x, int n_tokens, const void *dout,
+                           const float *saved, size_t saved_bytes, unsigned flags, float *dx,
+                           float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                           void *ws, size_t ws_bytes, void *stream);
+
 /* Expert health signals ("Step 3.5 Flash: Open Frontier-Level Intelligence with 11B Active
  * Parameters", section 4.1.2: monitor per-expert activation and parameter norms; "Step 3.5
  * Flash 技术论文深度解读", training stability, expert collapse: per-expert activation RMS

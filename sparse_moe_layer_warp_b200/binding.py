@@ -32,7 +32,8 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
            "moe_selftest_wait_timeout", "moe_expert_health", "moe_backward",
            "moe_backward_workspace_size", "moe_saved_size", "moe_forward_save",
-           "moe_backward_saved")
+           "moe_backward_saved", "moe_backward_ex")
+MOE_BACKWARD_OVERWRITE = 1
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -92,6 +93,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_saved_size.restype = Z
         lib.moe_forward_save.argtypes = [P, P, I, P, P, Z, P, Z, P]
         lib.moe_backward_saved.argtypes = [P, P, I, P, P, Z, P, P, P, P, P, P, Z, P]
+        lib.moe_backward_ex.argtypes = [P, P, I, P, P, Z, ctypes.c_uint, P, P, P, P, P, P, Z, P]
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -101,7 +103,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
                      "moe_update_router_bias", "moe_selftest_wait_timeout",
                      "moe_expert_health", "moe_backward", "moe_forward_save",
-                     "moe_backward_saved"):
+                     "moe_backward_saved", "moe_backward_ex"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -200,6 +202,16 @@ def moe_backward_saved(handle, x, n_tokens, dout, saved, dx, dw_router, dw_gate,
     _check("moe_backward_saved", load_library().moe_backward_saved(
         handle, _p(x), int(n_tokens), _p(dout), _p(saved), saved.numel() * saved.element_size(),
         _p(dx), _p(dw_router), _p(dw_gate), _p(dw_up), _p(dw_down), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_backward_ex(handle, x, n_tokens, dout, saved, flags, dx, dw_router, dw_gate, dw_up,
+                    dw_down, ws, stream=None) -> None:
+    """moe_backward with options: `saved` (or None) and flags (MOE_BACKWARD_OVERWRITE)."""
+    nbytes = 0 if saved is None else saved.numel() * saved.element_size()
+    _check("moe_backward_ex", load_library().moe_backward_ex(
+        handle, _p(x), int(n_tokens), _p(dout), None if saved is None else _p(saved), nbytes,
+        int(flags), _p(dx), _p(dw_router), _p(dw_gate), _p(dw_up), _p(dw_down), _p(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
 
 
@@ -332,11 +344,11 @@ class MoELayer:
         moe_forward_save(self.handle, x, T, out, saved, ws, stream)
         return out, saved
 
-    def backward(self, x, dout, stream=None, grads=None, saved=None):
+    def backward(self, x, dout, stream=None, grads=None, saved=None, overwrite=False):
         """dict of fp32 gradients dx, dw_router, dw_gate, dw_up, dw_down (device tensors); the
-        weight gradients are added to `grads`' tensors when given (new zeroed ones if not).
-        With `saved` (from forward_save of the same x) the pre-activations are not
-        recomputed."""
+        weight gradients are added to `grads`' tensors when given (new zeroed ones if not),
+        or set when `overwrite`.  With `saved` (from forward_save of the same x) the
+        pre-activations are not recomputed."""
         T = x.shape[0]
         need = moe_backward_workspace_size(self.handle, T)
         if self.bw_ws is None or self.bw_ws.numel() < need:
@@ -348,13 +360,23 @@ class MoELayer:
         if grads is not None:
             g = dict(grads)
             g["dx"] = torch.empty((T, self.d), **kw)
+        elif overwrite:  # every element is written
+            g = dict(dx=torch.empty((T, self.d), **kw),
+                     dw_router=torch.empty((self.E, self.d), **kw),
+                     dw_gate=torch.empty((G, f, self.d), **kw),
+                     dw_up=torch.empty((G, f, self.d), **kw),
+                     dw_down=torch.empty((G, self.d, f), **kw))
         else:  # the weight gradients accumulate: start them at zero
             g = dict(dx=torch.empty((T, self.d), **kw),
                      dw_router=torch.zeros((self.E, self.d), **kw),
                      dw_gate=torch.zeros((G, f, self.d), **kw),
                      dw_up=torch.zeros((G, f, self.d), **kw),
                      dw_down=torch.zeros((G, self.d, f), **kw))
-        if saved is not None:
+        if overwrite:
+            moe_backward_ex(self.handle, x, T, dout, saved, MOE_BACKWARD_OVERWRITE, g["dx"],
+                            g["dw_router"], g["dw_gate"], g["dw_up"], g["dw_down"], self.bw_ws,
+                            stream)
+        elif saved is not None:
             moe_backward_saved(self.handle, x, T, dout, saved, g["dx"], g["dw_router"],
                                g["dw_gate"], g["dw_up"], g["dw_down"], self.bw_ws, stream)
         else:

@@ -446,20 +446,27 @@ __device__ __forceinline__ float4 bw_load4(const float *p) {
 }
 
 // dW_r[e][i] += sum over the rows of routed group e (ascending token) of dl x_t[i]; experts
-// no token chose are left untouched.  Block (e, 512 columns): each thread two columns, the
-// rows four at a time (their loads issued together, the sums still in row order).
+// no token chose are left untouched (overwrite: dW_r[e][i] = the sum, zero for them).  Block
+// (e, 512 columns): each thread two columns, the rows four at a time (their loads issued
+// together, the sums still in row order).
 template <typename Tin>
 __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict__ x,
                                                            const float *__restrict__ dl,
                                                            const int *__restrict__ perm,
                                                            const int *__restrict__ offsets,
-                                                           int k, int d, float *dw_r) {
+                                                           int k, int d, float *dw_r,
+                                                           int overwrite) {
   griddep_wait();
   griddep_launch_dependents();
   const int e = blockIdx.x;
   const int i = 2 * (blockIdx.y * blockDim.x + threadIdx.x);
   const int lo = offsets[e], hi = offsets[e + 1];
-  if (i >= d || lo == hi) return;
+  if (i >= d) return;
+  if (lo == hi) {
+    if (overwrite)
+      *reinterpret_cast<float2 *>(dw_r + (size_t)e * d + i) = make_float2(0.f, 0.f);
+    return;
+  }
   float2 acc = make_float2(0.f, 0.f);
   int p = lo;
   for (; p + 4 <= hi; p += 4) {
@@ -487,8 +494,12 @@ __global__ void __launch_bounds__(256) bw_router_dw_kernel(const Tin *__restrict
     acc.y = fmaf(w, v.y, acc.y);
   }
   float2 *o = reinterpret_cast<float2 *>(dw_r + (size_t)e * d + i);
-  const float2 old = *o;
-  *o = make_float2(old.x + acc.x, old.y + acc.y);
+  if (overwrite) {
+    *o = acc;
+  } else {
+    const float2 old = *o;
+    *o = make_float2(old.x + acc.x, old.y + acc.y);
+  }
 }
 
 // dx[t][i] = sum_j dX[slot_row[t,j]][i] + dX[shared row][i] + sum_j dl[t,j] W_r[e_j][i],

@@ -86,6 +86,14 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, const 
       "r"(smem_u32(src)), "r"(c0), "r"(c1)
       : "memory");
 }
+// global[tile at (c0, c1)] = shared tile (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0,
+                                             int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::
+                   "l"(reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -942,7 +950,9 @@ struct BwWgradParams {
   BwRows rows;
   DevStatus *status;
   int n_groups;
-  int *sched;  // work counter (zero at launch)
+  int *sched;     // work counter (zero at launch)
+  int overwrite;  // 1: dW = this call's gradient (tiles stored, not added; experts no row
+                  // chose get zero tiles); 0: dW += it (experts no row chose untouched)
 };
 
 constexpr int kWgStgBytes = 32 * 32 * 4;  // one 32 x 32 fp32 reduction tile
@@ -952,24 +962,29 @@ constexpr int kWgStgBytes = 32 * 32 * 4;  // one 32 x 32 fp32 reduction tile
 // registers -> swizzled staging tile -> TMA reduction into dW at (col0 + 32 c, row).  The
 // warp cycles through NBUF staging tiles; lane 0 issues and tracks the reductions.  TMEM
 // loads run one chunk ahead.
+// `store`: tiles are stored instead of added; `zero`: the tiles are zeros (an expert no row
+// chose, in the overwrite mode; TMEM is not read).
 template <int NBUF>
 __device__ __forceinline__ void wgrad_epilogue(uint32_t taddr, int c_first, int c_step, int n_cols,
                                                const CUtensorMap *omap, int col0, int row,
-                                               uint8_t *stg, int &n_red, int lane) {
+                                               uint8_t *stg, int &n_red, int lane, bool store,
+                                               bool zero) {
   uint32_t n0[16], n1[16];
-  if (32 * c_first < n_cols) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) n0[i] = n1[i] = 0u;
+  if (!zero && 32 * c_first < n_cols) {
     tmem_ld16(taddr + 32 * c_first, n0);
     tmem_ld16(taddr + 32 * c_first + 16, n1);
   }
   for (int c = c_first; 32 * c < n_cols; c += c_step) {
     uint32_t v0[16], v1[16];
-    tmem_ld_wait_regs(n0, n1);
+    if (!zero) tmem_ld_wait_regs(n0, n1);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       v0[i] = n0[i];
       v1[i] = n1[i];
     }
-    if (32 * (c + c_step) < n_cols) {
+    if (!zero && 32 * (c + c_step) < n_cols) {
       tmem_ld16(taddr + 32 * (c + c_step), n0);
       tmem_ld16(taddr + 32 * (c + c_step) + 16, n1);
     }
@@ -993,7 +1008,8 @@ __device__ __forceinline__ void wgrad_epilogue(uint32_t taddr, int c_first, int 
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_reduce_add_2d(omap, buf, col0 + 32 * c, row);
+      if (store) tma_store_2d(omap, buf, col0 + 32 * c, row);
+      else tma_reduce_add_2d(omap, buf, col0 + 32 * c, row);
       bulk_commit_group();
     }
     ++n_red;
@@ -1013,7 +1029,8 @@ __device__ __forceinline__ void wgrad_unit_table(const BwWgradParams &p, int *un
     grp_count[g] = cnt;
     grp_row[g] = rowp;
     for (int pr = 0; pr < NP; ++pr)
-      unit_prefix[pr * G + g] = cnt > 0 ? (p.M[pr] / BMW) * (p.N[pr] / BNW) : 0;
+      unit_prefix[pr * G + g] =
+          (cnt > 0 || p.overwrite) ? (p.M[pr] / BMW) * (p.N[pr] / BNW) : 0;
   }
   __syncthreads();
   if (warp == 0) {
@@ -1219,14 +1236,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           qph ^= 1;
         }
         if (u < 0) break;
+        int pr, g, mt, nt;
+        wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
+        const int cnt = grp_count[g];
+        if (cnt == 0) continue;  // zero tile of the overwrite mode: no MMA, no accumulator
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         ++it;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 34)) break;
         tc_fence_after();
-        int pr, g, mt, nt;
-        wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
-        const int cnt = grp_count[g];
         const int kbs = (cnt + kBK - 1) / kBK;
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
         for (int kb = 0; kb < kbs; ++kb) {
@@ -1280,16 +1298,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         qph ^= 1;
       }
       if (u < 0) break;
+      int pr, g, mt, nt;
+      wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
+      const int out_row = g * p.M[pr] + mt * kBM + q * 32;
+      if (grp_count[g] == 0) {  // overwrite mode, expert no row chose: a zero tile
+        wgrad_epilogue<C::STG_BUFS>(0, 0, 1, BNW, &p.out[pr], nt * BNW, out_row, my_stg, n_red,
+                                    lane, true, true);
+        continue;
+      }
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       ++it;
       if (!warp_wait(&tfull[acc], acc_phase, 37)) break;
       tc_fence_after();
-      int pr, g, mt, nt;
-      wgrad_decode<BNW>(p, unit_prefix, u, pr, g, mt, nt);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
-      wgrad_epilogue<C::STG_BUFS>(taddr, 0, 1, BNW, &p.out[pr], nt * BNW,
-                                  g * p.M[pr] + mt * kBM + q * 32, my_stg, n_red, lane);
+      wgrad_epilogue<C::STG_BUFS>(taddr, 0, 1, BNW, &p.out[pr], nt * BNW, out_row, my_stg, n_red,
+                                  lane, p.overwrite != 0, false);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -1494,14 +1518,15 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
           qph ^= 1;
         }
         if (u < 0) break;
+        int pr, g, mt, nt;
+        wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
+        const int cnt = grp_count[g];
+        if (cnt == 0) continue;  // zero tile of the overwrite mode
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         ++it;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.status, 45)) break;
         tc_fence_after();
-        int pr, g, mt, nt;
-        wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
-        const int cnt = grp_count[g];
         const int kbs = (cnt + kBK - 1) / kBK;
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
         for (int kb = 0; kb < kbs; ++kb) {
@@ -1564,17 +1589,22 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
         qph ^= 1;
       }
       if (u < 0) break;
+      int pr, g, mt, nt;
+      wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
+      const int out_row = g * p.M[pr] + mt * 256 + (int)rank * 128 + q * 32;
+      if (grp_count[g] == 0) {  // overwrite mode, expert no row chose: a zero tile
+        wgrad_epilogue<C::STG_BUFS>(0, eh, 2, 256, &p.out[pr], nt * 256, out_row, my_stg, n_red,
+                                    lane, true, true);
+        continue;
+      }
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       ++it;
       if (!warp_wait(&tfull[acc], acc_phase, 48, false)) break;
       tc_fence_after();
-      int pr, g, mt, nt;
-      wgrad_decode<256>(p, unit_prefix, u, pr, g, mt, nt);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
-      wgrad_epilogue<C::STG_BUFS>(taddr, eh, 2, 256, &p.out[pr], nt * 256,
-                                  g * p.M[pr] + mt * 256 + (int)rank * 128 + q * 32, my_stg,
-                                  n_red, lane);
+      wgrad_epilogue<C::STG_BUFS>(taddr, eh, 2, 256, &p.out[pr], nt * 256, out_row, my_stg,
+                                  n_red, lane, p.overwrite != 0, false);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1695,7 +1725,8 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
     grp_count[g] = cnt;
     grp_row[g] = rowp;
     grp_rowu[g] = rowu;
-    unit_prefix[g] = cnt > 0 ? dx_mtiles * ((cnt + 255) / 256) + wg_units_per_group : 0;
+    unit_prefix[g] = (cnt > 0 ? dx_mtiles * ((cnt + 255) / 256) : 0) +
+                     ((cnt > 0 || pw.overwrite) ? wg_units_per_group : 0);
   }
   __syncthreads();
   if (warp == 0) {
@@ -1867,14 +1898,15 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
           qph ^= 1;
         }
         if (u < 0) break;
+        int g, pr, mt, nt;
+        decode(u, g, pr, mt, nt);
+        const int cnt = grp_count[g];
+        if (cnt == 0) continue;  // zero tile of the overwrite mode
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         ++it;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, pw.status, 65)) break;
         tc_fence_after();
-        int g, pr, mt, nt;
-        decode(u, g, pr, mt, nt);
-        const int cnt = grp_count[g];
         const int kbs = (pr < 0) ? dx_kblocks : (cnt + kBK - 1) / kBK;
         const uint32_t idesc = (pr < 0)
                                    ? idesc_bf16_f32_major(256, 2 * split(g, nt), true, false)
@@ -1948,13 +1980,19 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
         qph ^= 1;
       }
       if (u < 0) break;
+      int g, pr, mt, nt;
+      decode(u, g, pr, mt, nt);
+      if (grp_count[g] == 0) {  // overwrite mode, expert no row chose: a zero tile
+        wgrad_epilogue<C::STG_BUFS>(0, eh, 2, 256, &pw.out[pr], nt * 256,
+                                    g * pw.M[pr] + mt * 256 + (int)rank * 128 + q * 32, my_stg,
+                                    n_red, lane, true, true);
+        continue;
+      }
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       ++it;
       if (!warp_wait(&tfull[acc], acc_phase, 68, false)) break;
       tc_fence_after();
-      int g, pr, mt, nt;
-      decode(u, g, pr, mt, nt);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
       if (pr < 0) {
         // rows of dx: fp32, tokens of this unit at unpadded rows
@@ -1978,7 +2016,7 @@ __global__ void __launch_bounds__(kWgPairThreads, 1)
       } else {
         wgrad_epilogue<C::STG_BUFS>(taddr, eh, 2, 256, &pw.out[pr], nt * 256,
                                     g * pw.M[pr] + mt * 256 + (int)rank * 128 + q * 32, my_stg,
-                                    n_red, lane);
+                                    n_red, lane, pw.overwrite != 0, false);
       }
       tc_fence_before();
       __syncwarp();

@@ -551,7 +551,8 @@ BwLayout bw_layout(const moe_config &c, int T) {
 
 moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
                        int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
-                       float *dw_down, void *ws, cudaStream_t st, const float *saved);
+                       float *dw_down, void *ws, cudaStream_t st, const float *saved,
+                       bool overwrite);
 moe_status backward_f32(const moe_layer *L, const float *x, const float *dout, int T, float *dx,
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down, void *ws,
                         cudaStream_t st);
@@ -700,15 +701,30 @@ size_t moe_backward_workspace_size(moe_handle h, int n_tokens) {
 }
 
 static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, const void *dout,
-                                 const float *saved, float *dx, float *dw_router,
-                                 float *dw_gate, float *dw_up, float *dw_down, void *ws,
-                                 size_t ws_bytes, void *stream);
+                                 const float *saved, bool overwrite, float *dx,
+                                 float *dw_router, float *dw_gate, float *dw_up,
+                                 float *dw_down, void *ws, size_t ws_bytes, void *stream);
 
 moe_status moe_backward(moe_handle h, const void *x, int n_tokens, const void *dout, float *dx,
                         float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
                         void *ws, size_t ws_bytes, void *stream) {
-  return backward_entry(h, x, n_tokens, dout, nullptr, dx, dw_router, dw_gate, dw_up, dw_down,
-                        ws, ws_bytes, stream);
+  return backward_entry(h, x, n_tokens, dout, nullptr, false, dx, dw_router, dw_gate, dw_up,
+                        dw_down, ws, ws_bytes, stream);
+}
+
+moe_status moe_backward_ex(moe_handle h, const void *x, int n_tokens, const void *dout,
+                           const float *saved, size_t saved_bytes, unsigned flags, float *dx,
+                           float *dw_router, float *dw_gate, float *dw_up, float *dw_down,
+                           void *ws, size_t ws_bytes, void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)MOE_BACKWARD_OVERWRITE) return MOE_ERR_INVALID_ARG;
+  if (saved) {
+    if (h->cfg.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (n_tokens > 0 && saved_bytes < moe_saved_size(h, n_tokens)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(saved)) return MOE_ERR_ALIGNMENT;
+  }
+  return backward_entry(h, x, n_tokens, dout, saved, (flags & MOE_BACKWARD_OVERWRITE) != 0, dx,
+                        dw_router, dw_gate, dw_up, dw_down, ws, ws_bytes, stream);
 }
 
 moe_status moe_backward_saved(moe_handle h, const void *x, int n_tokens, const void *dout,
@@ -717,17 +733,15 @@ moe_status moe_backward_saved(moe_handle h, const void *x, int n_tokens, const v
                               void *ws, size_t ws_bytes, void *stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (h->cfg.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  if (n_tokens > 0 && (!saved || saved_bytes < moe_saved_size(h, n_tokens)))
-    return MOE_ERR_INVALID_ARG;
-  if (saved && !aligned16(saved)) return MOE_ERR_ALIGNMENT;
-  return backward_entry(h, x, n_tokens, dout, saved, dx, dw_router, dw_gate, dw_up, dw_down, ws,
-                        ws_bytes, stream);
+  if (n_tokens > 0 && !saved) return MOE_ERR_INVALID_ARG;
+  return moe_backward_ex(h, x, n_tokens, dout, saved, saved_bytes, 0u, dx, dw_router, dw_gate,
+                         dw_up, dw_down, ws, ws_bytes, stream);
 }
 
 static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, const void *dout,
-                                 const float *saved, float *dx, float *dw_router,
-                                 float *dw_gate, float *dw_up, float *dw_down, void *ws,
-                                 size_t ws_bytes, void *stream) {
+                                 const float *saved, bool overwrite, float *dx,
+                                 float *dw_router, float *dw_gate, float *dw_up,
+                                 float *dw_down, void *ws, size_t ws_bytes, void *stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
   if (n_tokens == 0) return MOE_OK;
@@ -743,7 +757,16 @@ static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, cons
   if (h->cfg.dtype == MOE_BF16)
     return backward_tc(h, static_cast<const __nv_bfloat16 *>(x),
                        static_cast<const __nv_bfloat16 *>(dout), n_tokens, dx, dw_router, dw_gate,
-                       dw_up, dw_down, ws, st, saved);
+                       dw_up, dw_down, ws, st, saved, overwrite);
+  if (overwrite) {  // fp32 layer: clear, then accumulate
+    const moe_config &c = h->cfg;
+    const size_t G = (size_t)c.n_experts + c.n_shared, fd = (size_t)c.d_ff * c.d_model;
+    if (cudaMemsetAsync(dw_router, 0, (size_t)c.n_experts * c.d_model * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(dw_gate, 0, G * fd * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(dw_up, 0, G * fd * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(dw_down, 0, G * fd * 4, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   return backward_f32(h, static_cast<const float *>(x), static_cast<const float *>(dout),
                       n_tokens, dx, dw_router, dw_gate, dw_up, dw_down, ws, st);
 }
@@ -1335,8 +1358,8 @@ moe_status backward_rows(const moe_layer *L, const T_ *x, const T_ *dout, int T,
   if ((s = launch(bw_router_dl_kernel, dim3(grid_for(T, 256, L->num_sms)), dim3(256), 0, st,
                   (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
       (s = launch(bw_router_dw_kernel<T_>, dim3(E, cdiv(d, 512)), dim3(256), 0, st, x,
-                  (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
-                  dw_router)) != MOE_OK)
+                  (const float *)dl, (const int *)perm, (const int *)offsets, k, d, dw_router,
+                  0)) != MOE_OK)
     return s;
   return launch(bw_dx_kernel<T_>, dim3(grid_for((size_t)T * d / 4, 256, L->num_sms)), dim3(256),
                 0, st, (const float *)wide, (const int *)slot_row, (const int *)idx,
@@ -1420,7 +1443,8 @@ moe_status launch_bw_wgrad_pair(const moe_layer *L, const BwWgradParams &p, cuda
 //   and dx.
 moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bfloat16 *dout,
                        int T, float *dx, float *dw_router, float *dw_gate, float *dw_up,
-                       float *dw_down, void *ws, cudaStream_t st, const float *saved) {
+                       float *dw_down, void *ws, cudaStream_t st, const float *saved,
+                       bool overwrite) {
   const moe_config &c = L->cfg;
   const int E = c.n_experts, G = E + c.n_shared, k = c.top_k, d = c.d_model, f = c.d_ff;
   const int Tk = T * k, P = Tk + c.n_shared * T;
@@ -1527,6 +1551,7 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
   pw.status = status;
   pw.n_groups = G;
   pw.sched = &status->sched[3];
+  pw.overwrite = overwrite ? 1 : 0;
   // CTA pairs (256 x 256 tiles) when the groups' K loops are long enough for their operand
   // traffic to matter; decode-sized groups (a row or two each) are bound by the gradient
   // read-modify-write, where the one-CTA kernel's shorter per-unit path is faster
@@ -1552,7 +1577,7 @@ moe_status backward_tc(const moe_layer *L, const __nv_bfloat16 *x, const __nv_bf
                   (const float *)gate, (const float *)dgate, T, k, dl)) != MOE_OK ||
       (s = launch(bw_router_dw_kernel<__nv_bfloat16>, dim3(E, (d + 511) / 512), dim3(256), 0,
                   st, x, (const float *)dl, (const int *)perm, (const int *)offsets, k, d,
-                  dw_router)) != MOE_OK)
+                  dw_router, overwrite ? 1 : 0)) != MOE_OK)
     return s;
   return launch(bw_dx_kernel<__nv_bfloat16>, dim3(grid_for((size_t)T * d / 4, 256, L->num_sms)),
                 dim3(256), 0, st, (const float *)wide, (const int *)slot_row, (const int *)idx,

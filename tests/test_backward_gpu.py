@@ -117,3 +117,41 @@ def test_training_pair_matches_forward_and_backward(cuda_ok, kw):
         err = (g[name] - ref).abs().max().item()
         assert err <= 1e-5 * ref.abs().max().item() + 1e-30, (name, err)
     assert layer.device_status() == 0
+
+
+@pytest.mark.parametrize("kw", [
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 128},             # 1-CTA, unchosen
+    {"dtype": "bf16", "T": 40, "d": 256, "E": 16, "k": 4, "f": 256},             # 1-CTA 128 x 256
+    {"dtype": "bf16", "T": 300, "d": 256, "E": 8, "k": 4, "f": 512, "seed": 10,  # fused pair tail,
+     "bias": "zipf"},                                                              # empty experts
+    {"dtype": "bf16", "T": 90, "d": 128, "E": 24, "k": 3, "f": 128, "bias": "zipf",
+     "n_shared": 0},
+    {"dtype": "f32"},
+])
+def test_backward_overwrite_sets_gradients(cuda_ok, kw):
+    """MOE_BACKWARD_OVERWRITE sets the weight gradients (whatever the buffers held, NaN here)
+    to exactly what an accumulating call adds to zeros, zeros for unchosen experts; with the
+    kept pre-activations as well."""
+    w = synth.WORKLOADS["tiny_fp32"].replace(**kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    dout = synth.make_x(w, w.T, device="cuda", seed=79)
+    ref = layer.backward(inp.x, dout)
+    torch.cuda.synchronize()
+    names = ("dw_router", "dw_gate", "dw_up", "dw_down")
+    runs = [None]
+    if w.dtype == "bf16":
+        runs.append(layer.forward_save(inp.x)[1])
+    for saved in runs:
+        grads = {n: torch.full_like(ref[n], float("nan")) for n in names}
+        g = layer.backward(inp.x, dout, grads=grads, saved=saved, overwrite=True)
+        torch.cuda.synchronize()
+        for n in names:
+            if saved is None:
+                assert torch.equal(g[n], ref[n]), n
+            else:  # as the saved-activation backward: within the recompute's rounding
+                assert not torch.isnan(g[n]).any(), n
+                err = (g[n] - ref[n]).abs().max().item()
+                assert err <= 1e-5 * ref[n].abs().max().item() + 1e-30, (n, err)
+        assert torch.equal(g["dx"], ref["dx"]) or saved is not None
+    assert layer.device_status() == 0
