@@ -181,6 +181,10 @@ def test_backward_rejects_bad_arguments(cuda_ok):
     dx_big = torch.zeros(T * d + 4, device="cuda")
     with pytest.raises(MoEError):
         call(dx=dx_big[1:1 + T * d].view(T, d))      # dx not 16-byte aligned
+    from sparse_moe_layer_warp_b200 import moe_backward_ex
+    with pytest.raises(MoEError):                   # unknown flag bits
+        moe_backward_ex(layer.handle, inp.x, T, dout, None, 2, g["dx"], g["dwr"], g["dwg"],
+                        g["dwu"], g["dwd"], ws)
     call()                                          # the valid call still works
     torch.cuda.synchronize()
     assert layer.device_status() == 0
