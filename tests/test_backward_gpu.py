@@ -17,15 +17,19 @@ CASES = [
     {"dtype": "bf16", "T": 90, "d": 128, "E": 24, "k": 3, "f": 128, "bias": "zipf",
      "n_shared": 0},                                                               # empty experts
     {"dtype": "bf16", "T": 400, "d": 128, "E": 8, "k": 4, "f": 128, "seed": 5},   # 256-row tiles
-    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 256, "seed": 6},   # pair wgrad,
-    {"dtype": "bf16", "T": 75, "d": 512, "E": 12, "k": 2, "f": 256, "seed": 7,    # small groups
+    {"dtype": "bf16", "T": 16, "d": 256, "E": 64, "k": 8, "f": 256, "seed": 6},   # 1-CTA 128x256
+    {"dtype": "bf16", "T": 75, "d": 512, "E": 12, "k": 2, "f": 256, "seed": 7,    # small groups,
      "routed_scale": 0.5},                                                       # ragged 16-row pads
     {"dtype": "bf16", "T": 200, "d": 256, "E": 16, "k": 4, "f": 256, "seed": 8,   # pair wgrad,
      "bias": "zipf"},                                                               # skewed groups
     {"dtype": "bf16", "T": 256, "d": 256, "E": 8, "k": 4, "f": 256, "seed": 9},   # pair dgrad
     {"dtype": "bf16", "T": 300, "d": 256, "E": 8, "k": 4, "f": 512, "seed": 10,   # pair dgrad,
      "bias": "zipf", "routed_scale": 1.5},                                          # skewed
+    {"dtype": "bf16", "T": 1, "d": 256, "E": 16, "k": 4, "f": 128, "seed": 11},   # one token
+    {"dtype": "bf16", "T": 17, "d": 128, "E": 8, "k": 2, "f": 128, "seed": 12,    # odd T, no
+     "n_shared": 0},                                                               # shared expert
     {"dtype": "f32"},
+    {"dtype": "f32", "T": 3, "seed": 13},
 ]
 
 
