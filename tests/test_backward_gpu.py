@@ -30,6 +30,7 @@ CASES = [
      "n_shared": 0},                                                               # shared expert
     {"dtype": "f32"},
     {"dtype": "f32", "T": 3, "seed": 13},
+    {"dtype": "f32", "T": 100, "seed": 14},                                       # chunked routing
 ]
 
 
