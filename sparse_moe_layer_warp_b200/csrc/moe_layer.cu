@@ -8,6 +8,12 @@
 //         (small token tiles: the up GEMM gathers the rows of x itself)
 //   fp32: SIMT up+SwiGLU -> SIMT down                                    (expert_simt.cuh)
 //   -> gate-weighted combine                                             (expert_simt.cuh)
+// (decode-sized batches: routing in one launch; large groups: CTA-pair GEMMs,
+// grouped_gemm_pair.cuh).  One call of moe_backward (bf16) launches:
+//   the forward's routing -> row bookkeeping, padded offsets, padded sorted rows
+//   -> [up GEMM recompute of a, b] -> DH -> dgate -> DX + weight gradients (one launch on
+//   CTA pairs, or two) -> router dl, dW_r -> dx                        (grouped_gemm_bw.cuh)
+// and the fp32 layer's backward runs the CUDA-core row kernels of backward.cuh.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
