@@ -586,10 +586,17 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) {
     int tot = 0, pre = 0;
-    for (int cc = 0; cc < n_chunks; ++cc) {
-      const int v = chunk_hist[(size_t)cc * E + e];
-      tot += v;
-      pre += (cc < c) ? v : 0;
+    // 16 chunk counts loaded before they are summed: independent L2 loads in flight
+    for (int cc0 = 0; cc0 < n_chunks; cc0 += 16) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        v[u] = (cc0 + u < n_chunks) ? chunk_hist[(size_t)(cc0 + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        tot += v[u];
+        pre += (cc0 + u < c) ? v[u] : 0;
+      }
     }
     s_tot[e] = tot;
     s_base[e] = pre;
