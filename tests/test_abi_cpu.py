@@ -64,3 +64,16 @@ def test_null_handle_calls_rejected(lib):
     assert lib.moe_forward(None, None, 16, None, None, 0, None) == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_destroy(None) == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_route(None, None, 1, None, None, None, None, None, None, None, None, 0, None) == binding.MOE_ERR_INVALID_ARG
+    # backward and training-pair entry points
+    assert lib.moe_backward_workspace_size(None, 16) == 0
+    assert lib.moe_saved_size(None, 16) == 0
+    assert lib.moe_backward(None, None, 1, None, None, None, None, None, None, None, 0,
+                            None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_backward_saved(None, None, 1, None, None, 0, None, None, None, None, None,
+                                  None, 0, None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_backward_ex(None, None, 1, None, None, 0, 0, None, None, None, None, None,
+                               None, 0, None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_save(None, None, 1, None, None, 0, None, 0,
+                                None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_health(None, 1, None, None, None, None, 0,
+                                 None) == binding.MOE_ERR_INVALID_ARG
