@@ -420,9 +420,12 @@ def run_reference(args, rank, world):
     import numpy as np
     import torch
 
-    from oracle import oracle_moe_forward, oracle_num_threads
+    from oracle import oracle_moe_forward, oracle_num_threads, oracle_set_num_threads
     from sparse_moe_layer_warp_b200 import synth
 
+    # rank 0 runs alone: every host core this process may use (torchrun sets
+    # OMP_NUM_THREADS=1 for each of its processes)
+    oracle_set_num_threads(len(os.sched_getaffinity(0)))
     w = synth.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = synth.make_inputs(w, device=dev)

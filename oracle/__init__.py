@@ -21,6 +21,7 @@ from .c_oracle import (  # noqa: F401
     oracle_expert_ffn,
     oracle_moe_forward,
     oracle_num_threads,
+    oracle_set_num_threads,
     oracle_router_stats,
     oracle_bias_update,
     oracle_expert_act_rms,

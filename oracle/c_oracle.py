@@ -43,6 +43,7 @@ def _load():
         lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
                                            ctypes.c_double, P, I, P, P, P, P, P]
         lib.oracle_num_threads.restype = I
+        lib.oracle_set_num_threads.argtypes = [I]
         lib.oracle_router_stats.argtypes = [P, P, I, I, I, I, P, P, P, P]
         lib.oracle_bias_update.argtypes = [P, I, I, ctypes.c_float, P]
         lib.oracle_expert_act_rms.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P]
@@ -72,6 +73,11 @@ def _as_input(a):
 
 def oracle_num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def oracle_set_num_threads(n: int) -> None:
+    """OpenMP threads for the following oracle calls (overrides OMP_NUM_THREADS)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def oracle_router_logits(x, w_r):

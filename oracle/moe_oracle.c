@@ -245,12 +245,17 @@ void oracle_moe_forward(const void *x, const void *w_r, const float *bias, const
   }
 }
 
-/* number of OpenMP threads the oracle runs with (1 when built without OpenMP) */
+/* number of OpenMP threads the oracle runs with (1 when built without OpenMP); the setter
+ * overrides OMP_NUM_THREADS (a launcher may have set it to 1 for every process) */
 #ifdef _OPENMP
 #include <omp.h>
 int oracle_num_threads(void) { return omp_get_max_threads(); }
+void oracle_set_num_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+}
 #else
 int oracle_num_threads(void) { return 1; }
+void oracle_set_num_threads(int n) { (void)n; }
 #endif
 
 /* ------------------------------------------------------------------------------------ */

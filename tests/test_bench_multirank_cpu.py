@@ -44,3 +44,29 @@ def test_single_rank_and_throughput():
     assert bench.max_over_ranks(3.5, 1, None) == 3.5
     # 2 replicas x 100 steps x 16 tokens in 50 ms
     assert bench.job_throughput(16, 100, 2, 50.0) == pytest.approx(64000.0)
+
+
+def test_reference_arm_under_torchrun_world2():
+    """`bench.py --impl reference` launched like the multi-GPU bench: rank 0 alone times the
+    oracle (on all the host cores it may use, despite torchrun's OMP_NUM_THREADS=1) and
+    prints the one JSON line; rank 1 exits 0 without work."""
+    import json
+    import subprocess
+
+    port = 29000 + os.getpid() % 500
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "2", "--warmup", "3",
+           "--workload", "tiny_fp32"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny_fp32"
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
+    assert d["cpu_baseline"]["value"] == d["value"] == d["e2e"]["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
