@@ -275,9 +275,13 @@ const char *moe_status_string(moe_status s);
  * allocator.  (No counterpart on the pages: this is a deployment convenience, not part of
  * the layer's method.)
  *
- * Computes logits_out[t, e] = x_t . W_r[e] (fp32, [n_tokens, E], row-major) with the same
- * split-K kernel and the same deterministic summation order as moe_route, so the values are
- * identical to moe_route's logits.  Its scratch (split partial sums and arrival counters)
+ * Computes logits_out[t, e] = x_t . W_r[e] (fp32, [n_tokens, E], row-major) with a split-K
+ * kernel in a fixed summation order (deterministic).  Where moe_route uses the same kernel
+ * (fp32 layers; bf16 layers with more than 288 experts or d_model > 8192) the values are
+ * identical to moe_route's logits; bf16 decode batches of moe_route go through its one-launch
+ * router, which sums in another fixed order, so there the two agree to fp32 rounding of the
+ * dot product (each within d_model * 2^-24 * sum_i |x_i w_i| of the exact value).
+ * Its scratch (split partial sums and arrival counters)
  * lives in a fixed 2 MiB buffer inside the library's own static device memory, which every
  * GPU that loads the library holds until the process exits.  Limits: 1 <= n_tokens <= 64 and
  * ceil(d_model / 256) * n_tokens * E * 4 bytes <= 2 MiB (for d_model = 4096, E = 288: up to
