@@ -1,0 +1,73 @@
+"""bench.py's work accounting (the numerators of every roofline fraction it reports), checked
+on the CPU against the closed forms of the layer's traffic and arithmetic:
+
+* bytes of one forward = the weights of every expert some token chose, plus the shared
+  expert's, each read once (gate + up + down = 3 d f elements), plus the router matrix, plus x
+  read and out written once;
+* flops = 2 (T k + T) 3 d f for the expert contractions (T k routed rows and T shared rows)
+  plus 2 T d E for the router.
+
+The expected values are written out from the shapes by hand, not from bench.py's formulas.
+"""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from sparse_moe_layer_warp_b200 import synth  # noqa: E402
+
+
+def _counts(E, touched, total):
+    c = np.zeros(E, dtype=np.int64)
+    c[:touched] = total // touched
+    c[0] += total - c.sum()
+    return c
+
+
+def test_decode_t16_bytes_and_flops():
+    w = synth.WORKLOADS["decode_t16"]  # T=16, d=4096, E=288, k=8, f=1280, bf16, 1 shared
+    a = bench.algorithmic(w, _counts(288, 104, 16 * 8), 16)
+    assert a["touched"] == 105
+    # 105 experts x 3 x 1280 x 4096 x 2 B, + W_r 288 x 4096 x 2 B, + x and out 2 x 16 x 4096 x 2 B
+    assert a["layer_bytes"] == 105 * 31_457_280 + 2_359_296 + 262_144 == 3_305_635_840
+    # (128 + 16) rows x 3 x 4096 x 1280 x 2, + 2 x 16 x 4096 x 288
+    assert a["layer_flops"] == 2 * 144 * 3 * 4096 * 1280 + 2 * 16 * 4096 * 288
+    # the up kernel: gate + up weights of the touched experts, its 144 operand rows of x,
+    # and the 144 x 1280 bf16 rows of h it writes
+    assert a["up_bytes"] == 105 * 2 * 1280 * 4096 * 2 + 144 * 4096 * 2 + 144 * 1280 * 2
+    # the down kernel: down weights, h read, fp32 y rows written
+    assert a["down_bytes"] == 105 * 4096 * 1280 * 2 + 144 * 1280 * 2 + 144 * 4096 * 4
+    assert a["up_flops"] + a["down_flops"] == 2 * 144 * 3 * 4096 * 1280
+
+
+def test_prefill_t8192_flops_match_the_ridge_arithmetic():
+    w = synth.WORKLOADS["prefill_t8192"]
+    a = bench.algorithmic(w, np.full(288, 8192 * 8 // 288 + 1), 8192)
+    assert a["touched"] == 289
+    assert a["layer_flops"] == pytest.approx(2.3386e12, rel=1e-4)  # 2.339 TFLOP
+    assert a["layer_bytes"] == pytest.approx(9.23e9, rel=2e-3)      # weights once + x + out
+    # arithmetic intensity on the measured ridge (about 251 flop/B on B200)
+    assert 240 < a["layer_flops"] / a["layer_bytes"] < 260
+
+
+def test_untouched_experts_cost_nothing_and_fp32_doubles_bytes():
+    w = synth.WORKLOADS["tiny_fp32"]  # T=64, d=256, E=16, k=2, f=64, fp32, 1 shared
+    a = bench.algorithmic(w, _counts(16, 3, 64 * 2), 64)
+    assert a["touched"] == 4
+    assert a["layer_bytes"] == 4 * 3 * 64 * 256 * 4 + 16 * 256 * 4 + 2 * 64 * 256 * 4
+    wb = w.replace(dtype="bf16")
+    b = bench.algorithmic(wb, _counts(16, 3, 64 * 2), 64)
+    assert a["layer_bytes"] == 2 * b["layer_bytes"]
+    assert a["layer_flops"] == b["layer_flops"]
+
+
+def test_dense_ffn_has_no_shared_rows():
+    w = synth.WORKLOADS["dense_ffn_t4096"]  # E=1, k=1, f=11264, no shared expert
+    a = bench.algorithmic(w, np.array([4096]), 4096)
+    assert a["touched"] == 1
+    assert a["layer_flops"] == 2 * 4096 * 3 * 4096 * 11264 + 2 * 4096 * 4096
+    assert a["layer_bytes"] == 3 * 11264 * 4096 * 2 + 4096 * 2 + 2 * 4096 * 4096 * 2
