@@ -118,8 +118,20 @@ def _check(fn: str, status: int) -> None:
         raise MoEError(fn, status)
 
 
+def _addr(t) -> int:
+    """Device address of a tensor handed to the C ABI.  The library reads and writes dense
+    row-major device memory through raw pointers, so a strided view or a host tensor is
+    refused here, before anything is launched."""
+    if not t.is_contiguous():
+        raise ValueError(f"the library takes contiguous (dense row-major) tensors; got shape "
+                         f"{tuple(t.shape)} with strides {tuple(t.stride())}")
+    if not t.is_cuda:
+        raise ValueError(f"the library takes CUDA tensors; got one on {t.device}")
+    return t.data_ptr()
+
+
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else ctypes.c_void_p(_addr(t))
 
 
 def _stream(stream):
@@ -130,8 +142,8 @@ def _stream(stream):
 # ------------------------------------------------------------------ C-ABI mirrors
 def moe_layer_init(cfg: moe_config, w_router, router_bias, w_gate, w_up, w_down):
     lib = load_library()
-    w = moe_weights(w_router.data_ptr(), None if router_bias is None else router_bias.data_ptr(),
-                    w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())
+    w = moe_weights(_addr(w_router), None if router_bias is None else _addr(router_bias),
+                    _addr(w_gate), _addr(w_up), _addr(w_down))
     h = ctypes.c_void_p()
     _check("moe_layer_init", lib.moe_layer_init(ctypes.byref(cfg), ctypes.byref(w),
                                                 ctypes.byref(h)))

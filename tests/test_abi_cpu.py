@@ -77,3 +77,22 @@ def test_null_handle_calls_rejected(lib):
                                 None) == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_health(None, 1, None, None, None, None, 0,
                                  None) == binding.MOE_ERR_INVALID_ARG
+
+
+def test_binding_refuses_strided_and_host_tensors(lib):
+    """The binding hands raw pointers to a library that reads dense device memory: a strided
+    view or a host tensor is refused in Python, before any library call or launch."""
+    import torch
+
+    strided = torch.zeros(8, 4).t()
+    with pytest.raises(ValueError, match="contiguous"):
+        binding._p(strided)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        binding._p(torch.zeros(8))
+    assert binding._p(None) is None
+    # the weights of a layer go through the same check
+    cfg = binding.moe_config(16, 256, 16, 2, 128, 1, binding.MOE_F32, 1.0)
+    w = [torch.zeros(16, 256), None, torch.zeros(17, 128, 256), torch.zeros(17, 128, 256),
+         torch.zeros(17, 256, 128)]
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        binding.moe_layer_init(cfg, *w)
