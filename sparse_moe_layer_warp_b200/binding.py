@@ -281,22 +281,46 @@ def moe_device_status(handle, ws, stream=None) -> int:
 
 
 # ------------------------------------------------------------------ convenience wrapper
+def _expect(t, shape, dtype, name):
+    """The C ABI sees only pointers: a tensor of another shape or type would be read or
+    written out of its bounds, so the class below checks every tensor it passes."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected shape {tuple(shape)} of {dtype}, got "
+                         f"{tuple(t.shape)} of {t.dtype}")
+
+
 class MoELayer:
     """Owns a handle and a workspace; holds references to the weight tensors."""
 
     def __init__(self, w_router, router_bias, w_gate, w_up, w_down, top_k: int,
                  max_tokens: int, n_shared: int = 1, routed_scale: float = 1.0):
-        dt = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32}[w_router.dtype]
+        if w_router.dtype not in (torch.bfloat16, torch.float32) or w_router.dim() != 2:
+            raise ValueError("w_router: expected a [E, d] bf16 or fp32 tensor")
+        dt = MOE_BF16 if w_router.dtype == torch.bfloat16 else MOE_F32
         E, d = w_router.shape
         f = w_gate.shape[1]
+        G = int(E) + int(n_shared)
+        _expect(w_gate, (G, f, d), w_router.dtype, "w_gate")
+        _expect(w_up, (G, f, d), w_router.dtype, "w_up")
+        _expect(w_down, (G, d, f), w_router.dtype, "w_down")
+        if router_bias is not None:
+            _expect(router_bias, (E,), torch.float32, "router_bias")
         self.cfg = moe_config(int(max_tokens), int(d), int(E), int(top_k), int(f),
                               int(n_shared), dt, float(routed_scale))
         self.tensors = (w_router, router_bias, w_gate, w_up, w_down)
         self.handle = moe_layer_init(self.cfg, *self.tensors)
         self.device = w_router.device
+        self.dtype = w_router.dtype
         self.ws = None
         self.bw_ws = None
         self.E, self.k, self.d = int(E), int(top_k), int(d)
+
+    def _rows(self, x, name="x"):
+        """Token count of a [T, d] activation of the layer's type."""
+        if x.dim() != 2:
+            raise ValueError(f"{name}: expected a [T, {self.d}] tensor, got {tuple(x.shape)}")
+        _expect(x, (x.shape[0], self.d), self.dtype, name)
+        return int(x.shape[0])
 
     def workspace(self, n_tokens: int):
         need = moe_workspace_size(self.handle, n_tokens)
@@ -306,13 +330,18 @@ class MoELayer:
         return self.ws
 
     def forward(self, x, out=None, stream=None):
-        T = x.shape[0]
+        T = self._rows(x)
         out = torch.empty_like(x) if out is None else out
+        _expect(out, x.shape, x.dtype, "out")
         moe_forward(self.handle, x, T, out, self.workspace(T), stream)
         return out
 
     def route(self, x=None, logits=None, want_logits=False, stream=None):
-        T = (x if x is not None else logits).shape[0]
+        if x is not None:
+            T = self._rows(x)
+        else:
+            T = int(logits.shape[0])
+            _expect(logits, (T, self.E), torch.float32, "logits")
         dev = self.device
         r = dict(
             idx=torch.empty((T, self.k), dtype=torch.int32, device=dev),
@@ -335,7 +364,9 @@ class MoELayer:
 
     def router_stats(self, logits, topk_idx, n_groups, stream=None):
         """p_mean [E], f_sel [E] and scalars [L_EP, routing confidence] (device tensors)."""
-        T = logits.shape[0]
+        T = int(logits.shape[0])
+        _expect(logits, (T, self.E), torch.float32, "logits")
+        _expect(topk_idx, (T, self.k), torch.int32, "topk_idx")
         p_mean = torch.empty(self.E, dtype=torch.float32, device=self.device)
         f_sel = torch.empty(self.E, dtype=torch.float32, device=self.device)
         scalars = torch.empty(2, dtype=torch.float32, device=self.device)
@@ -346,10 +377,11 @@ class MoELayer:
     def forward_save(self, x, out=None, saved=None, stream=None):
         """Training forward (bf16): (out, saved) with `saved` the fp32 pre-activations that
         backward(..., saved=saved) reads instead of recomputing them."""
-        T = x.shape[0]
+        T = self._rows(x)
         ws = self.workspace(T)
         if out is None:
             out = torch.empty_like(x)
+        _expect(out, x.shape, x.dtype, "out")
         if saved is None:
             saved = torch.empty(moe_saved_size(self.handle, T) // 4, dtype=torch.float32,
                                 device=self.device)
@@ -361,7 +393,8 @@ class MoELayer:
         weight gradients are added to `grads`' tensors when given (new zeroed ones if not),
         or set when `overwrite`.  With `saved` (from forward_save of the same x) the
         pre-activations are not recomputed."""
-        T = x.shape[0]
+        T = self._rows(x)
+        _expect(dout, x.shape, x.dtype, "dout")
         need = moe_backward_workspace_size(self.handle, T)
         if self.bw_ws is None or self.bw_ws.numel() < need:
             self.bw_ws = torch.empty(need, dtype=torch.uint8, device=self.device)
@@ -384,6 +417,9 @@ class MoELayer:
                      dw_gate=torch.zeros((G, f, self.d), **kw),
                      dw_up=torch.zeros((G, f, self.d), **kw),
                      dw_down=torch.zeros((G, self.d, f), **kw))
+        for name, shape in (("dw_router", (self.E, self.d)), ("dw_gate", (G, f, self.d)),
+                            ("dw_up", (G, f, self.d)), ("dw_down", (G, self.d, f))):
+            _expect(g[name], shape, torch.float32, name)
         if overwrite:
             moe_backward_ex(self.handle, x, T, dout, saved, MOE_BACKWARD_OVERWRITE, g["dx"],
                             g["dw_router"], g["dw_gate"], g["dw_up"], g["dw_down"], self.bw_ws,

@@ -96,3 +96,31 @@ def test_binding_refuses_strided_and_host_tensors(lib):
          torch.zeros(17, 256, 128)]
     with pytest.raises(ValueError, match="CUDA tensors"):
         binding.moe_layer_init(cfg, *w)
+
+
+def test_layer_class_checks_shapes_and_types(lib):
+    """MoELayer passes only pointers to the library, so it checks every weight's shape and
+    type against the configuration first (a mismatch would be read out of bounds)."""
+    import torch
+
+    E, d, f = 16, 256, 128
+    good = dict(w_router=torch.zeros(E, d), router_bias=torch.zeros(E),
+                w_gate=torch.zeros(E + 1, f, d), w_up=torch.zeros(E + 1, f, d),
+                w_down=torch.zeros(E + 1, d, f))
+    bad_cases = [
+        dict(w_gate=torch.zeros(E, f, d)),                    # no room for the shared expert
+        dict(w_up=torch.zeros(E + 1, f, d + 8)),              # wrong d
+        dict(w_down=torch.zeros(E + 1, f, d)),                # transposed down projection
+        dict(router_bias=torch.zeros(E, dtype=torch.float64)),
+        dict(w_up=torch.zeros(E + 1, f, d, dtype=torch.bfloat16)),  # mixed types
+        dict(w_router=torch.zeros(E, d, dtype=torch.float16)),
+    ]
+    for change in bad_cases:
+        kw = dict(good, **change)
+        with pytest.raises(ValueError):
+            binding.MoELayer(kw["w_router"], kw["router_bias"], kw["w_gate"], kw["w_up"],
+                             kw["w_down"], top_k=2, max_tokens=8)
+    # consistent shapes pass the Python checks and reach the pointer check (host tensors)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        binding.MoELayer(good["w_router"], good["router_bias"], good["w_gate"], good["w_up"],
+                         good["w_down"], top_k=2, max_tokens=8)
