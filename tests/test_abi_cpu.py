@@ -27,6 +27,18 @@ def test_header_and_binding_agree():
     assert _declared() == set(binding.EXPORTS)
 
 
+def test_header_constants_match_binding():
+    """Status codes, dtype codes, flags and the profile stage count are the header's values."""
+    text = open(os.path.join(ROOT, "include", "moe_layer.h")).read()
+    enums = dict((n, int(v)) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    defines = dict((n, int(v)) for n, v in
+                   re.findall(r"^#define\s+(MOE_[A-Z0-9_]+)\s+(\d+)u?\s*$", text, flags=re.M))
+    assert len(enums) == 9 and len(defines) == 2
+    for name, value in {**enums, **defines}.items():
+        assert getattr(binding, name) == value, name
+    assert len(binding.PROFILE_STAGE_NAMES) == binding.MOE_PROFILE_STAGES
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in _declared():
         assert hasattr(lib, name), name
