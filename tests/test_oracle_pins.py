@@ -16,6 +16,8 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from oracle import (oracle_expert_ffn, oracle_moe_forward, oracle_permute, oracle_route,
                     oracle_router_logits)
@@ -459,3 +461,30 @@ def test_sampled_backward_equals_full_backward(n_shared, rs, dtype):
     for name in ("dw_gate", "dw_up", "dw_down"):
         assert np.array_equal(got[name], full[name][exps]), name
     assert np.array_equal(got["dw_router"], full["dw_router"][rexps])
+
+
+# ------------------------------------------------------------ selection order, fuzzed
+_GRID = [float("nan"), float("inf"), float("-inf"), 0.0, -0.0, 0.5, -0.5, 1.0, 0.25, -2.0]
+
+
+@settings(max_examples=300, deadline=None)
+@given(st.data())
+def test_route_slot_order_equals_a_full_sort(data):
+    """Slot j holds the expert of rank j in one full sort of the biased scores: larger score
+    first, equal scores (-0.0 == +0.0) by lower id, NaN scores after every number (by id)."""
+    T = data.draw(st.integers(1, 5))
+    E = data.draw(st.integers(1, 20))
+    k = data.draw(st.integers(1, E))
+    vals = st.sampled_from(_GRID)
+    logits = np.array(data.draw(st.lists(vals, min_size=T * E, max_size=T * E)),
+                      dtype=np.float32).reshape(T, E)
+    bias = np.array(data.draw(st.lists(st.sampled_from([0.0, -0.0, 0.5, -0.25]),
+                                       min_size=E, max_size=E)), dtype=np.float32)
+    idx, _ = oracle_route(logits, bias, k)
+    s = logits + bias  # float32 add, as the selection rule states
+    for t in range(T):
+        def key(e):
+            v = float(s[t, e])
+            return (1, 0.0, e) if v != v else (0, -v, e)
+        want = sorted(range(E), key=key)[:k]
+        assert idx[t].tolist() == want, (logits[t], bias, k)
