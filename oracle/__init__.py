@@ -17,6 +17,7 @@ from .c_oracle import (  # noqa: F401
     build_oracle,
     oracle_router_logits,
     oracle_route,
+    oracle_gates,
     oracle_permute,
     oracle_expert_ffn,
     oracle_moe_forward,

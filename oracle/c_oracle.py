@@ -38,6 +38,7 @@ def _load():
         I = ctypes.c_int
         lib.oracle_router_logits.argtypes = [P, P, I, I, I, I, P]
         lib.oracle_route.argtypes = [P, P, I, I, I, P, P]
+        lib.oracle_gates.argtypes = [P, P, I, I, I, P]
         lib.oracle_permute.argtypes = [P, I, I, I, P, P, P, P]
         lib.oracle_expert_ffn.argtypes = [P, P, P, P, I, I, I, P]
         lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
@@ -99,6 +100,19 @@ def oracle_route(logits, bias, k):
     gates = np.empty((T, k), np.float32)
     _load().oracle_route(_ptr(logits), _ptr(bias), T, E, k, _ptr(idx), _ptr(gates))
     return idx, gates
+
+
+def oracle_gates(logits, idx):
+    """Gates [T, k] of a given selection idx [T, k] from fp32 logits [T, E]: softmax over
+    the selected unbiased logits (the same arithmetic oracle_route applies to its own)."""
+    logits = np.ascontiguousarray(logits, np.float32)
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, E = logits.shape
+    k = idx.shape[1]
+    assert idx.shape[0] == T and (idx >= 0).all() and (idx < E).all()
+    gates = np.empty((T, k), np.float32)
+    _load().oracle_gates(_ptr(logits), _ptr(idx), T, E, k, _ptr(gates))
+    return gates
 
 
 def oracle_permute(idx, E):

@@ -91,6 +91,21 @@ void oracle_router_logits(const void *x, const void *w_r, int dtype, int T, int 
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Gates of one token for a given selection sel[0..k): softmax over the k selected         */
+/* UNBIASED logits, max-shifted, in double, each rounded once to fp32.  [P2 2.2.2] p_{t,e} */
+/* renormalised over S_t; [P3 MoE] the bias takes no part in the gates.                    */
+static void orc_gates_of_selection(const float *l, const int *sel, int k, float *gates) {
+  double m = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    double v = (double)l[sel[j]];
+    if (v > m) m = v;
+  }
+  double z = 0.0;
+  for (int j = 0; j < k; ++j) z += exp((double)l[sel[j]] - m);
+  for (int j = 0; j < k; ++j) gates[j] = (float)(exp((double)l[sel[j]] - m) / z);
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Selection and gates for one token.                                                     */
 /* [P3 MoE] bias for selection only; [P2 2.2.2] S_t = top-K set; gates renormalised.       */
 static void orc_route_token(const float *l, const float *bias, int E, int k, int *idx,
@@ -112,18 +127,8 @@ static void orc_route_token(const float *l, const float *bias, int E, int k, int
     }
     order[b + 1] = cur;
   }
-  /* gates: softmax over the k selected unbiased logits (max-shifted), double */
-  double m = -INFINITY;
-  for (int j = 0; j < k; ++j) {
-    double v = (double)l[order[j]];
-    if (v > m) m = v;
-  }
-  double z = 0.0;
-  for (int j = 0; j < k; ++j) z += exp((double)l[order[j]] - m);
-  for (int j = 0; j < k; ++j) {
-    idx[j] = order[j];
-    gates[j] = (float)(exp((double)l[order[j]] - m) / z);
-  }
+  for (int j = 0; j < k; ++j) idx[j] = order[j];
+  orc_gates_of_selection(l, idx, k, gates);
   free(s);
   free(order);
 }
@@ -134,6 +139,15 @@ void oracle_route(const float *logits, const float *bias, int T, int E, int k, i
   for (int t = 0; t < T; ++t)
     orc_route_token(logits + (size_t)t * E, bias, E, k, idx + (size_t)t * k,
                     gates + (size_t)t * k);
+}
+
+/* Gates for a selection made elsewhere (e.g. the GPU's idx), from these logits: the same */
+/* softmax as oracle_route applies to its own selection.                                   */
+void oracle_gates(const float *logits, const int *idx, int T, int E, int k, float *gates) {
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t)
+    orc_gates_of_selection(logits + (size_t)t * E, idx + (size_t)t * k, k,
+                           gates + (size_t)t * k);
 }
 
 /* ------------------------------------------------------------------------------------ */

@@ -78,6 +78,31 @@ def test_topk_matches_torch_topk_without_ties():
     np.testing.assert_allclose(gates, ref_g, rtol=1e-6, atol=0)
 
 
+def test_gates_of_a_given_selection():
+    """oracle_gates (gates of a selection made elsewhere) against torch.softmax over the
+    selected unbiased logits, in any slot order, with repeated ids allowed by the softmax
+    definition; and exactly oracle_route's gates on oracle_route's own selection."""
+    from oracle import oracle_gates
+
+    logits = synth.make_logits(120, 288, seed=11).numpy()
+    bias = synth.make_bias(synth.WORKLOADS["skew_t4096"], torch.Generator().manual_seed(2),
+                           "cpu").numpy()
+    idx, gates = oracle_route(logits, bias, 8)
+    assert np.array_equal(oracle_gates(logits, idx), gates)
+    rng = np.random.default_rng(4)
+    sel = np.stack([rng.choice(288, 8, replace=False) for _ in range(120)]).astype(np.int32)
+    got = oracle_gates(logits, sel)
+    lg = np.take_along_axis(logits, sel.astype(np.int64), axis=1)
+    ref = torch.softmax(torch.from_numpy(lg).double(), dim=1).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-6, atol=0)
+    # permuting the slots permutes the gates
+    rev = np.ascontiguousarray(sel[:, ::-1])
+    assert np.array_equal(oracle_gates(logits, rev), got[:, ::-1])
+    # the bias does not enter: two selections with equal logits get equal gates
+    two = np.zeros((1, 4), np.float32)
+    assert (oracle_gates(two, np.array([[0, 3]], np.int32)) == 0.5).all()
+
+
 def test_gates_k_equals_E_zero_bias_is_full_softmax():
     logits = synth.make_logits(40, 16, seed=5).numpy()
     idx, gates = oracle_route(logits, np.zeros(16, np.float32), 16)
