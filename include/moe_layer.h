@@ -96,6 +96,32 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
 /* Releases the host-side handle.  Does not touch any device buffer. */
 moe_status moe_layer_destroy(moe_handle h);
 
+/* Launch-plan options of a handle (host only; takes effect from the next call):
+ *   MOE_OPTION_H_HANDOVER  1 (default): the bf16 forward's down-projection GEMM starts while
+ *                          the up GEMM still runs and takes each expert group's h as soon as
+ *                          that group's up units have stored it (per-group completion counts
+ *                          in the workspace) -- used only when the init-time occupancy check
+ *                          finds every persistent up grid co-resident on the device;
+ *                          0: the down GEMM waits for the whole up GEMM (same results, bit
+ *                          for bit; for callers that share the GPU's SMs with other
+ *                          persistent work and want no cross-kernel waiting at all).
+ *   MOE_OPTION_SHARED_SIDE_SMS  n >= 2: in bf16 forwards on CTA pairs (about 96 or more
+ *                          tokens per expert), the shared expert -- which needs no routing --
+ *                          runs its up and down GEMMs on a stream of the handle on n SMs
+ *                          (rounded down to whole pairs) while the caller's stream routes the
+ *                          tokens; the caller's stream waits for it (an event) before the
+ *                          combine, so the call stays asynchronous on `stream` and the results
+ *                          are the same bit for bit.  0 (default): everything on `stream`.
+ *                          The first non-zero value creates the stream and two events on the
+ *                          handle's device (make it before capturing a CUDA graph; a captured
+ *                          forward records the fork and join into the graph).  Calls on one
+ *                          handle from several host threads at once are not supported.
+ *                          Not used by moe_forward_profiled or moe_forward_save.
+ * MOE_ERR_INVALID_ARG for an unknown option or value. */
+#define MOE_OPTION_H_HANDOVER 1
+#define MOE_OPTION_SHARED_SIDE_SMS 2
+moe_status moe_set_option(moe_handle h, int option, int value);
+
 /* Bytes of device workspace a call with n_tokens tokens needs (0 on bad arguments).
  * The workspace holds the routing scratch, the expert-sorted activations, the SwiGLU
  * outputs h and the per-row expert outputs y between the kernels of one call. */
@@ -265,6 +291,82 @@ moe_status moe_router_stats(moe_handle h, const float *logits, const int *topk_i
 moe_status moe_update_router_bias(moe_handle h, const int *expert_counts, int n_tokens,
                                   float gamma, float *bias, void *stream);
 
+/* ------------------------------------------------------------------ expert parallelism
+ * The layer split by experts over R ranks ("Step 3.5 Flash: Open Frontier-Level Intelligence
+ * with 11B Active Parameters", section 3: the MoE layers run expert-parallel, EP8 within a
+ * node over NVLink / NVSwitch; section 2.2.2: the routed experts form G EP groups whose load
+ * the EP-group balance loss evens out).  Rank q holds EP group q, the E / R consecutive
+ * routed experts [q E / R, (q + 1) E / R) (the grouping moe_router_stats uses), plus the
+ * shared expert, and the full router: every rank routes its own tokens over all E experts.
+ * The exchanges themselves (all-to-all, all-gather, reduce-scatter) are the caller's (the
+ * Python package's expert_parallel module runs them over torch.distributed); these calls
+ * are the device steps around them.  bf16 layers only.
+ *
+ * moe_layer_init_ep: a handle over the routed experts [expert_begin, expert_end) of a layer
+ * of cfg->n_experts experts.  w->w_router [E, d] and router_bias [E] are the whole router;
+ * w_gate, w_up [(expert_end - expert_begin) + n_shared, f, d] and w_down [.., d, f] hold
+ * those experts in order, then the shared expert.  Such a handle routes (moe_route,
+ * moe_route_from_logits, moe_router_stats) and runs moe_forward_partial within its range;
+ * the whole-layer calls (moe_forward, the backward, moe_expert_health) return
+ * MOE_ERR_UNSUPPORTED on it.  moe_layer_init's handle holds [0, E). */
+moe_status moe_layer_init_ep(const moe_config *cfg, const moe_weights *w, int expert_begin,
+                             int expert_end, moe_handle *out);
+
+/* Part of the layer for n_tokens tokens, unrounded fp32:
+ *   out[t] = routed_scale * sum over slots j of t with expert_begin <= idx[t,j] < expert_end
+ *            of gate[t,j] FFN_{idx[t,j]}(x_t)
+ *          + FFN_shared(x_t) if shared_begin <= t < shared_end (else nothing)
+ * with the slots summed in j order and the shared expert last, in fp32.  The selection is
+ * topk_idx / topk_gate [n_tokens, k] (device; global expert ids, e.g. routed on another
+ * rank; ids outside [0, E) contribute nothing), or, with both null, the layer's own routing
+ * of x.  [expert_begin, expert_end) must lie in the handle's experts (it may be empty:
+ * shared expert only).  Summing the outputs of calls whose expert ranges partition [0, E)
+ * and whose shared ranges partition the tokens gives the layer output before its rounding.
+ * A given selection must name distinct experts within each token (as the router's does).
+ * out [n_tokens, d] fp32, 16-byte aligned; ws as for moe_forward.  MOE_ERR_UNSUPPORTED for
+ * the fp32 layer. */
+moe_status moe_forward_partial(moe_handle h, const void *x, int n_tokens, const int *topk_idx,
+                               const float *topk_gate, int expert_begin, int expert_end,
+                               int shared_begin, int shared_end, float *out, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* Dispatch plan of an all-to-all exchange over n_ranks ranks (E % n_ranks == 0, at most 512
+ * ranks) from the tokens' selections topk_idx [n_tokens, k]: token t goes once to every rank
+ * q that holds one of its experts.  The (token, rank) pairs are sorted by bucket, ascending
+ * token within a bucket: bucket q holds the tokens sent to rank q, bucket n_ranks + q the
+ * tokens that send nothing to rank q.  Outputs (device int32):
+ *   send_counts  [2 n_ranks]    tokens per bucket: entry q = rows sent to rank q
+ *   send_offsets [2 n_ranks + 1] exclusive prefix of send_counts: rank q's rows of the send
+ *                               buffer are [send_offsets[q], send_offsets[q + 1])
+ *   send_perm    [n_tokens * n_ranks]  row r of the send buffer carries pair send_perm[r]
+ *                               = t * n_ranks + q (the first send_offsets[n_ranks] rows)
+ *   send_slot    [n_tokens * n_ranks]  inverse: row of pair (t, q), >= send_offsets[n_ranks]
+ *                               when t sends nothing to q
+ * Deterministic (no atomic decides a position).  Uses the workspace of
+ * moe_workspace_size(h, n_tokens). */
+moe_status moe_ep_plan(moe_handle h, const int *topk_idx, int n_tokens, int n_ranks,
+                       int *send_counts, int *send_offsets, int *send_perm, int *send_slot,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Send buffer of the plan: row r < send_offsets[n_ranks] gets token t = send_perm[r] /
+ * n_ranks: x_send[r] = x[t] (layer dtype, [rows, d], 16-byte aligned), idx_send[r] =
+ * topk_idx[t], gate_send[r] = topk_gate[t] ([rows, k]).  The buffers need room for
+ * n_tokens * n_ranks rows (the largest possible send); rows past the send are not written. */
+moe_status moe_ep_pack(moe_handle h, const void *x, const int *topk_idx, const float *topk_gate,
+                       int n_tokens, int n_ranks, const int *send_perm, const int *send_offsets,
+                       void *x_send, int *idx_send, float *gate_send, void *stream);
+
+/* Output of the rank's own tokens:
+ *   out[t] = round( sum_{q = 0 .. n_ranks - 1, t sent to q} back[send_slot[t n_ranks + q]]
+ *                   + shared[t] )
+ * in fp32 in this order, one rounding to the layer dtype.  back: the fp32 partial rows the
+ * ranks returned, in the send buffer's row order ([send_offsets[n_ranks], d]; null: none,
+ * send_slot and send_offsets unused); shared: fp32 [n_tokens, d] (e.g. the shared expert's
+ * moe_forward_partial, or a reduce-scattered sum of partials; null: none). */
+moe_status moe_ep_combine(moe_handle h, const float *back, const int *send_slot,
+                          const int *send_offsets, const float *shared, int n_tokens,
+                          int n_ranks, void *out, void *stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 
@@ -287,7 +389,10 @@ const char *moe_status_string(moe_status s);
  * ceil(d_model / 256) * n_tokens * E * 4 bytes <= 2 MiB (for d_model = 4096, E = 288: up to
  * 64 tokens); larger requests return MOE_ERR_UNSUPPORTED before anything is launched.
  * The first call on each device looks up the buffer's device address (host-side set-up), so
- * make that first call before capturing a stream into a CUDA graph.  All calls on a device
+ * make that first call before capturing a stream into a CUDA graph.  The address is kept for
+ * the life of the process: do not use the library across a device reset
+ * (cudaDeviceReset), which may move the buffer.  The current device must be the one the
+ * handle was created on (MOE_ERR_INVALID_ARG otherwise).  All calls on a device
  * share the one buffer: calls that may overlap on the GPU (different streams without
  * ordering) race and give wrong results; serialise them.  Asynchronous on `stream`. */
 moe_status moe_router_logits_static(moe_handle h, const void *x, int n_tokens,

@@ -32,8 +32,11 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_router_stats", "moe_update_router_bias", "moe_forward_launch_count",
            "moe_selftest_wait_timeout", "moe_expert_health", "moe_backward",
            "moe_backward_workspace_size", "moe_saved_size", "moe_forward_save",
-           "moe_backward_saved", "moe_backward_ex")
+           "moe_backward_saved", "moe_backward_ex", "moe_set_option", "moe_layer_init_ep",
+           "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine")
 MOE_BACKWARD_OVERWRITE = 1
+MOE_OPTION_H_HANDOVER = 1
+MOE_OPTION_SHARED_SIDE_SMS = 2
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -94,6 +97,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_forward_save.argtypes = [P, P, I, P, P, Z, P, Z, P]
         lib.moe_backward_saved.argtypes = [P, P, I, P, P, Z, P, P, P, P, P, P, Z, P]
         lib.moe_backward_ex.argtypes = [P, P, I, P, P, Z, ctypes.c_uint, P, P, P, P, P, P, Z, P]
+        lib.moe_set_option.argtypes = [P, I, I]
+        lib.moe_layer_init_ep.argtypes = [ctypes.POINTER(moe_config),
+                                          ctypes.POINTER(moe_weights), I, I, ctypes.POINTER(P)]
+        lib.moe_forward_partial.argtypes = [P, P, I, P, P, I, I, I, I, P, P, Z, P]
+        lib.moe_ep_plan.argtypes = [P, P, I, I, P, P, P, P, P, Z, P]
+        lib.moe_ep_pack.argtypes = [P, P, P, P, I, I, P, P, P, P, P, P]
+        lib.moe_ep_combine.argtypes = [P, P, P, P, P, I, I, P, P]
         lib.moe_forward_launch_count.argtypes = [P, I]
         lib.moe_forward_launch_count.restype = I
         lib.moe_status_string.argtypes = [I]
@@ -103,7 +113,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                      "moe_device_status", "moe_router_logits_static", "moe_router_stats",
                      "moe_update_router_bias", "moe_selftest_wait_timeout",
                      "moe_expert_health", "moe_backward", "moe_forward_save",
-                     "moe_backward_saved", "moe_backward_ex"):
+                     "moe_backward_saved", "moe_backward_ex", "moe_set_option", "moe_layer_init_ep",
+           "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -150,8 +161,57 @@ def moe_layer_init(cfg: moe_config, w_router, router_bias, w_gate, w_up, w_down)
     return h
 
 
+def moe_layer_init_ep(cfg: moe_config, expert_begin: int, expert_end: int, w_router,
+                      router_bias, w_gate, w_up, w_down):
+    """Handle over the routed experts [expert_begin, expert_end) of a bf16 layer (weights:
+    those experts then the shared expert; the full router)."""
+    lib = load_library()
+    w = moe_weights(_addr(w_router), None if router_bias is None else _addr(router_bias),
+                    _addr(w_gate), _addr(w_up), _addr(w_down))
+    h = ctypes.c_void_p()
+    _check("moe_layer_init_ep", lib.moe_layer_init_ep(ctypes.byref(cfg), ctypes.byref(w),
+                                                      int(expert_begin), int(expert_end),
+                                                      ctypes.byref(h)))
+    return h
+
+
+def moe_forward_partial(handle, x, n_tokens, topk_idx, topk_gate, expert_begin, expert_end,
+                        shared_begin, shared_end, out, ws, stream=None) -> None:
+    """fp32 partial output of an expert range (see include/moe_layer.h)."""
+    _check("moe_forward_partial", load_library().moe_forward_partial(
+        handle, _p(x), int(n_tokens), _p(topk_idx), _p(topk_gate), int(expert_begin),
+        int(expert_end), int(shared_begin), int(shared_end), _p(out), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_ep_plan(handle, topk_idx, n_tokens, n_ranks, send_counts, send_offsets, send_perm,
+                send_slot, ws, stream=None) -> None:
+    _check("moe_ep_plan", load_library().moe_ep_plan(
+        handle, _p(topk_idx), int(n_tokens), int(n_ranks), _p(send_counts), _p(send_offsets),
+        _p(send_perm), _p(send_slot), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_ep_pack(handle, x, topk_idx, topk_gate, n_tokens, n_ranks, send_perm, send_offsets,
+                x_send, idx_send, gate_send, stream=None) -> None:
+    _check("moe_ep_pack", load_library().moe_ep_pack(
+        handle, _p(x), _p(topk_idx), _p(topk_gate), int(n_tokens), int(n_ranks), _p(send_perm),
+        _p(send_offsets), _p(x_send), _p(idx_send), _p(gate_send), _stream(stream)))
+
+
+def moe_ep_combine(handle, back, send_slot, send_offsets, shared, n_tokens, n_ranks, out,
+                   stream=None) -> None:
+    _check("moe_ep_combine", load_library().moe_ep_combine(
+        handle, _p(back), _p(send_slot), _p(send_offsets), _p(shared), int(n_tokens),
+        int(n_ranks), _p(out), _stream(stream)))
+
+
 def moe_layer_destroy(handle) -> None:
     _check("moe_layer_destroy", load_library().moe_layer_destroy(handle))
+
+
+def moe_set_option(handle, option: int, value: int) -> None:
+    """Launch-plan option of a handle (MOE_OPTION_H_HANDOVER; see include/moe_layer.h)."""
+    _check("moe_set_option", load_library().moe_set_option(handle, int(option), int(value)))
 
 
 def moe_workspace_size(handle, n_tokens: int) -> int:
@@ -256,9 +316,21 @@ def moe_forward_profiled(handle, x, n_tokens, out, ws, events, stream=None) -> N
         _stream(stream), arr, len(events)))
 
 
-def moe_router_logits_static(handle, x, n_tokens, logits_out, stream=None) -> None:
+def moe_router_logits_static(handle, x, n_tokens, logits_out, stream=None, *, d_model=None,
+                             n_experts=None, dtype=None) -> None:
     """Router logits with the library's own static scratch (no workspace argument), for
-    callers that cannot allocate device memory; see include/moe_layer.h for the limits."""
+    callers that cannot allocate device memory; see include/moe_layer.h for the limits.
+    With d_model, n_experts and dtype given (MoELayer passes them), x and logits_out are
+    checked to hold n_tokens rows before the library reads and writes them."""
+    if d_model is not None:
+        if x.dtype != dtype or x.numel() < int(n_tokens) * int(d_model):
+            raise ValueError(f"x: expected at least {int(n_tokens)} x {int(d_model)} elements "
+                             f"of {dtype}, got {tuple(x.shape)} of {x.dtype}")
+        if (logits_out.dtype != torch.float32 or
+                logits_out.numel() < int(n_tokens) * int(n_experts)):
+            raise ValueError(f"logits_out: expected at least {int(n_tokens)} x {int(n_experts)}"
+                             f" fp32 elements, got {tuple(logits_out.shape)} of "
+                             f"{logits_out.dtype}")
     _check("moe_router_logits_static", load_library().moe_router_logits_static(
         handle, _p(x), int(n_tokens), _p(logits_out), _stream(stream)))
 
@@ -321,6 +393,19 @@ class MoELayer:
             raise ValueError(f"{name}: expected a [T, {self.d}] tensor, got {tuple(x.shape)}")
         _expect(x, (x.shape[0], self.d), self.dtype, name)
         return int(x.shape[0])
+
+    def router_logits_static(self, x, logits_out=None, stream=None):
+        """Router logits [T, E] fp32 through the workspace-free entry point."""
+        T = self._rows(x)
+        if logits_out is None:
+            logits_out = torch.empty((T, self.E), dtype=torch.float32, device=self.device)
+        _expect(logits_out, (T, self.E), torch.float32, "logits_out")
+        moe_router_logits_static(self.handle, x, T, logits_out, stream, d_model=self.d,
+                                 n_experts=self.E, dtype=self.dtype)
+        return logits_out
+
+    def set_option(self, option: int, value: int) -> None:
+        moe_set_option(self.handle, option, value)
 
     def workspace(self, n_tokens: int):
         need = moe_workspace_size(self.handle, n_tokens)

@@ -55,6 +55,10 @@ struct GemmParams {
                      // UP, BN > 32: xs [Tk, d]; DOWN: h [Tk + n_shared*T, f]; LOGITS: x
                      // (box {64, BN} for all but the gather map)
   CUtensorMap tmBs;  // UP, BN > 32: x [T, d] (shared group)            box {64, BN}
+  // CTA-pair kernels with b_boxes set: the same matrices as tmB / tmBs with boxes of 16, 32
+  // and 64 rows, so a unit of few tokens stages only the rows it multiplies
+  CUtensorMap tmBr[3], tmBsr[3];
+  int b_boxes;
   const int *offsets;       // [E + 1] expert offsets in the sorted space
   const int *perm;          // [Tk] sorted row -> t*k + j (UP: token of a row; DOWN: gate)
   const float *topk_gate;   // [Tk] (DOWN)
@@ -79,10 +83,29 @@ struct GemmParams {
   int *done;
   int done_mt, done_bn;
   int done_warps;  // arrivals per up unit: its epilogue warps (all CTAs of the unit)
+  // Expert-range launches (a slice of the layer's experts, e.g. one expert-parallel rank's):
+  // routed group g reads the weights of weight group g + wg_off_routed, the shared group
+  // (g = E) those of E + wg_off_shared, and the shared group covers the T tokens from x row
+  // shared_t0 on.  All zero for the whole layer.
+  int wg_off_routed, wg_off_shared;
+  int shared_t0;
 };
+
+// Weight group of work group g (see GemmParams::wg_off_routed).
+__device__ __forceinline__ int weight_group(const GemmParams &p, int g) {
+  return g + (g < p.E ? p.wg_off_routed : p.wg_off_shared);
+}
 
 constexpr int kUnitQ = 4;  // depth of the producer -> MMA/epilogue unit queue
 constexpr int kGatherMaxBN = 32;  // MODE_UP token tiles up to this size gather rows from x
+
+// Launches with at most this many groups order their units by cost (build_unit_table);
+// larger ones keep the plain group order (the ordered list would not fit in shared memory
+// beside the deepest pipelines).
+constexpr int kOrderMaxGroups = 512;
+__host__ __device__ constexpr int order_words(int n_groups) {
+  return n_groups <= kOrderMaxGroups ? n_groups : 0;
+}
 
 constexpr int kBM = 128;         // weight rows per unit (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle atom of bf16
@@ -114,7 +137,8 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * kUnitQ) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
-           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * BN * 4 /*row scales*/ +
+           (size_t)(3 * n_groups + 1 + order_words(n_groups)) * 4 +
+           ACC_BUFS * BN * 4 /*row scales*/ +
            4 * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
   }
 };
@@ -170,6 +194,107 @@ __device__ __forceinline__ void store_block16_f32(float *out, int ld, int row0, 
   __syncwarp();
 }
 
+// Work list of a grouped GEMM launch, built by every CTA from the routing's offsets:
+// grp_count / grp_row [G] by group id; order [G] = the groups with at least one full token
+// tile of BN rows ("heavy": tensor-bound, their weight tiles shared by several token tiles)
+// in id order, then the others ("light": a few tokens each, bound by streaming their weights
+// from HBM) in id order; unit_prefix [G + 1] = exclusive prefix of the units (m tiles x
+// token tiles) over that order.  *n_heavy = units of the heavy groups.  With more than
+// kOrderMaxGroups groups the order is the identity (no array) and *n_heavy = 0.  Called by
+// all threads of the CTA (it synchronises them).
+template <int BN>
+__device__ __forceinline__ void build_unit_table(const GemmParams &p, int mtiles,
+                                                 int *unit_prefix, int *grp_count,
+                                                 int *grp_row, int *order, int *n_heavy) {
+  const int G = p.n_groups;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    int cnt, row;
+    if (g < p.E) {
+      row = p.offsets[g];
+      cnt = p.offsets[g + 1] - row;
+    } else {
+      row = p.Tk + (g - p.E) * p.T;
+      cnt = p.T;
+    }
+    grp_count[g] = cnt;
+    grp_row[g] = row;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // each lane a contiguous run of groups: heavy groups to the front, stable
+    const int per = (G + 31) / 32;
+    const int lo = min(G, lane * per), hi = min(G, lo + per);
+    int nh = 0;
+    if (order)
+      for (int g = lo; g < hi; ++g) nh += grp_count[g] >= BN;
+    int incl = nh;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int heavy_groups = __shfl_sync(0xffffffffu, incl, 31);
+    int hpos = incl - nh, lpos = heavy_groups + (lo - (incl - nh));
+    if (order)
+      for (int g = lo; g < hi; ++g) {
+        if (grp_count[g] >= BN) order[hpos++] = g;
+        else order[lpos++] = g;
+      }
+    __syncwarp();
+    // exclusive scan of the units over the ordered positions
+    auto grp_at = [&](int i) { return order ? order[i] : i; };
+    int run = 0;
+    for (int i = lo; i < hi; ++i) run += mtiles * ((grp_count[grp_at(i)] + BN - 1) / BN);
+    incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int excl = incl - run;
+    for (int i = lo; i < hi; ++i) {
+      const int u = mtiles * ((grp_count[grp_at(i)] + BN - 1) / BN);
+      unit_prefix[i] = excl;
+      excl += u;
+    }
+    if (lane == 31) unit_prefix[G] = incl;
+    __syncwarp();
+    if (lane == 0) *n_heavy = unit_prefix[heavy_groups];
+  }
+  __syncthreads();
+}
+
+// Claim order: ticket c of [0, total) -> unit.  The heavy units (the first n_heavy of the
+// ordered list) are spread evenly over the tickets (ticket c is heavy iff
+// floor((c+1) n_heavy / total) > floor(c n_heavy / total)), the light ones fill the rest in
+// order, so the CTAs run tensor-bound and HBM-bound units side by side instead of one kind
+// after the other.  A bijection of [0, total).
+__device__ __forceinline__ int unit_of_ticket(int c, int n_heavy, int total) {
+  const long long h0 = (long long)c * n_heavy / total;
+  const long long h1 = (long long)(c + 1) * n_heavy / total;
+  return h1 > h0 ? (int)h0 : n_heavy + (c - (int)h0);
+}
+
+// unit -> (group, m tile, token tile) over the ordered list: token tile innermost, so the
+// units that share a weight tile are claimed close together and run at about the same time
+// on different SMs (the tile is read from HBM about once).
+__device__ __forceinline__ void decode_unit(int u, int G, const int *unit_prefix,
+                                            const int *order, const int *grp_count, int bn,
+                                            int &g, int &mt, int &nt) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {  // last position with unit_prefix <= u
+    const int mid = (lo + hi + 1) >> 1;
+    if (unit_prefix[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  g = order ? order[lo] : lo;
+  const int nts = (grp_count[g] + bn - 1) / bn;
+  const int loc = u - unit_prefix[lo];
+  mt = loc / nts;
+  nt = loc % nts;
+}
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -193,12 +318,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
+  int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
+  // [G] when G <= kOrderMaxGroups, else none (identity order)
+  int *order = order_words(p.n_groups) ? grp_row + p.n_groups : nullptr;
   // [ACC_BUFS][BN], 16-byte aligned: read as float4
   float *row_scale = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups + order_words(p.n_groups)) + 15) &
+      ~static_cast<uintptr_t>(15));
   float *xbuf = row_scale + C::ACC_BUFS * BN;  // [4 warps][16][32] epilogue transposes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,60 +366,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // predecessor) could let it launch, and h, which it takes group by group through done[].
   if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
-  // group table: token count, first row in the sorted space, units per group
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    int cnt, row;
-    if (g < p.E) {
-      row = p.offsets[g];
-      cnt = p.offsets[g + 1] - row;
-    } else {
-      row = p.Tk + (g - p.E) * p.T;
-      cnt = p.T;
-    }
-    grp_count[g] = cnt;
-    grp_row[g] = row;
-    unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
-  }
-  __syncthreads();
-  if (warp == 0) {  // exclusive scan of units per group (each lane a contiguous run)
-    const int per = (G + 31) / 32;
-    const int lo = min(G, lane * per), hi = min(G, lo + per);
-    int run = 0;
-    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
-    int incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int excl = incl - run;
-    for (int g = lo; g < hi; ++g) {
-      const int u = unit_prefix[g];
-      unit_prefix[g] = excl;
-      excl += u;
-    }
-    if (lane == 31) unit_prefix[G] = incl;
-  }
+  // group table (token count, first row in the sorted space) and the cost-ordered work list
+  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_heavy_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = unit_prefix[G];
+  const int n_heavy = *n_heavy_s;
 
-  // unit -> (group, m tile, n tile); n tile innermost so the units that share a weight
-  // tile run back to back on neighbouring CTAs (the tile is read from HBM once).
   auto decode = [&](int u, int &g, int &mt, int &nt) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {  // last g with unit_prefix[g] <= u
-      const int mid = (lo + hi + 1) >> 1;
-      if (unit_prefix[mid] <= u) lo = mid;
-      else hi = mid - 1;
-    }
-    g = lo;
-    const int nts = (grp_count[g] + BN - 1) / BN;
-    const int loc = u - unit_prefix[g];
-    mt = loc / nts;
-    nt = loc % nts;
+    decode_unit(u, G, unit_prefix, order, grp_count, BN, g, mt, nt);
   };
 
   // Work distribution: the producer claims units (from the shared counter when p.sched is
@@ -324,7 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int uid = -1;
       if (lane == 0) {
         u = claim(u);
-        uid = (u < total_units) ? u : -1;
+        uid = (u < total_units) ? unit_of_ticket(u, n_heavy, total_units) : -1;
         if (mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 5)) {
           uq[qi] = uid;
           mbar_arrive(&uq_full[qi]);
@@ -342,12 +428,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (uid < 0) break;
       int g, mt, nt;
       decode(uid, g, mt, nt);
-      const int a_row = g * p.M + mt * kBM;
+      const int a_row = weight_group(p, g) * p.M + mt * kBM;
       const int valid = min(BN, grp_count[g] - nt * BN);
       // the shared group of a non-gathering up kernel reads x, not the sorted rows
       const bool shared_x = (MODE == MODE_UP) && !kGather && (g >= p.E);
       const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
-      const int b_row = shared_x ? nt * BN : grp_row[g] + nt * BN;
+      const int b_row = shared_x ? p.shared_t0 + nt * BN : grp_row[g] + nt * BN;
       // gathering: this lane's four token ids and the rows the MMA reads
       int tok[4] = {0, 0, 0, 0};
       int n_rows = BN;
@@ -357,7 +443,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int pos = 4 * lane + i;
           const int q = b_row + ((pos < valid) ? pos : 0);
-          if (4 * lane < n_rows) tok[i] = (g < p.E) ? p.perm[q] / p.topk : q - grp_row[g];
+          if (4 * lane < n_rows)
+            tok[i] = (g < p.E) ? p.perm[q] / p.topk : p.shared_t0 + q - grp_row[g];
         }
       }
       if (MODE == MODE_DOWN && p.done) {
@@ -607,6 +694,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      // every TMEM load of this unit has completed (tcgen05.wait::ld before each use), so
+      // the accumulator is handed back to the MMA thread before this warp's global stores
+      // drain: the h hand-over's fences below wait for them, off the MMA's critical path
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
       if (MODE == MODE_UP && p.done) {
         // publish this warp's rows of h for group g: stores, then a release of the count
         __threadfence();
@@ -616,8 +708,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           atomicAdd(p.done + g, 1);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
     }
   }
 

@@ -52,7 +52,7 @@ struct PairCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC_BUFS + 1 + 2 * kUnitQ) * 8;
   static constexpr size_t smem_bytes(int n_groups) {
     return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 64 +
-           (size_t)(3 * n_groups + 1) * 4 + ACC_BUFS * kPairBN * 4 +
+           (size_t)(3 * n_groups + 1 + order_words(n_groups)) * 4 + ACC_BUFS * kPairBN * 4 +
            kPairEpiWarps * 16 * 32 * 4 /*epilogue transpose buffers*/ + 16 /*alignment*/;
   }
 };
@@ -80,12 +80,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
+  int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
+  // [G] when G <= kOrderMaxGroups, else none (identity order)
+  int *order = order_words(p.n_groups) ? grp_row + p.n_groups : nullptr;
   // [ACC_BUFS][BN], 16-byte aligned: read as float4
   float *row_scale = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups) + 15) & ~static_cast<uintptr_t>(15));
+      (reinterpret_cast<uintptr_t>(grp_row + p.n_groups + order_words(p.n_groups)) + 15) &
+      ~static_cast<uintptr_t>(15));
   float *xbuf = row_scale + C::ACC_BUFS * BN;  // [8 warps][16][32] epilogue transposes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,39 +130,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   // except in a down kernel with the per-group hand-over of h (see grouped_gemm_kernel)
   if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    int cnt, row;
-    if (g < p.E) {
-      row = p.offsets[g];
-      cnt = p.offsets[g + 1] - row;
-    } else {
-      row = p.Tk + (g - p.E) * p.T;
-      cnt = p.T;
-    }
-    grp_count[g] = cnt;
-    grp_row[g] = row;
-    unit_prefix[g] = mtiles * ((cnt + BN - 1) / BN);
-  }
-  __syncthreads();
-  if (warp == 0) {  // exclusive scan of units per group (each lane a contiguous run)
-    const int per = (G + 31) / 32;
-    const int lo = min(G, lane * per), hi = min(G, lo + per);
-    int run = 0;
-    for (int g = lo; g < hi; ++g) run += unit_prefix[g];
-    int incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int excl = incl - run;
-    for (int g = lo; g < hi; ++g) {
-      const int u = unit_prefix[g];
-      unit_prefix[g] = excl;
-      excl += u;
-    }
-    if (lane == 31) unit_prefix[G] = incl;
-  }
+  // group table and the cost-ordered work list (see build_unit_table)
+  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_heavy_s);
   // both CTAs' barriers are initialised and TMEM allocated before any cross-CTA traffic
   tc_fence_before();
   __syncthreads();
@@ -166,19 +139,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = unit_prefix[G];
+  const int n_heavy = *n_heavy_s;
 
   auto decode = [&](int u, int &g, int &mt, int &nt) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (unit_prefix[mid] <= u) lo = mid;
-      else hi = mid - 1;
-    }
-    g = lo;
-    const int nts = (grp_count[g] + BN - 1) / BN;
-    const int loc = u - unit_prefix[g];
-    mt = loc / nts;
-    nt = loc % nts;
+    decode_unit(u, G, unit_prefix, order, grp_count, BN, g, mt, nt);
   };
   // token split of a unit: CTA r holds tokens [n0 + r*half, n0 + (r+1)*half), N = 2*half
   auto split = [&](int g, int nt) {
@@ -211,7 +175,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // the leader claims the next unit and publishes its id to both CTAs; the peer reads it
         if (leader) {
           u = claim(u);
-          const int uid = (u < total_units) ? u : -1;
+          const int uid = (u < total_units) ? unit_of_ticket(u, n_heavy, total_units) : -1;
           if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 15)) {
             ok = false;
             break;
@@ -237,10 +201,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         int g, mt, nt;
         decode(u, g, mt, nt);
         const int half = split(g, nt);
-        const int a_row = g * p.M + mt * kPairBM + (int)rank * 128;
+        const int a_row = weight_group(p, g) * p.M + mt * kPairBM + (int)rank * 128;
         const bool shared_x = (MODE == MODE_UP) && (g >= p.E);
-        const CUtensorMap *bmap = shared_x ? &p.tmBs : &p.tmB;
-        const int b_row = (shared_x ? nt * BN : grp_row[g] + nt * BN) + (int)rank * half;
+        // token rows of this CTA: a box of 16, 32, 64 or 128 rows, the smallest that holds
+        // the half tile (rows past it are never read by the MMA)
+        const int box = (!p.b_boxes || half > 64) ? 3 : (half > 32 ? 2 : (half > 16 ? 1 : 0));
+        const CUtensorMap *bmap = box == 3 ? (shared_x ? &p.tmBs : &p.tmB)
+                                           : (shared_x ? &p.tmBsr[box] : &p.tmBr[box]);
+        const uint32_t stage_tx = 2u * (C::NA * C::A_BYTES + (16u << box) * kBK * 2);
+        const int b_row =
+            (shared_x ? p.shared_t0 + nt * BN : grp_row[g] + nt * BN) + (int)rank * half;
         const uint64_t pw = (grp_count[g] <= BN) ? pol_w : pol_w_shared;
         if (MODE == MODE_DOWN && p.done && g != ready_group) {
           // both CTAs load h rows: each waits for every up unit of the group
@@ -259,7 +229,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             break;
           }
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           tma_load_2d_pair(sA0 + stage * C::A_BYTES, &p.tmA0, fbar, kb * kBK, a_row, pw);
           if (MODE == MODE_UP)
             tma_load_2d_pair(sA1 + stage * C::A_BYTES, &p.tmA1, fbar, kb * kBK, a_row, pw);
@@ -455,6 +425,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                             vals, wbuf, lane);
         }
       }
+      // every TMEM load of this unit has completed (tcgen05.wait::ld before each use): the
+      // accumulator goes back to the leader's MMA thread before this warp's global stores
+      // drain, so the h hand-over's fences below stay off the MMA's critical path (the up
+      // kernel has a single accumulator: its next unit's MMAs wait for this arrival)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_leader + acc * 8);
+      }
       if (MODE == MODE_UP && p.done) {
         // publish this warp's rows of h for group g: stores, then a release of the count
         __threadfence();
@@ -463,12 +443,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           __threadfence();
           atomicAdd(p.done + g, 1);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (leader) mbar_arrive(&tempty[acc]);
-        else mbar_arrive_remote(tempty_leader + acc * 8);
       }
     }
   }

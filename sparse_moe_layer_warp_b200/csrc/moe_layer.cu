@@ -26,6 +26,7 @@
 
 #include "moe_layer.h"
 #include "backward.cuh"
+#include "expert_parallel.cuh"
 #include "expert_simt.cuh"
 #include "expert_stats.cuh"
 #include "grouped_gemm.cuh"
@@ -45,12 +46,28 @@ struct moe_layer {
   int smem_optin;
   int pair_grid[2];  // CTAs of the CTA-pair GEMM (up, down): 2 x co-resident clusters
   CUtensorMap tm_wg, tm_wu, tm_wd, tm_wr;
+  CUtensorMap tm_wr2;  // W_r with a box of half the experts (256 < E <= 288, see below)
   // the same weights as MN-major operands of the backward (box {64, 64}): W_gate and W_up
   // as [G*f, d], W_down as [G*d, f]
   CUtensorMap tm_wg_mn, tm_wu_mn, tm_wd_mn;
   int wg_pair_grid;  // CTAs of the CTA-pair weight-gradient kernel (0: not available)
   int bw_pair_grid;  // CTAs of the CTA-pair dgrad kernels (0: not available)
   int tail_pair_grid;  // CTAs of the CTA-pair dx + weight-gradient kernel (0: not available)
+  // Per-group hand-over of h from the up to the down GEMM (see GemmParams::done):
+  // handover_fits is the init-time occupancy check (every persistent up grid the forward
+  // can launch fits on the device at once), opt_handover the caller's switch
+  // (MOE_OPTION_H_HANDOVER).  Without it the down GEMM waits for the whole up GEMM.
+  int handover_fits;
+  int opt_handover;
+  // experts whose weights the handle holds: [e0, e1) (the whole layer: [0, E)); the weight
+  // tensors hold e1 - e0 routed experts then the shared expert (moe_layer_init_ep)
+  int e0, e1;
+  // Shared expert beside the routing (MOE_OPTION_SHARED_SIDE_SMS): a stream of the handle on
+  // which the shared expert's up and down GEMMs run while the caller's stream routes, on
+  // side_sms SMs (0: off), forked from and joined back into the caller's stream by events.
+  int side_sms;
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
 };
 
 namespace {
@@ -105,6 +122,14 @@ bool encode_f32_2d(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The same matrix with token-row boxes of 16, 32 and 64 rows (the CTA-pair GEMMs' loads for
+// units of few tokens; see GemmParams::tmBr).
+bool encode_row_boxes(CUtensorMap (&m)[3], const void *base, uint64_t cols, uint64_t rows) {
+  for (int i = 0; i < 3; ++i)
+    if (!encode_bf16_2d(&m[i], base, cols, rows, 16u << i)) return false;
+  return true;
+}
 
 // Every kernel of the library starts with griddepcontrol.wait, so each launch may use
 // programmatic stream serialisation: its CTAs can be scheduled (and run their set-up)
@@ -176,11 +201,13 @@ WsLayout ws_layout(const moe_config &c, int T) {
   L.part = take((T <= kSplitKTokens ? (size_t)n_splits(c) : 0) * T * c.n_experts * 4);
   L.idx = take(Tk * 4);
   L.gate = take(Tk * 4);
-  L.counts = take((size_t)c.n_experts * 4);
-  L.offsets = take(((size_t)c.n_experts + 1) * 4);
+  // counts, offsets and chunk histograms hold kMaxTopK more buckets than experts: the drop
+  // buckets (one per slot) of an expert-range (partial) forward
+  L.counts = take(((size_t)c.n_experts + kMaxTopK) * 4);
+  L.offsets = take(((size_t)c.n_experts + kMaxTopK + 1) * 4);
   L.perm = take(Tk * 4);
   L.slot_row = take(Tk * 4);
-  L.chunk_hist = take(nch * c.n_experts * 4);
+  L.chunk_hist = take(nch * ((size_t)c.n_experts + kMaxTopK) * 4);
   L.stats = take(nch * (2 * (size_t)c.n_experts + 1) * 4);  // router statistics partials
   L.xs = (c.dtype == MOE_BF16 && !up_gathers_rows(c, T)) ? take(Tk * c.d_model * 2) : off;
   L.h = take(P * c.d_ff * esize(c));
@@ -446,18 +473,60 @@ int dgrad_pair_grid_size(const moe_layer *L) {
 }
 
 template <int MODE>
-moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_t st) {
-  const size_t smem = pair_smem<MODE>(L->cfg);
+moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_t st,
+                            int max_ctas = 0) {
+  // sized for this launch's groups (the kernel lays out its group table from p.n_groups)
+  const size_t smem = PairCfg<MODE>::smem_bytes(p.n_groups);
+  if (smem > (size_t)L->smem_optin) return MOE_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int grid = L->pair_grid[MODE == MODE_UP ? 0 : 1];
+  int grid = L->pair_grid[MODE == MODE_UP ? 0 : 1];
+  if (max_ctas >= 2 && max_ctas < grid) grid = max_ctas & ~1;
   return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(kPairThreads), smem, st, 2,
                    p);
 }
 
+// The per-group hand-over of h lets the down GEMM start while the up GEMM still runs.  Its
+// waits end because every up unit is claimed by an up CTA that is resident: a dependent
+// launch starts only after every CTA of the up grid has started (and signalled), and a CTA
+// leaves only once no unit is left to claim.  The persistent up grids are sized to be
+// co-resident (one CTA per SM, or the co-resident cluster count); this check repeats that
+// sizing with the occupancy calculator for every up kernel the forward can launch, and the
+// forward plans the down GEMM with a whole-grid wait instead when it fails.
+template <int BN>
+bool up_grid_fits(const moe_layer *L) {
+  using C = GemmCfg<MODE_UP, BN>;
+  const size_t smem = C::smem_bytes(L->cfg.n_experts + L->cfg.n_shared);
+  if (smem > (size_t)L->smem_optin) return true;  // not launchable: the forward refuses it
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE_UP, BN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return false;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_gemm_kernel<MODE_UP, BN>,
+                                                    kGemmThreads, smem) != cudaSuccess)
+    return false;
+  return (long long)per_sm * L->num_sms >= L->num_sms;  // grid = num_sms CTAs
+}
+
+bool up_grids_fit(const moe_layer *L) {
+  // the CTA-pair up grid is itself the occupancy calculator's co-resident cluster count
+  // (pair_grid_size), so only the one-CTA grids (num_sms CTAs) need the check
+  return up_grid_fits<16>(L) && up_grid_fits<32>(L) && up_grid_fits<64>(L) &&
+         up_grid_fits<128>(L);
+}
+
 // Token tile of the router GEMM.
 int pick_bn_router(int T) { return T <= 256 ? 16 : (T <= 1024 ? 32 : 64); }
+
+// Expert tile of the tokens-on-M router GEMM for 256 < E <= 288: two tiles of 144 experts
+// (0: tiles of 128).
+constexpr int kRouterHalfTile = 144;
+int router_half_tile(const moe_config &c) {
+  return (c.dtype == MOE_BF16 && c.n_experts > 256 && c.n_experts <= 2 * kRouterHalfTile)
+             ? kRouterHalfTile
+             : 0;
+}
 
 // From this many tokens the router GEMM puts tokens on M (see MODE_LOGITS, out_trans).
 constexpr int kRouterTokensOnM = 1024;
@@ -470,7 +539,11 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
   if (T >= kRouterTokensOnM) {
     // tokens on M (128 per unit), the E experts as the N side in tiles of 128
     if (!encode_bf16_2d(&p.tmA0, x, c.d_model, T, kBM)) return MOE_ERR_CUDA;
-    p.tmB = L->tm_wr;  // box {64, 128}: 128 experts per tile, rows past E zero-filled
+    // experts as the N side: tiles of 128 (rows past E zero-filled by TMA), or for
+    // 256 < E <= 288 two tiles of half of them, so the units of 128 tokens x one expert tile
+    // are 2 per token tile instead of 3 (8192 tokens: 128 units, one wave on 148 SMs)
+    const int half = router_half_tile(c);
+    p.tmB = half ? L->tm_wr2 : L->tm_wr;
     p.out = logits;
     p.status = status;
     p.E = 0;  // one group of E "rows": the experts
@@ -481,6 +554,7 @@ moe_status launch_gemm_logits(const moe_layer *L, const void *x, int T, float *l
     p.K = c.d_model;
     p.ld_out = c.n_experts;
     p.out_trans = 1;
+    if (half) return launch_gemm_bn<MODE_LOGITS, kRouterHalfTile>(L, p, st);
     return launch_gemm<MODE_LOGITS>(L, 128, p, st);
   }
   const int bn = pick_bn_router(T);
@@ -581,6 +655,8 @@ __global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(DevStatus *st
   counter_wait_bounded(flag, 1, &abort_flag, status, 102, limit_ns);
 }
 
+bool holds_all_experts(const moe_layer *L) { return L->e0 == 0 && L->e1 == L->cfg.n_experts; }
+
 moe_status check_call(const moe_layer *L, int T, void *ws, size_t ws_bytes) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
@@ -608,10 +684,12 @@ const char *moe_status_string(moe_status s) {
   return "unknown status";
 }
 
-moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handle *out) {
+static moe_status layer_init(const moe_config *cfg, const moe_weights *w, int e0, int e1,
+                             moe_handle *out) {
   if (!cfg || !w || !out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   const moe_config c = *cfg;
+  if (e0 < 0 || e1 <= e0 || e1 > c.n_experts) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.d_model < 1 || c.n_experts < 1 || c.top_k < 1 || c.d_ff < 1)
     return MOE_ERR_INVALID_ARG;
   if (c.top_k > c.n_experts || (c.n_shared != 0 && c.n_shared != 1)) return MOE_ERR_INVALID_ARG;
@@ -630,6 +708,8 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
   if (!L) return MOE_ERR_INVALID_ARG;
   L->cfg = c;
   L->w = *w;
+  L->e0 = e0;
+  L->e1 = e1;
 
   int major = 0;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
@@ -646,6 +726,7 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     free(L);
     return MOE_ERR_UNSUPPORTED;
   }
+  L->opt_handover = 1;
   if (c.dtype == MOE_BF16) {
     L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
@@ -654,12 +735,16 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
     L->tail_pair_grid = cluster_grid_size(bw_tail_pair_kernel,
                                           BwTailPairCfg::smem_bytes(c.n_experts + c.n_shared),
                                           kWgPairThreads, L);
+    L->handover_fits = up_grids_fit(L);
     cudaGetLastError();  // an unavailable cluster query only disables the pair path
-    const uint64_t G = (uint64_t)c.n_experts + c.n_shared;
+    const uint64_t G = (uint64_t)(e1 - e0) + c.n_shared;  // weight groups held
     if (!encode_bf16_2d(&L->tm_wg, w->w_gate, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wu, w->w_up, c.d_model, G * c.d_ff, kBM) ||
         !encode_bf16_2d(&L->tm_wd, w->w_down, c.d_ff, G * c.d_model, kBM) ||
         !encode_bf16_2d(&L->tm_wr, w->w_router, c.d_model, c.n_experts, kBM) ||
+        (router_half_tile(c) &&
+         !encode_bf16_2d(&L->tm_wr2, w->w_router, c.d_model, c.n_experts,
+                         (uint32_t)router_half_tile(c))) ||
         !encode_bf16_2d(&L->tm_wg_mn, w->w_gate, c.d_model, G * c.d_ff, 64) ||
         !encode_bf16_2d(&L->tm_wu_mn, w->w_up, c.d_model, G * c.d_ff, 64) ||
         !encode_bf16_2d(&L->tm_wd_mn, w->w_down, c.d_ff, G * c.d_model, 64)) {
@@ -671,10 +756,46 @@ moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handl
   return MOE_OK;
 }
 
+moe_status moe_layer_init(const moe_config *cfg, const moe_weights *w, moe_handle *out) {
+  return layer_init(cfg, w, 0, cfg ? cfg->n_experts : 0, out);
+}
+
+moe_status moe_layer_init_ep(const moe_config *cfg, const moe_weights *w, int expert_begin,
+                             int expert_end, moe_handle *out) {
+  if (cfg && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  return layer_init(cfg, w, expert_begin, expert_end, out);
+}
+
 moe_status moe_layer_destroy(moe_handle h) {
   if (!h) return MOE_ERR_INVALID_ARG;
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   free(h);
   return MOE_OK;
+}
+
+moe_status moe_set_option(moe_handle h, int option, int value) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  switch (option) {
+    case MOE_OPTION_H_HANDOVER:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      h->opt_handover = value;
+      return MOE_OK;
+    case MOE_OPTION_SHARED_SIDE_SMS:
+      if (value < 0 || value > h->num_sms) return MOE_ERR_INVALID_ARG;
+      if (value > 0 && !h->side) {
+        int cur = -1;
+        if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_INVALID_ARG;
+        if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      }
+      h->side_sms = value & ~1;  // whole CTA pairs
+      return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
 }
 
 size_t moe_workspace_size(moe_handle h, int n_tokens) {
@@ -750,6 +871,7 @@ static moe_status backward_entry(moe_handle h, const void *x, int n_tokens, cons
                                  float *dw_down, void *ws, size_t ws_bytes, void *stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (n_tokens < 0 || n_tokens > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (!holds_all_experts(h)) return MOE_ERR_UNSUPPORTED;  // an expert-parallel slice
   if (n_tokens == 0) return MOE_OK;
   if (!x || !dout || !dx || !dw_router || !dw_gate || !dw_up || !dw_down)
     return MOE_ERR_INVALID_ARG;
@@ -781,6 +903,7 @@ moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *
                              float *ratios, void *ws, size_t ws_bytes, void *stream) {
   moe_status s = check_call(h, n_tokens, ws, ws_bytes);
   if (s != MOE_OK) return s;
+  if (!holds_all_experts(h)) return MOE_ERR_UNSUPPORTED;  // an expert-parallel slice
   if (n_tokens == 0 || !act_rms || !param_norm || !ratios) return MOE_ERR_INVALID_ARG;
   const moe_config &c = h->cfg;
   const int T = n_tokens, Tk = T * c.top_k, G = c.n_experts + c.n_shared;
@@ -909,6 +1032,8 @@ struct ForwardPlan {
   bool small_route;   // selection + permutation in one launch after the router
   bool pair;          // CTA-pair grouped GEMMs
   bool gather_in_gemm;  // the up GEMM gathers x rows itself (no gather launch)
+  bool handover;        // the down GEMM takes h from the up GEMM group by group
+  bool side_shared;     // the shared expert's GEMMs run on the side stream during routing
   int launches;
 };
 
@@ -919,25 +1044,28 @@ ForwardPlan plan_forward(const moe_layer *L, int T) {
   f.small_route = !f.decode_route && T <= kChunk;
   f.pair = c.dtype == MOE_BF16 && use_pair(L, T);
   f.gather_in_gemm = c.dtype == MOE_BF16 && !f.pair && up_gathers_rows(c, T);
+  f.handover = c.dtype == MOE_BF16 && L->handover_fits && L->opt_handover;
+  f.side_shared = f.pair && c.n_shared && L->side_sms >= 2 && L->side != nullptr;
   if (T == 0) {
     f.launches = 0;
     return f;
   }
   const int routing = f.decode_route ? 1 : (f.small_route ? 2 : 3);
   const int gather = (c.dtype == MOE_BF16 && !f.gather_in_gemm) ? 1 : 0;
-  f.launches = routing + gather + 3;  // + up, down, combine
+  f.launches = routing + gather + 3 + (f.side_shared ? 2 : 0);  // + up, down, combine
   return f;
 }
 
 // bf16: the expert-sorted copy of x rows, unless the up GEMM gathers them itself.
 moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
-                             const WsLayout &W, const ForwardPlan &plan, cudaStream_t st) {
+                             const WsLayout &W, const ForwardPlan &plan, cudaStream_t st,
+                             const int *n_rows_dev = nullptr) {
   if (plan.gather_in_gemm) return MOE_OK;
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   return launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)), dim3(256), 0, st,
                 static_cast<const uint4 *>(x), (const int *)at<int>(ws, W.perm), c.top_k, Tk,
-                c.d_model / 8, at<uint4>(ws, W.xs));
+                c.d_model / 8, at<uint4>(ws, W.xs), n_rows_dev);
 }
 
 // bf16 expert up GEMM over the routing in `ws`: h (bf16, `out`) -- or, with out2 set, the
@@ -954,11 +1082,19 @@ struct UpRows {
   int xs_rows;
 };
 
+// Expert-range launch of the expert GEMMs (moe_forward_partial): `n_routed` routed groups
+// (the sorted space's first n_routed groups) whose weights start at weight group
+// wg_off_routed, and the shared expert (weight group n_routed + wg_off_shared) over the
+// shared_n tokens from shared_t0 on.  The whole layer: {E, 0, 0, 0, T}.
+struct Slice {
+  int n_routed, wg_off_routed, wg_off_shared, shared_t0, shared_n;
+};
+
 moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
                             const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
                             int *done, cudaStream_t st, GemmParams *used,
                             const UpRows *rows = nullptr, float *save_a = nullptr,
-                            float *save_b = nullptr) {
+                            float *save_b = nullptr, const Slice *slice = nullptr) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
@@ -967,12 +1103,19 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
   memset(&p1, 0, sizeof p1);
   p1.tmA0 = h->tm_wg;
   p1.tmA1 = h->tm_wu;
+  const void *xs = rows ? rows->xs : at<void>(ws, W.xs);
+  const int xs_rows = rows ? rows->xs_rows : Tk;
   if (plan.gather_in_gemm) {
     if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, 1)) return MOE_ERR_CUDA;  // gather4 map
-  } else if (!encode_bf16_2d(&p1.tmB, rows ? rows->xs : at<void>(ws, W.xs), c.d_model,
-                             rows ? rows->xs_rows : Tk, bn) ||
+  } else if (!encode_bf16_2d(&p1.tmB, xs, c.d_model, xs_rows, bn) ||
              !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, bn)) {
     return MOE_ERR_CUDA;
+  }
+  if (plan.pair) {  // smaller token-row boxes for units of few tokens
+    if (!encode_row_boxes(p1.tmBr, xs, c.d_model, xs_rows) ||
+        !encode_row_boxes(p1.tmBsr, x, c.d_model, T))
+      return MOE_ERR_CUDA;
+    p1.b_boxes = 1;
   }
   p1.offsets = at<int>(ws, W.offsets);
   p1.perm = at<int>(ws, W.perm);
@@ -998,7 +1141,131 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
     p1.perm = rows->perm;
     p1.Tk = rows->shared_row;
   }
+  if (slice) {
+    p1.E = slice->n_routed;
+    p1.n_groups = slice->n_routed + c.n_shared;
+    p1.T = slice->shared_n;
+    p1.shared_t0 = slice->shared_t0;
+    p1.wg_off_routed = slice->wg_off_routed;
+    p1.wg_off_shared = slice->wg_off_shared;
+  }
   return plan.pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st);
+}
+
+// bf16 expert stage of a forward, after the routing: [row gather] -> up + SwiGLU -> down,
+// leaving the per-row expert outputs in y.  events (if given) mark the ends of the gather,
+// up and down stages (indices 4, 5, 6); slice / n_rows_dev: an expert-range launch.
+moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *ws,
+                               const WsLayout &W, const ForwardPlan &plan, cudaStream_t st,
+                               void *const *events, float *saved, const Slice *slice,
+                               const int *n_rows_dev) {
+  const moe_config &c = h->cfg;
+  const int Tk = T * c.top_k;
+  const int P = Tk + (slice ? slice->shared_n : c.n_shared * T);
+  auto mark = [&](int i) -> moe_status {
+    if (!events) return MOE_OK;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+  };
+  moe_status s;
+  const bool pair = plan.pair;
+  const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
+  if ((s = launch_row_gather(h, x, T, ws, W, plan, st, n_rows_dev)) != MOE_OK ||
+      (s = mark(4)) != MOE_OK)
+    return s;
+  const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
+  __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
+  float *ybuf = at<float>(ws, W.y);
+  // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
+  // expert group for that group's rows of h (see grouped_gemm_kernel)
+  GemmParams p1;
+  if ((s = launch_expert_up(h, x, T, ws, W, plan, hbuf, nullptr,
+                            plan.handover ? at<int>(ws, W.done) : nullptr, st, &p1, nullptr,
+                            saved, saved ? saved + (size_t)P * c.d_ff : nullptr, slice)) !=
+      MOE_OK)
+    return s;
+  if ((s = mark(5)) != MOE_OK) return s;
+  GemmParams p2 = p1;
+  p2.tmA0 = h->tm_wd;
+  if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
+  p2.b_boxes = 0;
+  if (pair) {
+    if (!encode_row_boxes(p2.tmBr, hbuf, c.d_ff, P)) return MOE_ERR_CUDA;
+    p2.b_boxes = 1;
+  }
+  p2.out = ybuf;
+  p2.sched = &at<DevStatus>(ws, W.status)->sched[1];
+  p2.M = c.d_model;
+  p2.K = c.d_ff;
+  p2.ld_out = c.d_model;
+  // the up kernel's weight tiles per token tile, its token tile and its epilogue warps
+  p2.done_mt = c.d_ff / (pair ? kPairBM : kBM);
+  p2.done_bn = pair ? kPairBN : bn;
+  p2.done_warps = pair ? 2 * kPairEpiWarps : 4;
+  if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
+                : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
+    return s;
+  (void)ybuf;
+  return mark(6);
+}
+
+// The shared expert of a CTA-pair forward on the handle's side stream: forked from `st`
+// before the routing (it reads only x and writes only the shared rows of h and y, which no
+// routing kernel touches), up and down GEMMs on side_sms SMs with their own work counters,
+// and the join event recorded after them (the caller's stream waits for it before the
+// combine).
+moe_status launch_shared_side(const moe_layer *h, const void *x, int T, void *ws,
+                              const WsLayout &W, const ForwardPlan &plan, cudaStream_t st) {
+  const moe_config &c = h->cfg;
+  const int Tk = T * c.top_k;
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  cudaStream_t sd = h->side;
+  if (cudaEventRecord(h->ev_fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(sd, h->ev_fork, 0) != cudaSuccess ||
+      cudaMemsetAsync(status->side_sched, 0, sizeof(status->side_sched), sd) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const Slice shared{0, 0, h->e1 - h->e0, 0, T};  // no routed group; weight group E
+  __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
+  GemmParams p1;
+  memset(&p1, 0, sizeof p1);
+  p1.tmA0 = h->tm_wg;
+  p1.tmA1 = h->tm_wu;
+  if (!encode_bf16_2d(&p1.tmB, x, c.d_model, T, PairCfg<MODE_UP>::HALF_BN) ||
+      !encode_bf16_2d(&p1.tmBs, x, c.d_model, T, PairCfg<MODE_UP>::HALF_BN) ||
+      !encode_row_boxes(p1.tmBr, x, c.d_model, T) || !encode_row_boxes(p1.tmBsr, x, c.d_model, T))
+    return MOE_ERR_CUDA;
+  p1.b_boxes = 1;
+  p1.offsets = at<int>(ws, W.offsets);  // not read: no routed group
+  p1.perm = at<int>(ws, W.perm);
+  p1.topk_gate = at<float>(ws, W.gate);
+  p1.out = hbuf;
+  p1.status = status;
+  p1.routed_scale = c.routed_scale;
+  p1.E = shared.n_routed;
+  p1.n_groups = shared.n_routed + 1;
+  p1.T = T;
+  p1.Tk = Tk;
+  p1.M = c.d_ff;
+  p1.K = c.d_model;
+  p1.ld_out = c.d_ff;
+  p1.sched = &status->side_sched[0];
+  p1.topk = c.top_k;
+  p1.wg_off_shared = shared.wg_off_shared;
+  moe_status s;
+  if ((s = launch_gemm_pair<MODE_UP>(h, p1, sd, h->side_sms)) != MOE_OK) return s;
+  GemmParams p2 = p1;
+  p2.tmA0 = h->tm_wd;
+  if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, Tk + T, PairCfg<MODE_DOWN>::HALF_BN) ||
+      !encode_row_boxes(p2.tmBr, hbuf, c.d_ff, Tk + T))
+    return MOE_ERR_CUDA;
+  p2.out = at<float>(ws, W.y);
+  p2.sched = &status->side_sched[1];
+  p2.M = c.d_model;
+  p2.K = c.d_ff;
+  p2.ld_out = c.d_model;
+  if ((s = launch_gemm_pair<MODE_DOWN>(h, p2, sd, h->side_sms)) != MOE_OK) return s;
+  (void)plan;
+  return cudaEventRecord(h->ev_join, sd) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 }  // namespace
 
@@ -1013,7 +1280,9 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
                                size_t ws_bytes, void *stream, void *const *events,
                                float *saved = nullptr) {
   moe_status s = check_call(h, n_tokens, ws, ws_bytes);
-  if (s != MOE_OK || n_tokens == 0) return s;
+  if (s != MOE_OK) return s;
+  if (!holds_all_experts(h)) return MOE_ERR_UNSUPPORTED;  // an expert-parallel slice
+  if (n_tokens == 0) return MOE_OK;
   if (!x || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
   const moe_config &c = h->cfg;
@@ -1038,7 +1307,12 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   // the expert kernels' counters start from zero in every forward
   const CounterReset reset{at<DevStatus>(ws, W.status)->sched, at<int>(ws, W.done),
                            c.n_experts + c.n_shared};
-  const ForwardPlan plan = plan_forward(h, T);
+  ForwardPlan plan = plan_forward(h, T);
+  // the shared expert beside the routing: not with per-stage events (their stages would
+  // overlap) nor with kept pre-activations (the training forward stores all rows in one up
+  // launch)
+  if (events || saved) plan.side_shared = false;
+  if (plan.side_shared && (s = launch_shared_side(h, x, T, ws, W, plan, st)) != MOE_OK) return s;
   if (plan.decode_route) {
     if ((s = launch_route_decode(h, x, T, logits, idx, gate, at<int>(ws, W.counts), offsets,
                                  perm, slot_row, at<DevStatus>(ws, W.status), reset, st)) !=
@@ -1065,37 +1339,13 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   if ((s = mark(3)) != MOE_OK) return s;
 
   if (c.dtype == MOE_BF16) {
-    const bool pair = plan.pair;
-    const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
-    if ((s = launch_row_gather(h, x, T, ws, W, plan, st)) != MOE_OK || (s = mark(4)) != MOE_OK)
+    const Slice routed_only{c.n_experts, 0, 0, 0, 0};
+    if ((s = launch_experts_bf16(h, x, T, ws, W, plan, st, events, saved,
+                                 plan.side_shared ? &routed_only : nullptr, nullptr)) != MOE_OK)
       return s;
-    const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
-    __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
-    float *ybuf = at<float>(ws, W.y);
-    // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
-    // expert group for that group's rows of h (see grouped_gemm_kernel)
-    GemmParams p1;
-    if ((s = launch_expert_up(h, x, T, ws, W, plan, hbuf, nullptr, at<int>(ws, W.done), st,
-                              &p1, nullptr, saved, saved ? saved + (size_t)P * c.d_ff : nullptr)) !=
-        MOE_OK)
-      return s;
-    if ((s = mark(5)) != MOE_OK) return s;
-    GemmParams p2 = p1;
-    p2.tmA0 = h->tm_wd;
-    if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
-    p2.out = ybuf;
-    p2.sched = &at<DevStatus>(ws, W.status)->sched[1];
-    p2.M = c.d_model;
-    p2.K = c.d_ff;
-    p2.ld_out = c.d_model;
-    // the up kernel's weight tiles per token tile, its token tile and its epilogue warps
-    p2.done_mt = c.d_ff / (pair ? kPairBM : kBM);
-    p2.done_bn = pair ? kPairBN : bn;
-    p2.done_warps = pair ? 2 * kPairEpiWarps : 4;
-    if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
-                  : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
-      return s;
-    if ((s = mark(6)) != MOE_OK) return s;
+    if (plan.side_shared && cudaStreamWaitEvent(st, h->ev_join, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const float *ybuf = at<float>(ws, W.y);
     if ((s = launch(combine_kernel<__nv_bfloat16>,
                     dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0,
                     st, (const float *)ybuf, (const int *)slot_row, T, c.top_k, Tk, c.n_shared,
@@ -1207,6 +1457,147 @@ moe_status moe_update_router_bias(moe_handle h, const int *expert_counts, int n_
 
 }  // extern "C"
 
+// ================================================================ expert parallelism
+// The layer split by experts over ranks (expert_parallel.cuh): a forward of an expert range
+// returning unrounded fp32 partial outputs, the dispatch plan of an all-to-all exchange, the
+// packing of its send buffer and the combine of the partial rows that come back.
+extern "C" {
+
+moe_status moe_forward_partial(moe_handle h, const void *x, int n_tokens, const int *topk_idx,
+                               const float *topk_gate, int expert_begin, int expert_end,
+                               int shared_begin, int shared_end, float *out, void *ws,
+                               size_t ws_bytes, void *stream) {
+  moe_status s = check_call(h, n_tokens, ws, ws_bytes);
+  if (s != MOE_OK) return s;
+  const moe_config &c = h->cfg;
+  if (c.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (expert_begin < h->e0 || expert_end < expert_begin || expert_end > h->e1)
+    return MOE_ERR_INVALID_ARG;
+  if (expert_end - expert_begin + c.top_k > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (shared_end < shared_begin || shared_begin < 0 || shared_end > n_tokens)
+    return MOE_ERR_INVALID_ARG;
+  if (shared_end > shared_begin && !c.n_shared) return MOE_ERR_INVALID_ARG;
+  if ((topk_idx == nullptr) != (topk_gate == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!x || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+  const int T = n_tokens, k = c.top_k, Tk = T * k;
+  const int El = expert_end - expert_begin;  // routed groups of this launch
+  const WsLayout W = ws_layout(c, T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevStatus *status = at<DevStatus>(ws, W.status);
+  int *idx = at<int>(ws, W.idx);
+  float *gate = at<float>(ws, W.gate);
+  int *offsets = at<int>(ws, W.offsets);
+  int *perm = at<int>(ws, W.perm);
+  int *slot_row = at<int>(ws, W.slot_row);
+  int *lidx = at<int>(ws, W.y);  // local groups of the slots (y is written only later)
+  const CounterReset reset{status->sched, at<int>(ws, W.done), El + c.n_shared};
+  // 1. the selection: given, or the layer's own routing of x (full router, all E experts)
+  if (!topk_idx) {
+    if ((s = route_common(h, x, nullptr, T, nullptr, idx, gate, at<int>(ws, W.counts), offsets,
+                          perm, slot_row, ws, ws_bytes, stream)) != MOE_OK)
+      return s;
+    topk_idx = idx;
+    topk_gate = gate;
+  }
+  // 2. slots -> local groups (drop bucket El for other experts), sorted by group
+  const int nch = (T + kChunk - 1) / kChunk;
+  if ((s = launch(ep_local_hist_kernel, dim3(nch), dim3(256), 0, st, topk_idx, topk_gate, T, k,
+                  c.n_experts, expert_begin, expert_end, lidx, gate,
+                  at<int>(ws, W.chunk_hist))) != MOE_OK ||
+      (s = launch(permute_scatter_kernel, dim3(nch), dim3(256), 0, st, (const int *)lidx,
+                  (const int *)at<int>(ws, W.chunk_hist), T, El + k, k, nch,
+                  at<int>(ws, W.counts), offsets, perm, slot_row, reset)) != MOE_OK)
+    return s;
+  const int *n_valid = offsets + El;  // rows of the routed groups of this launch
+  // 3. the expert GEMMs over the local groups and the shared expert's token range
+  const ForwardPlan plan = plan_forward(h, T);
+  const Slice slice{El, expert_begin - h->e0, (h->e1 - h->e0) - El, shared_begin,
+                    shared_end - shared_begin};
+  if ((s = launch_experts_bf16(h, x, T, ws, W, plan, st, nullptr, nullptr, &slice, n_valid)) !=
+      MOE_OK)
+    return s;
+  // 4. per token: its slots in range, then the shared expert, fp32, not rounded
+  return launch(combine_partial_kernel,
+                dim3(grid_for((size_t)T * (c.d_model / 4), 256, h->num_sms)), dim3(256), 0, st,
+                (const float *)at<float>(ws, W.y), (const int *)slot_row, n_valid, T, k, Tk,
+                shared_begin, shared_end, c.d_model, out);
+}
+
+moe_status moe_ep_plan(moe_handle h, const int *topk_idx, int n_tokens, int n_ranks,
+                       int *send_counts, int *send_offsets, int *send_perm, int *send_slot,
+                       void *ws, size_t ws_bytes, void *stream) {
+  moe_status s = check_call(h, n_tokens, ws, ws_bytes);
+  if (s != MOE_OK) return s;
+  const moe_config &c = h->cfg;
+  if (n_ranks < 1 || 2 * n_ranks > kMaxExperts || c.n_experts % n_ranks != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!topk_idx || !send_counts || !send_offsets || !send_perm || !send_slot)
+    return MOE_ERR_INVALID_ARG;
+  if ((long long)n_tokens * n_ranks >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  const WsLayout W = ws_layout(c, n_tokens);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nch = (n_tokens + kChunk - 1) / kChunk;
+  int *pidx = at<int>(ws, W.y);  // (token, rank) buckets: scratch in the expert-output region
+  if ((s = launch(ep_plan_mask_kernel, dim3(nch), dim3(256), 0, st, topk_idx, n_tokens,
+                  c.top_k, c.n_experts, n_ranks, pidx, at<int>(ws, W.chunk_hist))) != MOE_OK)
+    return s;
+  return launch(permute_scatter_kernel, dim3(nch), dim3(256), 0, st, (const int *)pidx,
+                (const int *)at<int>(ws, W.chunk_hist), n_tokens, 2 * n_ranks, n_ranks, nch,
+                send_counts, send_offsets, send_perm, send_slot, CounterReset{nullptr, nullptr, 0});
+}
+
+moe_status moe_ep_pack(moe_handle h, const void *x, const int *topk_idx, const float *topk_gate,
+                       int n_tokens, int n_ranks, const int *send_perm,
+                       const int *send_offsets, void *x_send, int *idx_send, float *gate_send,
+                       void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config &c = h->cfg;
+  if (n_tokens < 0 || n_tokens > c.max_tokens || n_ranks < 1 || c.n_experts % n_ranks != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!x || !topk_idx || !topk_gate || !send_perm || !send_offsets || !x_send || !idx_send ||
+      !gate_send)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_send)) return MOE_ERR_ALIGNMENT;
+  const int n_pairs = n_tokens * n_ranks;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(grid_for((size_t)n_pairs, 8, h->num_sms));
+  if (c.dtype == MOE_BF16)
+    return launch(ep_pack_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                  static_cast<const __nv_bfloat16 *>(x), topk_idx, topk_gate, send_perm,
+                  send_offsets, n_ranks, n_pairs, c.d_model, c.top_k,
+                  static_cast<__nv_bfloat16 *>(x_send), idx_send, gate_send);
+  return launch(ep_pack_kernel<float>, grid, dim3(256), 0, st, static_cast<const float *>(x),
+                topk_idx, topk_gate, send_perm, send_offsets, n_ranks, n_pairs, c.d_model,
+                c.top_k, static_cast<float *>(x_send), idx_send, gate_send);
+}
+
+moe_status moe_ep_combine(moe_handle h, const float *back, const int *send_slot,
+                          const int *send_offsets, const float *shared, int n_tokens,
+                          int n_ranks, void *out, void *stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config &c = h->cfg;
+  if (n_tokens < 0 || n_tokens > c.max_tokens || n_ranks < 1 || c.n_experts % n_ranks != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MOE_OK;
+  if (!out || (back && (!send_slot || !send_offsets))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out) || (back && !aligned16(back)) || (shared && !aligned16(shared)))
+    return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(grid_for((size_t)n_tokens * (c.d_model / 4), 256, h->num_sms));
+  if (c.dtype == MOE_BF16)
+    return launch(ep_combine_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, back, send_slot,
+                  send_offsets, shared, n_tokens, n_ranks, c.d_model,
+                  static_cast<__nv_bfloat16 *>(out));
+  return launch(ep_combine_kernel<float>, grid, dim3(256), 0, st, back, send_slot, send_offsets,
+                shared, n_tokens, n_ranks, c.d_model, static_cast<float *>(out));
+}
+
+}  // extern "C"
+
 // ================================================== router logits with library-held scratch
 // For callers that cannot allocate device memory (see moe_router_logits_static in the
 // header): the split-K router's scratch -- partial sums [splits][T][E] and the per-expert-
@@ -1235,6 +1626,9 @@ extern "C" moe_status moe_router_logits_static(moe_handle h, const void *x, int 
     return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch size
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  // the scratch and the launch belong to the current device; the handle's weight pointers
+  // to the device it was created on
+  if (dev != h->device) return MOE_ERR_INVALID_ARG;
   void *base = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_static_mu);

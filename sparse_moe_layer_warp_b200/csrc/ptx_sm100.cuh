@@ -16,7 +16,9 @@ struct DevStatus {
   int error;             // 0 = ok, 1 = a bounded wait gave up
   int where;             // which wait (kernel-specific code)
   int sched[4];          // grouped-GEMM work counters (up, down), reset by the routing kernels
-  int pad[26];
+  int side_sched[2];     // the shared expert's up / down counters when it runs on the side
+                         // stream (cleared on that stream before its kernels)
+  int pad[24];
   int router_ticket[32]; // split-K router: arrivals per block of 32 experts; [31] also the
                          // decode router's last-CTA ticket (all self-resetting)
 };

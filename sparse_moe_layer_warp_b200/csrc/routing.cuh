@@ -670,14 +670,17 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
 }
 
 // ------------------------------------------------------------------ row gather
-// xs[p, :] = x[perm[p] / k, :] for p < n_rows: one warp per row (16-byte vectors, each lane
-// keeping several loads in flight), rows spread over all warps of the grid.
+// xs[p, :] = x[perm[p] / k, :] for p < n_rows (and p < *n_rows_dev when that is given: a
+// row count the routing computed on the device): one warp per row (16-byte vectors, each
+// lane keeping several loads in flight), rows spread over all warps of the grid.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
                                                           const int *__restrict__ perm, int k,
                                                           int n_rows, int vec_per_row,
-                                                          uint4 *__restrict__ xs) {
+                                                          uint4 *__restrict__ xs,
+                                                          const int *__restrict__ n_rows_dev) {
   griddep_wait();
   griddep_launch_dependents();
+  if (n_rows_dev) n_rows = min(n_rows, *n_rows_dev);
   const int lane = threadIdx.x & 31;
   const int n_warps = gridDim.x * (blockDim.x >> 5);
   for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < n_rows; p += n_warps) {

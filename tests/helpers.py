@@ -4,7 +4,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from oracle import oracle_moe_forward, oracle_permute, oracle_route
+from oracle import (oracle_gates, oracle_moe_forward, oracle_permute, oracle_route,
+                    oracle_router_logits)
 from sparse_moe_layer_warp_b200 import MoELayer, synth
 
 BF16_TOL = 2e-2   # max |err| <= 2e-2 * RMS(out) for bf16 weights/activations, fp32 accumulation
@@ -77,3 +78,76 @@ def check_routing_exact(layer: MoELayer, logits: torch.Tensor, bias_np, k, E):
     assert (g["slot_row"] == slot_row).all()
     np.testing.assert_allclose(g["gates"], gates, rtol=2e-6, atol=1e-30)
     return g
+
+
+def oracle_routing(inp: synth.LayerInputs):
+    """The oracle's own routing of the whole batch: logits [T, E], idx, gates [T, k],
+    counts [E], offsets [E + 1], perm [T*k], slot_row [T, k]."""
+    w = inp.w
+    x, wr, b, *_ = host_inputs(inp)
+    logits = oracle_router_logits(x, wr)
+    idx, gates = oracle_route(logits, b, w.k)
+    counts, offsets, perm, slot_row = oracle_permute(idx, w.E)
+    return dict(logits=logits, idx=idx, gates=gates, counts=counts, offsets=offsets,
+                perm=perm, slot_row=slot_row, bias=b)
+
+
+def check_full_routing(orc, gpu_idx, k):
+    """GPU selection of every token against the oracle's: identical slot by slot, except at
+    genuine near-ties (the oracle's k-th / (k+1)-th score gap below 1e-4), where the two
+    sides' fp32 logits (different accumulation orders) may order the scores differently.
+    Returns the number of such tokens."""
+    diff = ~(gpu_idx == orc["idx"]).all(axis=1)
+    if diff.any():
+        lg = orc["logits"][diff]
+        s = np.sort(lg.astype(np.float64) + orc["bias"].astype(np.float64), axis=1)[:, ::-1]
+        # a swap inside the selection needs a near-tie among the k selected scores, a
+        # different set one at the boundary: the smallest adjacent gap among the top k + 1
+        gaps = -np.diff(s[:, :min(k + 1, s.shape[1])], axis=1)
+        assert (gaps.min(axis=1) < 1e-4).all(), "routing differs away from a near-tie"
+    return int(diff.sum())
+
+
+def covering_tokens(orc, T, k, tile=128, extra=0, seed=7):
+    """Tokens whose outputs check every touched expert group of the oracle's routing: for
+    each group the first and last row (the last, ragged token tile), and both rows at every
+    multiple of `tile` inside it (the edges of the token tiles of 128 and 256 rows); the
+    shared group's first and last tokens and its first tile edges; plus `extra` random
+    tokens.  Returns sorted unique token ids."""
+    offs, perm = orc["offsets"], orc["perm"]
+    rows = []
+    for e in range(len(offs) - 1):
+        lo, hi = int(offs[e]), int(offs[e + 1])
+        if hi == lo:
+            continue
+        rows += [lo, hi - 1]
+        for m in range(tile, hi - lo, tile):
+            rows += [lo + m - 1, lo + m]
+    toks = set(int(perm[r]) // k for r in rows)
+    toks |= {t for t in (0, T - 1, tile - 1, tile, 2 * tile - 1, 2 * tile) if t < T}
+    if extra:
+        rng = np.random.default_rng(seed)
+        toks |= set(int(t) for t in rng.choice(T, min(extra, T), replace=False))
+    return np.array(sorted(toks), np.int32)
+
+
+def greedy_group_cover(orc, T, k, n_largest=8):
+    """A small token set whose selections together touch every touched routed expert (each
+    token covers its k experts; greedy set cover), plus the last token of each of the
+    `n_largest` largest groups (their last, ragged token tiles).  Every token also covers
+    the shared expert."""
+    idx = orc["idx"]
+    counts = orc["counts"]
+    touched = set(np.nonzero(counts)[0].tolist())
+    big = np.argsort(-counts, kind="stable")[:n_largest]
+    chosen = {int(orc["perm"][int(orc["offsets"][e + 1]) - 1]) // k for e in big
+              if counts[e] > 0}
+    covered = set()
+    for t in chosen:
+        covered |= set(idx[t].tolist())
+    while covered != touched:
+        gain = np.array([len(set(r.tolist()) - covered) for r in idx])
+        t = int(gain.argmax())
+        chosen.add(t)
+        covered |= set(idx[t].tolist())
+    return np.array(sorted(chosen), np.int32)

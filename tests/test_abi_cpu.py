@@ -33,7 +33,7 @@ def test_header_constants_match_binding():
     enums = dict((n, int(v)) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", text))
     defines = dict((n, int(v)) for n, v in
                    re.findall(r"^#define\s+(MOE_[A-Z0-9_]+)\s+(\d+)u?\s*$", text, flags=re.M))
-    assert len(enums) == 9 and len(defines) == 2
+    assert len(enums) == 9 and len(defines) == 4
     for name, value in {**enums, **defines}.items():
         assert getattr(binding, name) == value, name
     assert len(binding.PROFILE_STAGE_NAMES) == binding.MOE_PROFILE_STAGES
@@ -89,6 +89,8 @@ def test_null_handle_calls_rejected(lib):
                                 None) == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_health(None, 1, None, None, None, None, 0,
                                  None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_option(None, binding.MOE_OPTION_H_HANDOVER,
+                              0) == binding.MOE_ERR_INVALID_ARG
 
 
 def test_binding_refuses_strided_and_host_tensors(lib):

@@ -1,10 +1,12 @@
 """GPU parity for the layer backward (moe_backward) against the CPU oracle's chain rule, on
-the GPU's own selection (the oracle takes the same idx and gates)."""
+the GPU's own selection (the backward is defined for the forward's discrete choice of
+experts): the oracle takes the GPU's idx, and computes the gates of that selection itself
+from its own router logits."""
 import numpy as np
 import pytest
 import torch
 
-from oracle import oracle_moe_backward
+from oracle import oracle_gates, oracle_moe_backward, oracle_router_logits
 from sparse_moe_layer_warp_b200 import synth
 from tests.helpers import host_inputs, make_layer
 
@@ -57,8 +59,9 @@ def test_backward_matches_oracle(cuda_ok, kw):
     r = layer.route(x=inp.x)
     torch.cuda.synchronize()
     x, wr, _, wg, wu, wd = host_inputs(inp)
-    ref = oracle_moe_backward(x, synth.to_numpy_bits(dout), wr, wg, wu, wd,
-                              r["idx"].cpu().numpy(), r["gates"].cpu().numpy(),
+    idx = r["idx"].cpu().numpy()
+    gates = oracle_gates(oracle_router_logits(x, wr), idx)
+    ref = oracle_moe_backward(x, synth.to_numpy_bits(dout), wr, wg, wu, wd, idx, gates,
                               w.routed_scale, w.n_shared)
     counts = r["counts"].cpu().numpy()
     for name, want in ref.items():

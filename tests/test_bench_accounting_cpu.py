@@ -71,3 +71,22 @@ def test_dense_ffn_has_no_shared_rows():
     assert a["touched"] == 1
     assert a["layer_flops"] == 2 * 4096 * 3 * 4096 * 11264 + 2 * 4096 * 4096
     assert a["layer_bytes"] == 3 * 11264 * 4096 * 2 + 4096 * 2 + 2 * 4096 * 4096 * 2
+
+
+def test_layer_roofline_is_the_tensor_fraction_of_a_tensor_bound_forward():
+    """prefill_t8192 (every expert touched: 289 x 3 x 1280 x 4096 x 2 B + W_r + x + out =
+    9.23 GB, 2.34 TFLOP, 253 flop/B above the measured ridge of 1642.5 / 6554.2 = 250.6):
+    the bench line's roofline is the forward's flops over the step time against the burst
+    bf16 peak.  decode_t16 (1.4 flop/B) is HBM-bound: no layer tensor roofline."""
+    peaks = {"hbm_gbs": 6554.2, "bf16_tflops": 1642.5}
+    w = synth.WORKLOADS["prefill_t8192"]
+    a = bench.algorithmic(w, _counts(288, 288, 8192 * 8), 8192)
+    flops = 2 * (8192 * 8 + 8192) * 3 * 4096 * 1280 + 2 * 8192 * 4096 * 288
+    assert a["layer_flops"] == flops
+    r = bench.layer_roofline(a["layer_bytes"], a["layer_flops"], 2.85e-3, peaks)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["frac"] == round(flops / 2.85e-3 / 1e12 / 1642.5, 4)
+    assert 0.499 < r["frac"] < 0.501  # 2.3386 TFLOP in 2.85 ms is half the burst peak
+    d = synth.WORKLOADS["decode_t16"]
+    b = bench.algorithmic(d, _counts(288, 104, 16 * 8), 16)
+    assert bench.layer_roofline(b["layer_bytes"], b["layer_flops"], 0.5e-3, peaks) is None

@@ -7,7 +7,9 @@ import torch
 
 from oracle import oracle_router_logits
 from sparse_moe_layer_warp_b200 import synth
-from tests.helpers import check_routing_exact, compare_layer, host_inputs, make_layer
+from oracle import oracle_permute, oracle_route
+from tests.helpers import (check_full_routing, check_routing_exact, compare_layer,
+                           covering_tokens, host_inputs, make_layer, oracle_routing)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +40,45 @@ def test_route_nan_inf_signed_zero(cuda_ok):
     lg[1, 5] = -0.0
     lg[2, 10:20] = float("-inf")
     check_routing_exact(layer, lg.cuda(), np.zeros(40, np.float32), 6, 40)
+
+
+@pytest.mark.parametrize("T,bias,dup", [(1, "uniform", False), (5, "zipf", False),
+                                         (16, "uniform", False), (64, "zipf", False),
+                                         (16, "zero", True), (37, "uniform", False)])
+def test_decode_route_kernel_bit_exact(cuda_ok, T, bias, dup):
+    """moe_route(x) on a bf16 batch of at most 64 tokens runs the forward's one-launch
+    decode routing (router logits, top-k, gates, histogram, scan, permutation).  Its integer
+    outputs must equal the oracle's selection and permutation computed from the logits that
+    same launch wrote, bit for bit, and its gates the oracle's softmax of them.  dup: pairs
+    of experts with identical router rows and a zero bias, so their scores tie exactly and
+    the lower expert id must win."""
+    w = synth.Workload("route_dec", T=T, d=4096, E=288, k=8, f=128,
+                       bias="zipf" if bias == "zipf" else "uniform", seed=T)
+    inp = synth.make_inputs(w, device="cuda")
+    if bias == "zero":
+        inp.bias.zero_()
+    if dup:
+        inp.w_router[1::2] = inp.w_router[0::2]
+    layer = make_layer(inp)
+    from sparse_moe_layer_warp_b200 import moe_forward_launch_count
+    assert moe_forward_launch_count(layer.handle, T) == 4  # the one-launch routing plan
+    r = layer.route(x=inp.x, want_logits=True)
+    torch.cuda.synchronize()
+    lg = r["logits"].cpu().numpy()
+    b = inp.bias.cpu().numpy()
+    idx, gates = oracle_route(lg, b, w.k)
+    counts, offsets, perm, slot_row = oracle_permute(idx, w.E)
+    g = {kk: v.cpu().numpy() for kk, v in r.items()}
+    assert (g["idx"] == idx).all()
+    assert (g["counts"] == counts).all()
+    assert (g["offsets"] == offsets).all()
+    assert (g["perm"] == perm).all()
+    assert (g["slot_row"] == slot_row).all()
+    np.testing.assert_allclose(g["gates"], gates, rtol=2e-6, atol=1e-30)
+    if dup:  # some selection really contains a tied pair
+        assert any(((row // 2)[:, None] == (row // 2)[None, :]).sum() > len(row)
+                   for row in idx)
+    assert layer.device_status() == 0
 
 
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 64), ("decode_t16", 16), ("decode_t256", 256),
@@ -135,28 +176,45 @@ def test_forward_rejects_too_many_tokens(cuda_ok):
 
 
 # ------------------------------------------------------------ full-size workloads (sampled)
-FULL = [("decode_t16", None), ("decode_t256", 24), ("skew_t4096", 12), ("prefill_t8192", 12),
-        ("dense_ffn_t4096", 8)]
+# n_sample: None = every token; otherwise random tokens on top of the covering set
+FULL = [("decode_t16", None), ("decode_t256", None), ("skew_t4096", 16),
+        ("prefill_t8192", 16), ("dense_ffn_t4096", 8)]
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,n_sample", FULL)
 def test_forward_full_size_sampled(cuda_ok, name, n_sample):
+    """The bench's workloads at full size, in the launch configuration bench.py times
+    (max_tokens = the workload's T).  The oracle routes the whole batch itself; the GPU's
+    selection must equal it slot by slot for every token (near-ties aside), and the output
+    is compared on a token set that checks every touched expert group: each group's first
+    and last rows (the last, ragged token tile: e.g. the hottest expert of skew_t4096) and
+    the rows at both sides of every 128-row tile edge, the shared group's edges, plus random
+    tokens (every token with n_sample None)."""
     w = synth.WORKLOADS[name]
     inp = synth.make_inputs(w, device="cuda")
     layer = make_layer(inp)
     out = layer.forward(inp.x)
     r = layer.route(x=inp.x)
     torch.cuda.synchronize()
+    gpu_idx = r["idx"].cpu().numpy()
     counts = r["counts"].cpu().numpy()
     assert counts.sum() == w.T * w.k
-    rng = np.random.default_rng(7)
-    toks = None if n_sample is None else np.sort(rng.choice(w.T, n_sample, replace=False))
-    if toks is not None:
-        # always include the first and last tokens (edges of the last ragged tiles)
-        toks = np.unique(np.concatenate([[0, w.T - 1], toks]))
-    stats = compare_layer(inp, out, r["idx"].cpu().numpy(), tokens=toks)
-    print(name, stats, "empty experts:", int((counts == 0).sum()), "max load:", int(counts.max()))
+    orc = oracle_routing(inp)
+    n_diff = check_full_routing(orc, gpu_idx, w.k)
+    if n_diff == 0:
+        assert (counts == orc["counts"]).all()
+        assert (r["offsets"].cpu().numpy() == orc["offsets"]).all()
+        assert (r["perm"].cpu().numpy() == orc["perm"]).all()
+    if n_sample is None:
+        toks = None
+    else:
+        toks = covering_tokens(orc, w.T, w.k, extra=n_sample)
+        touched = set(np.nonzero(orc["counts"])[0].tolist())
+        assert set(orc["idx"][toks].ravel().tolist()) == touched
+    stats = compare_layer(inp, out, gpu_idx, tokens=toks)
+    print(name, stats, "routing near-tie tokens:", n_diff, "empty experts:",
+          int((counts == 0).sum()), "max load:", int(counts.max()))
     assert layer.device_status() == 0
     # properties that hold at any size: finite output, determinism
     assert torch.isfinite(out.float()).all()

@@ -1,0 +1,95 @@
+"""Launch-plan options of a handle (moe_set_option).
+
+MOE_OPTION_H_HANDOVER = 0 plans the bf16 forward's down-projection GEMM with a whole-grid
+wait on the up GEMM instead of the per-group hand-over of h (the plan the forward also takes
+when the init-time occupancy check finds an up grid that would not be co-resident).  Both
+plans run the same arithmetic in the same order, so their outputs must be equal bit for bit,
+and both must match the oracle."""
+import pytest
+import torch
+
+from sparse_moe_layer_warp_b200 import MOE_OPTION_H_HANDOVER, MoEError, synth
+from tests.helpers import compare_layer, make_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("kw", [
+    {"T": 16, "d": 512, "E": 64, "k": 8, "f": 256},               # one-CTA, rows gathered by TMA
+    {"T": 300, "d": 512, "E": 32, "k": 8, "f": 256},              # one-CTA, sorted copy of x
+    {"T": 700, "d": 768, "E": 8, "k": 4, "f": 512, "seed": 6},    # CTA pairs
+    {"T": 600, "d": 256, "E": 16, "k": 4, "f": 256, "seed": 4, "bias": "zipf"},  # skewed pairs
+])
+def test_whole_grid_wait_plan_matches_handover_plan(cuda_ok, kw):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", **kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    a = layer.forward(inp.x).clone()
+    layer.set_option(MOE_OPTION_H_HANDOVER, 0)
+    b = layer.forward(inp.x).clone()
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    compare_layer(inp, b, r["idx"].cpu().numpy())
+    layer.set_option(MOE_OPTION_H_HANDOVER, 1)
+    c = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+    assert layer.device_status() == 0
+
+
+def test_set_option_rejects_unknown(cuda_ok):
+    w = synth.WORKLOADS["tiny_fp32"]
+    layer = make_layer(synth.make_inputs(w, device="cuda"))
+    with pytest.raises(MoEError):
+        layer.set_option(99, 1)
+    with pytest.raises(MoEError):
+        layer.set_option(MOE_OPTION_H_HANDOVER, 2)
+
+
+PAIR_CASES = [
+    {"T": 700, "d": 768, "E": 8, "k": 4, "f": 512, "seed": 6},
+    {"T": 600, "d": 256, "E": 16, "k": 4, "f": 256, "seed": 4, "bias": "zipf"},
+    {"T": 1000, "d": 512, "E": 24, "k": 6, "f": 256, "seed": 8, "routed_scale": 1.5},
+]
+
+
+@pytest.mark.parametrize("kw", PAIR_CASES)
+@pytest.mark.parametrize("sms", [2, 32, 148])
+def test_shared_expert_on_side_stream_matches(cuda_ok, kw, sms):
+    """MOE_OPTION_SHARED_SIDE_SMS: the shared expert's GEMMs on the handle's side stream
+    during the routing give the same output bit for bit, eagerly and in a CUDA graph."""
+    from sparse_moe_layer_warp_b200 import MOE_OPTION_SHARED_SIDE_SMS, moe_forward_launch_count
+
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", **kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    ref = layer.forward(inp.x).clone()
+    n0 = moe_forward_launch_count(layer.handle, w.T)
+    layer.set_option(MOE_OPTION_SHARED_SIDE_SMS, sms)
+    assert moe_forward_launch_count(layer.handle, w.T) == n0 + 2  # the two side GEMMs
+    a = layer.forward(inp.x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
+    # captured: the fork and join are recorded into the graph
+    x = inp.x.clone()
+    out = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward(x, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, out=out)
+    x2 = synth.make_x(w, w.T, device="cuda", seed=11)
+    x.copy_(x2)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    layer.set_option(MOE_OPTION_SHARED_SIDE_SMS, 0)
+    b = layer.forward(x2)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), b.view(torch.int16))
+    del g
+    assert layer.device_status() == 0
