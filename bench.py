@@ -152,15 +152,15 @@ def layer_roofline(layer_bytes, layer_flops, step_s, peaks):
             "algorithmic_bytes_per_step": int(layer_bytes)}
 
 
-# the expert GEMM kernels' own sources (their device code and the PTX wrappers they use)
-GEMM_SOURCES = ("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx_sm100.cuh")
-
-
 def kernel_source_sha():
+    """sha256 (first 16 hex) of every kernel and launch source of the library: a committed
+    DRAM capture counts only while the code it measured is unchanged."""
     csrc = os.path.join(ROOT, "sparse_moe_layer_warp_b200", "csrc")
     h = hashlib.sha256()
-    for fn in GEMM_SOURCES:
-        h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(fn.encode())
+            h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
