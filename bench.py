@@ -525,7 +525,9 @@ def run_reference(args, rank, world):
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "tokens": w.T, "d_model": w.d, "n_experts": w.E,
-                       "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared},
+                       "top_k": w.k, "d_ff": w.f, "n_shared": w.n_shared,
+                       "parallelism": "rank 0 only (host cores)",
+                       "l2": "not applicable (host oracle)"},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
