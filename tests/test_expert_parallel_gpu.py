@@ -188,3 +188,58 @@ def test_slice_handle_refuses_whole_layer_calls(cuda_ok):
         binding.moe_forward_partial(ops.handle, inp.x, w.T, None, None, 0, e1, 0, 0, p, ws)
     assert e.value.status == binding.MOE_ERR_INVALID_ARG
     ops.close()
+
+
+@pytest.mark.parametrize("kw", CASES)
+def test_shared_expert_token_subranges(cuda_ok, kw):
+    """The shared expert on a token range that starts inside the batch (the all-gather
+    exchange gives each rank its own tokens' shared rows): three partials whose shared ranges
+    partition the tokens, one of them also holding every routed expert, sum to the layer."""
+    w, inp = _inputs(kw)
+    layer = make_layer(inp)
+    T = w.T
+    s0, s1 = T // 3, (2 * T) // 3 + 1
+    tot = _partial(layer, inp.x, 0, w.E, s0, s1)
+    tot += _partial(layer, inp.x, 0, 0, 0, s0)
+    tot += _partial(layer, inp.x, w.E, w.E, s1, T)
+    out = _round(layer, tot)
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    compare_layer(inp, out, r["idx"].cpu().numpy())
+    assert layer.device_status() == 0
+
+
+@pytest.mark.parametrize("kw", [CASES[0], CASES[2]])
+@pytest.mark.parametrize("R", [2, 4])
+def test_emulated_allgather_exchange_matches_oracle(cuda_ok, kw, R):
+    """ExpertParallelMoE's all-gather exchange emulated on one GPU: every rank (its own
+    handle over sliced weights) computes all ranks' tokens in its experts plus the shared
+    expert on its own tokens; the per-token sum of the ranks' partials (the reduce-scatter)
+    is rounded by moe_ep_combine."""
+    w, inp = _inputs(kw)
+    if w.E % R or w.T % R:
+        pytest.skip("experts or tokens do not split over the ranks")
+    T = w.T
+    Tr = T // R
+    ranks = []
+    for q in range(R):
+        e0, e1 = expert_range(w.E, q, R)
+        sl = lambda t: torch.cat([t[e0:e1], t[w.E:]]).contiguous()  # noqa: E731
+        ranks.append(LibraryOps(inp.w_router, inp.bias, sl(inp.w_gate), sl(inp.w_up),
+                                sl(inp.w_down), n_experts=w.E, top_k=w.k, max_tokens=Tr,
+                                rank=q, world=R, n_shared=w.n_shared,
+                                routed_scale=w.routed_scale))
+    # each rank routes its own tokens; the all-gather concatenates them in rank order
+    sel = [ranks[q].route(inp.x[q * Tr:(q + 1) * Tr].contiguous()) for q in range(R)]
+    ia = torch.cat([s[0] for s in sel])
+    ga = torch.cat([s[1] for s in sel])
+    tot = torch.zeros((T, w.d), dtype=torch.float32, device="cuda")
+    for q, ops in enumerate(ranks):
+        tot += ops.partial(inp.x, ia, ga, (ops.e0, ops.e1), (q * Tr, (q + 1) * Tr))
+    out = torch.cat([ranks[q].combine(None, None, None, tot[q * Tr:(q + 1) * Tr].contiguous(),
+                                      R, Tr) for q in range(R)])
+    full = make_layer(inp).route(x=inp.x)
+    torch.cuda.synchronize()
+    compare_layer(inp, out, full["idx"].cpu().numpy())
+    for ops in ranks:
+        ops.close()
