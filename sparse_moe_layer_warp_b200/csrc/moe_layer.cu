@@ -180,7 +180,7 @@ struct WsLayout {
 int pick_bn(const moe_config &c, int T, int mode);
 
 // The bf16 up GEMM gathers its token rows from x when its token tile is small; larger
-// tiles read an expert-sorted copy xs written by gather_rows_kernel.
+// tiles read an expert-sorted copy xs written by gather_rows_by_token_kernel.
 bool up_gathers_rows(const moe_config &c, int T) {
   return pick_bn(c, T, MODE_UP) <= kGatherMaxBN;
 }
@@ -1062,10 +1062,10 @@ moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
                              const int *n_rows_dev = nullptr) {
   if (plan.gather_in_gemm) return MOE_OK;
   const moe_config &c = h->cfg;
-  const int Tk = T * c.top_k;
-  return launch(gather_rows_kernel, dim3(grid_for((size_t)Tk, 8, h->num_sms)), dim3(256), 0, st,
-                static_cast<const uint4 *>(x), (const int *)at<int>(ws, W.perm), c.top_k, Tk,
-                c.d_model / 8, at<uint4>(ws, W.xs), n_rows_dev);
+  return launch(gather_rows_by_token_kernel, dim3(grid_for((size_t)T, 8, h->num_sms)),
+                dim3(256), 0, st, static_cast<const uint4 *>(x),
+                (const int *)at<int>(ws, W.slot_row), T, c.top_k, c.d_model / 8,
+                at<uint4>(ws, W.xs), n_rows_dev);
 }
 
 // bf16 expert up GEMM over the routing in `ws`: h (bf16, `out`) -- or, with out2 set, the

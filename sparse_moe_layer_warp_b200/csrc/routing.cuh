@@ -670,25 +670,41 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
 }
 
 // ------------------------------------------------------------------ row gather
-// xs[p, :] = x[perm[p] / k, :] for p < n_rows (and p < *n_rows_dev when that is given: a
-// row count the routing computed on the device): one warp per row (16-byte vectors, each
-// lane keeping several loads in flight), rows spread over all warps of the grid.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
-                                                          const int *__restrict__ perm, int k,
-                                                          int n_rows, int vec_per_row,
-                                                          uint4 *__restrict__ xs,
-                                                          const int *__restrict__ n_rows_dev) {
+// xs[p, :] = x[t, :] for every row p = slot_row[t, j] of the expert-sorted space (the sorted
+// copy of x that the up GEMM's larger token tiles load).
+// Written token by token: one warp per token reads its x row once
+// (chunks of four 16-byte vectors per lane in flight) and stores it to the k rows
+// slot_row[t, 0..k) of xs (rows at or past *n_rows_dev, when given, are skipped).  x is read
+// from HBM once instead of once per slot.
+__global__ void __launch_bounds__(256) gather_rows_by_token_kernel(
+    const uint4 *__restrict__ x, const int *__restrict__ slot_row, int T, int k,
+    int vec_per_row, uint4 *__restrict__ xs, const int *__restrict__ n_rows_dev) {
   griddep_wait();
   griddep_launch_dependents();
-  if (n_rows_dev) n_rows = min(n_rows, *n_rows_dev);
   const int lane = threadIdx.x & 31;
   const int n_warps = gridDim.x * (blockDim.x >> 5);
-  for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < n_rows; p += n_warps) {
-    const int t = __ldg(perm + p) / k;
+  const int n_rows = n_rows_dev ? *n_rows_dev : 0x7fffffff;
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += n_warps) {
+    const int my_row = lane < k ? __ldg(slot_row + (size_t)t * k + lane) : -1;
     const uint4 *__restrict__ src = x + (size_t)t * vec_per_row;
-    uint4 *__restrict__ dst = xs + (size_t)p * vec_per_row;
-#pragma unroll 4
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+    for (int v0 = 0; v0 < vec_per_row; v0 += 128) {
+      uint4 r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int v = v0 + 32 * i + lane;
+        if (v < vec_per_row) r[i] = __ldg(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const int p = __shfl_sync(0xffffffffu, my_row, j);
+        if (p >= n_rows) continue;
+        uint4 *__restrict__ dst = xs + (size_t)p * vec_per_row;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int v = v0 + 32 * i + lane;
+          if (v < vec_per_row) dst[v] = r[i];
+        }
+      }
+    }
   }
 }
 
