@@ -138,3 +138,39 @@ def test_layer_class_checks_shapes_and_types(lib):
     with pytest.raises(ValueError, match="CUDA tensors"):
         binding.MoELayer(good["w_router"], good["router_bias"], good["w_gate"], good["w_up"],
                          good["w_down"], top_k=2, max_tokens=8)
+
+
+def test_expert_parallel_and_option_calls_rejected_on_the_host(lib):
+    """The expert-parallel entry points and moe_set_option check their arguments before any
+    CUDA call: a null handle, an empty or out-of-range expert slice, a non-bf16 slice."""
+    cfg = binding.moe_config(16, 4096, 288, 8, 1280, 1, binding.MOE_BF16, 1.0)
+    w = binding.moe_weights(16, 0, 32, 48, 64)
+    h = ctypes.c_void_p()
+    ep = lib.moe_layer_init_ep
+    assert ep(None, ctypes.byref(w), 0, 36, ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+    for e0, e1 in ((36, 36), (40, 36), (-1, 36), (0, 289)):
+        assert ep(ctypes.byref(cfg), ctypes.byref(w), e0, e1,
+                  ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG, (e0, e1)
+    f32 = binding.moe_config(16, 4096, 288, 8, 1280, 1, binding.MOE_F32, 1.0)
+    assert ep(ctypes.byref(f32), ctypes.byref(w), 0, 36,
+              ctypes.byref(h)) == binding.MOE_ERR_UNSUPPORTED
+    assert lib.moe_forward_partial(None, None, 1, None, None, 0, 1, 0, 0, None, None, 0,
+                                   None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan(None, None, 1, 2, None, None, None, None, None, 0,
+                           None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_pack(None, None, None, None, 1, 2, None, None, None, None, None,
+                           None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_combine(None, None, None, None, None, 1, 2, None,
+                              None) == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_option(None, binding.MOE_OPTION_SHARED_SIDE_SMS,
+                              32) == binding.MOE_ERR_INVALID_ARG
+
+
+def test_expert_range_partition():
+    from sparse_moe_layer_warp_b200.expert_parallel import expert_range
+
+    parts = [expert_range(288, q, 8) for q in range(8)]
+    assert parts[0] == (0, 36) and parts[-1] == (252, 288)
+    assert all(parts[q][1] == parts[q + 1][0] for q in range(7))
+    with pytest.raises(ValueError):
+        expert_range(288, 0, 7)
