@@ -664,6 +664,91 @@ def run_backward(args, rank, world, local_rank):
         budget_s=min(args.cpu_budget, 10.0))})
 
 
+def run_ep_rank(args, rank, world, local_rank):
+    """One rank's device work in the expert-parallel layer (--ep-ranks R, emulated on this
+    GPU: no exchange is timed).  The global batch is R x T tokens (T = the workload's tokens
+    per rank); rank 0 holds EP group 0 (experts [0, E/R) and the shared expert).
+    allgather: its partial forward of all R x T tokens in its experts plus the shared expert
+    on its own T tokens, and the rounding of its T output rows.  alltoall: its partial forward
+    of the tokens the other ranks would send it (every token of the global batch with a slot
+    in its experts), and the per-token combine of its own T tokens' returned rows (taken as
+    the rows it computed itself) with its shared expert."""
+    import numpy as np
+    import torch
+
+    from sparse_moe_layer_warp_b200 import synth
+    from sparse_moe_layer_warp_b200.expert_parallel import LibraryOps, expert_range
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    R, T = args.ep_ranks, w.T
+    inp = synth.make_inputs(w, device=dev, T=1)
+    e0, e1 = expert_range(w.E, 0, R)
+    sl = lambda t: torch.cat([t[e0:e1], t[w.E:]]).contiguous()  # noqa: E731
+    ops = LibraryOps(inp.w_router, inp.bias, sl(inp.w_gate), sl(inp.w_up), sl(inp.w_down),
+                     n_experts=w.E, top_k=w.k, max_tokens=T, rank=0, world=R,
+                     n_shared=w.n_shared, routed_scale=w.routed_scale)
+    del inp
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    nb = args.steps + args.warmup
+    steps = []
+    for i in range(nb):
+        xg = synth.make_x(w, R * T, device=dev, seed=2000 + i)
+        idx, gates = ops.route(xg)
+        if args.ep_mode == "allgather":
+            steps.append((xg, idx, gates))
+        else:  # the received tokens: every token with a slot in this rank's experts
+            keep = ((idx >= e0) & (idx < e1)).any(dim=1).nonzero().squeeze(1)
+            steps.append((xg[keep].contiguous(), idx[keep].contiguous(),
+                          gates[keep].contiguous(), xg[:T].contiguous(), idx[:T].contiguous(),
+                          gates[:T].contiguous()))
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+
+    def one(s):
+        if args.ep_mode == "allgather":
+            xg, idx, gates = s
+            part = ops.partial(xg, idx, gates, (e0, e1), (0, T))
+            return ops.combine(None, None, None, part[:T].contiguous(), R, T)
+        xr, ir, gr, xo, io, go = s
+        part = ops.partial(xr, ir, gr, (e0, e1), (0, 0))
+        shared = ops.partial(xo, io, go, (e0, e0), (0, T))
+        return part, shared
+
+    for i in range(args.warmup):
+        flush.zero_()
+        one(steps[i])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(st)
+        one(steps[args.warmup + i])
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    rows = float(np.mean([s[0].shape[0] for s in steps[args.warmup:]]))
+    # bytes a rank must stream: its touched experts' weights once (plus the shared expert)
+    touched = float(np.mean([
+        int(torch.unique(s[1][((s[1] >= e0) & (s[1] < e1))]).numel()) for s in steps[args.warmup:]]))
+    wbytes = (touched + w.n_shared) * 3 * w.d * w.f * 2
+    # flops of the rank's expert work: its slots of the global batch and the shared expert
+    # on its own tokens (3 products of d x f per row)
+    slots = float(np.mean([int(((s[1] >= e0) & (s[1] < e1)).sum()) for s in steps[args.warmup:]]))
+    flops = 2.0 * (slots + T * w.n_shared) * 3 * w.d * w.f
+    peaks, src = load_peaks()
+    return {"pass": f"ep rank (emulated, {args.ep_mode})", "ep_ranks": R, "workload": w.name,
+            "tokens_per_rank": T, "rows_in_rank_partial": rows, "ms_per_step": round(ms, 4),
+            "rank_touched_experts": touched,
+            "rank_weight_bytes": int(wbytes),
+            "rank_weight_stream_frac_of_hbm": round(wbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "rank_slots": slots, "rank_flops": int(flops),
+            "rank_tensor_frac_burst": round(flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "note": "device steps of one rank only; the NCCL exchange is not timed (one GPU)"}
+
+
 def _routing_np(layer, x):
     r = layer.route(x=x)
     return r["idx"].cpu().numpy(), r["gates"].cpu().numpy()
@@ -684,8 +769,12 @@ def main():
     ap.add_argument("--saved", action="store_true",
                     help="with --pass backward: time moe_backward_saved on pre-activations "
                          "kept by a training forward (moe_forward_save) instead")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
-                    help="backward: time moe_backward instead (a separate measurement)")
+    ap.add_argument("--pass", dest="which", default="forward",
+                    choices=["forward", "backward", "ep"],
+                    help="backward: time moe_backward instead; ep: one rank's device work in "
+                         "the expert-parallel layer (separate measurements)")
+    ap.add_argument("--ep-ranks", type=int, default=8)
+    ap.add_argument("--ep-mode", default="allgather", choices=["allgather", "alltoall"])
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -708,8 +797,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=None)
     try:
-        res = (run_backward if args.which == "backward" else run_ours)(args, rank, world,
-                                                                       local_rank)
+        run = {"backward": run_backward, "ep": run_ep_rank}.get(args.which, run_ours)
+        res = run(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
