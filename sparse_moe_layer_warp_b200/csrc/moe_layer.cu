@@ -1175,7 +1175,6 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
     return s;
   const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
   __nv_bfloat16 *hbuf = at<__nv_bfloat16>(ws, W.h);
-  float *ybuf = at<float>(ws, W.y);
   // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
   // expert group for that group's rows of h (see grouped_gemm_kernel)
   GemmParams p1;
@@ -1193,7 +1192,7 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
     if (!encode_row_boxes(p2.tmBr, hbuf, c.d_ff, P)) return MOE_ERR_CUDA;
     p2.b_boxes = 1;
   }
-  p2.out = ybuf;
+  p2.out = at<float>(ws, W.y);
   p2.sched = &at<DevStatus>(ws, W.status)->sched[1];
   p2.M = c.d_model;
   p2.K = c.d_ff;
@@ -1205,7 +1204,6 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
   if ((s = pair ? launch_gemm_pair<MODE_DOWN>(h, p2, st)
                 : launch_gemm<MODE_DOWN>(h, bn2, p2, st)) != MOE_OK)
     return s;
-  (void)ybuf;
   return mark(6);
 }
 
@@ -1215,7 +1213,7 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
 // and the join event recorded after them (the caller's stream waits for it before the
 // combine).
 moe_status launch_shared_side(const moe_layer *h, const void *x, int T, void *ws,
-                              const WsLayout &W, const ForwardPlan &plan, cudaStream_t st) {
+                              const WsLayout &W, cudaStream_t st) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   DevStatus *status = at<DevStatus>(ws, W.status);
@@ -1264,7 +1262,6 @@ moe_status launch_shared_side(const moe_layer *h, const void *x, int T, void *ws
   p2.K = c.d_ff;
   p2.ld_out = c.d_model;
   if ((s = launch_gemm_pair<MODE_DOWN>(h, p2, sd, h->side_sms)) != MOE_OK) return s;
-  (void)plan;
   return cudaEventRecord(h->ev_join, sd) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 }  // namespace
@@ -1312,7 +1309,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   // overlap) nor with kept pre-activations (the training forward stores all rows in one up
   // launch)
   if (events || saved) plan.side_shared = false;
-  if (plan.side_shared && (s = launch_shared_side(h, x, T, ws, W, plan, st)) != MOE_OK) return s;
+  if (plan.side_shared && (s = launch_shared_side(h, x, T, ws, W, st)) != MOE_OK) return s;
   if (plan.decode_route) {
     if ((s = launch_route_decode(h, x, T, logits, idx, gate, at<int>(ws, W.counts), offsets,
                                  perm, slot_row, at<DevStatus>(ws, W.status), reset, st)) !=
