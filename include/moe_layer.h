@@ -117,9 +117,16 @@ moe_status moe_layer_destroy(moe_handle h);
  *                          forward records the fork and join into the graph).  Calls on one
  *                          handle from several host threads at once are not supported.
  *                          Not used by moe_forward_profiled or moe_forward_save.
+ *   MOE_OPTION_ROW_GATHER_IN_GEMM  1 (default): in bf16 forwards on CTA pairs with a shared
+ *                          expert, the up GEMM writes the expert-sorted copy of x itself (two
+ *                          warps of each CTA, while the CTAs run the shared expert's units,
+ *                          which read x directly and are claimed first); 0: a kernel of its own
+ *                          writes the copy before the up GEMM (same results, bit for bit).
+ *                          Off while the shared expert runs on the side stream.
  * MOE_ERR_INVALID_ARG for an unknown option or value. */
 #define MOE_OPTION_H_HANDOVER 1
 #define MOE_OPTION_SHARED_SIDE_SMS 2
+#define MOE_OPTION_ROW_GATHER_IN_GEMM 3
 moe_status moe_set_option(moe_handle h, int option, int value);
 
 /* Bytes of device workspace a call with n_tokens tokens needs (0 on bad arguments).
@@ -156,8 +163,9 @@ moe_status moe_forward(moe_handle h, const void *x, int n_tokens, void *out, voi
  * on `stream` around its kernel stages, for per-kernel timing with no profiler attached:
  *   events[0] before the router, then one event after each of the MOE_PROFILE_STAGES
  *   stages: 1 router logits, 2 top-k + gates + chunk histograms, 3 permutation scatter,
- *   4 row gather (bf16 with more than about 12 tokens per expert; otherwise empty, the
- *   expert-up kernel gathering the rows of x as it loads them), 5 expert up + SwiGLU,
+ *   4 row gather (bf16 with more than about 12 tokens per expert; empty when the expert-up
+ *   kernel gathers the rows of x as it loads them, or, on CTA pairs with
+ *   MOE_OPTION_ROW_GATHER_IN_GEMM, writes the sorted copy itself), 5 expert up + SwiGLU,
  *   6 expert down, 7 combine.
  *   For n_tokens <= 64 (bf16) stages 2-3 are one fused launch, timed as stage 2 (3 empty);
  *   with at most 288 experts and d_model <= 8192 stages 1-3 are one launch, timed as stage 1.

@@ -37,6 +37,7 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
 MOE_BACKWARD_OVERWRITE = 1
 MOE_OPTION_H_HANDOVER = 1
 MOE_OPTION_SHARED_SIDE_SMS = 2
+MOE_OPTION_ROW_GATHER_IN_GEMM = 3
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")

@@ -89,6 +89,19 @@ struct GemmParams {
   // shared_t0 on.  All zero for the whole layer.
   int wg_off_routed, wg_off_shared;
   int shared_t0;
+  // Claim the shared groups' units before all others (build_unit_table).
+  int shared_first;
+  // CTA-pair up kernel with gx_dst set: its gather warps write the expert-sorted copy of x
+  // (gx_dst [rows, d] = gx_src rows; token t to rows gx_slot_row[t*k .. t*k + k), rows at or
+  // past *gx_n_rows skipped when gx_n_rows is set) while the shared groups' units, which read
+  // x itself, run; a routed unit's loads wait until *gx_done = gx_T.  gx_claim and gx_done
+  // are zero at launch; gx_vec = 16-byte vectors per row.
+  const uint4 *gx_src;
+  uint4 *gx_dst;
+  const int *gx_slot_row;
+  const int *gx_n_rows;
+  int *gx_claim, *gx_done;
+  int gx_T, gx_vec;
 };
 
 // Weight group of work group g (see GemmParams::wg_off_routed).
@@ -195,17 +208,19 @@ __device__ __forceinline__ void store_block16_f32(float *out, int ld, int row0, 
 }
 
 // Work list of a grouped GEMM launch, built by every CTA from the routing's offsets:
-// grp_count / grp_row [G] by group id; order [G] = the groups with at least one full token
-// tile of BN rows ("heavy": tensor-bound, their weight tiles shared by several token tiles)
-// in id order, then the others ("light": a few tokens each, bound by streaming their weights
-// from HBM) in id order; unit_prefix [G + 1] = exclusive prefix of the units (m tiles x
-// token tiles) over that order.  *n_heavy = units of the heavy groups.  With more than
-// kOrderMaxGroups groups the order is the identity (no array) and *n_heavy = 0.  Called by
+// grp_count / grp_row [G] by group id; order [G] = the shared groups when p.shared_first is
+// set ("first"), then the groups with at least one full token tile of BN rows ("heavy":
+// tensor-bound, their weight tiles shared by several token tiles), then the others ("light":
+// a few tokens each, bound by streaming their weights from HBM), each class in id order;
+// unit_prefix [G + 1] = exclusive prefix of the units (m tiles x token tiles) over that
+// order.  *n_first = units of the first class, *n_heavy = units of the heavy class.  With more
+// than kOrderMaxGroups groups the order is the identity (no array) and both are 0.  Called by
 // all threads of the CTA (it synchronises them).
 template <int BN>
 __device__ __forceinline__ void build_unit_table(const GemmParams &p, int mtiles,
                                                  int *unit_prefix, int *grp_count,
-                                                 int *grp_row, int *order, int *n_heavy) {
+                                                 int *grp_row, int *order, int *n_first,
+                                                 int *n_heavy) {
   const int G = p.n_groups;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -222,23 +237,38 @@ __device__ __forceinline__ void build_unit_table(const GemmParams &p, int mtiles
   }
   __syncthreads();
   if (warp == 0) {
-    // each lane a contiguous run of groups: heavy groups to the front, stable
+    // each lane a contiguous run of groups, partitioned stably into the three classes
     const int per = (G + 31) / 32;
     const int lo = min(G, lane * per), hi = min(G, lo + per);
-    int nh = 0;
-    if (order)
-      for (int g = lo; g < hi; ++g) nh += grp_count[g] >= BN;
-    int incl = nh;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int heavy_groups = __shfl_sync(0xffffffffu, incl, 31);
-    int hpos = incl - nh, lpos = heavy_groups + (lo - (incl - nh));
+    auto cls = [&](int g) {
+      return (p.shared_first && g >= p.E) ? 0 : (grp_count[g] >= BN ? 1 : 2);
+    };
+    int nf = 0, nh = 0;
     if (order)
       for (int g = lo; g < hi; ++g) {
-        if (grp_count[g] >= BN) order[hpos++] = g;
+        const int c = cls(g);
+        nf += c == 0;
+        nh += c == 1;
+      }
+    int inf = nf, inh = nh;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yf = __shfl_up_sync(0xffffffffu, inf, o);
+      const int yh = __shfl_up_sync(0xffffffffu, inh, o);
+      if (lane >= o) {
+        inf += yf;
+        inh += yh;
+      }
+    }
+    const int first_groups = __shfl_sync(0xffffffffu, inf, 31);
+    const int heavy_groups = __shfl_sync(0xffffffffu, inh, 31);
+    int fpos = inf - nf, hpos = first_groups + inh - nh;
+    int lpos = first_groups + heavy_groups + (lo - (inf - nf) - (inh - nh));
+    if (order)
+      for (int g = lo; g < hi; ++g) {
+        const int c = cls(g);
+        if (c == 0) order[fpos++] = g;
+        else if (c == 1) order[hpos++] = g;
         else order[lpos++] = g;
       }
     __syncwarp();
@@ -246,7 +276,7 @@ __device__ __forceinline__ void build_unit_table(const GemmParams &p, int mtiles
     auto grp_at = [&](int i) { return order ? order[i] : i; };
     int run = 0;
     for (int i = lo; i < hi; ++i) run += mtiles * ((grp_count[grp_at(i)] + BN - 1) / BN);
-    incl = run;
+    int incl = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -260,20 +290,27 @@ __device__ __forceinline__ void build_unit_table(const GemmParams &p, int mtiles
     }
     if (lane == 31) unit_prefix[G] = incl;
     __syncwarp();
-    if (lane == 0) *n_heavy = unit_prefix[heavy_groups];
+    if (lane == 0) {
+      *n_first = unit_prefix[first_groups];
+      *n_heavy = unit_prefix[first_groups + heavy_groups] - unit_prefix[first_groups];
+    }
   }
   __syncthreads();
 }
 
-// Claim order: ticket c of [0, total) -> unit.  The heavy units (the first n_heavy of the
-// ordered list) are spread evenly over the tickets (ticket c is heavy iff
-// floor((c+1) n_heavy / total) > floor(c n_heavy / total)), the light ones fill the rest in
+// Claim order: ticket c of [0, total) -> unit.  The first n_first tickets take the first
+// class's units in order; over the rest the heavy units (the next n_heavy of the ordered
+// list) are spread evenly (ticket c' = c - n_first of rest = total - n_first is heavy iff
+// floor((c'+1) n_heavy / rest) > floor(c' n_heavy / rest)) and the light ones fill the gaps in
 // order, so the CTAs run tensor-bound and HBM-bound units side by side instead of one kind
 // after the other.  A bijection of [0, total).
-__device__ __forceinline__ int unit_of_ticket(int c, int n_heavy, int total) {
-  const long long h0 = (long long)c * n_heavy / total;
-  const long long h1 = (long long)(c + 1) * n_heavy / total;
-  return h1 > h0 ? (int)h0 : n_heavy + (c - (int)h0);
+__device__ __forceinline__ int unit_of_ticket(int c, int n_first, int n_heavy, int total) {
+  if (c < n_first) return c;
+  c -= n_first;
+  const int rest = total - n_first;
+  const long long h0 = (long long)c * n_heavy / rest;
+  const long long h1 = (long long)(c + 1) * n_heavy / rest;
+  return n_first + (h1 > h0 ? (int)h0 : n_heavy + (c - (int)h0));
 }
 
 // unit -> (group, m tile, token tile) over the ordered list: token tile innermost, so the
@@ -319,6 +356,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
+  int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -367,13 +405,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
   // group table (token count, first row in the sorted space) and the cost-ordered work list
-  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_heavy_s);
+  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_first_s,
+                       n_heavy_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = unit_prefix[G];
   const int n_heavy = *n_heavy_s;
+  const int n_first = *n_first_s;
 
   auto decode = [&](int u, int &g, int &mt, int &nt) {
     decode_unit(u, G, unit_prefix, order, grp_count, BN, g, mt, nt);
@@ -410,7 +450,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int uid = -1;
       if (lane == 0) {
         u = claim(u);
-        uid = (u < total_units) ? unit_of_ticket(u, n_heavy, total_units) : -1;
+        uid = (u < total_units) ? unit_of_ticket(u, n_first, n_heavy, total_units) : -1;
         if (mbar_wait_bounded(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 5)) {
           uq[qi] = uid;
           mbar_arrive(&uq_full[qi]);

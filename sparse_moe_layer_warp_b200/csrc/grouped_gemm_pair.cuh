@@ -18,6 +18,13 @@
 // signal it through the .cta_group::2 load form); the leader's MMA commits arrive on empty[s]
 // and tmem_full[a] of both CTAs; tmem_empty[a] (leader) collects one arrival per epilogue
 // warp of both CTAs.  All waits are bounded as in grouped_gemm.cuh.
+//
+// Row gather inside the up kernel (GemmParams::gx_dst): two more warps per CTA write the
+// expert-sorted copy of x, token by token (each x row read once, stored to its k rows), in
+// chunks claimed from a counter, while the CTAs run the shared expert's units -- claimed
+// first (shared_first), they read x itself and are tensor-bound with L2-resident operands, so
+// the copy's HBM writes overlap them instead of taking a launch of their own before the GEMM.
+// A routed unit's token loads wait (bounded) for the count of gathered tokens.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,11 +40,15 @@ constexpr int kPairBN = 256;  // tokens per unit (both CTAs)
 // warps: 0 producer, 1 MMA (leader) / TMEM owner, 2..9 epilogue -- two per TMEM lane
 // quadrant (warp % 4), splitting a unit's 16-column chunks between them
 constexpr int kPairEpiWarps = 8;
-constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
+// up kernel: warps 10, 11 gather rows of x (idle when the copy is already written)
+constexpr int kPairGatherWarps = 2;
+constexpr int kGatherChunk = 4;  // tokens per claim of a gather warp
 
 template <int MODE>
 struct PairCfg {
   static constexpr int NA = (MODE == MODE_UP) ? 2 : 1;
+  static constexpr int THREADS =
+      32 * (2 + kPairEpiWarps + (MODE == MODE_UP ? kPairGatherWarps : 0));
   static constexpr int HALF_BN = kPairBN / 2;
   static constexpr int A_BYTES = 128 * kBK * 2;      // this CTA's 128 weight rows
   static constexpr int B_BYTES = HALF_BN * kBK * 2;  // this CTA's token rows
@@ -57,8 +68,56 @@ struct PairCfg {
   }
 };
 
+// One gather warp of the up kernel: claims kGatherChunk tokens at a time until every token is
+// claimed; per token the warp reads the x row once (16-byte vectors, up to 16 per lane in
+// flight) and stores it to the token's k rows of the sorted copy (L2 evict-first: the copy is
+// far larger than L2 and is read back tile by tile later, while x and the running units'
+// operands should stay), then publishes the chunk (stores, fence, count).
+__device__ __forceinline__ void gather_token_rows(const GemmParams &p, int lane) {
+  const int k = p.topk, vec = p.gx_vec, T = p.gx_T;
+  const int n_rows = p.gx_n_rows ? *p.gx_n_rows : 0x7fffffff;
+  const uint64_t pol = policy_evict_first();
+  for (;;) {
+    int c = 0;
+    if (lane == 0) c = atomicAdd(p.gx_claim, 1);
+    c = __shfl_sync(0xffffffffu, c, 0);
+    const int t0 = c * kGatherChunk;
+    if (t0 >= T) break;
+    const int t1 = min(T, t0 + kGatherChunk);
+    for (int t = t0; t < t1; ++t) {
+      const int my_row = lane < k ? __ldg(p.gx_slot_row + (size_t)t * k + lane) : -1;
+      const uint4 *__restrict__ src = p.gx_src + (size_t)t * vec;
+      for (int v0 = 0; v0 < vec; v0 += 512) {
+        uint4 r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int v = v0 + 32 * i + lane;
+          if (v < vec) r[i] = __ldg(src + v);
+        }
+        for (int j = 0; j < k; ++j) {
+          const int row = __shfl_sync(0xffffffffu, my_row, j);
+          if (row >= n_rows) continue;
+          uint4 *__restrict__ dst = p.gx_dst + (size_t)row * vec;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int v = v0 + 32 * i + lane;
+            if (v < vec) st_global_v4_hint(dst + v, r[i], pol);
+          }
+        }
+      }
+    }
+    // publish: every lane's stores, then the count (as the h hand-over does)
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(p.gx_done, t1 - t0);
+    }
+  }
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kPairThreads, 1)
+__global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
   using C = PairCfg<MODE>;
   constexpr int S = C::STAGES;
@@ -81,6 +140,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
+  int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -131,7 +191,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (!(MODE == MODE_DOWN && p.done)) griddep_wait();
   griddep_launch_dependents();
   // group table and the cost-ordered work list (see build_unit_table)
-  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_heavy_s);
+  build_unit_table<BN>(p, mtiles, unit_prefix, grp_count, grp_row, order, n_first_s,
+                       n_heavy_s);
   // both CTAs' barriers are initialised and TMEM allocated before any cross-CTA traffic
   tc_fence_before();
   __syncthreads();
@@ -140,6 +201,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = unit_prefix[G];
   const int n_heavy = *n_heavy_s;
+  const int n_first = *n_first_s;
 
   auto decode = [&](int u, int &g, int &mt, int &nt) {
     decode_unit(u, G, unit_prefix, order, grp_count, BN, g, mt, nt);
@@ -171,11 +233,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       uint32_t qph = 0;
       int u = -1;
       int ready_group = -1;  // down kernel: group whose h is known to be complete
+      bool gathered = !(MODE == MODE_UP && p.gx_dst);  // up: the sorted copy is complete
       while (ok) {
         // the leader claims the next unit and publishes its id to both CTAs; the peer reads it
         if (leader) {
           u = claim(u);
-          const int uid = (u < total_units) ? unit_of_ticket(u, n_heavy, total_units) : -1;
+          const int uid =
+              (u < total_units) ? unit_of_ticket(u, n_first, n_heavy, total_units) : -1;
           if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 15)) {
             ok = false;
             break;
@@ -222,6 +286,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
           fence_proxy_async_global();  // the h rows are read through TMA below
           ready_group = g;
+        }
+        if (MODE == MODE_UP && !gathered && !shared_x) {
+          // both CTAs load rows of the sorted copy: each waits for every token's rows
+          if (!counter_wait_bounded(p.gx_done, p.gx_T, abort_flag, p.status, 20)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // written by the gather warps' stores, read by TMA
+          gathered = true;
         }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 11)) {
@@ -314,6 +387,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       mbar_wait_bounded(drain, 0, &no_abort, nullptr, 0);
     }
     __syncwarp();
+  } else if (warp >= 2 + kPairEpiWarps) {
+    // ---------------------------------------------------------------- row gather (up)
+    if (MODE == MODE_UP && p.gx_dst) gather_token_rows(p, lane);
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;         // TMEM lane quadrant

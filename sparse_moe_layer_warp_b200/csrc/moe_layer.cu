@@ -59,6 +59,7 @@ struct moe_layer {
   // (MOE_OPTION_H_HANDOVER).  Without it the down GEMM waits for the whole up GEMM.
   int handover_fits;
   int opt_handover;
+  int opt_gather_in_gemm;  // MOE_OPTION_ROW_GATHER_IN_GEMM
   // experts whose weights the handle holds: [e0, e1) (the whole layer: [0, E)); the weight
   // tensors hold e1 - e0 routed experts then the shared expert (moe_layer_init_ep)
   int e0, e1;
@@ -382,7 +383,7 @@ int pair_grid_size(const moe_layer *L) {
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3(L->num_sms & ~1);
-  cfg.blockDim = dim3(kPairThreads);
+  cfg.blockDim = dim3(PairCfg<MODE>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -483,7 +484,8 @@ moe_status launch_gemm_pair(const moe_layer *L, const GemmParams &p, cudaStream_
     return MOE_ERR_CUDA;
   int grid = L->pair_grid[MODE == MODE_UP ? 0 : 1];
   if (max_ctas >= 2 && max_ctas < grid) grid = max_ctas & ~1;
-  return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(kPairThreads), smem, st, 2,
+  return launch_cl(grouped_gemm_pair_kernel<MODE>, dim3(grid), dim3(PairCfg<MODE>::THREADS), smem,
+                   st, 2,
                    p);
 }
 
@@ -727,6 +729,7 @@ static moe_status layer_init(const moe_config *cfg, const moe_weights *w, int e0
     return MOE_ERR_UNSUPPORTED;
   }
   L->opt_handover = 1;
+  L->opt_gather_in_gemm = 1;
   if (c.dtype == MOE_BF16) {
     L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
@@ -793,6 +796,10 @@ moe_status moe_set_option(moe_handle h, int option, int value) {
           return MOE_ERR_CUDA;
       }
       h->side_sms = value & ~1;  // whole CTA pairs
+      return MOE_OK;
+    case MOE_OPTION_ROW_GATHER_IN_GEMM:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      h->opt_gather_in_gemm = value;
       return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
@@ -1032,6 +1039,8 @@ struct ForwardPlan {
   bool small_route;   // selection + permutation in one launch after the router
   bool pair;          // CTA-pair grouped GEMMs
   bool gather_in_gemm;  // the up GEMM gathers x rows itself (no gather launch)
+  bool gather_in_pair;  // the CTA-pair up GEMM's gather warps write the sorted copy of x
+                        // during the shared expert's units (no gather launch)
   bool handover;        // the down GEMM takes h from the up GEMM group by group
   bool side_shared;     // the shared expert's GEMMs run on the side stream during routing
   int launches;
@@ -1046,12 +1055,13 @@ ForwardPlan plan_forward(const moe_layer *L, int T) {
   f.gather_in_gemm = c.dtype == MOE_BF16 && !f.pair && up_gathers_rows(c, T);
   f.handover = c.dtype == MOE_BF16 && L->handover_fits && L->opt_handover;
   f.side_shared = f.pair && c.n_shared && L->side_sms >= 2 && L->side != nullptr;
+  f.gather_in_pair = f.pair && c.n_shared && !f.side_shared && L->opt_gather_in_gemm;
   if (T == 0) {
     f.launches = 0;
     return f;
   }
   const int routing = f.decode_route ? 1 : (f.small_route ? 2 : 3);
-  const int gather = (c.dtype == MOE_BF16 && !f.gather_in_gemm) ? 1 : 0;
+  const int gather = (c.dtype == MOE_BF16 && !f.gather_in_gemm && !f.gather_in_pair) ? 1 : 0;
   f.launches = routing + gather + 3 + (f.side_shared ? 2 : 0);  // + up, down, combine
   return f;
 }
@@ -1060,7 +1070,7 @@ ForwardPlan plan_forward(const moe_layer *L, int T) {
 moe_status launch_row_gather(const moe_layer *h, const void *x, int T, void *ws,
                              const WsLayout &W, const ForwardPlan &plan, cudaStream_t st,
                              const int *n_rows_dev = nullptr) {
-  if (plan.gather_in_gemm) return MOE_OK;
+  if (plan.gather_in_gemm || plan.gather_in_pair) return MOE_OK;
   const moe_config &c = h->cfg;
   return launch(gather_rows_by_token_kernel, dim3(grid_for((size_t)T, 8, h->num_sms)),
                 dim3(256), 0, st, static_cast<const uint4 *>(x),
@@ -1090,11 +1100,14 @@ struct Slice {
   int n_routed, wg_off_routed, wg_off_shared, shared_t0, shared_n;
 };
 
+// gather_rows: the CTA-pair kernel writes the sorted copy of x itself (rows at or past
+// *n_rows_dev skipped, when given) and claims the shared group's units first.
 moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
                             const WsLayout &W, const ForwardPlan &plan, void *out, float *out2,
                             int *done, cudaStream_t st, GemmParams *used,
                             const UpRows *rows = nullptr, float *save_a = nullptr,
-                            float *save_b = nullptr, const Slice *slice = nullptr) {
+                            float *save_b = nullptr, const Slice *slice = nullptr,
+                            bool gather_rows = false, const int *n_rows_dev = nullptr) {
   const moe_config &c = h->cfg;
   const int Tk = T * c.top_k;
   // token rows per TMA box: the pair kernels stage half of a 256-token tile per CTA
@@ -1149,6 +1162,18 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
     p1.wg_off_routed = slice->wg_off_routed;
     p1.wg_off_shared = slice->wg_off_shared;
   }
+  if (gather_rows && plan.pair && !rows) {
+    DevStatus *status = at<DevStatus>(ws, W.status);
+    p1.shared_first = 1;
+    p1.gx_src = static_cast<const uint4 *>(x);
+    p1.gx_dst = at<uint4>(ws, W.xs);
+    p1.gx_slot_row = at<int>(ws, W.slot_row);
+    p1.gx_n_rows = n_rows_dev;
+    p1.gx_claim = &status->sched[4];
+    p1.gx_done = &status->sched[5];
+    p1.gx_T = T;
+    p1.gx_vec = c.d_model / 8;
+  }
   return plan.pair ? launch_gemm_pair<MODE_UP>(h, p1, st) : launch_gemm<MODE_UP>(h, bn, p1, st);
 }
 
@@ -1168,9 +1193,13 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
                                                                                  : MOE_ERR_CUDA;
   };
   moe_status s;
-  const bool pair = plan.pair;
+  ForwardPlan pl = plan;
+  // the up kernel gathers the rows while it runs the shared expert's units: not in a launch
+  // without them
+  if (slice && slice->shared_n == 0) pl.gather_in_pair = false;
+  const bool pair = pl.pair;
   const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
-  if ((s = launch_row_gather(h, x, T, ws, W, plan, st, n_rows_dev)) != MOE_OK ||
+  if ((s = launch_row_gather(h, x, T, ws, W, pl, st, n_rows_dev)) != MOE_OK ||
       (s = mark(4)) != MOE_OK)
     return s;
   const int bn2 = pair ? PairCfg<MODE_DOWN>::HALF_BN : pick_bn(c, T, MODE_DOWN);
@@ -1178,13 +1207,14 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
   // the down kernel starts on the SMs the up kernel leaves in its last wave and waits per
   // expert group for that group's rows of h (see grouped_gemm_kernel)
   GemmParams p1;
-  if ((s = launch_expert_up(h, x, T, ws, W, plan, hbuf, nullptr,
-                            plan.handover ? at<int>(ws, W.done) : nullptr, st, &p1, nullptr,
-                            saved, saved ? saved + (size_t)P * c.d_ff : nullptr, slice)) !=
-      MOE_OK)
+  if ((s = launch_expert_up(h, x, T, ws, W, pl, hbuf, nullptr,
+                            pl.handover ? at<int>(ws, W.done) : nullptr, st, &p1, nullptr,
+                            saved, saved ? saved + (size_t)P * c.d_ff : nullptr, slice,
+                            pl.gather_in_pair, n_rows_dev)) != MOE_OK)
     return s;
   if ((s = mark(5)) != MOE_OK) return s;
-  GemmParams p2 = p1;
+  GemmParams p2 = p1;  // shared_first carries over: the shared group's h is complete first
+  p2.gx_dst = nullptr;
   p2.tmA0 = h->tm_wd;
   if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
   p2.b_boxes = 0;
@@ -1308,7 +1338,10 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   // the shared expert beside the routing: not with per-stage events (their stages would
   // overlap) nor with kept pre-activations (the training forward stores all rows in one up
   // launch)
-  if (events || saved) plan.side_shared = false;
+  if (events || saved) {
+    plan.side_shared = false;
+    plan.gather_in_pair = plan.pair && c.n_shared && h->opt_gather_in_gemm;
+  }
   if (plan.side_shared && (s = launch_shared_side(h, x, T, ws, W, st)) != MOE_OK) return s;
   if (plan.decode_route) {
     if ((s = launch_route_decode(h, x, T, logits, idx, gate, at<int>(ws, W.counts), offsets,

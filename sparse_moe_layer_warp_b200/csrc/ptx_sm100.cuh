@@ -15,10 +15,12 @@ namespace moe {
 struct DevStatus {
   int error;             // 0 = ok, 1 = a bounded wait gave up
   int where;             // which wait (kernel-specific code)
-  int sched[4];          // grouped-GEMM work counters (up, down), reset by the routing kernels
+  int sched[8];          // work counters reset by the routing kernels: [0] up and [1] down
+                         // grouped-GEMM units ([2], [3] the backward's), [4] row-gather
+                         // chunks claimed and [5] tokens gathered by the CTA-pair up kernel
   int side_sched[2];     // the shared expert's up / down counters when it runs on the side
                          // stream (cleared on that stream before its kernels)
-  int pad[24];
+  int pad[20];
   int router_ticket[32]; // split-K router: arrivals per block of 32 experts; [31] also the
                          // decode router's last-CTA ticket (all self-resetting)
 };
@@ -216,6 +218,13 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// 16-byte global store with an L2 cache policy (createpolicy)
+__device__ __forceinline__ void st_global_v4_hint(uint4 *dst, const uint4 &v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
 }
 
 // ------------------------------------------------------------------------- tcgen05

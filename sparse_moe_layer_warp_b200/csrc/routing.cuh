@@ -15,17 +15,17 @@
 namespace moe {
 
 // Work counters of the expert kernels that follow a routing launch, zeroed by that launch
-// (block 0) so every forward starts from zero: the grouped GEMMs' unit counters (two ints)
-// and the fused FFN's per-group completion counts.
+// (block 0) so every forward starts from zero: the grouped GEMMs' unit and row-gather
+// counters (DevStatus::sched) and the per-group completion counts of the h hand-over.
 struct CounterReset {
-  int *sched;  // [4] or null
+  int *sched;  // [8] or null
   int *done;   // [n_done] or null
   int n_done;
   __device__ __forceinline__ void apply() const {
     if (blockIdx.x == 0) run();
   }
   __device__ __forceinline__ void run() const {  // by the whole of one CTA
-    if (sched && threadIdx.x < 4) sched[threadIdx.x] = 0;
+    if (sched && threadIdx.x < 8) sched[threadIdx.x] = 0;
     if (done)
       for (int i = threadIdx.x; i < n_done; i += blockDim.x) done[i] = 0;
   }

@@ -33,7 +33,7 @@ def test_header_constants_match_binding():
     enums = dict((n, int(v)) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", text))
     defines = dict((n, int(v)) for n, v in
                    re.findall(r"^#define\s+(MOE_[A-Z0-9_]+)\s+(\d+)u?\s*$", text, flags=re.M))
-    assert len(enums) == 9 and len(defines) == 4
+    assert len(enums) == 9 and len(defines) == 5
     for name, value in {**enums, **defines}.items():
         assert getattr(binding, name) == value, name
     assert len(binding.PROFILE_STAGE_NAMES) == binding.MOE_PROFILE_STAGES

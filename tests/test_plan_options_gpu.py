@@ -4,11 +4,14 @@ MOE_OPTION_H_HANDOVER = 0 plans the bf16 forward's down-projection GEMM with a w
 wait on the up GEMM instead of the per-group hand-over of h (the plan the forward also takes
 when the init-time occupancy check finds an up grid that would not be co-resident).  Both
 plans run the same arithmetic in the same order, so their outputs must be equal bit for bit,
-and both must match the oracle."""
+and both must match the oracle.  MOE_OPTION_ROW_GATHER_IN_GEMM = 0 writes the expert-sorted
+copy of x with a kernel of its own instead of the CTA-pair up GEMM's gather warps: same
+bytes in the copy, same results bit for bit."""
 import pytest
 import torch
 
-from sparse_moe_layer_warp_b200 import MOE_OPTION_H_HANDOVER, MoEError, synth
+from sparse_moe_layer_warp_b200 import (MOE_OPTION_H_HANDOVER, MOE_OPTION_ROW_GATHER_IN_GEMM,
+                                        MoEError, synth)
 from tests.helpers import compare_layer, make_layer
 
 pytestmark = pytest.mark.gpu
@@ -67,7 +70,9 @@ def test_shared_expert_on_side_stream_matches(cuda_ok, kw, sms):
     ref = layer.forward(inp.x).clone()
     n0 = moe_forward_launch_count(layer.handle, w.T)
     layer.set_option(MOE_OPTION_SHARED_SIDE_SMS, sms)
-    assert moe_forward_launch_count(layer.handle, w.T) == n0 + 2  # the two side GEMMs
+    # the two side GEMMs, and the row gather's own launch (the up GEMM gathers the rows
+    # itself only while it runs the shared expert's units)
+    assert moe_forward_launch_count(layer.handle, w.T) == n0 + 3
     a = layer.forward(inp.x).clone()
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
@@ -93,3 +98,35 @@ def test_shared_expert_on_side_stream_matches(cuda_ok, kw, sms):
     assert torch.equal(out.view(torch.int16), b.view(torch.int16))
     del g
     assert layer.device_status() == 0
+
+
+@pytest.mark.parametrize("kw", PAIR_CASES + [
+    {"T": 900, "d": 512, "E": 16, "k": 4, "f": 256, "seed": 9, "n_shared": 0},  # no shared
+])
+def test_row_gather_in_up_gemm_matches_own_launch(cuda_ok, kw):
+    """The CTA-pair up GEMM's own row gather (default) against the gather kernel: outputs
+    equal bit for bit, both equal to the oracle; one launch fewer with a shared expert."""
+    from sparse_moe_layer_warp_b200 import moe_forward_launch_count
+
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", **kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    n1 = moe_forward_launch_count(layer.handle, w.T)
+    a = layer.forward(inp.x).clone()
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 0)
+    assert moe_forward_launch_count(layer.handle, w.T) == n1 + (1 if w.n_shared else 0)
+    b = layer.forward(inp.x).clone()
+    r = layer.route(x=inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    compare_layer(inp, a, r["idx"].cpu().numpy())
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 1)
+    x2 = synth.make_x(w, w.T, device="cuda", seed=21)
+    c = layer.forward(x2).clone()
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 0)
+    d = layer.forward(x2)
+    torch.cuda.synchronize()
+    assert torch.equal(c.view(torch.int16), d.view(torch.int16))
+    assert layer.device_status() == 0
+    with pytest.raises(MoEError):
+        layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 2)
