@@ -202,7 +202,8 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from sparse_moe_layer_warp_b200 import (MOE_PROFILE_STAGES, PROFILE_STAGE_NAMES, MoELayer,
+    from sparse_moe_layer_warp_b200 import (MOE_OPTION_GEMM_CLOCK, MOE_PROFILE_STAGES,
+                                            PROFILE_STAGE_NAMES, MoELayer,
                                             moe_forward_launch_count,
                                             moe_forward, moe_forward_profiled, synth)
 
@@ -268,6 +269,17 @@ def run_ours(args, rank, world, local_rank):
     status = layer.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
+    # the clock the expert GEMMs actually ran at (SM cycles over %globaltimer inside every
+    # CTA, MOE_OPTION_GEMM_CLOCK), outside the timed region, with the same flushed steps:
+    # under the 1 kW cap it sits well below the sampled clock of the lines above
+    layer.set_option(MOE_OPTION_GEMM_CLOCK, 1)
+    layer.gemm_clock_mhz()
+    for i in range(min(args.steps, 10)):
+        flush.zero_()
+        moe_forward(layer.handle, batches[args.warmup + i], T, out, ws)
+    gemm_mhz = layer.gemm_clock_mhz()
+    layer.set_option(MOE_OPTION_GEMM_CLOCK, 0)
+    clocks["gemm_effective_mhz"] = {"up": round(gemm_mhz[0], 1), "down": round(gemm_mhz[1], 1)}
 
     # end to end through the public API, serial (the bench line's e2e): per step, outside
     # the events the L2 flush as in the device-timed region; inside them the copy of that

@@ -123,10 +123,15 @@ moe_status moe_layer_destroy(moe_handle h);
  *                          which read x directly and are claimed first); 0: a kernel of its own
  *                          writes the copy before the up GEMM (same results, bit for bit).
  *                          Off while the shared expert runs on the side stream.
+ *   MOE_OPTION_GEMM_CLOCK  1: the bf16 forward's expert GEMMs add each CTA's SM cycles and
+ *                          %globaltimer nanoseconds from entry to exit to the workspace's
+ *                          status block, for moe_gemm_clock (two 64-bit atomics per CTA);
+ *                          0 (default): nothing recorded.  Results are the same either way.
  * MOE_ERR_INVALID_ARG for an unknown option or value. */
 #define MOE_OPTION_H_HANDOVER 1
 #define MOE_OPTION_SHARED_SIDE_SMS 2
 #define MOE_OPTION_ROW_GATHER_IN_GEMM 3
+#define MOE_OPTION_GEMM_CLOCK 4
 moe_status moe_set_option(moe_handle h, int option, int value);
 
 /* Bytes of device workspace a call with n_tokens tokens needs (0 on bad arguments).
@@ -183,6 +188,14 @@ int moe_forward_launch_count(moe_handle h, int n_tokens);
 /* Waits for `stream`, then reads and clears the workspace's device status word:
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last query. */
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream);
+
+/* Effective SM clock of the expert GEMMs of the forwards run on this workspace with
+ * MOE_OPTION_GEMM_CLOCK since the last call: mhz[0] the up GEMM's, mhz[1] the down GEMM's
+ * (CTA-time-weighted SM cycles per microsecond of %globaltimer; 0 when none ran).  Waits for
+ * `stream`, reads the sums and clears them.  Under a power or thermal cap this is the clock
+ * the tensor cores actually ran at, which a sampling tool (nvidia-smi) may not resolve inside
+ * a millisecond-long kernel.  MOE_ERR_INVALID_ARG on null arguments or a short workspace. */
+moe_status moe_gemm_clock(moe_handle h, void *ws, size_t ws_bytes, double *mhz, void *stream);
 
 /* Backward of moe_forward: gradients of <out, dout> with respect to x and the weights, for
  * the forward's own selection (recomputed here with the same kernels; the selection carries

@@ -33,11 +33,13 @@ EXPORTS = ("moe_layer_init", "moe_layer_destroy", "moe_workspace_size", "moe_wor
            "moe_selftest_wait_timeout", "moe_expert_health", "moe_backward",
            "moe_backward_workspace_size", "moe_saved_size", "moe_forward_save",
            "moe_backward_saved", "moe_backward_ex", "moe_set_option", "moe_layer_init_ep",
-           "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine")
+           "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine",
+           "moe_gemm_clock")
 MOE_BACKWARD_OVERWRITE = 1
 MOE_OPTION_H_HANDOVER = 1
 MOE_OPTION_SHARED_SIDE_SMS = 2
 MOE_OPTION_ROW_GATHER_IN_GEMM = 3
+MOE_OPTION_GEMM_CLOCK = 4
 MOE_PROFILE_STAGES = 7
 PROFILE_STAGE_NAMES = ("router_logits", "topk_gates_hist", "permute_scatter", "row_gather",
                        "expert_up_swiglu", "expert_down", "combine")
@@ -85,6 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.moe_forward.argtypes = [P, P, I, P, P, Z, P]
         lib.moe_forward_profiled.argtypes = [P, P, I, P, P, Z, P, ctypes.POINTER(P), I]
         lib.moe_device_status.argtypes = [P, P, Z, P]
+        lib.moe_gemm_clock.argtypes = [P, P, Z, ctypes.POINTER(ctypes.c_double), P]
         lib.moe_router_logits_static.argtypes = [P, P, I, P, P]
         lib.moe_router_stats.argtypes = [P, P, P, I, I, P, P, P, P, Z, P]
         lib.moe_update_router_bias.argtypes = [P, P, I, ctypes.c_float, P, P]
@@ -115,7 +118,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                      "moe_update_router_bias", "moe_selftest_wait_timeout",
                      "moe_expert_health", "moe_backward", "moe_forward_save",
                      "moe_backward_saved", "moe_backward_ex", "moe_set_option", "moe_layer_init_ep",
-           "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine"):
+                     "moe_forward_partial", "moe_ep_plan", "moe_ep_pack", "moe_ep_combine",
+                     "moe_gemm_clock"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -353,6 +357,15 @@ def moe_device_status(handle, ws, stream=None) -> int:
                                                  _stream(stream)))
 
 
+def moe_gemm_clock(handle, ws, stream=None) -> tuple:
+    """(up, down) effective SM clock in MHz of the expert GEMMs run with MOE_OPTION_GEMM_CLOCK
+    since the last call (0.0 when none ran); clears the sums."""
+    mhz = (ctypes.c_double * 2)()
+    _check("moe_gemm_clock", load_library().moe_gemm_clock(
+        handle, _p(ws), ws.numel() * ws.element_size(), mhz, _stream(stream)))
+    return float(mhz[0]), float(mhz[1])
+
+
 # ------------------------------------------------------------------ convenience wrapper
 def _expect(t, shape, dtype, name):
     """The C ABI sees only pointers: a tensor of another shape or type would be read or
@@ -527,6 +540,11 @@ class MoELayer:
         moe_expert_health(self.handle, n_tokens, act, par, ratios, self.workspace(n_tokens),
                           stream)
         return act, par, ratios
+
+    def gemm_clock_mhz(self, stream=None) -> tuple:
+        """(up, down) effective SM clock of the forward's expert GEMMs since the last call, for
+        forwards run with MOE_OPTION_GEMM_CLOCK set (see moe_gemm_clock)."""
+        return moe_gemm_clock(self.handle, self.ws, stream)
 
     def device_status(self, stream=None) -> int:
         """Device status of the forward's and the backward's workspaces (0: no bounded wait

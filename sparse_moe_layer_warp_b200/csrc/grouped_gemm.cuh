@@ -96,6 +96,9 @@ struct GemmParams {
   // past *gx_n_rows skipped when gx_n_rows is set) while the shared groups' units, which read
   // x itself, run; a routed unit's loads wait until *gx_done = gx_T.  gx_claim and gx_done
   // are zero at launch; gx_vec = 16-byte vectors per row.
+  // Effective SM clock (null: not measured): each CTA adds its SM cycles and %globaltimer ns
+  // from entry to exit to clock_sum[0] and clock_sum[1].
+  unsigned long long *clock_sum;
   const uint4 *gx_src;
   uint4 *gx_dst;
   const int *gx_slot_row;
@@ -357,6 +360,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
+  ClockSpan *span = reinterpret_cast<ClockSpan *>(tmem_slot + 12);  // effective-clock probe
+  if (p.clock_sum && threadIdx.x == 0) *span = clock_span_start();
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -757,6 +762,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  if (p.clock_sum && threadIdx.x == 0) clock_span_add(*span, p.clock_sum);
 }
 
 }  // namespace moe

@@ -141,6 +141,8 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
+  ClockSpan *span = reinterpret_cast<ClockSpan *>(tmem_slot + 12);  // effective-clock probe
+  if (p.clock_sum && threadIdx.x == 0) *span = clock_span_start();
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                // [G]
   int *grp_row = grp_count + p.n_groups;                        // [G]
@@ -532,6 +534,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
+  if (p.clock_sum && threadIdx.x == 0) clock_span_add(*span, p.clock_sum);
 }
 
 }  // namespace moe

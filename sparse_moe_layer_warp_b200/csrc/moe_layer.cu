@@ -60,6 +60,7 @@ struct moe_layer {
   int handover_fits;
   int opt_handover;
   int opt_gather_in_gemm;  // MOE_OPTION_ROW_GATHER_IN_GEMM
+  int opt_gemm_clock;      // MOE_OPTION_GEMM_CLOCK
   // experts whose weights the handle holds: [e0, e1) (the whole layer: [0, E)); the weight
   // tensors hold e1 - e0 routed experts then the shared expert (moe_layer_init_ep)
   int e0, e1;
@@ -730,6 +731,7 @@ static moe_status layer_init(const moe_config *cfg, const moe_weights *w, int e0
   }
   L->opt_handover = 1;
   L->opt_gather_in_gemm = 1;
+  L->opt_gemm_clock = 0;
   if (c.dtype == MOE_BF16) {
     L->pair_grid[0] = pair_grid_size<MODE_UP>(L);
     L->pair_grid[1] = pair_grid_size<MODE_DOWN>(L);
@@ -800,6 +802,10 @@ moe_status moe_set_option(moe_handle h, int option, int value) {
     case MOE_OPTION_ROW_GATHER_IN_GEMM:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       h->opt_gather_in_gemm = value;
+      return MOE_OK;
+    case MOE_OPTION_GEMM_CLOCK:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      h->opt_gemm_clock = value;
       return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
@@ -943,6 +949,20 @@ moe_status moe_expert_health(moe_handle h, int n_tokens, float *act_rms, float *
   return launch(expert_health_final_kernel, dim3(1), dim3(1024), 0, st, (const double *)act_part,
                 (const double *)par_part, offsets, c.n_experts, G, T, c.d_ff, act_rms,
                 param_norm, ratios);
+}
+
+moe_status moe_gemm_clock(moe_handle h, void *ws, size_t ws_bytes, double *mhz, void *stream) {
+  if (!h || !ws || !mhz || ws_bytes < sizeof(DevStatus)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevStatus *d = static_cast<DevStatus *>(ws);
+  unsigned long long v[4];
+  if (cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemcpy(v, d->gemm_clock, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(d->gemm_clock, 0, sizeof v) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int i = 0; i < 2; ++i)  // cycles per microsecond
+    mhz[i] = v[2 * i + 1] ? 1e3 * (double)v[2 * i] / (double)v[2 * i + 1] : 0.0;
+  return MOE_OK;
 }
 
 moe_status moe_device_status(moe_handle h, void *ws, size_t ws_bytes, void *stream) {
@@ -1162,6 +1182,7 @@ moe_status launch_expert_up(const moe_layer *h, const void *x, int T, void *ws,
     p1.wg_off_routed = slice->wg_off_routed;
     p1.wg_off_shared = slice->wg_off_shared;
   }
+  if (h->opt_gemm_clock && !rows) p1.clock_sum = at<DevStatus>(ws, W.status)->gemm_clock;
   if (gather_rows && plan.pair && !rows) {
     DevStatus *status = at<DevStatus>(ws, W.status);
     p1.shared_first = 1;
@@ -1215,6 +1236,7 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
   if ((s = mark(5)) != MOE_OK) return s;
   GemmParams p2 = p1;  // shared_first carries over: the shared group's h is complete first
   p2.gx_dst = nullptr;
+  if (p1.clock_sum) p2.clock_sum = p1.clock_sum + 2;
   p2.tmA0 = h->tm_wd;
   if (!encode_bf16_2d(&p2.tmB, hbuf, c.d_ff, P, bn2)) return MOE_ERR_CUDA;
   p2.b_boxes = 0;

@@ -20,7 +20,10 @@ struct DevStatus {
                          // chunks claimed and [5] tokens gathered by the CTA-pair up kernel
   int side_sched[2];     // the shared expert's up / down counters when it runs on the side
                          // stream (cleared on that stream before its kernels)
-  int pad[20];
+  // bf16 expert GEMMs with MOE_OPTION_GEMM_CLOCK: SM cycles and %globaltimer ns from entry to
+  // exit of every CTA, summed ([0], [1] up; [2], [3] down), read and cleared by moe_gemm_clock
+  unsigned long long gemm_clock[4];
+  int pad[12];
   int router_ticket[32]; // split-K router: arrivals per block of 32 experts; [31] also the
                          // decode router's last-CTA ticket (all self-resetting)
 };
@@ -32,6 +35,20 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+
+// Per-CTA span of a kernel in SM cycles and %globaltimer ns (for the effective SM clock):
+// start() at entry, add() at exit by the same thread.
+struct ClockSpan {
+  long long c0;
+  unsigned long long t0;
+};
+__device__ __forceinline__ ClockSpan clock_span_start() {
+  return ClockSpan{clock64(), globaltimer_ns()};
+}
+__device__ __forceinline__ void clock_span_add(const ClockSpan &s, unsigned long long *sum) {
+  atomicAdd(sum, (unsigned long long)(clock64() - s.c0));
+  atomicAdd(sum + 1, globaltimer_ns() - s.t0);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

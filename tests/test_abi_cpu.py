@@ -33,7 +33,7 @@ def test_header_constants_match_binding():
     enums = dict((n, int(v)) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", text))
     defines = dict((n, int(v)) for n, v in
                    re.findall(r"^#define\s+(MOE_[A-Z0-9_]+)\s+(\d+)u?\s*$", text, flags=re.M))
-    assert len(enums) == 9 and len(defines) == 5
+    assert len(enums) == 9 and len(defines) == 6
     for name, value in {**enums, **defines}.items():
         assert getattr(binding, name) == value, name
     assert len(binding.PROFILE_STAGE_NAMES) == binding.MOE_PROFILE_STAGES
@@ -164,6 +164,8 @@ def test_expert_parallel_and_option_calls_rejected_on_the_host(lib):
                               None) == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_set_option(None, binding.MOE_OPTION_SHARED_SIDE_SMS,
                               32) == binding.MOE_ERR_INVALID_ARG
+    mhz = (ctypes.c_double * 2)()
+    assert lib.moe_gemm_clock(None, None, 0, mhz, None) == binding.MOE_ERR_INVALID_ARG
 
 
 def test_expert_range_partition():

@@ -10,8 +10,8 @@ bytes in the copy, same results bit for bit."""
 import pytest
 import torch
 
-from sparse_moe_layer_warp_b200 import (MOE_OPTION_H_HANDOVER, MOE_OPTION_ROW_GATHER_IN_GEMM,
-                                        MoEError, synth)
+from sparse_moe_layer_warp_b200 import (MOE_OPTION_GEMM_CLOCK, MOE_OPTION_H_HANDOVER,
+                                        MOE_OPTION_ROW_GATHER_IN_GEMM, MoEError, synth)
 from tests.helpers import compare_layer, make_layer
 
 pytestmark = pytest.mark.gpu
@@ -130,3 +130,28 @@ def test_row_gather_in_up_gemm_matches_own_launch(cuda_ok, kw):
     assert layer.device_status() == 0
     with pytest.raises(MoEError):
         layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 2)
+
+
+@pytest.mark.parametrize("kw", [
+    {"T": 16, "d": 512, "E": 64, "k": 8, "f": 256},               # one-CTA GEMMs
+    {"T": 700, "d": 768, "E": 8, "k": 4, "f": 512, "seed": 6},    # CTA pairs
+])
+def test_gemm_clock_option(cuda_ok, kw):
+    w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", **kw)
+    inp = synth.make_inputs(w, device="cuda")
+    layer = make_layer(inp)
+    a = layer.forward(inp.x).clone()
+    assert layer.gemm_clock_mhz() == (0.0, 0.0)  # off by default: nothing recorded
+    layer.set_option(MOE_OPTION_GEMM_CLOCK, 1)
+    for _ in range(3):
+        b = layer.forward(inp.x)
+    up, down = layer.gemm_clock_mhz()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert 100.0 < up < 3000.0 and 100.0 < down < 3000.0, (up, down)
+    assert layer.gemm_clock_mhz() == (0.0, 0.0)  # read and cleared
+    layer.set_option(MOE_OPTION_GEMM_CLOCK, 0)
+    layer.forward(inp.x)
+    assert layer.gemm_clock_mhz() == (0.0, 0.0)
+    with pytest.raises(MoEError):
+        layer.set_option(MOE_OPTION_GEMM_CLOCK, 2)
