@@ -117,12 +117,14 @@ moe_status moe_layer_destroy(moe_handle h);
  *                          forward records the fork and join into the graph).  Calls on one
  *                          handle from several host threads at once are not supported.
  *                          Not used by moe_forward_profiled or moe_forward_save.
- *   MOE_OPTION_ROW_GATHER_IN_GEMM  1 (default): in bf16 forwards on CTA pairs with a shared
- *                          expert, the up GEMM writes the expert-sorted copy of x itself (two
+ *   MOE_OPTION_ROW_GATHER_IN_GEMM  in bf16 forwards on CTA pairs with a shared expert, who
+ *                          writes the expert-sorted copy of x: 2: the up GEMM itself (two
  *                          warps of each CTA, while the CTAs run the shared expert's units,
- *                          which read x directly and are claimed first); 0: a kernel of its own
- *                          writes the copy before the up GEMM (same results, bit for bit).
- *                          Off while the shared expert runs on the side stream.
+ *                          which read x directly and are claimed first); 1 (default): the
+ *                          same when the shared expert's up units are at least one per CTA
+ *                          pair of the device (d_ff/256 x ceil(T/256) >= SMs/2), else as 0;
+ *                          0: a kernel of its own before the up GEMM.  Same results, bit for
+ *                          bit.  Off while the shared expert runs on the side stream.
  *   MOE_OPTION_GEMM_CLOCK  1: the bf16 forward's expert GEMMs add each CTA's SM cycles and
  *                          %globaltimer nanoseconds from entry to exit to the workspace's
  *                          status block, for moe_gemm_clock (two 64-bit atomics per CTA);

@@ -800,7 +800,7 @@ moe_status moe_set_option(moe_handle h, int option, int value) {
       h->side_sms = value & ~1;  // whole CTA pairs
       return MOE_OK;
     case MOE_OPTION_ROW_GATHER_IN_GEMM:
-      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
       h->opt_gather_in_gemm = value;
       return MOE_OK;
     case MOE_OPTION_GEMM_CLOCK:
@@ -1066,6 +1066,18 @@ struct ForwardPlan {
   int launches;
 };
 
+// The CTA-pair up GEMM writes the sorted copy of x itself (MOE_OPTION_ROW_GATHER_IN_GEMM):
+// 2 always with a shared expert; 1 when the shared expert's n_shared_tokens rows make at
+// least one up unit per CTA pair, so the copy's writes have a wave of shared units to overlap.
+bool gather_in_pair_ok(const moe_layer *L, bool pair, bool side_shared, int n_shared_tokens) {
+  const moe_config &c = L->cfg;
+  if (!pair || !c.n_shared || side_shared || n_shared_tokens <= 0) return false;
+  if (L->opt_gather_in_gemm == 2) return true;
+  const long long units = (long long)(c.d_ff / kPairBM) *
+                          ((n_shared_tokens + kPairBN - 1) / kPairBN) * c.n_shared;
+  return L->opt_gather_in_gemm == 1 && units >= L->pair_grid[0] / 2;
+}
+
 ForwardPlan plan_forward(const moe_layer *L, int T) {
   const moe_config &c = L->cfg;
   ForwardPlan f;
@@ -1075,7 +1087,7 @@ ForwardPlan plan_forward(const moe_layer *L, int T) {
   f.gather_in_gemm = c.dtype == MOE_BF16 && !f.pair && up_gathers_rows(c, T);
   f.handover = c.dtype == MOE_BF16 && L->handover_fits && L->opt_handover;
   f.side_shared = f.pair && c.n_shared && L->side_sms >= 2 && L->side != nullptr;
-  f.gather_in_pair = f.pair && c.n_shared && !f.side_shared && L->opt_gather_in_gemm;
+  f.gather_in_pair = gather_in_pair_ok(L, f.pair, f.side_shared, T);
   if (T == 0) {
     f.launches = 0;
     return f;
@@ -1215,9 +1227,9 @@ moe_status launch_experts_bf16(const moe_layer *h, const void *x, int T, void *w
   };
   moe_status s;
   ForwardPlan pl = plan;
-  // the up kernel gathers the rows while it runs the shared expert's units: not in a launch
-  // without them
-  if (slice && slice->shared_n == 0) pl.gather_in_pair = false;
+  // the up kernel gathers the rows while it runs the shared expert's units: an expert-range
+  // launch decides by its own shared rows
+  if (slice) pl.gather_in_pair = gather_in_pair_ok(h, pl.pair, pl.side_shared, slice->shared_n);
   const bool pair = pl.pair;
   const int bn = pair ? PairCfg<MODE_UP>::HALF_BN : pick_bn(c, T, MODE_UP);
   if ((s = launch_row_gather(h, x, T, ws, W, pl, st, n_rows_dev)) != MOE_OK ||
@@ -1362,7 +1374,7 @@ static moe_status forward_impl(moe_handle h, const void *x, int n_tokens, void *
   // launch)
   if (events || saved) {
     plan.side_shared = false;
-    plan.gather_in_pair = plan.pair && c.n_shared && h->opt_gather_in_gemm;
+    plan.gather_in_pair = gather_in_pair_ok(h, plan.pair, false, T);
   }
   if (plan.side_shared && (s = launch_shared_side(h, x, T, ws, W, st)) != MOE_OK) return s;
   if (plan.decode_route) {

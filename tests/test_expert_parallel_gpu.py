@@ -42,12 +42,15 @@ def _round(layer, s):
 
 @pytest.mark.parametrize("kw", CASES)
 @pytest.mark.parametrize("R", [2, 4])
-def test_partials_over_expert_slices_sum_to_the_layer(cuda_ok, kw, R):
+@pytest.mark.parametrize("gather", [1, 2])
+def test_partials_over_expert_slices_sum_to_the_layer(cuda_ok, kw, R, gather):
     """Partials of a partition of the experts (the shared expert in one of them) add up to
     the layer: within fp32 reordering of the forward's sum, and within the parity bound of
-    the oracle."""
+    the oracle.  gather = 2: CTA-pair partials write the sorted copy inside the up GEMM,
+    skipping the rows of other ranks' experts."""
     w, inp = _inputs(kw)
     layer = make_layer(inp)
+    layer.set_option(binding.MOE_OPTION_ROW_GATHER_IN_GEMM, gather)
     full = layer.forward(inp.x)
     T = w.T
     tot = torch.zeros((T, w.d), dtype=torch.float32, device="cuda")

@@ -68,11 +68,13 @@ def test_shared_expert_on_side_stream_matches(cuda_ok, kw, sms):
     inp = synth.make_inputs(w, device="cuda")
     layer = make_layer(inp)
     ref = layer.forward(inp.x).clone()
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 0)
     n0 = moe_forward_launch_count(layer.handle, w.T)
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 1)
     layer.set_option(MOE_OPTION_SHARED_SIDE_SMS, sms)
-    # the two side GEMMs, and the row gather's own launch (the up GEMM gathers the rows
+    # the two side GEMMs; the row gather has its own launch (the up GEMM gathers the rows
     # itself only while it runs the shared expert's units)
-    assert moe_forward_launch_count(layer.handle, w.T) == n0 + 3
+    assert moe_forward_launch_count(layer.handle, w.T) == n0 + 2
     a = layer.forward(inp.x).clone()
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
@@ -104,32 +106,49 @@ def test_shared_expert_on_side_stream_matches(cuda_ok, kw, sms):
     {"T": 900, "d": 512, "E": 16, "k": 4, "f": 256, "seed": 9, "n_shared": 0},  # no shared
 ])
 def test_row_gather_in_up_gemm_matches_own_launch(cuda_ok, kw):
-    """The CTA-pair up GEMM's own row gather (default) against the gather kernel: outputs
-    equal bit for bit, both equal to the oracle; one launch fewer with a shared expert."""
+    """The CTA-pair up GEMM's own row gather (2: forced; these shapes have too few shared
+    units for the default to choose it) against the gather kernel (0): outputs equal bit for
+    bit, both equal to the oracle, one launch fewer with a shared expert; the in-GEMM gather
+    replays from a CUDA graph."""
     from sparse_moe_layer_warp_b200 import moe_forward_launch_count
 
     w = synth.WORKLOADS["tiny_fp32"].replace(dtype="bf16", **kw)
     inp = synth.make_inputs(w, device="cuda")
     layer = make_layer(inp)
     n1 = moe_forward_launch_count(layer.handle, w.T)
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 2)
+    n2 = moe_forward_launch_count(layer.handle, w.T)
+    assert n2 == n1 - (1 if w.n_shared else 0)
     a = layer.forward(inp.x).clone()
     layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 0)
-    assert moe_forward_launch_count(layer.handle, w.T) == n1 + (1 if w.n_shared else 0)
+    assert moe_forward_launch_count(layer.handle, w.T) == n1
     b = layer.forward(inp.x).clone()
     r = layer.route(x=inp.x)
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     compare_layer(inp, a, r["idx"].cpu().numpy())
-    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 1)
-    x2 = synth.make_x(w, w.T, device="cuda", seed=21)
-    c = layer.forward(x2).clone()
+    # captured with the in-GEMM gather, replayed on another batch
+    layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 2)
+    x = inp.x.clone()
+    out = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward(x, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, out=out)
+    x.copy_(synth.make_x(w, w.T, device="cuda", seed=21))
+    g.replay()
     layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 0)
-    d = layer.forward(x2)
+    d = layer.forward(x)
     torch.cuda.synchronize()
-    assert torch.equal(c.view(torch.int16), d.view(torch.int16))
+    assert torch.equal(out.view(torch.int16), d.view(torch.int16))
+    del g
     assert layer.device_status() == 0
     with pytest.raises(MoEError):
-        layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 2)
+        layer.set_option(MOE_OPTION_ROW_GATHER_IN_GEMM, 3)
 
 
 @pytest.mark.parametrize("kw", [
