@@ -15,6 +15,7 @@ decode_t256        256    4096   288  8   1280   bf16; batched decode
 prefill_t8192      8192   4096   288  8   1280   bf16; prefill chunk
 skew_t4096         4096   4096   288  8   1280   bf16; Zipf(1.1)-skewed expert selection
 prefill_e32_t1024  1024   4096   32   8   1280   bf16; profiler-sized prefill-like case
+prefill_e128_t4096 4096   4096   128  8   1280   bf16; same, with a wave of shared-expert units
 decode_e32_t16     16     4096   32   8   1280   bf16; profiler-sized decode-like case
 dense_ffn_t4096    4096   4096   1    1   11264  bf16; dense SwiGLU FFN, no shared expert
 =================  =====  =====  ===  ==  =====  ======================================
@@ -67,6 +68,10 @@ WORKLOADS = {
     # small case with prefill's per-expert load (~256 tokens per expert) and full-size
     # expert matrices, ~1 GB of weights: for profiler captures that must stay small
     "prefill_e32_t1024": Workload("prefill_e32_t1024", T=1024, d=4096, E=32, k=8, f=1280),
+    # the same per-expert load with enough tokens (80 shared-expert up units, more than the
+    # 74 CTA pairs) that the CTA-pair up GEMM writes the sorted copy of x itself; ~4 GB of
+    # weights
+    "prefill_e128_t4096": Workload("prefill_e128_t4096", T=4096, d=4096, E=128, k=8, f=1280),
     # small case with decode's per-expert load (~4 tokens per expert, the same 16-token tiles
     # with rows gathered by TMA) and full-size expert matrices, ~1 GB of weights
     "decode_e32_t16": Workload("decode_e32_t16", T=16, d=4096, E=32, k=8, f=1280),
