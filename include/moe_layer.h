@@ -394,11 +394,9 @@ moe_status moe_ep_combine(moe_handle h, const float *back, const int *send_slot,
 const char *moe_status_string(moe_status s);
 
 /* Router logits without any caller workspace, for callers that cannot allocate device
- * memory: for example code that runs while a CUDA graph is being captured (a device
- * allocation is not allowed there), plugin or embedding hosts that hand the library only its
- * input and output buffers, and latency-critical decode loops that must not touch an
- * allocator.  (No counterpart on the pages: this is a deployment convenience, not part of
- * the layer's method.)
+ * memory: plugin or embedding hosts that hand the library only its input and output buffers,
+ * and latency-critical decode loops that must not touch an allocator.  (No counterpart on
+ * the pages: this is a deployment convenience, not part of the layer's method.)
  *
  * Computes logits_out[t, e] = x_t . W_r[e] (fp32, [n_tokens, E], row-major) with a split-K
  * kernel in a fixed summation order (deterministic).  Where moe_route uses the same kernel
@@ -411,13 +409,12 @@ const char *moe_status_string(moe_status s);
  * GPU that loads the library holds until the process exits.  Limits: 1 <= n_tokens <= 64 and
  * ceil(d_model / 256) * n_tokens * E * 4 bytes <= 2 MiB (for d_model = 4096, E = 288: up to
  * 64 tokens); larger requests return MOE_ERR_UNSUPPORTED before anything is launched.
- * The first call on each device looks up the buffer's device address (host-side set-up), so
- * make that first call before capturing a stream into a CUDA graph.  The address is kept for
- * the life of the process: do not use the library across a device reset
- * (cudaDeviceReset), which may move the buffer.  The current device must be the one the
- * handle was created on (MOE_ERR_INVALID_ARG otherwise).  All calls on a device
- * share the one buffer: calls that may overlap on the GPU (different streams without
- * ordering) race and give wrong results; serialise them.  Asynchronous on `stream`. */
+ * The first call on each device looks up the buffer's device address (host-side set-up).
+ * The address is kept for the life of the process: do not use the library across a device
+ * reset (cudaDeviceReset), which may move the buffer.  The current device must be the one
+ * the handle was created on (MOE_ERR_INVALID_ARG otherwise).  All calls on a device share
+ * the one buffer: calls that may overlap on the GPU (different streams without ordering)
+ * race and give wrong results; serialise them.  Asynchronous on `stream`. */
 moe_status moe_router_logits_static(moe_handle h, const void *x, int n_tokens,
                                     float *logits_out, void *stream);
 

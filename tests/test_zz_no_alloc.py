@@ -1,7 +1,7 @@
 """The allocation-free router entry point (moe_router_logits_static).
 
-Some callers cannot allocate device memory -- for example code running while a CUDA graph
-is captured, or a plugin host that only hands over input and output buffers -- so this
+Some callers cannot allocate device memory -- for example a plugin host that only hands
+over input and output buffers -- so this
 entry point keeps its scratch in the library's own static device buffer instead of a
 caller workspace.  These tests call it through the C ABI and check it against the regular
 workspace-based routing call, twice in a row (the shared buffer keeps the previous call's
