@@ -234,14 +234,16 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
       int qi = 0;
       uint32_t qph = 0;
       int u = -1;
+      int ticket = -1;       // leader: its claim cursor
       int ready_group = -1;  // down kernel: group whose h is known to be complete
       bool gathered = !(MODE == MODE_UP && p.gx_dst);  // up: the sorted copy is complete
       while (ok) {
         // the leader claims the next unit and publishes its id to both CTAs; the peer reads it
         if (leader) {
-          u = claim(u);
-          const int uid =
-              (u < total_units) ? unit_of_ticket(u, n_first, n_heavy, total_units) : -1;
+          ticket = claim(ticket);
+          const int uid = (ticket < total_units)
+                              ? unit_of_ticket(ticket, n_first, n_heavy, total_units)
+                              : -1;
           if (!mbar_wait_bounded<true>(&uq_empty[qi], qph ^ 1, abort_flag, p.status, 15)) {
             ok = false;
             break;
