@@ -360,6 +360,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
+  uint64_t *epi_bar = reinterpret_cast<uint64_t *>(tmem_slot + 2);  // epilogue warps' barrier
   ClockSpan *span = reinterpret_cast<ClockSpan *>(tmem_slot + 12);  // effective-clock probe
   if (p.clock_sum && threadIdx.x == 0) *span = clock_span_start();
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
@@ -388,6 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(epi_bar, 4);
     for (int q = 0; q < kUnitQ; ++q) {
       mbar_init(&uq_full[q], 1);
       mbar_init(&uq_empty[q], 5);  // the MMA thread and the four epilogue warps
@@ -659,7 +661,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
           row_scale[acc * BN + n] = sc;
         }
-        named_bar_sync(1, 128);
+        // all epilogue warps' scales are staged before any reads them: a bounded mbarrier (one
+        // arrival per warp) instead of bar.sync, so a warp that aborts leaves none waiting
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_bar);
+        if (!warp_wait(epi_bar, (uint32_t)(it - 1) & 1, 71)) break;
       }
       float *wbuf = xbuf + q * 16 * 32;
       const int col_base = mt * kBM + q * 32;  // first output column of this warp

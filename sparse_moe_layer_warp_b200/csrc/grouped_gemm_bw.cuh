@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *uq_empty = uq_full + kUnitQ;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint64_t *epi_bar = reinterpret_cast<uint64_t *>(tmem_slot + 2);  // epilogue warps' barrier
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);        // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                     // [G]
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(epi_bar, 4);
     for (int q = 0; q < kUnitQ; ++q) {
       mbar_init(&uq_full[q], 1);
       mbar_init(&uq_empty[q], 5);
@@ -459,7 +461,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (MODE == BW_DH) {
         for (int n = threadIdx.x - 64; n < BN; n += 128)
           row_scale[acc * BN + n] = (n < valid) ? p.row_scale[rowu0 + n] : 0.f;
-        named_bar_sync(1, 128);
+        // all epilogue warps' scales are staged before any reads them: a bounded mbarrier (one
+        // arrival per warp) instead of bar.sync, so a warp that aborts leaves none waiting
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_bar);
+        if (!warp_wait(epi_bar, (uint32_t)(it - 1) & 1, 73)) break;
       }
       uint32_t nx[16];
       tmem_ld16(taddr, nx);
@@ -583,6 +589,7 @@ __global__ void __launch_bounds__(kBwPairThreads, 1)
   uint64_t *uq_empty = uq_full + kUnitQ;  // used in the leader only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(uq_empty + kUnitQ);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint64_t *epi_bar = reinterpret_cast<uint64_t *>(tmem_slot + 2);  // epilogue warps' barrier
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ]
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);        // [G + 1]
   int *grp_count = unit_prefix + p.n_groups + 1;                     // [G]
@@ -611,6 +618,7 @@ __global__ void __launch_bounds__(kBwPairThreads, 1)
       mbar_init(&tempty[a], 2 * kBwPairEpiWarps);
     }
     mbar_init(drain, 1);
+    mbar_init(epi_bar, kBwPairEpiWarps);
     for (int q = 0; q < kUnitQ; ++q) {
       mbar_init(&uq_full[q], 1);
       mbar_init(&uq_empty[q], 2 + 2 * kBwPairEpiWarps);
@@ -858,7 +866,11 @@ __global__ void __launch_bounds__(kBwPairThreads, 1)
       if (MODE == BW_DH) {
         for (int n = threadIdx.x - 64; n < BN; n += 32 * kBwPairEpiWarps)
           row_scale[acc * BN + n] = (n < valid) ? p.row_scale[rowu0 + n] : 0.f;
-        named_bar_sync(1, 32 * kBwPairEpiWarps);
+        // all epilogue warps' scales are staged before any reads them: a bounded mbarrier (one
+        // arrival per warp) instead of bar.sync, so a warp that aborts leaves none waiting
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_bar);
+        if (!warp_wait(epi_bar, (uint32_t)(it - 1) & 1, 74, false)) break;
       }
       uint32_t nx[16];
       const int c_first = 16 * eh;

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
   volatile int *uq = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kUnitQ] unit ids
   int *n_heavy_s = reinterpret_cast<int *>(tmem_slot + 8);
   int *n_first_s = reinterpret_cast<int *>(tmem_slot + 9);
+  uint64_t *epi_bar = reinterpret_cast<uint64_t *>(tmem_slot + 2);  // epilogue warps' barrier
   ClockSpan *span = reinterpret_cast<ClockSpan *>(tmem_slot + 12);  // effective-clock probe
   if (p.clock_sum && threadIdx.x == 0) *span = clock_span_start();
   int *unit_prefix = reinterpret_cast<int *>(tmem_slot + 16);  // [G + 1]
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
       mbar_init(&tempty[a], 2 * kPairEpiWarps);  // one per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    mbar_init(epi_bar, kPairEpiWarps);
     for (int q = 0; q < kUnitQ; ++q) {
       mbar_init(&uq_full[q], 1);
       // readers of a published unit id: the leader's MMA thread and epilogue warps, the
@@ -444,7 +446,11 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
           if (n < valid) sc = (g < p.E) ? p.routed_scale * p.topk_gate[p.perm[row0 + n]] : 1.f;
           row_scale[acc * BN + n] = sc;
         }
-        named_bar_sync(1, 32 * kPairEpiWarps);
+        // all epilogue warps' scales are staged before any reads them: a bounded mbarrier (one
+        // arrival per warp) instead of bar.sync, so a warp that aborts leaves none waiting
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_bar);
+        if (!warp_wait(epi_bar, (uint32_t)(it - 1) & 1, 72, false)) break;
       }
       float *wbuf = xbuf + (warp - 2) * 16 * 32;
       const int col_base = mt * kPairBM + (int)rank * 128 + q * 32;
