@@ -166,15 +166,19 @@ class ExpertParallelMoE:
         xr = torch.empty((n_recv, x.shape[1]), dtype=x.dtype, device=x.device)
         ir = torch.empty((n_recv, ids.shape[1]), dtype=ids.dtype, device=x.device)
         gr = torch.empty((n_recv, gs.shape[1]), dtype=gs.dtype, device=x.device)
-        dist.all_to_all_single(xr, xs, recv, send, group=self.group)
-        dist.all_to_all_single(ir, ids, recv, send, group=self.group)
-        dist.all_to_all_single(gr, gs, recv, send, group=self.group)
+        pending = [dist.all_to_all_single(xr, xs, recv, send, group=self.group, async_op=True),
+                   dist.all_to_all_single(ir, ids, recv, send, group=self.group, async_op=True),
+                   dist.all_to_all_single(gr, gs, recv, send, group=self.group, async_op=True)]
+        # the shared expert on this rank's own tokens needs nothing from the exchange: it runs
+        # while the rows are in flight (on the compute stream, beside the collectives' own)
+        shared = ops.partial(x, idx, gates, (self.experts[0], self.experts[0]), (0, T))
+        for work in pending:
+            work.wait()
         # the received tokens' slots in this rank's experts (no shared expert here)
         part = ops.partial(xr, ir, gr, self.experts, (0, 0))
         back = torch.empty((n_send, x.shape[1]), dtype=torch.float32, device=x.device)
         dist.all_to_all_single(back, part, send, recv, group=self.group)
-        # the shared expert on this rank's own tokens, then the per-token sum in rank order
-        shared = ops.partial(x, idx, gates, (self.experts[0], self.experts[0]), (0, T))
+        # the per-token sum in rank order
         return ops.combine(back, slot, offsets, shared, R, T)
 
     def _forward_allgather(self, x):
