@@ -140,9 +140,9 @@ def kernel_roofline(algo, key, dur_s, peaks):
 
 
 def tensor_peak_regime(peaks, gemm_mhz):
-    """The measured bf16 peak whose clock regime the expert GEMMs ran in: the sustained figure
-    (the GEMM loop held at the 1 kW cap) when the GEMMs' own effective clock is within 10 % of
-    that loop's median SM clock, else the burst figure.  Returns (TFLOP/s, regime, note)."""
+    """Which measured bf16 peak's clock regime the expert GEMMs ran in: "sustained" (the GEMM
+    loop held at the 1 kW cap) when the GEMMs' own effective clock is within 10 % of that
+    loop's median SM clock, else "burst".  Returns (TFLOP/s of that regime, regime, note)."""
     sus = peaks.get("bf16_tflops_sustained")
     med = (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")
     if sus and med and gemm_mhz and abs(gemm_mhz - med) <= 0.1 * med:
@@ -153,17 +153,18 @@ def tensor_peak_regime(peaks, gemm_mhz):
 
 
 def layer_roofline(layer_bytes, layer_flops, step_s, peaks, gemm_mhz=None):
-    """The whole forward against the bf16 peak of its clock regime when it is tensor-bound
-    (layer flops per algorithmic byte above the ridge of the burst peaks), else None."""
+    """The whole forward against the burst bf16 peak when it is tensor-bound (layer flops per
+    algorithmic byte above the ridge of the burst peaks), else None.  Beside it: the fraction
+    of the peak whose clock regime the GEMMs were measured in (gemm_mhz), with the evidence."""
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if layer_flops / layer_bytes <= ridge:
         return None
-    peak, regime, note = tensor_peak_regime(peaks, gemm_mhz)
+    peak_rg, regime, note = tensor_peak_regime(peaks, gemm_mhz)
     achieved = layer_flops / step_s / 1e12
-    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-            "peak_regime": regime, "peak_regime_evidence": note,
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "clock_regime": regime, "frac_of_clock_regime_peak": round(achieved / peak_rg, 4),
+            "clock_regime_evidence": note,
             "scope": "layer", "algorithmic_flops_per_step": int(layer_flops),
             "algorithmic_bytes_per_step": int(layer_bytes)}
 
@@ -393,9 +394,9 @@ def run_ours(args, rank, world, local_rank):
     kern["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
     # the roofline of the whole forward when the workload is tensor-bound (its flops per
     # algorithmic byte above the ridge of the burst peaks): one forward's flops over the
-    # plain step time against the measured bf16 peak of the clock regime the GEMMs ran in
-    # (their effective clock, measured above); otherwise the dominant kernel's, which
-    # streams the weights at the HBM bound
+    # plain step time against the burst bf16 peak, and beside it against the peak of the
+    # clock regime the GEMMs were measured in (their effective clock, above); otherwise the
+    # dominant kernel's, which streams the weights at the HBM bound
     t_up, t_down = mean_stage[up_i], mean_stage[down_i]
     gemm_mhz = ((t_up * gemm_mhz_pair[0] + t_down * gemm_mhz_pair[1]) / (t_up + t_down)
                 if (t_up + t_down) > 0 and min(gemm_mhz_pair) > 0 else None)
@@ -405,7 +406,7 @@ def run_ours(args, rank, world, local_rank):
     else:
         roof["traffic"] = ncu_traffic("layer", args.workload)
         roof["kernel"] = "moe_forward (all kernels of one forward)"
-        roof["peak_source"] = kern["peak_source"] + f", {roof['peak_regime']} bf16"
+        roof["peak_source"] = kern["peak_source"] + ", burst bf16"
     value = job_throughput(T, args.steps, world, total_ms)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

@@ -76,8 +76,8 @@ def test_dense_ffn_has_no_shared_rows():
 def test_layer_roofline_is_the_tensor_fraction_of_a_tensor_bound_forward():
     """prefill_t8192 (every expert touched: 289 x 3 x 1280 x 4096 x 2 B + W_r + x + out =
     9.23 GB, 2.34 TFLOP, 253 flop/B above the measured ridge of 1642.5 / 6554.2 = 250.6):
-    the bench line's roofline is the forward's flops over the step time against the bf16
-    peak (burst when no GEMM clock is given).  decode_t16 (1.4 flop/B) is HBM-bound: no layer tensor roofline."""
+    the bench line's roofline is the forward's flops over the step time against the burst
+    bf16 peak.  decode_t16 (1.4 flop/B) is HBM-bound: no layer tensor roofline."""
     peaks = {"hbm_gbs": 6554.2, "bf16_tflops": 1642.5}
     w = synth.WORKLOADS["prefill_t8192"]
     a = bench.algorithmic(w, _counts(288, 288, 8192 * 8), 8192)
@@ -93,8 +93,9 @@ def test_layer_roofline_is_the_tensor_fraction_of_a_tensor_bound_forward():
 
 
 def test_layer_roofline_peak_follows_the_measured_gemm_clock():
-    """The sustained bf16 peak is the denominator only when the GEMMs' own effective clock is
-    within 10 % of the sustained loop's median clock; otherwise (or unmeasured) the burst."""
+    """frac stays the burst fraction; the clock-regime fraction beside it uses the sustained
+    peak only when the GEMMs' own effective clock is within 10 % of the sustained loop's
+    median clock; otherwise (or unmeasured) the burst peak."""
     peaks = {"hbm_gbs": 6554.2, "bf16_tflops": 1642.5, "bf16_tflops_sustained": 1394.5,
              "clocks_under_load": {"sm_mhz_median": 1335.0}}
     w = synth.WORKLOADS["prefill_t8192"]
@@ -102,10 +103,11 @@ def test_layer_roofline_peak_follows_the_measured_gemm_clock():
     args = (a["layer_bytes"], a["layer_flops"], 2.85e-3, peaks)
     ach = a["layer_flops"] / 2.85e-3 / 1e12
     r = bench.layer_roofline(*args, gemm_mhz=1370.0)
-    assert r["peak_regime"] == "sustained" and r["peak"] == 1394.5
-    assert r["frac"] == round(ach / 1394.5, 4) and r["frac_of_burst"] == round(ach / 1642.5, 4)
+    assert r["peak"] == 1642.5 and r["frac"] == round(ach / 1642.5, 4)
+    assert r["clock_regime"] == "sustained"
+    assert r["frac_of_clock_regime_peak"] == round(ach / 1394.5, 4)
     for mhz in (None, 1900.0, 1100.0):
         r = bench.layer_roofline(*args, gemm_mhz=mhz)
-        assert r["peak_regime"] == "burst" and r["frac"] == r["frac_of_burst"]
+        assert r["clock_regime"] == "burst" and r["frac_of_clock_regime_peak"] == r["frac"]
     del peaks["bf16_tflops_sustained"]
-    assert bench.layer_roofline(*args, gemm_mhz=1370.0)["peak_regime"] == "burst"
+    assert bench.layer_roofline(*args, gemm_mhz=1370.0)["clock_regime"] == "burst"
